@@ -1,0 +1,13 @@
+"""fp64 CPU oracle for the multi-pattern dilated-attention forward.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the package smoke check
+and by the benchmark's CPU-baseline leg, never by the product path.  It shares
+no code with the CUDA library (see oracle.c for the method it restates).
+"""
+from .oracle import (  # noqa: F401
+    build_oracle,
+    dilated_attn_fp64,
+    dilated_attn_rows_fp64,
+    num_threads,
+)
+from .brute import dilated_attn_bruteforce  # noqa: F401

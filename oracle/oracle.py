@@ -1,0 +1,111 @@
+"""ctypes wrapper around oracle.c (TEST INFRASTRUCTURE ONLY).
+
+The C file holds the arithmetic; this wrapper only builds it with gcc, widens
+inputs to float64 and passes pointers.  Nothing here is imported by the
+product path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, OpenMP, -O2)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-Wall", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load_library(path: str | None = None):
+    """Load liboracle.so (or another build of oracle.c given by path)."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(path or build_oracle())
+    i64, dp, ip = ctypes.c_int64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_dilated_attn_fp64.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64,
+                                             ctypes.c_int, ip, ip, ctypes.c_int]
+    lib.oracle_dilated_attn_fp64.restype = ctypes.c_int
+    lib.oracle_dilated_attn_rows_fp64.argtypes = [dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
+                                                  ip, ip, ctypes.c_int, i64, ip, dp, dp]
+    lib.oracle_dilated_attn_rows_fp64.restype = ctypes.c_int
+    lib.oracle_num_threads.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact widening to a C-contiguous float64 array (bf16/fp32 -> fp64 is exact)."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, t=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(t))
+
+
+def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None):
+    """Full fp64 forward.  q, k, v: [B, N, H, D].  patterns: [(w, r), ...].
+
+    Returns (out [B, N, H, D] float64, lse [B, H, N] float64).
+    """
+    lib = lib or load_library()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N, H, D = q.shape
+    w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)
+    r = np.ascontiguousarray([p[1] for p in patterns], dtype=np.int64)
+    out = np.empty_like(q)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    rc = lib.oracle_dilated_attn_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H, D,
+                                      len(patterns), _ptr(w, ctypes.c_int64), _ptr(r, ctypes.c_int64),
+                                      int(bool(causal)))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out, lse
+
+
+def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None):
+    """fp64 forward of selected rows only.  rows_bph: int array [n, 3] of (b, pos, h).
+
+    Returns (out_rows [n, D], lse_rows [n]).
+    """
+    lib = lib or load_library()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N, H, D = q.shape
+    rows = np.ascontiguousarray(np.asarray(rows_bph, dtype=np.int64).reshape(-1, 3))
+    w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)
+    r = np.ascontiguousarray([p[1] for p in patterns], dtype=np.int64)
+    out = np.empty((rows.shape[0], D), dtype=np.float64)
+    lse = np.empty((rows.shape[0],), dtype=np.float64)
+    rc = lib.oracle_dilated_attn_rows_fp64(_ptr(q), _ptr(k), _ptr(v), B, N, H, D, len(patterns),
+                                           _ptr(w, ctypes.c_int64), _ptr(r, ctypes.c_int64),
+                                           int(bool(causal)), rows.shape[0],
+                                           _ptr(rows, ctypes.c_int64), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return out, lse
+
+
+def num_threads(lib=None) -> int:
+    """OpenMP threads the oracle runs on."""
+    return int((lib or load_library()).oracle_num_threads())

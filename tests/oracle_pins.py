@@ -1,0 +1,259 @@
+"""Pins for the fp64 oracle, written as plain check functions.
+
+Each check takes a loaded build of oracle.c (``lib``) and raises AssertionError
+when the oracle disagrees with something fixed independently of it: a library
+routine on a case that reduces to textbook attention, a second formulation,
+a closed form, a hand-written fixture, or an invariant of the mathematics.
+tests/test_oracle_pins.py runs them on the real oracle; tests/test_oracle_mutants.py
+runs them on deliberately broken copies and expects each copy to fail one.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle.oracle as orc
+from oracle.brute import dilated_attn_bruteforce
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rand(shape, seed):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape)
+
+
+def _sdpa(q, k, v, mask=None, causal=False):
+    """torch's scaled_dot_product_attention in fp64; inputs [N, D] per head."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x))[None, None] for x in (q, k, v))
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=m, is_causal=causal)
+    return o[0, 0].numpy()
+
+
+def _logsumexp_masked(q, k, mask):
+    s = torch.from_numpy(q) @ torch.from_numpy(k).T / math.sqrt(q.shape[-1])
+    s = s.masked_fill(~torch.from_numpy(mask), -math.inf)
+    return torch.logsumexp(s, dim=-1).numpy()
+
+
+def check_dense_causal(lib):
+    """One pattern with w = N, r = 1 is ordinary causal softmax attention."""
+    B, N, H, D = 2, 48, 3, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (1, 2, 3))
+    out, lse = orc.dilated_attn_fp64(q, k, v, [(N, 1)], causal=True, lib=lib)
+    tri = np.tril(np.ones((N, N), dtype=bool))
+    for b in range(B):
+        for h in range(H):
+            ref = _sdpa(q[b, :, h], k[b, :, h], v[b, :, h], causal=True)
+            np.testing.assert_allclose(out[b, :, h], ref, atol=1e-12, rtol=0)
+            ref_l = _logsumexp_masked(q[b, :, h], k[b, :, h], tri)
+            np.testing.assert_allclose(lse[b, h], ref_l, atol=1e-12, rtol=0)
+
+
+def check_dense_noncausal(lib):
+    """One pattern with w = N, r = 1, non-causal is full softmax attention."""
+    B, N, H, D = 1, 40, 2, 16
+    q, k, v = (_rand((B, N, H, D), s) for s in (4, 5, 6))
+    out, lse = orc.dilated_attn_fp64(q, k, v, [(N, 1)], causal=False, lib=lib)
+    full = np.ones((N, N), dtype=bool)
+    for h in range(H):
+        ref = _sdpa(q[0, :, h], k[0, :, h], v[0, :, h], causal=False)
+        np.testing.assert_allclose(out[0, :, h], ref, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse[0, h], _logsumexp_masked(q[0, :, h], k[0, :, h], full),
+                                   atol=1e-12, rtol=0)
+
+
+def check_block_diagonal(lib):
+    """r = 1 with w < N is block-diagonal attention (causal inside each block)."""
+    B, N, H, D, w = 1, 60, 2, 8, 12
+    q, k, v = (_rand((B, N, H, D), s) for s in (7, 8, 9))
+    for causal in (True, False):
+        out, _ = orc.dilated_attn_fp64(q, k, v, [(w, 1)], causal=causal, lib=lib)
+        blk = np.arange(N) // w
+        mask = blk[:, None] == blk[None, :]
+        if causal:
+            mask &= np.tril(np.ones((N, N), dtype=bool))
+        for h in range(H):
+            ref = _sdpa(q[0, :, h], k[0, :, h], v[0, :, h], mask=mask)
+            np.testing.assert_allclose(out[0, :, h], ref, atol=1e-12, rtol=0)
+
+
+def read_selection_fixture():
+    sel = {}
+    with open(os.path.join(GOLDEN, "selection_N24_w12_r5_H3.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, rest = line.split(":")
+            segs = [[int(t) for t in part.split()] for part in rest.split("|")]
+            sel[int(head)] = segs
+    return sel
+
+
+def check_dilated_equals_gathered(lib):
+    """One dilated pattern is dense attention on the rows listed by hand in
+    the selection fixture; rows no head keeps come out as 0 / -inf."""
+    sel = read_selection_fixture()
+    B, N, H, D = 1, 24, 3, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (10, 11, 12))
+    for causal in (True, False):
+        out, lse = orc.dilated_attn_fp64(q, k, v, [(12, 5)], causal=causal, lib=lib)
+        for h in range(H):
+            kept = set()
+            for rows in sel[h]:
+                kept.update(rows)
+                idx = np.array(rows)
+                ref = _sdpa(q[0, idx, h], k[0, idx, h], v[0, idx, h], causal=causal)
+                np.testing.assert_allclose(out[0, idx, h], ref, atol=1e-12, rtol=0)
+                m = np.tril(np.ones((len(rows),) * 2, dtype=bool)) if causal else \
+                    np.ones((len(rows),) * 2, dtype=bool)
+                np.testing.assert_allclose(lse[0, h, idx],
+                                           _logsumexp_masked(q[0, idx, h], k[0, idx, h], m),
+                                           atol=1e-12, rtol=0)
+            for pos in range(N):
+                if pos not in kept:
+                    assert np.all(out[0, pos, h] == 0.0)
+                    assert lse[0, h, pos] == -math.inf
+
+
+def read_support_fixture():
+    sup = {}
+    with open(os.path.join(GOLDEN, "support_N12_mix.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            left, right = line.split(":")
+            h, pos = (int(t) for t in left.split())
+            sup[(h, pos)] = [int(t) for t in right.split()]
+    return sup
+
+
+def check_support_and_uniform_weights(lib):
+    """Q = 0 makes every score 0, so each row averages V over the multiset of
+    keys that reach it, and lse = log(count).  With V one-hot over positions
+    (D = N), out[pos] is the key histogram / count: compared with the
+    hand-written multiset fixture."""
+    sup = read_support_fixture()
+    B, N, H = 1, 12, 2
+    D = N
+    q = np.zeros((B, N, H, D))
+    k = _rand((B, N, H, D), 13)
+    v = np.zeros((B, N, H, D))
+    for pos in range(N):
+        v[0, pos, :, pos] = 1.0
+    out, lse = orc.dilated_attn_fp64(q, k, v, [(4, 1), (6, 2), (12, 3)], causal=True, lib=lib)
+    for (h, pos), keys in sup.items():
+        hist = np.bincount(keys, minlength=N) / len(keys)
+        np.testing.assert_allclose(out[0, pos, h], hist, atol=1e-14, rtol=0)
+        assert abs(lse[0, h, pos] - math.log(len(keys))) < 1e-14
+
+
+def check_bruteforce_agreement(lib):
+    """Per-pattern attention + combination agrees with one softmax over the
+    multiset union of (pattern, key) pairs, on shapes where r does not divide
+    w, heads have different offsets and rows are reached by 1..3 patterns."""
+    cases = [
+        (1, 36, 5, 4, [(12, 5), (18, 3), (36, 7)], True, 21),
+        (2, 30, 3, 6, [(10, 1), (15, 4), (30, 6)], True, 22),
+        (1, 24, 4, 5, [(8, 3), (24, 5)], False, 23),
+        (1, 32, 2, 8, [(16, 1), (16, 1)], True, 24),  # duplicated pattern
+    ]
+    for (B, N, H, D, pats, causal, seed) in cases:
+        q, k, v = (_rand((B, N, H, D), seed + 100 * i) for i in range(3))
+        o1, l1 = orc.dilated_attn_fp64(q, k, v, pats, causal=causal, lib=lib)
+        o2, l2 = dilated_attn_bruteforce(q, k, v, pats, causal=causal)
+        np.testing.assert_allclose(o1, o2, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(l1, l2, atol=1e-12, rtol=0)
+
+
+def check_disjoint_rows_single_pattern(lib):
+    """Rows kept by exactly one pattern equal that pattern's attention alone
+    (the disjoint case: the combination adds nothing)."""
+    B, N, H, D = 1, 32, 2, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (31, 32, 33))
+    pats = [(16, 2), (32, 4)]
+    both, _ = orc.dilated_attn_fp64(q, k, v, pats, causal=True, lib=lib)
+    only_a, _ = orc.dilated_attn_fp64(q, k, v, pats[:1], causal=True, lib=lib)
+    # head 1 of (16, 2) keeps odd rows; (32, 4) keeps rows 1, 5, 9, ... for head 1
+    for pos in range(1, N, 2):
+        if (pos - 1) % 4 != 0:
+            np.testing.assert_allclose(both[0, pos, 1], only_a[0, pos, 1], atol=1e-13, rtol=0)
+
+
+def check_invariants(lib):
+    """Order of patterns does not matter; a duplicated pattern keeps out and
+    raises lse by log 2 on its rows; V + c shifts out by c; adding a constant
+    vector c to every key shifts each row's scores (in every pattern) by the
+    same <q, c>/sqrt(D), so out is unchanged and lse moves by that amount."""
+    B, N, H, D = 1, 48, 3, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (41, 42, 43))
+    pats = [(12, 1), (24, 2), (48, 5)]
+    o, l = orc.dilated_attn_fp64(q, k, v, pats, causal=True, lib=lib)
+    o2, l2 = orc.dilated_attn_fp64(q, k, v, pats[::-1], causal=True, lib=lib)
+    np.testing.assert_allclose(o2, o, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(l2, l, atol=1e-13, rtol=0)
+    # duplicate the (48, 5) pattern alone
+    od, ld = orc.dilated_attn_fp64(q, k, v, [(48, 5), (48, 5)], causal=True, lib=lib)
+    os_, ls_ = orc.dilated_attn_fp64(q, k, v, [(48, 5)], causal=True, lib=lib)
+    np.testing.assert_allclose(od, os_, atol=1e-13, rtol=0)
+    fin = np.isfinite(ls_)
+    np.testing.assert_allclose(ld[fin], ls_[fin] + math.log(2.0), atol=1e-13, rtol=0)
+    assert np.all(~np.isfinite(ld[~fin]))
+    # V + c
+    c = 0.75
+    oc, _ = orc.dilated_attn_fp64(q, k, v + c, pats, causal=True, lib=lib)
+    np.testing.assert_allclose(oc, o + c, atol=1e-12, rtol=0)
+    # K + const vector
+    cvec = _rand((D,), 44)
+    ok, lk = orc.dilated_attn_fp64(q, k + cvec, v, pats, causal=True, lib=lib)
+    np.testing.assert_allclose(ok, o, atol=1e-12, rtol=0)
+    shift = np.einsum("bnhd,d->bhn", q, cvec) / math.sqrt(D)
+    np.testing.assert_allclose(lk, l + shift, atol=1e-12, rtol=0)
+
+
+def check_uncovered_rows(lib):
+    """With no r = 1 pattern some rows are kept by no pattern: out 0, lse -inf."""
+    B, N, H, D = 1, 24, 2, 4
+    q, k, v = (_rand((B, N, H, D), s) for s in (51, 52, 53))
+    out, lse = orc.dilated_attn_fp64(q, k, v, [(12, 3), (24, 4)], causal=True, lib=lib)
+    for h in range(H):
+        for pos in range(N):
+            kept3 = (pos % 12 - h % 3) >= 0 and (pos % 12 - h % 3) % 3 == 0
+            kept4 = (pos - h % 4) >= 0 and (pos - h % 4) % 4 == 0
+            if not (kept3 or kept4):
+                assert np.all(out[0, pos, h] == 0.0) and lse[0, h, pos] == -math.inf
+            else:
+                assert np.isfinite(lse[0, h, pos])
+
+
+def check_rows_function(lib):
+    """The per-row entry point returns the same rows as the full forward."""
+    B, N, H, D = 2, 36, 3, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (61, 62, 63))
+    pats = [(12, 1), (18, 4), (36, 5)]
+    for causal in (True, False):
+        o, l = orc.dilated_attn_fp64(q, k, v, pats, causal=causal, lib=lib)
+        rows = [(b, pos, h) for b in range(B) for pos in range(0, N, 5) for h in range(H)]
+        orow, lrow = orc.dilated_attn_rows_fp64(q, k, v, pats, rows, causal=causal, lib=lib)
+        for t, (b, pos, h) in enumerate(rows):
+            np.testing.assert_allclose(orow[t], o[b, pos, h], atol=1e-13, rtol=0)
+            assert abs(lrow[t] - l[b, h, pos]) < 1e-13
+
+
+ALL_CHECKS = [
+    check_dense_causal,
+    check_dense_noncausal,
+    check_block_diagonal,
+    check_dilated_equals_gathered,
+    check_support_and_uniform_weights,
+    check_bruteforce_agreement,
+    check_disjoint_rows_single_pattern,
+    check_invariants,
+    check_uncovered_rows,
+    check_rows_function,
+]
