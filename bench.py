@@ -1,0 +1,451 @@
+"""Benchmark of the multi-pattern dilated-attention forward on B200.
+
+One step = one forward over the whole workload (all patterns, segment split,
+dilated gather, attention, scatter and combination: a single launch of the
+library) on inputs already resident in HBM.  Default workload: 32K tokens,
+5 patterns (the pages' experiment pattern set), bf16, causal.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference] [--sweep]
+
+With N > 1 (launched under torch.distributed.run) every rank runs its own
+independent copy of the workload (different seed): the path has no data
+exchange, so this is weak scaling with no collective on the data path.
+
+Prints one JSON line (rank 0).  Timing: CUDA events on the launch stream per
+step, with a 512 MiB L2 flush between steps (outside the events), barrier +
+synchronize around the timed region, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Dilated-attn fwd tokens/s @32K, 5 patterns; % of bf16 tensor-core peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_long_sequence_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(workload: str, impl_name: str):
+    """DRAM bytes per launch from a committed ncu summary, when it was taken
+    on the current kernel sources; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(f"{impl_name}:{workload}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running
+    (read-only; no setting of the GPU is touched)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            import torch
+
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                uuid = None
+            if uuid:
+                u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(u.encode() if isinstance(u, str) else u)
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                t = time.time()
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((t, mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = None
+        if not inside:
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "timed region shorter than the sampling period; nearest samples"
+        reasons = set()
+        for _, _, bits in inside:
+            for bit, name in self.REASONS.items():
+                if bits & bit and name != "gpu_idle":
+                    reasons.add(name)
+        out = {"sm_mhz": statistics.median([s[1] for s in inside]) if inside else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(inside)}
+        if note:
+            out["note"] = note
+        return out
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+_INPUT_CACHE = {}
+
+
+def oracle_cpu_sample(wl, n_positions: int, seed: int):
+    """Time the fp64 oracle (as it stands) on n_positions random positions of
+    the workload, all heads of each position.  Returns (tokens/s, seconds,
+    threads, description)."""
+    import numpy as np
+
+    import oracle
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    key = (wl.name, wl.N)
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE.clear()
+        _INPUT_CACHE[key] = wlm.make_inputs(wl)
+    q, k, v = _INPUT_CACHE[key]
+    g = np.random.default_rng(seed)
+    pos = g.choice(wl.N, size=n_positions, replace=False)
+    bs = g.integers(0, wl.B, size=n_positions)
+    rows = np.array([(b, p, h) for b, p in zip(bs, pos) for h in range(wl.H)], dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.dilated_attn_rows_fp64(q, k, v, wl.patterns, rows, wl.causal)
+    dt = time.perf_counter() - t0
+    desc = (f"{n_positions} random positions (all {wl.H} heads each) of workload {wl.name}, "
+            f"fp64 oracle rows entry point")
+    return n_positions / dt, dt, oracle.num_threads(), desc
+
+
+def run_reference(args, wl):
+    """Reference arm: the fp64 CPU oracle timed on the host cores, on a
+    bounded sample of the same workload per step."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+
+    n_pos = args.ref_positions
+    times = []
+    threads = None
+    desc = None
+    for i in range(args.warmup + args.steps):
+        tps, dt, threads, desc = oracle_cpu_sample(wl, n_pos, seed=1000 + i)
+        if i >= args.warmup:
+            times.append(dt)
+    mean_dt = sum(times) / len(times)
+    value = n_pos / mean_dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+                   "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
+                   "sample_positions_per_step": n_pos},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long32k")
+    ap.add_argument("--impl", default="ours", help="ours | reference")
+    ap.add_argument("--kernel", default="auto", help="auto | simt | tcgen05 | smallseg")
+    ap.add_argument("--ref-positions", type=int, default=48)
+    ap.add_argument("--cpu-positions", type=int, default=0,
+                    help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="linear-scaling sweep instead")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    if args.sweep:
+        return run_sweep(args)
+    return run_ours(args, wl)
+
+
+def _impl_code(name):
+    from sparse_long_sequence_attn_b200 import binding as bd
+
+    return {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT,
+            "tcgen05": bd.LONGNET_IMPL_TCGEN05, "smallseg": bd.LONGNET_IMPL_SMALLSEG}[name]
+
+
+def _impl_name(code):
+    return {1: "simt", 2: "tcgen05", 3: "smallseg"}.get(code, str(code))
+
+
+def time_steps(fn, steps, warmup, stream, flush_buf):
+    """Warm up, then time each step with CUDA events on `stream`, flushing L2
+    between steps outside the events.  Returns per-step seconds."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush_buf.zero_()
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) * 1e-3 for a, b in evs]
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_long_sequence_attn_b200 import binding as bd
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    bd.load_library()
+
+    q, k, v = wlm.make_inputs(wl, seed=wl.seed + 7919 * rank)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    out = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.H, wl.N), device=dev, dtype=torch.float32)
+    impl = _impl_code(args.kernel)
+    chosen = bd.longnet_select_impl(wl.B, wl.N, wl.H, wl.D, wl.patterns, wl.causal, wl.torch_dtype) \
+        if impl == bd.LONGNET_IMPL_AUTO else impl
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, wl.patterns, wl.causal, impl, stream)
+
+    # device-resident timed region
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    per_step = time_steps(step, args.steps, args.warmup, stream, flush)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    sampler.stop()
+    st = bd.longnet_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after the timed region: {bd.status_string(st)}")
+    total = sum(per_step)
+    if ws > 1:
+        t = torch.tensor([total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    mean_step = total / args.steps
+
+    # end-to-end through the public API with host buffers: pinned H2D of the
+    # inputs, the forward, D2H of out and lse, every step
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, wl.patterns, wl.causal, impl, stream)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    if ws > 1:
+        dist.barrier()
+    per_e2e = time_steps(e2e_step, e2e_steps, 2, stream, flush)
+    e2e_total = sum(per_e2e)
+    if ws > 1:
+        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    tokens = wl.B * wl.N
+    value = ws * tokens / mean_step
+    flops = wlm.algorithmic_flops(wl)
+    peaks, peak_kind = load_peaks()
+    kname = _impl_name(chosen)
+    if kname == "smallseg":
+        achieved = wlm.algorithmic_bytes(wl) / mean_step / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = flops / mean_step / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
+    roof["traffic"] = traffic_from_profiles(wl.name, kname)
+    roof["algorithmic_flops_per_launch"] = flops
+    roof["algorithmic_bytes_per_launch"] = wlm.algorithmic_bytes(wl)
+    roof["frac_of_sustained_bf16"] = flops / mean_step / 1e12 / peaks.get("bf16_tflops_sustained", 1400.0)
+    roof["frac_of_nominal_bf16"] = flops / mean_step / 1e12 / NOMINAL_BF16_TFLOPS
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic: seeded N(0,1) q/k/v at the workload's shape (no dataset)",
+        "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+                   "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
+                   "global_batch": wl.B * ws, "seq_len": wl.N,
+                   "parallelism": f"independent replicas x{ws}" if ws > 1 else "single GPU",
+                   "kernel": kname, "l2": "512 MiB flush between timed steps (outside events)"},
+        "roofline": roof,
+        "e2e": {"value": ws * tokens * e2e_steps / e2e_total, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        n = args.cpu_positions
+        if n <= 0:
+            tps, dt, _, _ = oracle_cpu_sample(wl, 16, seed=1)
+            n = int(max(16, min(wl.N, 10.0 * tps)))
+        tps, dt, threads, desc = oracle_cpu_sample(wl, n, seed=2)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc + f" ({dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sweep(args):
+    """Linear-scaling sweep: tokens/s at N = 65536, 262144, 1048576."""
+    import torch
+
+    from sparse_long_sequence_attn_b200 import binding as bd
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    impl = _impl_code(args.kernel)
+    res = []
+    for N in wlm.SWEEP_NS:
+        wl = wlm.sweep_workload(N)
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.seed)
+        # device-side draws: the sweep measures speed only (parity is tested separately)
+        qd, kd, vd = (torch.randn(wl.B, N, wl.H, wl.D, device=dev, generator=g,
+                                  dtype=torch.float32).to(torch.bfloat16) for _ in range(3))
+        out = torch.empty_like(qd)
+        lse = torch.empty((wl.B, wl.H, N), device=dev, dtype=torch.float32)
+
+        def step():
+            bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, wl.patterns, wl.causal, impl, stream)
+
+        per = time_steps(step, args.steps, args.warmup, stream, flush)
+        t = sum(per) / len(per)
+        res.append({"N": N, "ms": t * 1e3, "tokens_per_s": N / t,
+                    "tflops": wlm.algorithmic_flops(wl) / t / 1e12})
+        del qd, kd, vd, out, lse
+        torch.cuda.empty_cache()
+    base = res[0]["tokens_per_s"]
+    for r in res:
+        r["tokens_per_s_vs_65536"] = r["tokens_per_s"] / base
+    print(json.dumps({"sweep": res}), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,139 @@
+/*
+ * longnet.h — C ABI of the B200 (sm_100a) multi-pattern dilated-attention
+ * forward of LongNet.
+ *
+ * The operation ("LONGNET: Scaling Transformer to 1 billion tokens", section
+ * "LongNet's attention allocation principle"; "LongNet论文精读", section
+ * "Dilated Attention的工作原理"):
+ *   for every pattern p = (w_p, r_p):
+ *     - split the sequence into segments of w_p tokens;
+ *     - in each segment head h keeps the rows at offsets o + r_p*k < w_p,
+ *       with o = h mod r_p (each head has its own offset);
+ *     - attend with softmax(Q K^T / sqrt(D)) V over the kept rows of the
+ *       segment (causal: a kept row sees kept rows at or before itself);
+ *     - put the rows back at their positions;
+ *   then combine the patterns row by row, each weighted by its softmax
+ *   denominator:  out = sum_p e^{lse_p} O_p / sum_p e^{lse_p},
+ *   lse = log sum_p e^{lse_p}, over the patterns that keep the row (the
+ *   reading adopted for "combine local attention into global attention",
+ *   same page, section "Token expansion reaches 1 billion+").  A row kept by
+ *   no pattern gets out = 0 and lse = -inf.
+ *
+ * Conventions shared by every entry point
+ *   - q, k, v, out: device pointers, contiguous [B, N, H, D] in the dtype
+ *     given (LONGNET_DTYPE_F32 or LONGNET_DTYPE_BF16); 16-byte aligned.
+ *   - lse: device pointer to fp32 [B, H, N] (natural log, scale included),
+ *     or NULL when not wanted.  4-byte aligned.
+ *   - w, r: HOST arrays of n_pat pattern parameters, read during the call
+ *     and not kept.  1 <= n_pat <= LONGNET_MAX_PATTERNS, r >= 1,
+ *     1 <= w <= N, N % w == 0.  Patterns may repeat and come in any order;
+ *     a repeated pattern counts twice.
+ *   - causal: 1 = causal inside each sparsified segment, 0 = full.
+ *   - stream: a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns before it finishes.
+ *   - Memory: every pointer is owned by the caller.  The library allocates
+ *     no device or host memory in any call.  Its only global state is one
+ *     status word per device (see longnet_last_device_status).
+ *   - Errors: every entry point returns LONGNET_OK (0) or a negative code,
+ *     never aborts, traps or exits.  Arguments are checked before anything is
+ *     enqueued: a rejected call enqueues nothing.
+ *   - Calls may run concurrently on different streams.
+ */
+#ifndef LONGNET_H_
+#define LONGNET_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA. */
+typedef struct CUstream_st* longnet_stream_t;
+
+#define LONGNET_MAX_PATTERNS 16
+
+enum longnet_status {
+  LONGNET_OK = 0,
+  LONGNET_ERR_INVALID_ARG = -1,   /* a size <= 0, bad pattern, NULL tensor */
+  LONGNET_ERR_UNSUPPORTED = -2,   /* a valid shape the chosen kernel lacks */
+  LONGNET_ERR_MISALIGNED = -3,    /* a pointer misses its alignment */
+  LONGNET_ERR_CUDA = -4,          /* a CUDA call failed (launch, config) */
+  LONGNET_ERR_DEVICE_TIMEOUT = -5,/* a kernel wait ran out of time (status word) */
+  LONGNET_ERR_DEVICE_BOUNDS = -6, /* a kernel index check failed (status word) */
+  LONGNET_ERR_NO_DEVICE = -7      /* no usable sm_100 device */
+};
+
+enum longnet_dtype { LONGNET_DTYPE_F32 = 0, LONGNET_DTYPE_BF16 = 1 };
+
+/* Kernel families.  AUTO picks per shape; the others force one (tests). */
+enum longnet_impl {
+  LONGNET_IMPL_AUTO = 0,
+  LONGNET_IMPL_SIMT = 1,     /* fp32 FMA, any D in {16,32,64,128}, both dtypes */
+  LONGNET_IMPL_TCGEN05 = 2,  /* bf16, D = 64: TMA + tcgen05/TMEM flash kernel,
+                                patterns fused in shared memory */
+  LONGNET_IMPL_SMALLSEG = 3  /* bf16, D = 64, w/r <= 128: memory-bound kernel */
+};
+
+/*
+ * longnet_dilated_attn_fwd — the forward described at the top of this file.
+ * Chooses the kernel (LONGNET_IMPL_AUTO).  Returns a longnet_status.
+ */
+int longnet_dilated_attn_fwd(const void* q, const void* k, const void* v,
+                             void* out, float* lse,
+                             int64_t B, int64_t N, int64_t H, int64_t D,
+                             int n_pat, const int64_t* w, const int64_t* r,
+                             int causal, int dtype, longnet_stream_t stream);
+
+/*
+ * longnet_dilated_attn_fwd_impl — same operation, with the kernel family
+ * forced (enum longnet_impl).  Returns LONGNET_ERR_UNSUPPORTED when that
+ * family does not cover the arguments.
+ */
+int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
+                                  void* out, float* lse,
+                                  int64_t B, int64_t N, int64_t H, int64_t D,
+                                  int n_pat, const int64_t* w, const int64_t* r,
+                                  int causal, int dtype, int impl,
+                                  longnet_stream_t stream);
+
+/*
+ * longnet_select_impl — which family AUTO would run for these arguments
+ * (a longnet_impl >= 1), or a negative longnet_status when the arguments
+ * are invalid.  Host-only; touches no device.
+ */
+int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
+                        const int64_t* w, const int64_t* r, int causal,
+                        int dtype);
+
+/*
+ * longnet_last_device_status — synchronises `stream`, then returns and
+ * clears the current device's status word: LONGNET_OK, or
+ * LONGNET_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave up, or
+ * LONGNET_ERR_DEVICE_BOUNDS when a kernel's index check failed (such a kernel
+ * skips the access and finishes early; its outputs are then undefined).
+ * LONGNET_ERR_CUDA if the synchronisation itself failed.
+ */
+int longnet_last_device_status(longnet_stream_t stream);
+
+/*
+ * longnet_watchdog_selftest — enqueues one tiny kernel on `stream` that waits
+ * on a shared-memory barrier nothing ever completes, with a wait limit of
+ * `limit_ns` nanoseconds (clamped to [1e3, 1e9]).  The wait runs out, the
+ * kernel records LONGNET_ERR_DEVICE_TIMEOUT in the status word and returns,
+ * leaving the context usable.  Lets tests exercise the timeout path without
+ * hanging a GPU.  Returns a longnet_status for the launch.
+ */
+int longnet_watchdog_selftest(int64_t limit_ns, longnet_stream_t stream);
+
+/* Static text for a longnet_status code ("unknown status" otherwise). */
+const char* longnet_status_string(int status);
+
+/* Library version, e.g. "longnet-b200 1.0 sm_100a". */
+const char* longnet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LONGNET_H_ */

@@ -1,0 +1,21 @@
+"""B200 (sm_100a) multi-pattern dilated-attention forward of LongNet.
+
+The product is the C-ABI library liblongnet.so (include/longnet.h); this
+package holds its CUDA sources (csrc/), the build script, a thin ctypes
+binding and the named synthetic workloads.
+"""
+from .binding import (  # noqa: F401
+    LONGNET_IMPL_AUTO,
+    LONGNET_IMPL_SIMT,
+    LONGNET_IMPL_SMALLSEG,
+    LONGNET_IMPL_TCGEN05,
+    LongNetError,
+    dilated_attn,
+    load_library,
+    longnet_dilated_attn_fwd,
+    longnet_last_device_status,
+    longnet_select_impl,
+    longnet_watchdog_selftest,
+    status_string,
+    version,
+)

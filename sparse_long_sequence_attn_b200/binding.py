@@ -1,0 +1,167 @@
+"""Thin Python binding of liblongnet (include/longnet.h) over ctypes.
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch provides device memory and streams.  If the in-tree
+library is missing, loading raises: there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblongnet.so")
+
+LONGNET_OK = 0
+LONGNET_ERR_INVALID_ARG = -1
+LONGNET_ERR_UNSUPPORTED = -2
+LONGNET_ERR_MISALIGNED = -3
+LONGNET_ERR_CUDA = -4
+LONGNET_ERR_DEVICE_TIMEOUT = -5
+LONGNET_ERR_DEVICE_BOUNDS = -6
+LONGNET_ERR_NO_DEVICE = -7
+LONGNET_MAX_PATTERNS = 16
+
+LONGNET_DTYPE_F32 = 0
+LONGNET_DTYPE_BF16 = 1
+
+LONGNET_IMPL_AUTO = 0
+LONGNET_IMPL_SIMT = 1
+LONGNET_IMPL_TCGEN05 = 2
+LONGNET_IMPL_SMALLSEG = 3
+
+# Every symbol include/longnet.h declares, with its ctypes signature.
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+_i64p = ctypes.POINTER(ctypes.c_int64)
+SIGNATURES = {
+    "longnet_dilated_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                                ctypes.c_int, _i64p, _i64p, ctypes.c_int,
+                                                ctypes.c_int, _vp]),
+    "longnet_dilated_attn_fwd_impl": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                     _i64, ctypes.c_int, _i64p, _i64p,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     _vp]),
+    "longnet_select_impl": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
+                                           ctypes.c_int, ctypes.c_int]),
+    "longnet_last_device_status": (ctypes.c_int, [_vp]),
+    "longnet_watchdog_selftest": (ctypes.c_int, [_i64, _vp]),
+    "longnet_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "longnet_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class LongNetError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} (code {code})")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH):
+    """Load liblongnet.so; raises if it was not built (no fallback)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"liblongnet.so not built at {path}; run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().longnet_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return load_library().longnet_version().decode()
+
+
+def _patterns(patterns: Sequence[Tuple[int, int]]):
+    n = len(patterns)
+    w = (ctypes.c_int64 * max(n, 1))(*[int(p[0]) for p in patterns])
+    r = (ctypes.c_int64 * max(n, 1))(*[int(p[1]) for p in patterns])
+    return n, w, r
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LONGNET_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return LONGNET_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) or None
+
+
+def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                             out: torch.Tensor, lse: torch.Tensor | None,
+                             patterns: Sequence[Tuple[int, int]], causal: bool = True,
+                             impl: int = LONGNET_IMPL_AUTO, stream=None) -> None:
+    """Enqueue the forward on `stream` (default: torch's current stream).
+
+    q, k, v, out: contiguous CUDA tensors [B, N, H, D] of one dtype (fp32/bf16);
+    lse: contiguous fp32 [B, H, N] or None.  Raises LongNetError on a non-zero
+    status.
+    """
+    lib = load_library()
+    for t in (q, k, v, out):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("q, k, v, out must be contiguous CUDA tensors")
+    if lse is not None and not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor")
+    B, N, H, D = q.shape
+    for t in (k, v, out):
+        if tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must share shape and dtype")
+    if lse is not None and tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_fwd_impl(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        None if lse is None else lse.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), int(impl), _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_fwd")
+
+
+def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 patterns: Sequence[Tuple[int, int]], causal: bool = True,
+                 impl: int = LONGNET_IMPL_AUTO, want_lse: bool = True, stream=None):
+    """Allocate out (and lse) with torch and run the forward.  Returns (out, lse)."""
+    B, N, H, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if want_lse else None
+    longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream)
+    return out, lse
+
+
+def longnet_select_impl(B: int, N: int, H: int, D: int, patterns, causal: bool, dtype) -> int:
+    """Kernel family AUTO would use (>= 1) or a negative status (host only)."""
+    n, w, r = _patterns(patterns)
+    code = dtype if isinstance(dtype, int) else (LONGNET_DTYPE_F32 if dtype == torch.float32 else LONGNET_DTYPE_BF16)
+    return int(load_library().longnet_select_impl(B, N, H, D, n, w, r, int(bool(causal)), code))
+
+
+def longnet_last_device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear this device's status word."""
+    return int(load_library().longnet_last_device_status(_stream_handle(stream)))
+
+
+def longnet_watchdog_selftest(limit_ns: int = 1_000_000, stream=None) -> int:
+    """Launch the kernel whose barrier wait must run out (see longnet.h)."""
+    return int(load_library().longnet_watchdog_selftest(int(limit_ns), _stream_handle(stream)))

@@ -1,0 +1,233 @@
+// C ABI of liblongnet: argument checks, kernel-family choice, status word.
+//
+// Everything the caller passes is checked on the host before anything is
+// enqueued; the device work itself lives in the family files (simt.cu,
+// tcgen05.cu, smallseg.cu).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "device_util.cuh"
+#include "longnet.h"
+#include "params.h"
+
+namespace longnet {
+
+// One status word per device: the first error a kernel of this library
+// records (wait timeout, failed index check).  Cleared by
+// longnet_last_device_status.
+__device__ int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+int* g_status_addr[kMaxDevices] = {nullptr};
+int g_dev_checked[kMaxDevices] = {0};  // 0 unknown, 1 ok, -1 not sm_100
+
+// Device checks and the status word's device address, once per device.
+int current_device_state(int* dev_out, int** status_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LONGNET_ERR_NO_DEVICE;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return LONGNET_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_dev_checked[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return LONGNET_ERR_NO_DEVICE;
+    }
+    if (major != 10 || minor != 0) {
+      g_dev_checked[dev] = -1;
+    } else {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess || addr == nullptr) {
+        cudaGetLastError();
+        return LONGNET_ERR_CUDA;
+      }
+      g_status_addr[dev] = static_cast<int*>(addr);
+      g_dev_checked[dev] = 1;
+    }
+  }
+  if (g_dev_checked[dev] != 1) return LONGNET_ERR_NO_DEVICE;
+  *dev_out = dev;
+  *status_out = g_status_addr[dev];
+  return LONGNET_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Argument checks common to every family; fills the problem block.
+int check_args(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,
+               int64_t N, int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r,
+               int causal, int dtype, Problem* pb) {
+  if (!q || !k || !v || !out) return LONGNET_ERR_INVALID_ARG;
+  if (B <= 0 || N <= 0 || H <= 0 || D <= 0) return LONGNET_ERR_INVALID_ARG;
+  if (N > (int64_t)INT32_MAX || H > 65535 || D > 65535) return LONGNET_ERR_INVALID_ARG;
+  if (B > (int64_t)1 << 40 || B * N > ((int64_t)1 << 40) || B * N * H * D > ((int64_t)1 << 50))
+    return LONGNET_ERR_INVALID_ARG;
+  if (n_pat < 1 || n_pat > LONGNET_MAX_PATTERNS || !w || !r) return LONGNET_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return LONGNET_ERR_INVALID_ARG;
+  if (dtype != LONGNET_DTYPE_F32 && dtype != LONGNET_DTYPE_BF16) return LONGNET_ERR_INVALID_ARG;
+  for (int i = 0; i < n_pat; ++i) {
+    if (r[i] < 1 || w[i] < 1 || w[i] > N || N % w[i] != 0) return LONGNET_ERR_INVALID_ARG;
+  }
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return LONGNET_ERR_MISALIGNED;
+  if (lse && !aligned(lse, 4)) return LONGNET_ERR_MISALIGNED;
+  memset(pb, 0, sizeof(*pb));
+  pb->q = q;
+  pb->k = k;
+  pb->v = v;
+  pb->out = out;
+  pb->lse = lse;
+  pb->B = B;
+  pb->N = N;
+  pb->H = H;
+  pb->D = D;
+  pb->n_pat = n_pat;
+  pb->causal = causal;
+  pb->dtype = dtype;
+  for (int i = 0; i < n_pat; ++i) {
+    pb->w[i] = w[i];
+    pb->r[i] = r[i];
+  }
+  return LONGNET_OK;
+}
+
+bool simt_supports(const Problem& p) { return p.D == 16 || p.D == 32 || p.D == 64 || p.D == 128; }
+
+int choose_impl(const Problem& p) {
+  if (smallseg_supports(p)) return LONGNET_IMPL_SMALLSEG;
+  if (tcgen05_supports(p)) return LONGNET_IMPL_TCGEN05;
+  if (simt_supports(p)) return LONGNET_IMPL_SIMT;
+  return LONGNET_ERR_UNSUPPORTED;
+}
+
+// The watchdog self-test: a barrier that expects one arrival which never
+// comes.  The bounded wait gives up after limit_ns and records a timeout.
+__global__ void watchdog_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!mbar_wait(&bar, 0, limit_ns)) record_status(status, kStatusTimeout);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace longnet
+
+using namespace longnet;
+
+extern "C" int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
+                                             void* out, float* lse, int64_t B, int64_t N,
+                                             int64_t H, int64_t D, int n_pat, const int64_t* w,
+                                             const int64_t* r, int causal, int dtype, int impl,
+                                             longnet_stream_t stream) {
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
+  if (rc) return rc;
+  int dev = 0;
+  rc = current_device_state(&dev, &pb.status);
+  if (rc) return rc;
+  if (impl == LONGNET_IMPL_AUTO) {
+    impl = choose_impl(pb);
+    if (impl < 0) return impl;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (impl) {
+    case LONGNET_IMPL_SIMT:
+      if (!simt_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+      return launch_simt(pb, s);
+    case LONGNET_IMPL_TCGEN05:
+      if (!tcgen05_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+      return launch_tcgen05(pb, s);
+    case LONGNET_IMPL_SMALLSEG:
+      if (!smallseg_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+      return launch_smallseg(pb, s);
+    default:
+      return LONGNET_ERR_INVALID_ARG;
+  }
+}
+
+extern "C" int longnet_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                        float* lse, int64_t B, int64_t N, int64_t H, int64_t D,
+                                        int n_pat, const int64_t* w, const int64_t* r, int causal,
+                                        int dtype, longnet_stream_t stream) {
+  return longnet_dilated_attn_fwd_impl(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype,
+                                       LONGNET_IMPL_AUTO, stream);
+}
+
+extern "C" int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
+                                   const int64_t* w, const int64_t* r, int causal, int dtype) {
+  // Stand-in pointers: only their alignment is looked at here.
+  static __align__(16) char dummy[16];
+  Problem pb;
+  int rc = check_args(dummy, dummy, dummy, dummy, nullptr, B, N, H, D, n_pat, w, r, causal, dtype,
+                      &pb);
+  if (rc) return rc;
+  return choose_impl(pb);
+}
+
+extern "C" int longnet_last_device_status(longnet_stream_t stream) {
+  int dev = 0;
+  int* addr = nullptr;
+  int rc = current_device_state(&dev, &addr);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LONGNET_ERR_CUDA;
+  }
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return LONGNET_ERR_CUDA;
+  }
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return LONGNET_ERR_CUDA;
+  }
+  return word;
+}
+
+extern "C" int longnet_watchdog_selftest(int64_t limit_ns, longnet_stream_t stream) {
+  int dev = 0;
+  int* addr = nullptr;
+  int rc = current_device_state(&dev, &addr);
+  if (rc) return rc;
+  if (limit_ns < 1000) limit_ns = 1000;
+  if (limit_ns > 1000000000) limit_ns = 1000000000;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      addr, static_cast<uint64_t>(limit_ns));
+  if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
+  return LONGNET_OK;
+}
+
+extern "C" const char* longnet_status_string(int status) {
+  switch (status) {
+    case LONGNET_OK: return "ok";
+    case LONGNET_ERR_INVALID_ARG: return "invalid argument";
+    case LONGNET_ERR_UNSUPPORTED: return "unsupported shape or dtype for this kernel family";
+    case LONGNET_ERR_MISALIGNED: return "pointer misaligned";
+    case LONGNET_ERR_CUDA: return "CUDA call failed";
+    case LONGNET_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case LONGNET_ERR_DEVICE_BOUNDS: return "device index check failed";
+    case LONGNET_ERR_NO_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* longnet_version(void) { return "longnet-b200 1.0 sm_100a"; }

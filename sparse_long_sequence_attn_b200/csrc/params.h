@@ -1,0 +1,43 @@
+// Host/device parameter block shared by the kernels of liblongnet.
+#pragma once
+
+#include <stdint.h>
+
+#include "longnet.h"
+
+namespace longnet {
+
+// One call's arguments after validation.  Pattern arrays are copied in so a
+// kernel can read them from its parameter space.
+struct Problem {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;  // may be null
+  int64_t B, N, H, D;
+  int n_pat;
+  int causal;
+  int dtype;
+  int64_t w[LONGNET_MAX_PATTERNS];
+  int64_t r[LONGNET_MAX_PATTERNS];
+  int* status;  // device address of this device's status word
+};
+
+// Status codes written into the device status word (first error wins).
+constexpr int kStatusTimeout = LONGNET_ERR_DEVICE_TIMEOUT;
+constexpr int kStatusBounds = LONGNET_ERR_DEVICE_BOUNDS;
+
+// Wait limit of every bounded device-side wait in the library.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Kernel launchers (one per family).  Return a longnet_status.
+int launch_simt(const Problem& p, cudaStream_t stream);
+int launch_tcgen05(const Problem& p, cudaStream_t stream);
+int launch_smallseg(const Problem& p, cudaStream_t stream);
+
+// Shape checks of the specialised families (host only, no device access).
+bool tcgen05_supports(const Problem& p);
+bool smallseg_supports(const Problem& p);
+
+}  // namespace longnet

@@ -1,0 +1,80 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol include/longnet.h declares, rejects bad arguments before touching a
+device, and reports the missing device instead of crashing (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from sparse_long_sequence_attn_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "longnet.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(longnet_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = bd.load_library()
+    names = declared_functions()
+    assert len(names) >= 7
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in longnet.h but not exported"
+        assert name in bd.SIGNATURES, f"{name} missing from the Python binding"
+
+
+def test_status_strings_and_version():
+    assert bd.status_string(0) == "ok"
+    assert "invalid" in bd.status_string(bd.LONGNET_ERR_INVALID_ARG)
+    assert bd.status_string(12345) == "unknown status"
+    assert bd.version().startswith("longnet-b200")
+
+
+def _call(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, ptr=None, lse=None, impl=0):
+    buf = ptr if ptr is not None else ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    n = len(pats)
+    w = (ctypes.c_int64 * max(n, 1))(*[p[0] for p in pats])
+    r = (ctypes.c_int64 * max(n, 1))(*[p[1] for p in pats])
+    return lib.longnet_dilated_attn_fwd_impl(buf, buf, buf, buf, lse, B, N, H, D, n, w, r, causal,
+                                             dtype, impl, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=0), dict(N=-1), dict(H=0), dict(D=0), dict(pats=()), dict(pats=((16, 0),)),
+    dict(pats=((0, 1),)), dict(pats=((128, 1),)), dict(pats=((24, 1),)), dict(causal=2),
+    dict(dtype=7), dict(pats=tuple((16, 1) for _ in range(17))), dict(impl=9),
+])
+def test_invalid_arguments_rejected_on_host(kw):
+    lib = bd.load_library()
+    rc = _call(lib, **kw)
+    assert rc == bd.LONGNET_ERR_INVALID_ARG, rc
+
+
+def test_null_and_misaligned_pointers():
+    lib = bd.load_library()
+    assert _call(lib, ptr=ctypes.c_void_p(0)) == bd.LONGNET_ERR_INVALID_ARG
+    assert _call(lib, ptr=ctypes.c_void_p(0x1008)) == bd.LONGNET_ERR_MISALIGNED
+    assert _call(lib, lse=ctypes.c_void_p(0x1002)) == bd.LONGNET_ERR_MISALIGNED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_no_device():
+    lib = bd.load_library()
+    assert _call(lib) == bd.LONGNET_ERR_NO_DEVICE
+    assert lib.longnet_last_device_status(None) == bd.LONGNET_ERR_NO_DEVICE
+    assert lib.longnet_watchdog_selftest(1000, None) == bd.LONGNET_ERR_NO_DEVICE
+
+
+def test_select_impl_host_logic():
+    f32, bf16 = torch.float32, torch.bfloat16
+    assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 1), (128, 2)), True, f32) == bd.LONGNET_IMPL_SIMT
+    assert bd.longnet_select_impl(1, 256, 2, 48, ((64, 1),), True, f32) == bd.LONGNET_ERR_UNSUPPORTED
+    assert bd.longnet_select_impl(1, 255, 2, 16, ((64, 1),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
+    impl = bd.longnet_select_impl(1, 32768, 12, 64, ((2048, 1), (4096, 2)), True, bf16)
+    assert impl in (bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05)

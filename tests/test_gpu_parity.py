@@ -1,0 +1,142 @@
+"""GPU parity: every kernel family through the C ABI against the fp64 oracle
+on the same seeded inputs (needs a B200)."""
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_long_sequence_attn_b200 import binding as bd
+from sparse_long_sequence_attn_b200 import workloads as wl
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = {"simt": bd.LONGNET_IMPL_SIMT, "tcgen05": bd.LONGNET_IMPL_TCGEN05,
+         "smallseg": bd.LONGNET_IMPL_SMALLSEG}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    bd.load_library()
+    yield
+
+
+# Small cases spanning several tiles and ragged tails: r not dividing w,
+# rows reached by 1..n patterns, rows reached by none, duplicates, B > 1.
+SMALL_CASES = [
+    # name, B, N, H, D, dtype, causal, patterns
+    ("tiny_cfg", 1, 256, 2, 16, torch.float32, True, ((64, 1), (128, 2), (256, 4))),
+    ("fp32_d32_rdivw", 2, 384, 3, 32, torch.float32, True, ((96, 1), (192, 5), (384, 7))),
+    ("fp32_d64_noncausal", 1, 512, 2, 64, torch.float32, False, ((128, 1), (256, 3))),
+    ("fp32_d128_uncovered", 1, 240, 3, 128, torch.float32, True, ((48, 3), (240, 4))),
+    ("bf16_d64_lm_like", 2, 2048, 4, 64, torch.bfloat16, True, ((512, 1), (1024, 2), (2048, 4))),
+    ("bf16_d64_paper_like", 1, 3072, 6, 64, torch.bfloat16, True,
+     ((256, 1), (512, 2), (1024, 4), (1536, 6), (3072, 12))),
+    ("bf16_d64_dup_unordered", 1, 1024, 3, 64, torch.bfloat16, True, ((1024, 4), (256, 1), (256, 1))),
+    ("bf16_d64_noncausal_small", 2, 1024, 4, 64, torch.bfloat16, False, ((64, 1), (64, 2))),
+    ("bf16_d64_no_r1", 1, 1536, 5, 64, torch.bfloat16, True, ((384, 3), (768, 4), (1536, 8))),
+    ("bf16_d64_w_eq_N", 1, 640, 2, 64, torch.bfloat16, True, ((640, 1),)),
+    ("bf16_d64_r_gt_w", 1, 512, 4, 64, torch.bfloat16, True, ((512, 1), (2, 3))),
+    ("bf16_d32", 1, 512, 2, 32, torch.bfloat16, True, ((128, 1), (512, 2))),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
+@pytest.mark.parametrize("impl_name", ["auto", "simt"])
+def test_small_cases_vs_oracle(case, impl_name):
+    name, B, N, H, D, dtype, causal, pats = case
+    impl = bd.LONGNET_IMPL_AUTO if impl_name == "auto" else IMPLS[impl_name]
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=zlib.crc32(name.encode()) % 100000)
+    o, l = gh.run_cuda(q, k, v, pats, causal, impl)
+    gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c[5] == torch.bfloat16 and c[4] == 64],
+                         ids=[c[0] for c in SMALL_CASES if c[5] == torch.bfloat16 and c[4] == 64])
+@pytest.mark.parametrize("impl_name", ["tcgen05", "smallseg"])
+def test_specialised_families_vs_oracle(case, impl_name):
+    name, B, N, H, D, dtype, causal, pats = case
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=zlib.crc32(name.encode()) % 100000)
+    try:
+        o, l = gh.run_cuda(q, k, v, pats, causal, IMPLS[impl_name])
+    except bd.LongNetError as e:
+        if e.code == bd.LONGNET_ERR_UNSUPPORTED:
+            pytest.skip(f"{impl_name} does not take {name}")
+        raise
+    gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
+
+
+def test_named_tiny_workload_fp32():
+    w = wl.WORKLOADS["tiny"]
+    q, k, v = wl.make_inputs(w)
+    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
+    err = gh.compare_full(o, l, q, k, v, w.patterns, w.causal, torch.float32, "tiny")
+    assert err <= 1e-4
+
+
+@pytest.mark.parametrize("name", ["lm", "long32k", "smallseg"])
+def test_named_workloads_sampled_rows(name):
+    """Full-size workloads in the launch configuration the benchmark times
+    (AUTO), checked on sampled rows: every segment's first and last row for
+    every pattern and head, plus random rows."""
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.make_inputs(w)
+    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
+    assert gh.lse_is_finite_everywhere(l)  # every row is kept by an r = 1 pattern
+    rows = gh.sample_rows(w.B, w.N, w.H, w.patterns, n_random=1500, seed=w.seed)
+    gh.compare_rows(o, l, q, k, v, w.patterns, w.causal, torch.bfloat16, rows, label=name)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("N", wl.SWEEP_NS)
+def test_sweep_sampled_rows(N):
+    w = wl.sweep_workload(N)
+    q, k, v = wl.make_inputs(w)
+    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
+    assert gh.lse_is_finite_everywhere(l)
+    rows = gh.sample_rows(w.B, w.N, w.H, w.patterns, n_random=1000, seed=w.seed + N)
+    gh.compare_rows(o, l, q, k, v, w.patterns, w.causal, torch.bfloat16, rows, label=f"sweep{N}")
+
+
+def test_lse_optional_and_deterministic():
+    pats = ((256, 1), (512, 2), (1024, 4))
+    q, k, v = wl.random_inputs(1, 1024, 4, 64, torch.bfloat16, seed=5)
+    o1, _ = gh.run_cuda(q, k, v, pats, True, bd.LONGNET_IMPL_AUTO, want_lse=False)
+    o2, l2 = gh.run_cuda(q, k, v, pats, True, bd.LONGNET_IMPL_AUTO, want_lse=True)
+    assert np.array_equal(o1, o2), "two runs differ"
+    gh.compare_full(o2, l2, q, k, v, pats, True, torch.bfloat16, "lse_optional")
+
+
+def test_runs_on_a_side_stream():
+    pats = ((128, 1), (256, 2))
+    q, k, v = wl.random_inputs(1, 512, 2, 64, torch.bfloat16, seed=6)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o, l = gh.run_cuda(q, k, v, pats, True, bd.LONGNET_IMPL_AUTO, stream=s)
+    gh.compare_full(o, l, q, k, v, pats, True, torch.bfloat16, "side_stream")
+
+
+def test_misaligned_device_pointer_rejected():
+    dev = torch.device("cuda:0")
+    buf = torch.zeros(1 * 64 * 2 * 16 + 8, dtype=torch.float32, device=dev)
+    x = buf[1:1 + 64 * 2 * 16].view(1, 64, 2, 16)  # 4-byte offset
+    with pytest.raises(bd.LongNetError) as ei:
+        bd.longnet_dilated_attn_fwd(x, x, x, x, None, ((64, 1),), True)
+    assert ei.value.code == bd.LONGNET_ERR_MISALIGNED
+
+
+def test_watchdog_timeout_is_reported_and_context_survives():
+    assert bd.longnet_last_device_status() == 0
+    assert bd.longnet_watchdog_selftest(200_000) == 0
+    assert bd.longnet_last_device_status() == bd.LONGNET_ERR_DEVICE_TIMEOUT
+    assert bd.longnet_last_device_status() == 0  # cleared
+    w = wl.WORKLOADS["tiny"]
+    q, k, v = wl.make_inputs(w)
+    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
+    gh.compare_full(o, l, q, k, v, w.patterns, w.causal, torch.float32, "after_watchdog")
