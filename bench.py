@@ -149,10 +149,9 @@ class ClockSampler:
 
 
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from sparse_long_sequence_attn_b200.replicas import dist_env as _de
+
+    return _de()
 
 
 _INPUT_CACHE = {}
@@ -291,7 +290,9 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
     bd.load_library()
 
-    q, k, v = wlm.make_inputs(wl, seed=wl.seed + 7919 * rank)
+    from sparse_long_sequence_attn_b200.replicas import max_over_ranks, replica_seed, weak_scaling_rate
+
+    q, k, v = wlm.make_inputs(wl, seed=replica_seed(wl.seed, rank))
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to(dev) for x in (q, k, v))
     out = torch.empty_like(qd)
@@ -321,11 +322,7 @@ def run_ours(args, wl):
     st = bd.longnet_last_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status after the timed region: {bd.status_string(st)}")
-    total = sum(per_step)
-    if ws > 1:
-        t = torch.tensor([total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(sum(per_step), dev)
     mean_step = total / args.steps
 
     # end-to-end through the public API with host buffers: pinned H2D of the
@@ -346,11 +343,7 @@ def run_ours(args, wl):
     if ws > 1:
         dist.barrier()
     per_e2e = time_steps(e2e_step, e2e_steps, 2, stream, flush)
-    e2e_total = sum(per_e2e)
-    if ws > 1:
-        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = max_over_ranks(sum(per_e2e), dev)
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
 
@@ -361,7 +354,7 @@ def run_ours(args, wl):
         return 0
 
     tokens = wl.B * wl.N
-    value = ws * tokens / mean_step
+    value = weak_scaling_rate(tokens, ws, mean_step)
     flops = wlm.algorithmic_flops(wl)
     peaks, peak_kind = load_peaks()
     kname = _impl_name(chosen)
@@ -391,7 +384,7 @@ def run_ours(args, wl):
                    "parallelism": f"independent replicas x{ws}" if ws > 1 else "single GPU",
                    "kernel": kname, "l2": "512 MiB flush between timed steps (outside events)"},
         "roofline": roof,
-        "e2e": {"value": ws * tokens * e2e_steps / e2e_total, "unit": UNIT,
+        "e2e": {"value": weak_scaling_rate(tokens * e2e_steps, ws, e2e_total), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),

@@ -245,7 +245,36 @@ def check_rows_function(lib):
             assert abs(lrow[t] - l[b, h, pos]) < 1e-13
 
 
+def check_rows_function_direct(lib):
+    """The per-row entry point pinned on its own: against the multiset
+    brute force, and against the Q = 0 closed form of the support fixture."""
+    B, N, H, D = 1, 30, 3, 4
+    q, k, v = (_rand((B, N, H, D), s) for s in (71, 72, 73))
+    pats = [(10, 1), (15, 4), (30, 7)]
+    rows = [(0, pos, h) for pos in range(N) for h in range(H)]
+    orow, lrow = orc.dilated_attn_rows_fp64(q, k, v, pats, rows, causal=True, lib=lib)
+    o2, l2 = dilated_attn_bruteforce(q, k, v, pats, causal=True)
+    for t, (b, pos, h) in enumerate(rows):
+        np.testing.assert_allclose(orow[t], o2[b, pos, h], atol=1e-12, rtol=0)
+        assert abs(lrow[t] - l2[b, h, pos]) < 1e-12
+    sup = read_support_fixture()
+    D = 12
+    qz = np.zeros((1, 12, 2, D))
+    kz = _rand((1, 12, 2, D), 74)
+    vz = np.zeros((1, 12, 2, D))
+    for pos in range(12):
+        vz[0, pos, :, pos] = 1.0
+    rows = sorted(sup)
+    orow, lrow = orc.dilated_attn_rows_fp64(qz, kz, vz, [(4, 1), (6, 2), (12, 3)],
+                                            [(0, pos, h) for (h, pos) in rows], causal=True, lib=lib)
+    for t, key in enumerate(rows):
+        keys = sup[key]
+        np.testing.assert_allclose(orow[t], np.bincount(keys, minlength=12) / len(keys), atol=1e-14, rtol=0)
+        assert abs(lrow[t] - math.log(len(keys))) < 1e-14
+
+
 ALL_CHECKS = [
+    check_rows_function_direct,
     check_dense_causal,
     check_dense_noncausal,
     check_block_diagonal,
