@@ -90,11 +90,11 @@ struct __align__(64) TmaMaps {
 struct Params {
   Problem pb;
   int n_r;                    // distinct dilations
-  int64_t r_val[kMaxR];       // their values
-  int64_t tail[kMaxR];        // N mod r
-  int64_t kfull[kMaxR];       // N div r
+  int r_val[kMaxR];           // their values
+  int tail[kMaxR];            // N mod r
+  int kfull[kMaxR];           // N div r
   int pat_r[kMaxPat];         // index into r_val of each pattern
-  int64_t range_len;          // R
+  int range_len;              // R
   int n_ranges;
   int uncovered_possible;     // some position may be kept by no pattern
   uint64_t wait_limit_ns;
@@ -222,27 +222,27 @@ constexpr uint32_t kIdescPV = idesc_bf16(kBM, kD, true);
 
 struct Tile {
   int p;          // pattern index
-  int64_t seg;    // segment index
-  int64_t k0;     // first kept row (sparse index within the segment)
+  int seg;    // segment index
+  int k0;     // first kept row (sparse index within the segment)
   int nrows;      // rows in this tile (<= 128)
   int nkv;        // KV blocks of 128 keys
-  int64_t start;  // position of the first row
+  int start;  // position of the first row
 };
 
 // Walks the unit's tiles in processing order.  All roles run identical copies.
 struct TileWalker {
   int n_pat;
-  int64_t A, Bnd;  // range [A, Bnd)
-  int64_t w[kMaxPat], r[kMaxPat], o[kMaxPat], m[kMaxPat];
-  int64_t seg[kMaxPat], k0[kMaxPat], khi[kMaxPat], seg_last[kMaxPat];
+  int A, Bnd;  // range [A, Bnd)
+  int w[kMaxPat], r[kMaxPat], o[kMaxPat], m[kMaxPat];
+  int seg[kMaxPat], k0[kMaxPat], khi[kMaxPat], seg_last[kMaxPat];
   bool causal;
 
   __host__ __device__ void seg_bounds(int p) {
     // kept rows of segment seg[p] whose positions fall in [A, Bnd)
-    const int64_t base = seg[p] * w[p] + o[p];
-    int64_t lo = A - base;
+    const int base = seg[p] * w[p] + o[p];
+    int lo = A - base;
     lo = lo <= 0 ? 0 : (lo + r[p] - 1) / r[p];
-    int64_t hi = Bnd - base;
+    int hi = Bnd - base;
     hi = hi <= 0 ? 0 : (hi + r[p] - 1) / r[p];
     if (hi > m[p]) hi = m[p];
     k0[p] = lo;
@@ -254,7 +254,7 @@ struct TileWalker {
       if (seg[p] <= seg_last[p]) seg_bounds(p);
     }
   }
-  __host__ __device__ void init(const Params& P, int64_t h, int64_t a, int64_t bnd) {
+  __host__ __device__ void init(const Params& P, int h, int a, int bnd) {
     n_pat = P.pb.n_pat;
     A = a;
     Bnd = bnd;
@@ -272,10 +272,10 @@ struct TileWalker {
   }
   __host__ __device__ bool next(Tile& t) {
     int best = -1;
-    int64_t best_start = 0;
+    int best_start = 0;
     for (int p = 0; p < n_pat; ++p) {
       if (seg[p] > seg_last[p]) continue;
-      const int64_t st = seg[p] * w[p] + o[p] + r[p] * k0[p];
+      const int st = seg[p] * w[p] + o[p] + r[p] * k0[p];
       if (best < 0 || st < best_start || (st == best_start && r[p] > r[best])) {
         best = p;
         best_start = st;
@@ -286,10 +286,10 @@ struct TileWalker {
     t.p = p;
     t.seg = seg[p];
     t.k0 = k0[p];
-    const int64_t n = khi[p] - k0[p];
+    const int n = khi[p] - k0[p];
     t.nrows = (int)(n < kBM ? n : kBM);
     t.start = best_start;
-    const int64_t nkeys = causal ? k0[p] + t.nrows : m[p];
+    const int nkeys = causal ? k0[p] + t.nrows : m[p];
     t.nkv = (int)((nkeys + kBN - 1) / kBN);
     k0[p] += t.nrows;
     advance_to_nonempty(p);
@@ -300,26 +300,26 @@ struct TileWalker {
 // Processing-order key of the tile of pattern q that covers position x in
 // the unit [A, Bnd); returns false when q does not keep x.
 struct Cover {
-  int64_t start;
+  int start;
   int slot_row;
 };
-__host__ __device__ inline bool cover_of(const TileWalker& tw, int q, int64_t x, Cover& c) {
-  const int64_t sq = x / tw.w[q];
-  const int64_t rel = x - sq * tw.w[q] - tw.o[q];
+__host__ __device__ inline bool cover_of(const TileWalker& tw, int q, int x, Cover& c) {
+  const int sq = x / tw.w[q];
+  const int rel = x - sq * tw.w[q] - tw.o[q];
   if (rel < 0) return false;
-  const int64_t kq = rel / tw.r[q];
+  const int kq = rel / tw.r[q];
   if (kq * tw.r[q] != rel) return false;
   if (kq >= tw.m[q]) return false;
-  const int64_t base = sq * tw.w[q] + tw.o[q];
-  int64_t lo = tw.A - base;
+  const int base = sq * tw.w[q] + tw.o[q];
+  int lo = tw.A - base;
   lo = lo <= 0 ? 0 : (lo + tw.r[q] - 1) / tw.r[q];
-  const int64_t t = (kq - lo) / kBM;
+  const int t = (kq - lo) / kBM;
   c.start = base + tw.r[q] * (lo + t * kBM);
   c.slot_row = (int)((kq - lo) - t * kBM);
   return true;
 }
-__host__ __device__ inline bool key_before(int64_t s_a, int64_t r_a, int p_a, int64_t s_b,
-                                           int64_t r_b, int p_b) {
+__host__ __device__ inline bool key_before(int s_a, int r_a, int p_a, int s_b,
+                                           int r_b, int p_b) {
   if (s_a != s_b) return s_a < s_b;
   if (r_a != r_b) return r_a > r_b;
   return p_a < p_b;
@@ -362,13 +362,13 @@ struct TmaCoord {
   int map;  // 0 base map, 1 shifted map
   int c, kk;
 };
-__host__ __device__ inline TmaCoord tma_coord(const Params& P, int ri, int64_t first_pos,
-                                              int64_t need) {
-  const int64_t r = P.r_val[ri];
-  const int64_t last_pos = first_pos + r * (need - 1);
+__host__ __device__ inline TmaCoord tma_coord(const Params& P, int ri, int first_pos,
+                                              int need) {
+  const int r = P.r_val[ri];
+  const int last_pos = first_pos + r * (need - 1);
   TmaCoord t;
   if (last_pos >= r * P.kfull[ri]) {
-    const int64_t x = first_pos - P.tail[ri];  // >= 0 by the host's shape check
+    const int x = first_pos - P.tail[ri];  // >= 0 by the host's shape check
     t.map = 1;
     t.c = (int)(x % r);
     t.kk = (int)(x / r);
@@ -414,9 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t bh = blockIdx.x - rank * BH;
   const int64_t b = bh / P.pb.H;
   const int64_t h = bh - b * P.pb.H;
-  const int64_t ri_range = (P.range_order[0] >= 0 && rank < kMaxRangeOrder) ? P.range_order[rank] : rank;
-  const int64_t A = ri_range * P.range_len;
-  const int64_t Bnd = (A + P.range_len < P.pb.N) ? A + P.range_len : P.pb.N;
+  const int ri_range = (P.range_order[0] >= 0 && rank < kMaxRangeOrder) ? P.range_order[rank] : (int)rank;
+  const int A = ri_range * P.range_len;
+  const int Bnd = (int64_t)A + P.range_len < P.pb.N ? A + P.range_len : (int)P.pb.N;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
@@ -465,24 +465,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && tw.next(t)) {
         const int ri = P.pat_r[t.p];
-        const int64_t seg_base = t.seg * tw.w[t.p] + tw.o[t.p];
+        const int seg_base = t.seg * tw.w[t.p] + tw.o[t.p];
         if (tile_it > 0) ok = sy.wait(bar_q_empty, (tile_it - 1) & 1);
         if (!ok) break;
         {
-          const int64_t first = seg_base + tw.r[t.p] * t.k0;
+          const int first = seg_base + tw.r[t.p] * t.k0;
           const TmaCoord c = tma_coord(P, ri, first, t.nrows);
           mbar_arrive_expect_tx(bar_q_full, kTileBytes);
           tma_load_5d(sQ, &maps.m[ri][c.map][0], bar_q_full, 0, (int)h, c.c, c.kk, (int)b);
         }
-        const int64_t n_keys_total = tw.causal ? t.k0 + t.nrows : tw.m[t.p];
+        const int n_keys_total = tw.causal ? t.k0 + t.nrows : tw.m[t.p];
         for (int j = 0; j < t.nkv; ++j) {
           const int s = kv_it % kStages;
           if (kv_it >= kStages) ok = sy.wait(bar_kv_empty + s, ((kv_it / kStages) - 1) & 1);
           if (!ok) break;
-          const int64_t kstart = (int64_t)j * kBN;
-          int64_t need = n_keys_total - kstart;
+          const int kstart = j * kBN;
+          int need = n_keys_total - kstart;
           if (need > kBN) need = kBN;
-          const int64_t first = seg_base + tw.r[t.p] * kstart;
+          const int first = seg_base + tw.r[t.p] * kstart;
           const TmaCoord c = tma_coord(P, ri, first, need);
           mbar_arrive_expect_tx(bar_kv_full + s, 2 * kTileBytes);
           tma_load_5d(sK + s * kTileBytes, &maps.m[ri][c.map][1], bar_kv_full + s, 0, (int)h, c.c,
@@ -585,33 +585,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
     while (ok && tw.next(t)) {
       float m_use = -INFINITY, l_run = 0.f;
-      const int64_t krow = t.k0 + row;  // this thread's sparse row
+      const int krow = t.k0 + row;  // this thread's sparse row
       for (int j = 0; j < t.nkv; ++j) {
         const uint32_t sb = s_it & 1;
         ok = sy.wait_warp(bar_s_full + sb, (s_it >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         const uint32_t s_col = tmem + lane_base + (sb ? kColS1 : kColS0);
+        uint32_t sr[kBN];
+        // four loads in flight, one wait
+        LN_TMEM_LD32(s_col + 0, (sr + 0));
+        LN_TMEM_LD32(s_col + 32, (sr + 32));
+        LN_TMEM_LD32(s_col + 64, (sr + 64));
+        LN_TMEM_LD32(s_col + 96, (sr + 96));
+        tmem_wait_ld();
         float s[kBN];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t rr[32];
-          LN_TMEM_LD32(s_col + c * 32, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
-        }
+        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
         // masks: causal (key <= row) and keys past the segment's kept rows
-        const int64_t kbase = (int64_t)j * kBN;
-        int64_t lim = tw.causal ? krow - kbase : tw.m[t.p] - 1 - kbase;
+        const int kbase = j * kBN;
+        const int lim = tw.causal ? krow - kbase : tw.m[t.p] - 1 - kbase;
         if (lim < kBN - 1) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if ((int64_t)c > lim) s[c] = -INFINITY;
+            if (c > lim) s[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max as a tree (independent partial maxima)
+        float pm[8];
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) pm[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         const float m_blk = mx * scale_log2;
         float corr = 1.f;
         bool rescale = false;
@@ -624,7 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_use = m_blk;
           }
         }
-        float lsum = 0.f;
+        float ps[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ps[e] = 0.f;
         const uint32_t p_col = s_col;  // P overwrites the first 64 columns of S
 #pragma unroll
         for (int c = 0; c < kBN / 64; ++c) {
@@ -633,11 +643,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) {
             const float a = ex2(fmaf(s[c * 64 + 2 * e], scale_log2, -m_use));
             const float bq = ex2(fmaf(s[c * 64 + 2 * e + 1], scale_log2, -m_use));
-            lsum += a + bq;
+            ps[e & 7] += a + bq;
             pk[e] = pack_bf16(a, bq);
           }
           LN_TMEM_ST32(p_col + c * 32, pk);
         }
+        const float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         tmem_wait_st();
         l_run = l_run * corr + lsum;
         if (j > 0) {
@@ -647,15 +658,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (__any_sync(0xffffffffu, rescale)) {
             const uint32_t o_col = tmem + lane_base + kColO;
+            uint32_t rr[kD];
+            LN_TMEM_LD32(o_col, (rr + 0));
+            LN_TMEM_LD32(o_col + 32, (rr + 32));
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kD / 32; ++c) {
-              uint32_t rr[32];
-              LN_TMEM_LD32(o_col + c * 32, rr);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
-              LN_TMEM_ST32(o_col + c * 32, rr);
-            }
+            for (int e = 0; e < kD; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
+            LN_TMEM_ST32(o_col, (rr + 0));
+            LN_TMEM_ST32(o_col + 32, (rr + 32));
             tmem_wait_st();
           }
         }
@@ -671,14 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[kD];
       {
         const uint32_t o_col = tmem + lane_base + kColO;
+        uint32_t rr[kD];
+        LN_TMEM_LD32(o_col, (rr + 0));
+        LN_TMEM_LD32(o_col + 32, (rr + 32));
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t rr[32];
-          LN_TMEM_LD32(o_col + c * 32, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[c * 32 + e] = __uint_as_float(rr[e]);
-        }
+        for (int e = 0; e < kD; ++e) o[e] = __uint_as_float(rr[e]);
       }
       tc_fence_before();
       mbar_arrive(bar_o_free);
@@ -687,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int d = 0; d < kD; ++d) o[d] *= inv;
         float lse2 = m_use + __log2f(l_run);  // log2 domain
-        const int64_t x = t.start + tw.r[t.p] * (int64_t)row;
+        const int x = t.start + tw.r[t.p] * row;
         // last tile covering x?  (all other covering tiles come earlier)
         bool final_row = true;
         for (int q = 0; q < tw.n_pat && final_row; ++q) {
@@ -753,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && P.uncovered_possible) {
       // positions of this range that no pattern keeps: out = 0, lse = -inf
-      for (int64_t x = A + row; x < Bnd; x += 128) {
+      for (int x = A + row; x < Bnd; x += 128) {
         bool any = false;
         for (int q = 0; q < tw.n_pat && !any; ++q) {
           Cover cv;
@@ -901,7 +909,7 @@ void fill_params(const Problem& pb, tc::Params& P) {
   if (P.n_ranges <= kMaxRangeOrder) {
     std::vector<int64_t> cost(P.n_ranges);
     for (int i = 0; i < P.n_ranges; ++i)
-      cost[i] = range_cost(pb, i * P.range_len, std::min(pb.N, (i + 1) * P.range_len));
+      cost[i] = range_cost(pb, (int64_t)i * P.range_len, std::min<int64_t>(pb.N, (int64_t)(i + 1) * P.range_len));
     std::vector<int> idx(P.n_ranges);
     std::iota(idx.begin(), idx.end(), 0);
     std::stable_sort(idx.begin(), idx.end(), [&](int a, int c) { return cost[a] > cost[c]; });
