@@ -48,6 +48,7 @@
 #include <algorithm>
 #include <mutex>
 #include <numeric>
+#include <type_traits>
 #include <vector>
 
 #include "device_util.cuh"
@@ -58,30 +59,83 @@ namespace tc {
 
 constexpr int kD = 64;          // head dimension of this family
 constexpr int kBM = 128;        // query rows per tile (MMA M)
-constexpr int kBN = 128;        // keys per KV block (MMA N of Q K^T)
-constexpr int kStages = 3;      // K/V shared-memory ring depth
+constexpr int kBN = 64;         // keys per KV block (MMA N of Q K^T)
 constexpr int kMaxPat = 6;      // patterns (and combination slots) supported
 constexpr int kMaxR = 8;        // distinct dilations supported
-constexpr int kThreads = 256;   // 8 warps: TMA, MMA, 2 idle, 4 softmax/epilogue
-constexpr int kTileBytes = kBM * kD * 2;  // 16 KB per 128 x 64 bf16 tile
+constexpr int kThreads = 512;   // 16 warps: TMA, MMA, 2 idle, 2x4 softmax, 4 epilogue
+constexpr int kTileBytes = kBM * kD * 2;  // 16 KB per 128 x 64 bf16 Q tile
+constexpr int kKVBytes = kBN * kD * 2;    // 8 KB per 64 x 64 bf16 K or V block
 constexpr int kMaxRangeOrder = 4096;
+constexpr int kSmemLimit = 232448;       // dynamic shared memory per block on sm_100
+constexpr int kTileOverhead = 1;         // block-equivalents charged per tile (stream balance)
 
-// TMEM columns: two S buffers (128 fp32 columns each) and O (64 columns).
+// TMEM columns: two S buffers per softmax stream (64 fp32 columns each) and
+// two O buffers per stream (64 columns each).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+__host__ __device__ constexpr uint32_t col_s(int g, int sb) { return (uint32_t)(2 * g + sb) * 64u; }
+__host__ __device__ constexpr uint32_t col_o(int g, int ob) { return 256u + (uint32_t)(2 * g + ob) * 64u; }
 
-struct SmemLayout {
-  static constexpr int q = 0;
-  static constexpr int k = q + kTileBytes;
-  static constexpr int v = k + kStages * kTileBytes;
-  static constexpr int slot_o = v + kStages * kTileBytes;
-  static constexpr int slot_l = slot_o + kMaxPat * kTileBytes;
-  static constexpr int bars = slot_l + kMaxPat * kBM * 4;
-  static constexpr int n_bars = 2 + 2 * kStages + 2 + 2 + 3;
-  static constexpr int misc = bars + n_bars * 8;
-  static constexpr int total = misc + 64;
+// Descriptors the TMA thread publishes for the other roles.
+constexpr int kQE = 16;  // element queue entries per softmax stream
+constexpr int kQT = 32;  // tile queue entries (epilogue)
+struct ElemMeta {        // one KV block of one tile
+  int info;              // bit0 stream, bit1 O buffer, bit2 use parity, bit3 use > 0, bit4 end
+  int j;                 // KV block within the tile
+  int nkv;               // KV blocks of the tile
+  int lim0;              // causal: first kept row of the tile; full: kept rows - 1
 };
-constexpr int kSmemBytes = SmemLayout::total + 1024;  // + alignment slack
+struct TileMeta {        // one tile, in processing order
+  int info;              // as ElemMeta
+  int p;                 // pattern
+  int start;             // position of the first row
+  int nrows;
+  int seq;               // processing-order index; written last (release)
+  int pad[3];
+};
+constexpr int kInfoEnd = 16;
+// element queues [2][kQE], tile queue [kQT], stage descriptors [kMaxStages],
+// pattern table [kMaxPat] (w, r, o, m), counters (16 ints)
+constexpr int kMaxStages = 4;   // K/V ring depth per stream (runtime, 2..4)
+constexpr int kMetaBytes = 2 * kQE * 16 + kQT * 32 + 2 * kMaxStages * 16 + kMaxPat * 16 + 64;
+constexpr int kWalkerBytes = 512;  // per stream
+
+// Shared-memory carve-up, sized at run time from the pattern count.
+struct SmemLayout {
+  int q;       // 2 Q tiles (one per stream)
+  int kv;      // [stream][stages] x (K block, V block)
+  int slot_o;  // n_pat x 128 parked rows (bf16)
+  int slot_l;  // n_pat x 128 parked lse (fp32, log2 domain)
+  int stats;   // [stream][O buffer][use parity][row] (m, l)
+  int meta;    // element queues, tile queue, stage descriptors, pattern table, counters
+  int walker;  // the TMA thread's block-sequence state (kept out of local memory)
+  int bars;
+  int misc;
+  int total;
+  int stages;
+  __host__ __device__ void make(int n_pat, int n_stages) {
+    stages = n_stages;
+    q = 0;
+    kv = q + 2 * kTileBytes;
+    slot_o = kv + 2 * stages * 2 * kKVBytes;
+    slot_l = slot_o + n_pat * kTileBytes;
+    stats = slot_l + n_pat * kBM * 4;
+    meta = stats + 2 * 2 * 2 * kBM * 8;
+    walker = meta + kMetaBytes;
+    bars = walker + 2 * kWalkerBytes;
+    misc = bars + 48 * 8;
+    total = misc + 64;
+  }
+};
+// Largest per-stream K/V ring that fits with n_pat slots (>= 2: a stream's MMA
+// issues the S of its next block before the PV of the current one).
+inline int pick_stages(int n_pat) {
+  for (int st = kMaxStages; st >= 2; --st) {
+    SmemLayout L;
+    L.make(n_pat, st);
+    if (L.total + 1024 <= kSmemLimit) return st;
+  }
+  return 0;
+}
 
 struct __align__(64) TmaMaps {
   CUtensorMap m[kMaxR][2][3];  // [distinct r][base / shifted][q, k, v]
@@ -97,6 +151,8 @@ struct Params {
   int range_len;              // R
   int n_ranges;
   int uncovered_possible;     // some position may be kept by no pattern
+  int stages;                 // K/V ring depth
+  int smem_bytes;             // dynamic shared memory requested
   uint64_t wait_limit_ns;
   int range_order[kMaxRangeOrder];  // longest-first order of ranges (or -1: identity)
 };
@@ -215,7 +271,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
-constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false);
+constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false);  // S: 128 x 64
 constexpr uint32_t kIdescPV = idesc_bf16(kBM, kD, true);
 
 // ---------------------------------------------------------------- tiles
@@ -303,20 +359,25 @@ struct Cover {
   int start;
   int slot_row;
 };
-__host__ __device__ inline bool cover_of(const TileWalker& tw, int q, int x, Cover& c) {
-  const int sq = x / tw.w[q];
-  const int rel = x - sq * tw.w[q] - tw.o[q];
+// Tile of one pattern (segment length w, dilation r, head offset o, m kept
+// rows per segment) covering position x in a unit starting at A.
+__host__ __device__ inline bool cover_pat(int w, int r, int o, int m, int A, int x, Cover& c) {
+  const int sq = x / w;
+  const int rel = x - sq * w - o;
   if (rel < 0) return false;
-  const int kq = rel / tw.r[q];
-  if (kq * tw.r[q] != rel) return false;
-  if (kq >= tw.m[q]) return false;
-  const int base = sq * tw.w[q] + tw.o[q];
-  int lo = tw.A - base;
-  lo = lo <= 0 ? 0 : (lo + tw.r[q] - 1) / tw.r[q];
+  const int kq = rel / r;
+  if (kq * r != rel) return false;
+  if (kq >= m) return false;
+  const int base = sq * w + o;
+  int lo = A - base;
+  lo = lo <= 0 ? 0 : (lo + r - 1) / r;
   const int t = (kq - lo) / kBM;
-  c.start = base + tw.r[q] * (lo + t * kBM);
-  c.slot_row = (int)((kq - lo) - t * kBM);
+  c.start = base + r * (lo + t * kBM);
+  c.slot_row = (kq - lo) - t * kBM;
   return true;
+}
+__host__ __device__ inline bool cover_of(const TileWalker& tw, int q, int x, Cover& c) {
+  return cover_pat(tw.w[q], tw.r[q], tw.o[q], tw.m[q], tw.A, x, c);
 }
 __host__ __device__ inline bool key_before(int s_a, int r_a, int p_a, int s_b,
                                            int r_b, int p_b) {
@@ -380,30 +441,313 @@ __host__ __device__ inline TmaCoord tma_coord(const Params& P, int ri, int first
   return t;
 }
 
+// ---------------------------------------------------------------- block sequence
+
+// One KV block of one tile, as emitted in the order the K/V ring is filled.
+struct Elem {
+  int g;         // softmax stream (warpgroup) that owns the tile
+  Tile t;
+  int j;         // KV block within the tile
+  int tile_idx;  // position of the tile in processing order
+  int ob;        // O buffer (TMEM) of the tile within its stream
+  int use;       // earlier tiles of this stream that used the same O buffer
+};
+
+// Deterministic interleaving of the unit's tiles over two softmax streams.
+// Every role runs an identical copy, so the TMA warp and the MMA warp agree
+// on the K/V ring order and each softmax stream knows its own tiles.
+//  * Tiles are taken in processing order by whichever stream is ahead least
+//    (a simulated clock in KV blocks), so the streams stay balanced.
+//  * A stream may start a tile that reuses an O buffer only when the other
+//    stream has emitted every block of every tile up to the previous user of
+//    that buffer: the epilogue (which runs in processing order) can then
+//    always free the buffer without waiting on work queued behind it.
+struct BlockSeq {
+  TileWalker tw;
+  Tile cur[2];
+  int j[2], clk[2], nt[2], cur_idx[2], last_user[2][2];
+  bool alive[2];
+  int fetched;
+
+  __host__ __device__ void init(const Params& P, int h, int A, int Bnd) {
+    tw.init(P, h, A, Bnd);
+    fetched = 0;
+    for (int g = 0; g < 2; ++g) {
+      cur[g].nkv = 0;
+      j[g] = 0;
+      clk[g] = 0;
+      nt[g] = 0;
+      cur_idx[g] = -1;
+      last_user[g][0] = last_user[g][1] = -1;
+      alive[g] = true;
+    }
+  }
+  __host__ __device__ bool in_progress(int g) const { return alive[g] && j[g] < cur[g].nkv; }
+  __host__ __device__ bool next(Elem& e) {
+    for (;;) {
+      int g;
+      if (alive[0] && (!alive[1] || clk[0] <= clk[1])) g = 0;
+      else if (alive[1]) g = 1;
+      else return false;
+      if (!in_progress(g)) {
+        const int og = 1 - g;
+        if (nt[g] >= 2) {
+          const int prev = last_user[g][nt[g] & 1];
+          if (in_progress(og) && cur_idx[og] <= prev) g = og;  // the other stream first
+        }
+        if (!in_progress(g)) {
+          Tile t;
+          if (!tw.next(t)) {
+            alive[g] = false;
+            continue;
+          }
+          cur[g] = t;
+          j[g] = 0;
+          cur_idx[g] = fetched++;
+          last_user[g][nt[g] & 1] = cur_idx[g];
+          ++nt[g];
+          clk[g] += kTileOverhead;
+        }
+      }
+      e.g = g;
+      e.t = cur[g];
+      e.j = j[g];
+      e.tile_idx = cur_idx[g];
+      e.ob = (nt[g] - 1) & 1;
+      e.use = (nt[g] - 1) >> 1;
+      ++j[g];
+      ++clk[g];
+      return true;
+    }
+  }
+};
+
+// ---------------------------------------------------------------- single-thread roles
+
+// The TMA thread's block sequence, with every per-stream field in registers
+// (stream indices are compile-time constants; only the tile walk, touched
+// once per tile, lives in shared memory).  Emits exactly the sequence of
+// BlockSeq above.
+struct StreamState {
+  Tile t;
+  int j, clk, nt, cur_idx, lu0, lu1;
+  bool alive;
+};
+struct FastSeq {
+  TileWalker* tw;
+  StreamState s0, s1;
+  int fetched;
+  template <int G>
+  __host__ __device__ __forceinline__ StreamState& st() {
+    if constexpr (G == 0) return s0;
+    else return s1;
+  }
+  __host__ __device__ __forceinline__ void init(TileWalker* w) {
+    tw = w;
+    fetched = 0;
+    s0.t.nkv = s1.t.nkv = 0;
+    s0.j = s1.j = 0;
+    s0.clk = s1.clk = 0;
+    s0.nt = s1.nt = 0;
+    s0.cur_idx = s1.cur_idx = -1;
+    s0.lu0 = s0.lu1 = s1.lu0 = s1.lu1 = -1;
+    s0.alive = s1.alive = true;
+  }
+  template <int G>
+  __host__ __device__ __forceinline__ void emit(Elem& e) {
+    StreamState& me = st<G>();
+    e.g = G;
+    e.t = me.t;
+    e.j = me.j;
+    e.tile_idx = me.cur_idx;
+    e.ob = (me.nt - 1) & 1;
+    e.use = (me.nt - 1) >> 1;
+    ++me.j;
+    ++me.clk;
+  }
+  template <int G>
+  __host__ __device__ __forceinline__ bool step(Elem& e) {  // false: pick again
+    StreamState& me = st<G>();
+    StreamState& ot = st<1 - G>();
+    if (me.j >= me.t.nkv) {
+      if (me.nt >= 2) {
+        const int prev = (me.nt & 1) ? me.lu1 : me.lu0;
+        if (ot.alive && ot.j < ot.t.nkv && ot.cur_idx <= prev) {  // the other stream first
+          emit<1 - G>(e);
+          return true;
+        }
+      }
+      Tile t;
+      if (!tw->next(t)) {
+        me.alive = false;
+        return false;
+      }
+      me.t = t;
+      me.j = 0;
+      me.cur_idx = fetched++;
+      if (me.nt & 1) me.lu1 = me.cur_idx;
+      else me.lu0 = me.cur_idx;
+      ++me.nt;
+      me.clk += kTileOverhead;
+    }
+    emit<G>(e);
+    return true;
+  }
+  __host__ __device__ __forceinline__ bool next(Elem& e) {
+    for (;;) {
+      if (s0.alive && (!s1.alive || s0.clk <= s1.clk)) {
+        if (step<0>(e)) return true;
+      } else if (s1.alive) {
+        if (step<1>(e)) return true;
+      } else {
+        return false;
+      }
+    }
+  }
+};
+
+// Pending PV of one block, packed: stage (bits 0-2), S buffer (3), its
+// phase parity (4), first block of the tile (5), last block (6), O buffer
+// (7), O-buffer use parity (8), O buffer used before (9), P seen (10).
+enum : uint32_t {
+  kEStage = 7u, kESb = 1u << 3, kEPar = 1u << 4, kEFirst = 1u << 5, kELast = 1u << 6,
+  kEOb = 1u << 7, kEUpar = 1u << 8, kEUgt0 = 1u << 9, kESeen = 1u << 10
+};
+
+// Shared-memory matrix descriptor from a precomputed low word.
+__device__ __forceinline__ uint64_t desc_from(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
+}
+// High word: SBO 1024 B, sm_100 version, 128-byte swizzle.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+struct MmaCtx {
+  uint32_t tmem;
+  uint32_t kv_lo;  // (smem address of the K/V ring) >> 4
+  uint64_t* bar_p_full;
+  uint64_t* bar_o_free;
+  uint64_t* bar_o_full;
+  uint64_t* bar_o_done;
+  uint64_t* bar_kv_empty;
+  Sync* sy;
+  uint32_t f0, f1;  // FIFO of pending PVs per stream (two 16-bit entries)
+  int n0, n1;
+  uint32_t busy;    // bit per ring stage: a pending PV still holds it
+  uint32_t owner1;  // bit per ring stage: that PV is stream 1's
+};
+template <int G>
+__device__ __forceinline__ uint32_t& fifo_of(MmaCtx& c) {
+  if constexpr (G == 0) return c.f0;
+  else return c.f1;
+}
+template <int G>
+__device__ __forceinline__ int& nf_of(MmaCtx& c) {
+  if constexpr (G == 0) return c.n0;
+  else return c.n1;
+}
+template <int G>
+__device__ __forceinline__ void pv_issue_front(MmaCtx& c) {
+  uint32_t& f = fifo_of<G>(c);
+  const uint32_t e = f & 0xFFFFu;
+  const int st = (int)(e & kEStage), sb = (e & kESb) ? 1 : 0, ob = (e & kEOb) ? 1 : 0;
+  const bool first = (e & kEFirst) != 0;
+  tc_fence_after();
+  const uint32_t v_lo = c.kv_lo + (uint32_t)st * ((2 * kKVBytes) >> 4) + (kKVBytes >> 4) +
+                        ((uint32_t)(kBN * 128) >> 4 << 16);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    mma_ts(c.tmem + col_o(G, ob), c.tmem + col_s(G, sb) + kk * 8, desc_from(v_lo + kk * 128, kDescHi),
+           kIdescPV, (first && kk == 0) ? 0u : 1u);
+  tc_commit(c.bar_kv_empty + st);
+  tc_commit((e & kELast) ? c.bar_o_full + 2 * G + ob : c.bar_o_done + G);
+  c.busy &= ~(1u << st);
+  f >>= 16;
+  --nf_of<G>(c);
+}
+// Has the front PV's P landed (and, for a tile's first block, its O buffer
+// been freed)?  Blocking or not.
+template <int G>
+__device__ __forceinline__ bool pv_front_ready(MmaCtx& c, bool block) {
+  uint32_t& f = fifo_of<G>(c);
+  const uint32_t e = f & 0xFFFFu;
+  if (!(e & kESeen)) {
+    uint64_t* bar = c.bar_p_full + 2 * G + ((e & kESb) ? 1 : 0);
+    const uint32_t par = (e & kEPar) ? 1u : 0u;
+    if (block ? !c.sy->wait(bar, par) : !mbar_test_wait(bar, par)) return false;
+    f |= kESeen;
+  }
+  if ((e & kEFirst) && (e & kEUgt0)) {
+    uint64_t* bar = c.bar_o_free + 2 * G + ((e & kEOb) ? 1 : 0);
+    const uint32_t par = (e & kEUpar) ? 0u : 1u;  // the previous use's phase
+    if (block ? !c.sy->wait(bar, par) : !mbar_test_wait(bar, par)) return false;
+  }
+  return true;
+}
+// Blocking issue of the front PV; before waiting for an O buffer, the other
+// stream's pending PVs go first (without nesting further).
+template <int G>
+__device__ __forceinline__ bool pv_force_front(MmaCtx& c, bool flush) {
+  const uint32_t e = fifo_of<G>(c) & 0xFFFFu;
+  if (flush && (e & kEFirst) && (e & kEUgt0)) {
+    while (nf_of<1 - G>(c) > 0) {
+      if (!pv_front_ready<1 - G>(c, true)) return false;
+      pv_issue_front<1 - G>(c);
+    }
+  }
+  if (!pv_front_ready<G>(c, true)) return false;
+  pv_issue_front<G>(c);
+  return true;
+}
+template <int G>
+__device__ __forceinline__ void pv_issue_ready(MmaCtx& c) {
+  while (nf_of<G>(c) > 0 && pv_front_ready<G>(c, false)) pv_issue_front<G>(c);
+}
+
 // ---------------------------------------------------------------- kernel
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     dilated_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ TmaMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + SmemLayout::q;
-  uint8_t* sK = smem + SmemLayout::k;
-  uint8_t* sV = smem + SmemLayout::v;
-  uint8_t* sSlotO = smem + SmemLayout::slot_o;
-  float* sSlotL = reinterpret_cast<float*>(smem + SmemLayout::slot_l);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
-  uint64_t* bar_q_full = bars + 0;
-  uint64_t* bar_q_empty = bars + 1;
-  uint64_t* bar_kv_full = bars + 2;
-  uint64_t* bar_kv_empty = bars + 2 + kStages;
-  uint64_t* bar_s_full = bars + 2 + 2 * kStages;
-  uint64_t* bar_p_full = bar_s_full + 2;
-  uint64_t* bar_o_done = bar_p_full + 2;
-  uint64_t* bar_o_free = bar_o_done + 1;
-  uint64_t* bar_drain = bar_o_free + 1;
-  uint64_t* bar_epi = bar_drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 8);
+  SmemLayout L;
+  L.make(P.pb.n_pat, P.stages);
+  const int NS = P.stages;
+  uint8_t* sQ = smem + L.q;
+  uint8_t* sKV = smem + L.kv;  // stream g, stage s at (g*NS + s)*16K: K, then V at +8K
+  uint8_t* sSlotO = smem + L.slot_o;
+  float* sSlotL = reinterpret_cast<float*>(smem + L.slot_l);
+  float2* sStats = reinterpret_cast<float2*>(smem + L.stats);
+  ElemMeta* sElemQ = reinterpret_cast<ElemMeta*>(smem + L.meta);     // [2][kQE]
+  TileMeta* sTileQ = reinterpret_cast<TileMeta*>(sElemQ + 2 * kQE);   // [kQT]
+  ElemMeta* sStageMeta = reinterpret_cast<ElemMeta*>(sTileQ + kQT);   // [2][kMaxStages]
+  int4* sPat = reinterpret_cast<int4*>(sStageMeta + 2 * kMaxStages);  // [kMaxPat] (w, r, o, m)
+  int* sCnt = reinterpret_cast<int*>(sPat + kMaxPat);
+  int* cnt_elem = sCnt + 0;       // [2] elements published per stream
+  int* cnt_soft = sCnt + 4;       // [2] elements consumed per stream
+  int* cnt_epi = sCnt + 6;        // tiles consumed
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* bar_q_full = bars + 0;        // [2]
+  uint64_t* bar_q_empty = bars + 2;       // [2]
+  uint64_t* bar_s_full = bars + 4;        // [2][2] stream, S buffer
+  uint64_t* bar_p_full = bars + 8;        // [2][2]
+  uint64_t* bar_o_done = bars + 12;       // [2]
+  uint64_t* bar_o_full = bars + 14;       // [2][2] stream, O buffer
+  uint64_t* bar_o_free = bars + 18;       // [2][2]
+  uint64_t* bar_epi = bars + 22;
+  uint64_t* bar_drain = bars + 23;        // [2]
+  uint64_t* bar_kv_full = bars + 26;      // [2][kMaxStages]
+  uint64_t* bar_kv_empty = bars + 26 + 2 * kMaxStages;  // [2][kMaxStages]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -417,29 +761,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ri_range = (P.range_order[0] >= 0 && rank < kMaxRangeOrder) ? P.range_order[rank] : (int)rank;
   const int A = ri_range * P.range_len;
   const int Bnd = (int64_t)A + P.range_len < P.pb.N ? A + P.range_len : (int)P.pb.N;
+  const int n_pat = P.pb.n_pat;
+  const bool causal = P.pb.causal != 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_kv_full + s, 1);
-      mbar_init(bar_kv_empty + s, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar_q_full + g, 1);
+      mbar_init(bar_q_empty + g, 1);
+      for (int sb = 0; sb < 2; ++sb) {
+        mbar_init(bar_s_full + 2 * g + sb, 1);
+        mbar_init(bar_p_full + 2 * g + sb, 128);
+      }
+      mbar_init(bar_o_done + g, 1);
+      for (int ob = 0; ob < 2; ++ob) {
+        mbar_init(bar_o_full + 2 * g + ob, 1 + 128);  // last PV commit + softmax stats
+        mbar_init(bar_o_free + 2 * g + ob, 128);
+      }
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_s_full + s, 1);
-      mbar_init(bar_p_full + s, 128);
-    }
-    mbar_init(bar_o_done, 1);
-    mbar_init(bar_o_free, 128);
-    mbar_init(bar_drain, 1);
     mbar_init(bar_epi, 128);
+    mbar_init(bar_drain + 0, 1);
+    mbar_init(bar_drain + 1, 1);
+    for (int st = 0; st < 2 * kMaxStages; ++st) {
+      mbar_init(bar_kv_full + st, 1);
+      mbar_init(bar_kv_empty + st, 1);
+    }
+    for (int i = 0; i < kQT; ++i) sTileQ[i].seq = -1;
+    for (int p = 0; p < n_pat; ++p) {
+      const int w = (int)P.pb.w[p], r = (int)P.pb.r[p], o = (int)(h % r);
+      sPat[p] = make_int4(w, r, o, o >= w ? 0 : (w - o + r - 1) / r);
+    }
+    for (int i = 0; i < 16; ++i) sCnt[i] = 0;
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if ((warp == 0 || warp == 2) && lane == 0) {
     for (int i = 0; i < P.n_r; ++i)
-      for (int j = 0; j < 2; ++j)
-        for (int t = 0; t < 3; ++t) prefetch_tmap(&maps.m[i][j][t]);
+      for (int jj = 0; jj < 2; ++jj)
+        for (int t = 0; t < 3; ++t) prefetch_tmap(&maps.m[i][jj][t]);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -454,261 +812,406 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   Sync sy{bars, abort_flag, P.pb.status, P.wait_limit_ns};
-  TileWalker tw;
-  tw.init(P, h, A, Bnd);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t kv_it = 0, tile_it = 0;
-      Tile t;
-      bool ok = true;
-      while (ok && tw.next(t)) {
-        const int ri = P.pat_r[t.p];
-        const int seg_base = t.seg * tw.w[t.p] + tw.o[t.p];
-        if (tile_it > 0) ok = sy.wait(bar_q_empty, (tile_it - 1) & 1);
-        if (!ok) break;
-        {
-          const int first = seg_base + tw.r[t.p] * t.k0;
-          const TmaCoord c = tma_coord(P, ri, first, t.nrows);
-          mbar_arrive_expect_tx(bar_q_full, kTileBytes);
-          tma_load_5d(sQ, &maps.m[ri][c.map][0], bar_q_full, 0, (int)h, c.c, c.kk, (int)b);
+  // Bounded spin until *cnt > need (acquire); false on timeout or abort.
+  auto wait_count = [&](const int* cnt, int need) -> bool {
+    if (ld_acquire(cnt) > need) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(64);
+      if (ld_acquire(cnt) > need) return true;
+      if ((it & 15u) == 0) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > P.wait_limit_ns) {
+          *abort_flag = 1;
+          record_status(P.pb.status, kStatusTimeout);
+          return false;
         }
-        const int n_keys_total = tw.causal ? t.k0 + t.nrows : tw.m[t.p];
-        for (int j = 0; j < t.nkv; ++j) {
-          const int s = kv_it % kStages;
-          if (kv_it >= kStages) ok = sy.wait(bar_kv_empty + s, ((kv_it / kStages) - 1) & 1);
+      }
+    }
+  };
+
+  // Register split across warpgroups (512 threads x 128 registers at launch,
+  // 65536 in all): TMA/MMA warpgroup 96, two softmax warpgroups 152 each,
+  // epilogue 112 (96*128 + 152*256 + 112*128 = 65536).  Each role sets its
+  // own limit first thing in its branch.
+  // Bounded spin until *p == v (acquire); false on timeout or abort.
+  auto wait_seq = [&](const int* p, int v) -> bool {
+    if (ld_acquire(p) == v) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(64);
+      if (ld_acquire(p) == v) return true;
+      if ((it & 15u) == 0) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > P.wait_limit_ns) {
+          *abort_flag = 1;
+          record_status(P.pb.status, kStatusTimeout);
+          return false;
+        }
+      }
+    }
+  };
+
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ TMA, one warp per stream
+    // Both run the same block sequence (so they agree on which tiles are
+    // whose); each loads only its own stream's Q tiles and K/V blocks into its
+    // own ring, and publishes its own descriptors.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+    const int g = warp >> 1;
+    if (lane == 0) {
+      TileWalker* twp = reinterpret_cast<TileWalker*>(smem + L.walker + g * kWalkerBytes);
+      twp->init(P, (int)h, A, Bnd);
+      FastSeq seq;
+      seq.init(twp);
+      Elem e;
+      uint8_t* ring = sKV + g * NS * 2 * kKVBytes;
+      uint64_t* kv_full = bar_kv_full + g * kMaxStages;
+      uint64_t* kv_empty = bar_kv_empty + g * kMaxStages;
+      ElemMeta* stage_meta = sStageMeta + g * kMaxStages;
+      uint32_t kv_it = 0, qc = 0;
+      int st = 0;
+      uint32_t st_par = 0;
+      int ne = 0;
+      bool ok = true;
+      while (ok && seq.next(e)) {
+        if (e.g != g) continue;
+        const Tile& t = e.t;
+        const int ri = P.pat_r[t.p];
+        const int4 pt = sPat[t.p];  // (w, r, o, m)
+        const int seg_base = t.seg * pt.x + pt.z;
+        const int info = g | (e.ob << 1) | ((e.use & 1) << 2) | ((e.use > 0) << 3);
+        if (e.j == 0) {
+          ok = wait_count(cnt_epi, e.tile_idx - kQT);  // tile queue entry is free
           if (!ok) break;
-          const int kstart = j * kBN;
-          int need = n_keys_total - kstart;
-          if (need > kBN) need = kBN;
-          const int first = seg_base + tw.r[t.p] * kstart;
-          const TmaCoord c = tma_coord(P, ri, first, need);
-          mbar_arrive_expect_tx(bar_kv_full + s, 2 * kTileBytes);
-          tma_load_5d(sK + s * kTileBytes, &maps.m[ri][c.map][1], bar_kv_full + s, 0, (int)h, c.c,
-                      c.kk, (int)b);
-          tma_load_5d(sV + s * kTileBytes, &maps.m[ri][c.map][2], bar_kv_full + s, 0, (int)h, c.c,
-                      c.kk, (int)b);
+          TileMeta& tm = sTileQ[e.tile_idx % kQT];
+          tm.info = info;
+          tm.p = t.p;
+          tm.start = t.start;
+          tm.nrows = t.nrows;
+          st_release(&tm.seq, e.tile_idx);
+          if (qc > 0) ok = sy.wait(bar_q_empty + g, (qc - 1) & 1);
+          if (!ok) break;
+          const TmaCoord c = tma_coord(P, ri, seg_base + pt.y * t.k0, t.nrows);
+          mbar_arrive_expect_tx(bar_q_full + g, kTileBytes);
+          tma_load_5d(sQ + g * kTileBytes, &maps.m[ri][c.map][0], bar_q_full + g, 0, (int)h, c.c, c.kk,
+                      (int)b);
+          ++qc;
+        }
+        ElemMeta em;
+        em.info = info;
+        em.j = e.j;
+        em.nkv = t.nkv;
+        em.lim0 = causal ? t.k0 : pt.w - 1;
+        ok = wait_count(cnt_soft + g, ne - kQE);  // element queue has room
+        if (!ok) break;
+        sElemQ[g * kQE + (ne & (kQE - 1))] = em;
+        st_release(cnt_elem + g, ++ne);
+        if (kv_it >= (uint32_t)NS) ok = sy.wait(kv_empty + st, st_par ^ 1);
+        if (!ok) break;
+        stage_meta[st] = em;
+        const int n_keys_total = causal ? t.k0 + t.nrows : pt.w;
+        const int kstart = e.j * kBN;
+        const int need = n_keys_total - kstart < kBN ? n_keys_total - kstart : kBN;
+        const TmaCoord c = tma_coord(P, ri, seg_base + pt.y * kstart, need);
+        mbar_arrive_expect_tx(kv_full + st, 2 * kKVBytes);
+        tma_load_5d(ring + st * 2 * kKVBytes, &maps.m[ri][c.map][1], kv_full + st, 0, (int)h, c.c, c.kk,
+                    (int)b);
+        tma_load_5d(ring + st * 2 * kKVBytes + kKVBytes, &maps.m[ri][c.map][2], kv_full + st, 0, (int)h,
+                    c.c, c.kk, (int)b);
+        ++kv_it;
+        if (++st == NS) {
+          st = 0;
+          st_par ^= 1;
+        }
+      }
+      if (ok) {
+        // end markers: one more ring stage (plain arrive) and the element
+        // queue; stream 0 also closes the tile queue
+        ElemMeta end;
+        end.info = kInfoEnd;
+        end.j = end.nkv = end.lim0 = 0;
+        if (kv_it >= (uint32_t)NS) ok = sy.wait(kv_empty + st, st_par ^ 1);
+        if (ok) {
+          stage_meta[st] = end;
+          mbar_arrive(kv_full + st);
           ++kv_it;
         }
-        ++tile_it;
+        if (ok) ok = wait_count(cnt_soft + g, ne - kQE);
+        if (ok) {
+          sElemQ[g * kQE + (ne & (kQE - 1))] = end;
+          st_release(cnt_elem + g, ++ne);
+        }
+        if (ok && g == 0) {
+          const int n_tile = seq.fetched;
+          ok = wait_count(cnt_epi, n_tile - kQT);
+          if (ok) {
+            TileMeta& tm = sTileQ[n_tile % kQT];
+            tm.info = kInfoEnd;
+            tm.p = tm.start = tm.nrows = 0;
+            st_release(&tm.seq, n_tile);
+          }
+        }
       }
-      // drain: every issued K/V load has landed before the CTA may exit
-      for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(bar_kv_full + s, (i / kStages) & 1, P.wait_limit_ns)) {
+      // drain: every issued load has landed before the CTA may exit
+      for (uint32_t i = (kv_it > (uint32_t)NS ? kv_it - NS : 0); i < kv_it; ++i) {
+        if (!mbar_wait(kv_full + (i % NS), (i / NS) & 1, P.wait_limit_ns)) {
           record_status(P.pb.status, kStatusTimeout);
           break;
         }
       }
-      if (tile_it > 0) {
-        if (!mbar_wait(bar_q_full, (tile_it - 1) & 1, P.wait_limit_ns))
-          record_status(P.pb.status, kStatusTimeout);
-      }
+      if (qc > 0 && !mbar_wait(bar_q_full + g, (qc - 1) & 1, P.wait_limit_ns))
+        record_status(P.pb.status, kStatusTimeout);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA, one warp per stream
+    // Per stream, in its ring order: the block's S = Q K^T into one of the
+    // stream's two S buffers, then the previous block's O += P V once its P
+    // is ready (for a tile's first block, once the epilogue has freed the O
+    // buffer).  So a block's S is computed while the softmax works on the one
+    // before, and the S buffer reused next is released by the PV just issued.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+    const int g = warp >> 1;
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ);
-      uint32_t kv_it = 0, tile_it = 0, s_it = 0;
-      Tile t;
+      uint8_t* ring = sKV + g * NS * 2 * kKVBytes;
+      uint64_t* kv_full = bar_kv_full + g * kMaxStages;
+      uint64_t* kv_empty = bar_kv_empty + g * kMaxStages;
+      const ElemMeta* stage_meta = sStageMeta + g * kMaxStages;
+      const uint32_t ring_lo = smem_u32(ring) >> 4;
+      const uint32_t q_lo = (smem_u32(sQ + g * kTileBytes) >> 4) | (1u << 16);
+      const uint32_t s_tmem0 = tmem + col_s(g, 0), s_tmem1 = tmem + col_s(g, 1);
+      const uint32_t o_tmem0 = tmem + col_o(g, 0), o_tmem1 = tmem + col_o(g, 1);
+      uint32_t idx = 0, qc = 0;
+      int st = 0;
+      uint32_t st_par = 0;
+      // the previous block, whose PV is still to be issued
+      bool have_prev = false;
+      int pv_st = 0, pv_info = 0;
+      uint32_t pv_idx = 0;
+      bool pv_first = false, pv_last = false;
       bool ok = true;
-      while (ok && tw.next(t)) {
-        ok = sy.wait(bar_q_full, tile_it & 1);
-        if (!ok) break;
+      auto issue_prev = [&]() -> bool {
+        const int sb = pv_idx & 1, ob = (pv_info >> 1) & 1;
+        if (!sy.wait(bar_p_full + 2 * g + sb, (pv_idx >> 1) & 1)) return false;
+        if (pv_first && (pv_info & 8) &&
+            !sy.wait(bar_o_free + 2 * g + ob, ((pv_info >> 2) & 1) ^ 1))
+          return false;
         tc_fence_after();
-        int pend_stage = -1;
-        uint32_t pend_s = 0;
-        bool pend_first = false;
-        for (int j = 0; j <= t.nkv && ok; ++j) {
-          if (j < t.nkv) {
-            const int st = kv_it % kStages;
-            ok = sy.wait(bar_kv_full + st, (kv_it / kStages) & 1);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t sb = s_it & 1;
-            const uint32_t d = tmem + (sb ? kColS1 : kColS0);
-            const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
+        const uint32_t v_lo = (ring_lo + (uint32_t)pv_st * ((2 * kKVBytes) >> 4) + (kKVBytes >> 4)) |
+                              (((uint32_t)(kBN * 128) >> 4) << 16);
+        const uint32_t a_tmem = sb ? s_tmem1 : s_tmem0;
+        const uint32_t d_tmem = ob ? o_tmem1 : o_tmem0;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(q_addr + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(k_addr + kk * 32, 16, 1024);
-              mma_ss(d, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_s_full + sb);
-            if (j == t.nkv - 1) tc_commit(bar_q_empty);
-          }
-          if (pend_stage >= 0) {
-            // O += P V for the previous block
-            const uint32_t sb = pend_s & 1;
-            ok = sy.wait(bar_p_full + sb, (pend_s >> 1) & 1);
-            if (!ok) break;
-            if (pend_first && tile_it > 0) {
-              ok = sy.wait(bar_o_free, (tile_it - 1) & 1);
-              if (!ok) break;
-            }
-            tc_fence_after();
-            const uint32_t v_addr = smem_u32(sV + pend_stage * kTileBytes);
-            const uint32_t p_tmem = tmem + (sb ? kColS1 : kColS0);
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, kBN * 128, 1024);
-              mma_ts(tmem + kColO, p_tmem + kk * 8, bd, kIdescPV,
-                     (pend_first && kk == 0) ? 0u : 1u);
-            }
-            tc_commit(bar_kv_empty + pend_stage);
-            tc_commit(bar_o_done);
-            pend_stage = -1;
-          }
-          if (j < t.nkv) {
-            pend_stage = kv_it % kStages;
-            pend_s = s_it;
-            pend_first = (j == 0);
-            ++kv_it;
-            ++s_it;
-          }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, desc_from(v_lo + kk * 128, kDescHi), kIdescPV,
+                 (pv_first && kk == 0) ? 0u : 1u);
+        tc_commit(kv_empty + pv_st);
+        tc_commit(pv_last ? bar_o_full + 2 * g + ob : bar_o_done + g);
+        return true;
+      };
+      while (ok) {
+        ok = sy.wait(kv_full + st, st_par);
+        if (!ok) break;
+        const ElemMeta em = stage_meta[st];
+        if (em.info & kInfoEnd) break;
+        if (em.j == 0) {
+          ok = sy.wait(bar_q_full + g, qc & 1);
+          if (!ok) break;
+          ++qc;
         }
-        ++tile_it;
+        tc_fence_after();
+        const int sb = idx & 1;
+        const uint32_t k_lo = (ring_lo + (uint32_t)st * ((2 * kKVBytes) >> 4)) | (1u << 16);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk)
+          mma_ss(sb ? s_tmem1 : s_tmem0, desc_from(q_lo + kk * 2, kDescHi),
+                 desc_from(k_lo + kk * 2, kDescHi), kIdescQK, kk > 0 ? 1u : 0u);
+        tc_commit(bar_s_full + 2 * g + sb);
+        if (em.j == em.nkv - 1) tc_commit(bar_q_empty + g);
+        if (have_prev) {
+          ok = issue_prev();
+          if (!ok) break;
+        }
+        have_prev = true;
+        pv_st = st;
+        pv_info = em.info;
+        pv_idx = idx;
+        pv_first = em.j == 0;
+        pv_last = em.j == em.nkv - 1;
+        ++idx;
+        if (++st == NS) {
+          st = 0;
+          st_par ^= 1;
+        }
       }
+      if (ok && have_prev) ok = issue_prev();
       // drain: all issued MMAs complete before TMEM is released
-      tc_commit(bar_drain);
-      if (!mbar_wait(bar_drain, 0, P.wait_limit_ns)) record_status(P.pb.status, kStatusTimeout);
+      tc_commit(bar_drain + g);
+      if (!mbar_wait(bar_drain + g, 0, P.wait_limit_ns)) record_status(P.pb.status, kStatusTimeout);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int row = (warp - 4) * 32 + lane;
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 152;" ::: "memory");
+    // ------------------------------------------------------------ softmax streams
+    const int g = (warp - 4) >> 2;
+    const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
-    uint32_t s_it = 0, tile_it = 0;
-    Tile t;
+    uint32_t s_cnt = 0, od_cnt = 0;
+    float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
-    while (ok && tw.next(t)) {
-      float m_use = -INFINITY, l_run = 0.f;
-      const int krow = t.k0 + row;  // this thread's sparse row
-      for (int j = 0; j < t.nkv; ++j) {
-        const uint32_t sb = s_it & 1;
-        ok = sy.wait_warp(bar_s_full + sb, (s_it >> 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t s_col = tmem + lane_base + (sb ? kColS1 : kColS0);
-        uint32_t sr[kBN];
-        // four loads in flight, one wait
-        LN_TMEM_LD32(s_col + 0, (sr + 0));
-        LN_TMEM_LD32(s_col + 32, (sr + 32));
-        LN_TMEM_LD32(s_col + 64, (sr + 64));
-        LN_TMEM_LD32(s_col + 96, (sr + 96));
-        tmem_wait_ld();
-        float s[kBN];
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
-        // masks: causal (key <= row) and keys past the segment's kept rows
-        const int kbase = j * kBN;
-        const int lim = tw.causal ? krow - kbase : tw.m[t.p] - 1 - kbase;
-        if (lim < kBN - 1) {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (c > lim) s[c] = -INFINITY;
-        }
-        // row max as a tree (independent partial maxima)
-        float pm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pm[e] = s[e];
-#pragma unroll
-        for (int c = 8; c < kBN; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        const float m_blk = mx * scale_log2;
-        float corr = 1.f;
-        bool rescale = false;
-        if (m_blk > m_use + 8.f || m_use == -INFINITY) {
-          if (m_blk != -INFINITY) {
-            if (m_use != -INFINITY) {
-              corr = ex2(m_use - m_blk);
-              rescale = true;
-            }
-            m_use = m_blk;
-          }
-        }
-        float ps[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-        const uint32_t p_col = s_col;  // P overwrites the first 64 columns of S
-#pragma unroll
-        for (int c = 0; c < kBN / 64; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float a = ex2(fmaf(s[c * 64 + 2 * e], scale_log2, -m_use));
-            const float bq = ex2(fmaf(s[c * 64 + 2 * e + 1], scale_log2, -m_use));
-            ps[e & 7] += a + bq;
-            pk[e] = pack_bf16(a, bq);
-          }
-          LN_TMEM_ST32(p_col + c * 32, pk);
-        }
-        const float lsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        tmem_wait_st();
-        l_run = l_run * corr + lsum;
-        if (j > 0) {
-          // PV of the previous block must be done before O is touched
-          ok = sy.wait_warp(bar_o_done, (s_it - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            const uint32_t o_col = tmem + lane_base + kColO;
-            uint32_t rr[kD];
-            LN_TMEM_LD32(o_col, (rr + 0));
-            LN_TMEM_LD32(o_col + 32, (rr + 32));
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < kD; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
-            LN_TMEM_ST32(o_col, (rr + 0));
-            LN_TMEM_ST32(o_col + 32, (rr + 32));
-            tmem_wait_st();
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar_p_full + sb);
-        ++s_it;
-      }
+    for (int i = 0; ok; ++i) {
+      ok = wait_count(cnt_elem + g, i);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      // ---- epilogue of this tile
-      ok = sy.wait_warp(bar_o_done, (s_it - 1) & 1);
+      const ElemMeta em = sElemQ[g * kQE + i % kQE];
+      __syncwarp();
+      if ((warp & 3) == 0 && lane == 0) {
+        // Released by the first warp: the producer runs at most NS ring stages
+        // ahead of the MMA warp, which cannot pass this stream's next block
+        // before all four warps have arrived for this one, so slot i % kQE is
+        // not rewritten while another warp of this warpgroup may still read it.
+        st_release(cnt_soft + g, i + 1);
+      }
+      if (em.info & kInfoEnd) break;
+      const int ob = (em.info >> 1) & 1;
+      if (em.j == 0) {
+        m_use = -INFINITY;
+        l_run = 0.f;
+      }
+      const int sb = s_cnt & 1;
+      ok = sy.wait_warp(bar_s_full + 2 * g + sb, (s_cnt >> 1) & 1);
+      if (!ok) break;
+      ++s_cnt;
+      tc_fence_after();
+      const uint32_t s_col = tmem + lane_base + col_s(g, sb);
+      const int lim = causal ? em.lim0 + row - em.j * kBN : em.lim0 - em.j * kBN;
+      uint32_t sr[kBN];
+      LN_TMEM_LD32(s_col + 0, (sr + 0));
+      LN_TMEM_LD32(s_col + 32, (sr + 32));
+      tmem_wait_ld();
+      if (lim < kBN - 1) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float pm[8];
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
+#pragma unroll
+      for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float m_blk = mx * scale_log2;
+      float corr = 1.f;
+      bool rescale = false;
+      if (m_blk > m_use + 8.f || m_use == -INFINITY) {
+        if (m_blk != -INFINITY) {
+          if (m_use != -INFINITY) {
+            corr = ex2(m_use - m_blk);
+            rescale = true;
+          }
+          m_use = m_blk;
+        }
+      }
+      // P = 2^(s*scale - m) as bf16 over the first 32 columns of this S buffer
+      float ps[8];
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float a = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, -m_use));
+          const float bq = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, -m_use));
+          ps[c & 7] += a + bq;
+          pk[c] = pack_bf16(a, bq);
+        }
+        LN_TMEM_ST32(s_col, pk);
+      }
+      tmem_wait_st();
+      l_run = l_run * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+      if (em.j > 0) {
+        // PV of the previous block must be done before O is touched
+        ok = sy.wait_warp(bar_o_done + g, od_cnt & 1);
+        if (!ok) break;
+        ++od_cnt;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+          const uint32_t o_col = tmem + lane_base + col_o(g, ob);
+          uint32_t rr[kD];
+          LN_TMEM_LD32(o_col, (rr + 0));
+          LN_TMEM_LD32(o_col + 32, (rr + 32));
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < kD; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
+          LN_TMEM_ST32(o_col, (rr + 0));
+          LN_TMEM_ST32(o_col + 32, (rr + 32));
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_p_full + 2 * g + sb);
+      if (em.j == em.nkv - 1) {
+        // row statistics for the epilogue, then hand the tile over; indexed by
+        // use parity too: a one-block tile writes its statistics before
+        // anything orders it after the epilogue's read of the previous user
+        // of this O buffer, but always after the one before that
+        sStats[((2 * g + ob) * 2 + ((em.info >> 2) & 1)) * kBM + row] = make_float2(m_use, l_run);
+        mbar_arrive(bar_o_full + 2 * g + ob);
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 112;" ::: "memory");
+    // ------------------------------------------------------------ epilogue (processing order)
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      ok = wait_seq(&sTileQ[i % kQT].seq, i);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const TileMeta tm = sTileQ[i % kQT];
+      if (tm.info & kInfoEnd) break;
+      const int g = tm.info & 1, ob = (tm.info >> 1) & 1, up = (tm.info >> 2) & 1;
+      ok = sy.wait_warp(bar_o_full + 2 * g + ob, up);
       if (!ok) break;
       tc_fence_after();
       float o[kD];
       {
-        const uint32_t o_col = tmem + lane_base + kColO;
+        const uint32_t o_col = tmem + lane_base + col_o(g, ob);
         uint32_t rr[kD];
         LN_TMEM_LD32(o_col, (rr + 0));
         LN_TMEM_LD32(o_col + 32, (rr + 32));
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < kD; ++e) o[e] = __uint_as_float(rr[e]);
+        for (int c = 0; c < kD; ++c) o[c] = __uint_as_float(rr[c]);
       }
+      const float2 st = sStats[((2 * g + ob) * 2 + up) * kBM + row];
       tc_fence_before();
-      mbar_arrive(bar_o_free);
-      if (row < t.nrows) {
-        const float inv = 1.f / l_run;
+      mbar_arrive(bar_o_free + 2 * g + ob);
+      if (row < tm.nrows) {
+        const int4 pt = sPat[tm.p];  // (w, r, o, m) of this tile's pattern
+        const float inv = 1.f / st.y;
 #pragma unroll
         for (int d = 0; d < kD; ++d) o[d] *= inv;
-        float lse2 = m_use + __log2f(l_run);  // log2 domain
-        const int x = t.start + tw.r[t.p] * row;
+        float lse2 = st.x + __log2f(st.y);  // log2 domain
+        const int x = tm.start + pt.y * row;
         // last tile covering x?  (all other covering tiles come earlier)
         bool final_row = true;
-        for (int q = 0; q < tw.n_pat && final_row; ++q) {
-          if (q == t.p) continue;
+        for (int q = 0; q < n_pat && final_row; ++q) {
+          if (q == tm.p) continue;
+          const int4 pq = sPat[q];
           Cover cv;
-          if (!cover_of(tw, q, x, cv)) continue;
-          if (!key_before(cv.start, tw.r[q], q, t.start, tw.r[t.p], t.p)) final_row = false;
+          if (!cover_pat(pq.x, pq.y, pq.z, pq.w, A, x, cv)) continue;
+          if (!key_before(cv.start, pq.y, q, tm.start, pt.y, tm.p)) final_row = false;
         }
         if (final_row) {
-          for (int q = 0; q < tw.n_pat; ++q) {
-            if (q == t.p) continue;
+          for (int q = 0; q < n_pat; ++q) {
+            if (q == tm.p) continue;
+            const int4 pq = sPat[q];
             Cover cv;
-            if (!cover_of(tw, q, x, cv)) continue;
+            if (!cover_pat(pq.x, pq.y, pq.z, pq.w, A, x, cv)) continue;
             const float lq = sSlotL[q * kBM + cv.slot_row];
             const float mxl = fmaxf(lse2, lq);
             const float wa = ex2(lse2 - mxl), wb = ex2(lq - mxl);
@@ -719,9 +1222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint4 u = src[ch ^ (cv.slot_row & 7)];
               const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&wv[e]);
-                const int d = ch * 8 + e * 2;
+              for (int q2 = 0; q2 < 4; ++q2) {
+                __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&wv[q2]);
+                const int d = ch * 8 + q2 * 2;
                 o[d] = (wa * o[d] + wb * __bfloat162float(pr.x)) * inv2;
                 o[d + 1] = (wa * o[d + 1] + wb * __bfloat162float(pr.y)) * inv2;
               }
@@ -740,7 +1243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (P.pb.lse) P.pb.lse[(b * P.pb.H + h) * P.pb.N + x] = lse2 * 0.69314718055994531f;
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(sSlotO + t.p * kTileBytes + row * 128);
+          uint4* dst = reinterpret_cast<uint4*>(sSlotO + tm.p * kTileBytes + row * 128);
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             uint4 u;
@@ -750,22 +1253,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             u.w = pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]);
             dst[ch ^ (row & 7)] = u;
           }
-          sSlotL[t.p * kBM + row] = lse2;
+          sSlotL[tm.p * kBM + row] = lse2;
         }
       }
-      // parked rows become visible to the next epilogue's threads (a bounded
-      // barrier of the 128 softmax threads)
+      // parked rows become visible to the next tile's epilogue threads, and
+      // the tile queue entry is released once all 128 threads have read it
       mbar_arrive(bar_epi);
-      ok = sy.wait_warp(bar_epi, tile_it & 1);
-      ++tile_it;
+      ok = sy.wait_warp(bar_epi, i & 1);
+      if (warp == 12 && lane == 0) st_release(cnt_epi, i + 1);
     }
     if (ok && P.uncovered_possible) {
       // positions of this range that no pattern keeps: out = 0, lse = -inf
       for (int x = A + row; x < Bnd; x += 128) {
         bool any = false;
-        for (int q = 0; q < tw.n_pat && !any; ++q) {
+        for (int q = 0; q < n_pat && !any; ++q) {
+          const int4 pq = sPat[q];
           Cover cv;
-          any = cover_of(tw, q, x, cv);
+          any = cover_pat(pq.x, pq.y, pq.z, pq.w, A, x, cv);
         }
         if (!any) {
           uint4* dst = reinterpret_cast<uint4*>(outp + ((b * P.pb.N + x) * P.pb.H + h) * kD);
@@ -811,14 +1315,14 @@ EncodeTiledFn get_encoder() {
 // View [B, N, H, D] bf16 (starting `shift` positions in) as (d, h, c, k, b)
 // with position = shift + r*k + c, k < kcount.
 bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem& p, int64_t r,
-                int64_t shift, int64_t kcount) {
+                int64_t shift, int64_t kcount, int box_rows) {
   const int64_t es = 2;
   const char* ptr = static_cast<const char*>(base) + shift * p.H * kD * es;
   cuuint64_t dims[5] = {(cuuint64_t)kD, (cuuint64_t)p.H, (cuuint64_t)r, (cuuint64_t)kcount,
                         (cuuint64_t)p.B};
   cuuint64_t strides[4] = {(cuuint64_t)(kD * es), (cuuint64_t)(p.H * kD * es),
                            (cuuint64_t)(r * p.H * kD * es), (cuuint64_t)(p.N * p.H * kD * es)};
-  cuuint32_t box[5] = {(cuuint32_t)kD, 1, 1, (cuuint32_t)kBM, 1};
+  cuuint32_t box[5] = {(cuuint32_t)kD, 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult rc = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<char*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -860,7 +1364,8 @@ int64_t range_cost(const Problem& pb, int64_t A, int64_t Bnd) {
 bool tcgen05_supports(const Problem& p) {
   using namespace tc;
   if (p.dtype != LONGNET_DTYPE_BF16 || p.D != kD) return false;
-  if (p.n_pat > kMaxPat) return false;
+  static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
+  if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 2) return false;
   if (p.H > 65535 || p.B > 65535) return false;
   int n_r = 0;
   int64_t rv[kMaxR];
@@ -904,6 +1409,12 @@ void fill_params(const Problem& pb, tc::Params& P) {
   bool has_r1 = false;
   for (int i = 0; i < pb.n_pat; ++i) has_r1 |= (pb.r[i] == 1);
   P.uncovered_possible = has_r1 ? 0 : 1;
+  P.stages = pick_stages(pb.n_pat);
+  {
+    SmemLayout L;
+    L.make(pb.n_pat, P.stages);
+    P.smem_bytes = L.total + 1024;
+  }
   P.range_len = kBM * r_max_of(pb);
   P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
   if (P.n_ranges <= kMaxRangeOrder) {
@@ -931,23 +1442,25 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
   const void* bases[3] = {pb.q, pb.k, pb.v};
   for (int i = 0; i < P.n_r; ++i) {
     for (int t = 0; t < 3; ++t) {
-      if (!encode_map(enc, &maps.m[i][0][t], bases[t], pb, P.r_val[i], 0, P.kfull[i]))
+      const int rows = t == 0 ? kBM : kBN;  // Q tiles 128 rows, K/V blocks 64 rows
+      if (!encode_map(enc, &maps.m[i][0][t], bases[t], pb, P.r_val[i], 0, P.kfull[i], rows))
         return LONGNET_ERR_CUDA;
-      if (!encode_map(enc, &maps.m[i][1][t], bases[t], pb, P.r_val[i], P.tail[i], P.kfull[i]))
+      if (!encode_map(enc, &maps.m[i][1][t], bases[t], pb, P.r_val[i], P.tail[i], P.kfull[i], rows))
         return LONGNET_ERR_CUDA;
     }
   }
-  static bool attr_set[64] = {false};
+  const int smem_bytes = P.smem_bytes;
+  static int attr_set[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LONGNET_ERR_CUDA;
-  if (!attr_set[dev]) {
+  if (attr_set[dev] < smem_bytes) {
     if (cudaFuncSetAttribute(dilated_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
+                             kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev] = kSmemLimit;
   }
   const int64_t grid = (int64_t)P.n_ranges * pb.B * pb.H;
-  dilated_fwd_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(P, maps);
+  dilated_fwd_kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 
