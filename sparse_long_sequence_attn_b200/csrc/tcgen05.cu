@@ -1131,12 +1131,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       l_run = l_run * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
       if (em.j > 0) {
-        // PV of the previous block must be done before O is touched
-        ok = sy.wait_warp(bar_o_done + g, od_cnt & 1);
-        if (!ok) break;
-        ++od_cnt;
-        tc_fence_after();
+        // O may be rescaled only once the previous block's PV has completed.
+        // Every PV before that one has: this block's S, committed after them
+        // by the same thread, is complete.  So at most the o_done phase of
+        // the previous PV is pending, and its parity can be waited on
+        // without having waited on the phases before it; a warp with no row
+        // to rescale skips the wait (the lazy threshold makes that the rule).
+        const uint32_t ph = od_cnt++;
         if (__any_sync(0xffffffffu, rescale)) {
+          ok = sy.wait_warp(bar_o_done + g, ph & 1);
+          if (!ok) break;
+          tc_fence_after();
           const uint32_t o_col = tmem + lane_base + col_o(g, ob);
           uint32_t rr[kD];
           LN_TMEM_LD32(o_col, (rr + 0));
