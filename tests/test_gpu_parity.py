@@ -44,6 +44,9 @@ SMALL_CASES = [
     ("bf16_d64_w_eq_N", 1, 640, 2, 64, torch.bfloat16, True, ((640, 1),)),
     ("bf16_d64_r_gt_w", 1, 512, 4, 64, torch.bfloat16, True, ((512, 1), (2, 3))),
     ("bf16_d32", 1, 512, 2, 32, torch.bfloat16, True, ((128, 1), (512, 2))),
+    ("bf16_d64_seg32_causal", 2, 512, 3, 64, torch.bfloat16, True, ((32, 4), (32, 2), (32, 1))),
+    ("bf16_d64_seg64_r3_noncausal", 1, 1024, 4, 64, torch.bfloat16, False, ((64, 3), (64, 1))),
+    ("bf16_d64_seg64_r2_causal", 1, 1024, 4, 64, torch.bfloat16, True, ((64, 1), (64, 2))),
 ]
 
 
