@@ -4,16 +4,18 @@
 // (the DilatedAttention usage example of the "LongNet" docs page: segment 64,
 // dilation 2), so this kernel is built for HBM bandwidth, not tensor peak.
 //
-// Each warp owns one (batch, segment, head) item at a time, in a persistent
-// grid (one CTA per SM, several warps):
+// Each pair of warps owns one (batch, segment, head) item at a time, in a
+// persistent grid (one CTA per SM, several pairs); the two warps split every
+// pattern's 16-row chunks:
 //   * three TMA tile loads (Q, K, V: W rows x 128 B, 128-byte swizzle) bring
-//     the segment's rows of that head into the warp's shared memory;
+//     the segment's rows of that head into the pair's shared memory;
 //   * every pattern's sparsified segment (head offset o = h mod r, rows
 //     o + r*k < W) is read straight from shared memory by ldmatrix (the
 //     dilated gather is just a choice of row addresses) and attended with
 //     mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an fp32 softmax;
-//   * patterns other than the r = 1 one park their normalised rows and lse
-//     in the warp's shared memory; the r = 1 pattern, processed last, merges
+//   * patterns other than the r = 1 one park their normalised rows (16-byte
+//     chunks rotated by row, like the TMA swizzle, so a fragment's 8 rows hit
+//     distinct banks) and lse in the pair's shared memory; the r = 1 pattern, processed last, merges
 //     them row by row with weights e^{lse_p} ("LONGNET: Scaling Transformer
 //     to 1 billion tokens", section "Token expansion reaches 1 billion+",
 //     read as the softmax-denominator-weighted combination) and the rows go
@@ -45,9 +47,10 @@ struct Params {
   Problem pb;
   int W;                    // common segment length
   int order[kMaxPat];       // patterns in processing order (the r = 1 one last)
-  int park_off[kMaxPat];    // byte offset of each parked pattern's rows in a warp's region
-  int warp_bytes;           // shared memory per warp (1024-aligned)
-  int n_warps;
+  int park_off[kMaxPat];    // byte offset of each parked pattern's rows in a pair's region
+  int park_rows[kMaxPat];   // rows reserved for it (ceil(W / r))
+  int pair_bytes;           // shared memory per warp pair (1024-aligned)
+  int n_pairs;
   int64_t n_items;          // B * (N / W) * H
   uint64_t wait_limit_ns;
 };
@@ -103,24 +106,35 @@ __device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int ch) {
 
 // ------------------------------------------------------------ kernel
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
     smallseg_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp >= P.n_warps) return;
-  uint8_t* region = smem + (size_t)warp * P.warp_bytes;
+  const int pair = warp >> 1, wsub = warp & 1;
+  uint8_t* region = smem + (size_t)pair * P.pair_bytes;
   uint8_t* sQ = region;
   uint8_t* sK = region + kTile;
   uint8_t* sV = region + 2 * kTile;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(region + P.warp_bytes - 16);
-  if (lane == 0) {
+  uint64_t* bar = reinterpret_cast<uint64_t*>(region + P.pair_bytes - 32);  // TMA landed
+  uint64_t* pbar = bar + 1;                                                 // the pair's hand-off
+  if (wsub == 0 && lane == 0) {
     mbar_init(bar, 1);
+    mbar_init(pbar, 64);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int t = 0; t < 3; ++t)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[t])) : "memory");
   }
-  __syncwarp();
+  __syncthreads();
+  uint32_t pphase = 0;
+  // Bounded barrier of the warp pair (both warps arrive, both wait).
+  auto pair_sync = [&]() -> bool {
+    mbar_arrive_cta(pbar);
+    const bool ok = mbar_wait(pbar, pphase, P.wait_limit_ns);
+    pphase ^= 1;
+    if (!ok) record_status(P.pb.status, kStatusTimeout);
+    return ok;
+  };
 
   const int W = P.W;
   const int64_t H = P.pb.H, N = P.pb.N;
@@ -131,15 +145,16 @@ __global__ void __launch_bounds__(256, 1)
   __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
   uint32_t phase = 0;
 
-  for (int64_t item = (int64_t)blockIdx.x * P.n_warps + warp; item < P.n_items;
-       item += (int64_t)gridDim.x * P.n_warps, phase ^= 1) {
+  for (int64_t item = (int64_t)blockIdx.x * P.n_pairs + pair; item < P.n_items;
+       item += (int64_t)gridDim.x * P.n_pairs, phase ^= 1) {
     const int h = (int)(item % H);
     const int64_t bs = item / H;
     const int seg = (int)(bs % n_seg);
     const int b = (int)(bs / n_seg);
-    // ---- load the segment's rows of this head
+    // ---- load the segment's rows of this head (both warps are done with the
+    // previous item: the pair synchronised at its end)
     __syncwarp();
-    if (lane == 0) {
+    if (wsub == 0 && lane == 0) {
       // the previous item's rows were staged here with ordinary stores
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
@@ -154,17 +169,20 @@ __global__ void __launch_bounds__(256, 1)
       return;
     }
 
+    bool ok = true;
     for (int pi = 0; pi < P.pb.n_pat; ++pi) {
       const int p = P.order[pi];
       const bool last = pi == P.pb.n_pat - 1;
+      // the other warp's parked rows are complete before the merging pattern
+      if (last && pi > 0 && !(ok = pair_sync())) break;
       const int r = (int)P.pb.r[p];
       const int o = h % r;
       const int m = o >= W ? 0 : (W - o + r - 1) / r;  // kept rows of this head
       if (m == 0) continue;
       const int n_kt = (m + 15) >> 4;  // 16-key steps
       uint8_t* park = region + P.park_off[p];
-      float* park_l = reinterpret_cast<float*>(park + kMaxW * 128);
-      for (int rc = 0; rc < ((m + 15) >> 4); ++rc) {
+      float* park_l = reinterpret_cast<float*>(park + P.park_rows[p] * 128);
+      for (int rc = wsub; rc < ((m + 15) >> 4); rc += 2) {
         // ---- S = Q K^T for rows [16 rc, 16 rc + 16) of the sparsified segment
         float acc[8][4];
 #pragma unroll
@@ -275,7 +293,7 @@ __global__ void __launch_bounds__(256, 1)
             if (row < m) {
 #pragma unroll
               for (int nt = 0; nt < 8; ++nt)
-                *reinterpret_cast<uint32_t*>(park + row * 128 + nt * 16 + 4 * t4) =
+                *reinterpret_cast<uint32_t*>(park + row * 128 + ((nt ^ (row & 7)) << 4) + 4 * t4) =
                     pack2(ov[nt][2 * half], ov[nt][2 * half + 1]);
               if (t4 == 0) park_l[row] = half ? lse1 : lse0;
             }
@@ -293,14 +311,14 @@ __global__ void __launch_bounds__(256, 1)
                 if (rel < 0 || rel % rq) continue;
                 const int kq = rel / rq;
                 const uint8_t* pk = region + P.park_off[q];
-                const float lq = reinterpret_cast<const float*>(pk + kMaxW * 128)[kq];
+                const float lq = reinterpret_cast<const float*>(pk + P.park_rows[q] * 128)[kq];
                 const float mxl = fmaxf(lse, lq);
                 const float wa = ex2(lse - mxl), wb = ex2(lq - mxl);
                 const float iw = 1.f / (wa + wb);
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
                   const __nv_bfloat162 pv =
-                      *reinterpret_cast<const __nv_bfloat162*>(pk + kq * 128 + nt * 16 + 4 * t4);
+                      *reinterpret_cast<const __nv_bfloat162*>(pk + kq * 128 + ((nt ^ (kq & 7)) << 4) + 4 * t4);
                   ov[nt][2 * half] = (wa * ov[nt][2 * half] + wb * __bfloat162float(pv.x)) * iw;
                   ov[nt][2 * half + 1] = (wa * ov[nt][2 * half + 1] + wb * __bfloat162float(pv.y)) * iw;
                 }
@@ -320,14 +338,19 @@ __global__ void __launch_bounds__(256, 1)
         __syncwarp();
       }
     }
-    // ---- coalesced store of the staged rows: 16-byte chunks, 8 per row
+    if (!ok) return;
+    // ---- coalesced store of the rows this warp staged (its 16-row chunks):
+    // 16-byte chunks, 8 per row
     __syncwarp();
-    for (int idx = lane; idx < W * 8; idx += 32) {
-      const int row = idx >> 3, ch = idx & 7;
-      const uint4 u = *reinterpret_cast<const uint4*>(sQ + sw_addr(0, row, ch));
-      *reinterpret_cast<uint4*>(outp + (((int64_t)b * N + (int64_t)seg * W + row) * H + h) * kD + ch * 8) = u;
+    for (int rc = wsub; rc * 16 < W; rc += 2) {
+      for (int idx = lane; idx < 16 * 8; idx += 32) {
+        const int row = rc * 16 + (idx >> 3), ch = idx & 7;
+        if (row >= W) break;
+        const uint4 u = *reinterpret_cast<const uint4*>(sQ + sw_addr(0, row, ch));
+        *reinterpret_cast<uint4*>(outp + (((int64_t)b * N + (int64_t)seg * W + row) * H + h) * kD + ch * 8) = u;
+      }
     }
-    __syncwarp();
+    if (!pair_sync()) return;
   }
 }
 
@@ -352,8 +375,8 @@ EncodeTiledFn get_encoder() {
   return fn;
 }
 
-// Layout of one warp's shared memory for these patterns; 0 if unsupported.
-int warp_bytes(const Problem& p, int* park_off, int* order) {
+// Layout of one warp pair's shared memory for these patterns; 0 if unsupported.
+int pair_bytes(const Problem& p, int* park_off, int* park_rows, int* order) {
   int n1 = 0, k = 0;
   for (int i = 0; i < p.n_pat; ++i) {
     if (p.r[i] == 1) ++n1;
@@ -364,16 +387,18 @@ int warp_bytes(const Problem& p, int* park_off, int* order) {
     if (p.r[i] != 1) {
       order[k++] = i;
       park_off[i] = off;
-      off += kMaxW * 128 + kMaxW * 4;
+      park_rows[i] = (int)((p.w[0] + p.r[i] - 1) / p.r[i]);
+      off += park_rows[i] * 128 + park_rows[i] * 4;
     }
   }
   for (int i = 0; i < p.n_pat; ++i) {
     if (p.r[i] == 1) {
       order[k++] = i;
       park_off[i] = 0;
+      park_rows[i] = 0;
     }
   }
-  off += 16;                                 // mbarrier
+  off += 32;                                 // mbarriers
   return (off + 1023) & ~1023;
 }
 
@@ -388,9 +413,9 @@ bool smallseg_supports(const Problem& p) {
   for (int i = 0; i < p.n_pat; ++i)
     if (p.w[i] != W) return false;
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
-  int off[kMaxPat], order[kMaxPat];
-  const int wb = warp_bytes(p, off, order);
-  return wb > 0 && wb + 1024 <= kSmemLimit;
+  int off[kMaxPat], rows[kMaxPat], order[kMaxPat];
+  const int pb = pair_bytes(p, off, rows, order);
+  return pb > 0 && pb + 1024 <= kSmemLimit;
 }
 
 int launch_smallseg(const Problem& pb, cudaStream_t stream) {
@@ -405,11 +430,11 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   P.pb = pb;
   P.W = (int)pb.w[0];
   P.wait_limit_ns = kWaitLimitNs;
-  P.warp_bytes = warp_bytes(pb, P.park_off, P.order);
-  if (P.warp_bytes <= 0) return LONGNET_ERR_UNSUPPORTED;
-  P.n_warps = (kSmemLimit - 1024) / P.warp_bytes;
-  if (P.n_warps > 8) P.n_warps = 8;
-  if (P.n_warps < 1) return LONGNET_ERR_UNSUPPORTED;
+  P.pair_bytes = pair_bytes(pb, P.park_off, P.park_rows, P.order);
+  if (P.pair_bytes <= 0) return LONGNET_ERR_UNSUPPORTED;
+  P.n_pairs = (kSmemLimit - 1024) / P.pair_bytes;
+  if (P.n_pairs > 8) P.n_pairs = 8;
+  if (P.n_pairs < 1) return LONGNET_ERR_UNSUPPORTED;
   P.n_items = pb.B * (pb.N / P.W) * pb.H;
   const void* bases[3] = {pb.q, pb.k, pb.v};
   for (int t = 0; t < 3; ++t) {
@@ -435,10 +460,10 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
       return LONGNET_ERR_CUDA;
     attr_set[dev] = 1;
   }
-  const int smem = P.n_warps * P.warp_bytes + 1024;
-  int64_t grid = (P.n_items + P.n_warps - 1) / P.n_warps;
+  const int smem = P.n_pairs * P.pair_bytes + 1024;
+  int64_t grid = (P.n_items + P.n_pairs - 1) / P.n_pairs;
   if (grid > n_sm) grid = n_sm;
-  smallseg_kernel<<<(unsigned)grid, P.n_warps * 32, smem, stream>>>(P, maps);
+  smallseg_kernel<<<(unsigned)grid, P.n_pairs * 64, smem, stream>>>(P, maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 

@@ -1395,7 +1395,8 @@ bool tcgen05_supports(const Problem& p) {
 }
 
 // Host half of the launch: everything in Params but the tensor maps.
-void fill_params(const Problem& pb, tc::Params& P) {
+// n_sm: multiprocessors of the device (units are halved while fewer).
+void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
   using namespace tc;
   memset(&P, 0, sizeof(P));
   P.pb = pb;
@@ -1420,8 +1421,14 @@ void fill_params(const Problem& pb, tc::Params& P) {
     L.make(pb.n_pat, P.stages);
     P.smem_bytes = L.total + 1024;
   }
+  // A unit spans 128 * r_max positions, so the coarsest pattern's tiles are
+  // full; while that leaves SMs idle, halve it (its tiles are then partial).
   P.range_len = kBM * r_max_of(pb);
   P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
+  while ((int64_t)P.n_ranges * pb.B * pb.H < n_sm && P.range_len >= 2 * kBM && P.range_len % 2 == 0) {
+    P.range_len /= 2;
+    P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
+  }
   if (P.n_ranges <= kMaxRangeOrder) {
     std::vector<int64_t> cost(P.n_ranges);
     for (int i = 0; i < P.n_ranges; ++i)
@@ -1443,7 +1450,10 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
   static TmaMaps maps;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
-  fill_params(pb, P);
+  int dev_sm = 0, n_sm = 148;
+  if (cudaGetDevice(&dev_sm) == cudaSuccess)
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev_sm);
+  fill_params(pb, P, n_sm);
   const void* bases[3] = {pb.q, pb.k, pb.v};
   for (int i = 0; i < P.n_r; ++i) {
     for (int t = 0; t < 3; ++t) {

@@ -47,6 +47,10 @@ SMALL_CASES = [
     ("bf16_d64_seg32_causal", 2, 512, 3, 64, torch.bfloat16, True, ((32, 4), (32, 2), (32, 1))),
     ("bf16_d64_seg64_r3_noncausal", 1, 1024, 4, 64, torch.bfloat16, False, ((64, 3), (64, 1))),
     ("bf16_d64_seg64_r2_causal", 1, 1024, 4, 64, torch.bfloat16, True, ((64, 1), (64, 2))),
+    # segment lengths that are not a multiple of 16, four patterns, r > W
+    ("bf16_d64_seg40_4pat", 1, 800, 5, 64, torch.bfloat16, True, ((40, 1), (40, 3), (40, 7), (40, 48))),
+    ("bf16_d64_seg8_noncausal", 2, 256, 3, 64, torch.bfloat16, False, ((8, 1), (8, 2))),
+    ("bf16_d64_seg56_r5", 1, 560, 6, 64, torch.bfloat16, False, ((56, 5), (56, 1), (56, 2))),
 ]
 
 
