@@ -621,88 +621,6 @@ __device__ __forceinline__ uint64_t desc_from(uint32_t lo, uint32_t hi) {
 // High word: SBO 1024 B, sm_100 version, 128-byte swizzle.
 constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
 
-struct MmaCtx {
-  uint32_t tmem;
-  uint32_t kv_lo;  // (smem address of the K/V ring) >> 4
-  uint64_t* bar_p_full;
-  uint64_t* bar_o_free;
-  uint64_t* bar_o_full;
-  uint64_t* bar_o_done;
-  uint64_t* bar_kv_empty;
-  Sync* sy;
-  uint32_t f0, f1;  // FIFO of pending PVs per stream (two 16-bit entries)
-  int n0, n1;
-  uint32_t busy;    // bit per ring stage: a pending PV still holds it
-  uint32_t owner1;  // bit per ring stage: that PV is stream 1's
-};
-template <int G>
-__device__ __forceinline__ uint32_t& fifo_of(MmaCtx& c) {
-  if constexpr (G == 0) return c.f0;
-  else return c.f1;
-}
-template <int G>
-__device__ __forceinline__ int& nf_of(MmaCtx& c) {
-  if constexpr (G == 0) return c.n0;
-  else return c.n1;
-}
-template <int G>
-__device__ __forceinline__ void pv_issue_front(MmaCtx& c) {
-  uint32_t& f = fifo_of<G>(c);
-  const uint32_t e = f & 0xFFFFu;
-  const int st = (int)(e & kEStage), sb = (e & kESb) ? 1 : 0, ob = (e & kEOb) ? 1 : 0;
-  const bool first = (e & kEFirst) != 0;
-  tc_fence_after();
-  const uint32_t v_lo = c.kv_lo + (uint32_t)st * ((2 * kKVBytes) >> 4) + (kKVBytes >> 4) +
-                        ((uint32_t)(kBN * 128) >> 4 << 16);
-#pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_ts(c.tmem + col_o(G, ob), c.tmem + col_s(G, sb) + kk * 8, desc_from(v_lo + kk * 128, kDescHi),
-           kIdescPV, (first && kk == 0) ? 0u : 1u);
-  tc_commit(c.bar_kv_empty + st);
-  tc_commit((e & kELast) ? c.bar_o_full + 2 * G + ob : c.bar_o_done + G);
-  c.busy &= ~(1u << st);
-  f >>= 16;
-  --nf_of<G>(c);
-}
-// Has the front PV's P landed (and, for a tile's first block, its O buffer
-// been freed)?  Blocking or not.
-template <int G>
-__device__ __forceinline__ bool pv_front_ready(MmaCtx& c, bool block) {
-  uint32_t& f = fifo_of<G>(c);
-  const uint32_t e = f & 0xFFFFu;
-  if (!(e & kESeen)) {
-    uint64_t* bar = c.bar_p_full + 2 * G + ((e & kESb) ? 1 : 0);
-    const uint32_t par = (e & kEPar) ? 1u : 0u;
-    if (block ? !c.sy->wait(bar, par) : !mbar_test_wait(bar, par)) return false;
-    f |= kESeen;
-  }
-  if ((e & kEFirst) && (e & kEUgt0)) {
-    uint64_t* bar = c.bar_o_free + 2 * G + ((e & kEOb) ? 1 : 0);
-    const uint32_t par = (e & kEUpar) ? 0u : 1u;  // the previous use's phase
-    if (block ? !c.sy->wait(bar, par) : !mbar_test_wait(bar, par)) return false;
-  }
-  return true;
-}
-// Blocking issue of the front PV; before waiting for an O buffer, the other
-// stream's pending PVs go first (without nesting further).
-template <int G>
-__device__ __forceinline__ bool pv_force_front(MmaCtx& c, bool flush) {
-  const uint32_t e = fifo_of<G>(c) & 0xFFFFu;
-  if (flush && (e & kEFirst) && (e & kEUgt0)) {
-    while (nf_of<1 - G>(c) > 0) {
-      if (!pv_front_ready<1 - G>(c, true)) return false;
-      pv_issue_front<1 - G>(c);
-    }
-  }
-  if (!pv_front_ready<G>(c, true)) return false;
-  pv_issue_front<G>(c);
-  return true;
-}
-template <int G>
-__device__ __forceinline__ void pv_issue_ready(MmaCtx& c) {
-  while (nf_of<G>(c) > 0 && pv_front_ready<G>(c, false)) pv_issue_front<G>(c);
-}
-
 // ---------------------------------------------------------------- kernel
 
 __device__ __forceinline__ void st_release(int* p, int v) {
