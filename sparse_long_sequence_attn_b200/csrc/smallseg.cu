@@ -15,13 +15,16 @@
 //     mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an fp32 softmax;
 //   * patterns other than the r = 1 one park their normalised rows (16-byte
 //     chunks rotated by row, like the TMA swizzle, so a fragment's 8 rows hit
-//     distinct banks) and lse in the pair's shared memory; the r = 1 pattern, processed last, merges
-//     them row by row with weights e^{lse_p} ("LONGNET: Scaling Transformer
-//     to 1 billion tokens", section "Token expansion reaches 1 billion+",
-//     read as the softmax-denominator-weighted combination) and the rows go
-//     out as coalesced 128-byte stores.
-// Warps of an SM sit at different points of their load/compute/store cycle,
-// which keeps bytes in flight while others compute.
+//     distinct banks) and lse in the pair's shared memory;
+//   * the r = 1 pattern, processed last, merges them row by row with weights
+//     e^{lse_p} ("LONGNET: Scaling Transformer to 1 billion tokens", section
+//     "Token expansion reaches 1 billion+", read as the softmax-denominator-
+//     weighted combination) and the rows go out as coalesced 128-byte stores.
+// Pairs of an SM sit at different points of their load/compute/store cycle,
+// which keeps bytes in flight while others compute.  The work per item is
+// issue-bound (index arithmetic, softmax, mma.sync), so the per-item set-up
+// is hoisted and the unmasked case (non-causal, m a multiple of 16) has its
+// own instantiation; six pairs leave 168 registers per thread.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -40,6 +43,7 @@ namespace ss {
 constexpr int kD = 64;
 constexpr int kMaxW = 64;
 constexpr int kMaxPat = 4;
+constexpr int kMaxPairs = 6;  // 12 warps, 3 per SM sub-partition: up to 168 registers each
 constexpr int kTile = kMaxW * kD * 2;  // 8 KB
 constexpr int kSmemLimit = 232448;
 
@@ -49,6 +53,8 @@ struct Params {
   int order[kMaxPat];       // patterns in processing order (the r = 1 one last)
   int park_off[kMaxPat];    // byte offset of each parked pattern's rows in a pair's region
   int park_rows[kMaxPat];   // rows reserved for it (ceil(W / r))
+  int r32[kMaxPat];         // dilations (the host checks they fit)
+  uint32_t rcp16[kMaxPat];  // ceil(2^16 / r): (x * rcp16) >> 16 = x / r for 0 <= x < 64
   int pair_bytes;           // shared memory per warp pair (1024-aligned)
   int n_pairs;
   int64_t n_items;          // B * (N / W) * H
@@ -106,7 +112,134 @@ __device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int ch) {
 
 // ------------------------------------------------------------ kernel
 
-__global__ void __launch_bounds__(512, 1)
+// One 16-row chunk (rows [16 rc, 16 rc + 16) of a sparsified segment with m
+// kept rows at o, o + r, ...): S = Q K^T over its m keys, softmax, O = P V,
+// normalised.  In the mma fragment layout this lane holds rows g and g + 8 of
+// the chunk; their O goes to ov and their lse (log2 domain) to lse0, lse1.
+// kMasked: some of the n_kt * 16 key columns are not keys of every row
+// (causal, or m not a multiple of 16).
+template <bool kMasked>
+__device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, uint32_t v_base, int o,
+                                             int r, int m, int n_kt, int rc, bool causal,
+                                             float scale_log2, int lane, float (&ov)[8][4],
+                                             float& lse0, float& lse1) {
+  const int g = lane >> 2, t4 = lane & 3;
+  float acc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  {
+    // A fragments address row 16 rc + (lane & 15); B fragments key
+    // 16 np + (lane & 7) + 8 (lane >> 4); rows past m are clamped (their
+    // results are never used, their keys are masked or absent)
+    int qi = rc * 16 + (lane & 15);
+    if (qi >= m) qi = m - 1;
+    const int qrow = o + r * qi;
+    const uint32_t qa = q_base + (uint32_t)qrow * 128u;
+    const int qsw = qrow & 7;
+    uint32_t ka[4];
+    int ksw[4];
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      int kj = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+      if (kj >= m) kj = m - 1;
+      const int krow = o + r * kj;
+      ka[np] = k_base + (uint32_t)krow * 128u;
+      ksw[np] = krow & 7;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(qa + ((uint32_t)((2 * kk + (lane >> 4)) ^ qsw) << 4), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        if (np < n_kt) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(ka[np] + ((uint32_t)((2 * kk + ((lane >> 3) & 1)) ^ ksw[np]) << 4), b0, b1, b2, b3);
+          mma16816(acc[2 * np], a, b0, b1);
+          mma16816(acc[2 * np + 1], a, b2, b3);
+        }
+      }
+    }
+  }
+  // ---- softmax over the keys (rows g and g + 8 of this chunk)
+  const int row0 = rc * 16 + g, row1 = row0 + 8;
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    if (nt < 2 * n_kt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (kMasked) {
+          const int c = nt * 8 + 2 * t4 + e;
+          const bool k_ok = c < m;
+          if (!(k_ok && (!causal || c <= row0))) acc[nt][e] = -INFINITY;
+          if (!(k_ok && (!causal || c <= row1))) acc[nt][2 + e] = -INFINITY;
+        }
+        mx0 = fmaxf(mx0, acc[nt][e]);
+        mx1 = fmaxf(mx1, acc[nt][2 + e]);
+      }
+    }
+  }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float ms0 = mx0 * scale_log2, ms1 = mx1 * scale_log2;  // every row has a key: finite
+  float l0 = 0.f, l1 = 0.f;
+  uint32_t pa[4][4];  // P as A fragments, one per 16-key step
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    if (nt < 2 * n_kt) {
+      const float p0 = ex2(fmaf(acc[nt][0], scale_log2, -ms0)), p1 = ex2(fmaf(acc[nt][1], scale_log2, -ms0));
+      const float p2 = ex2(fmaf(acc[nt][2], scale_log2, -ms1)), p3 = ex2(fmaf(acc[nt][3], scale_log2, -ms1));
+      l0 += p0 + p1;
+      l1 += p2 + p3;
+      const int kk = nt >> 1, hi = nt & 1;
+      pa[kk][hi * 2 + 0] = pack2(p0, p1);
+      pa[kk][hi * 2 + 1] = pack2(p2, p3);
+    }
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  // ---- O = P V (16 rows x 64 dims)
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ov[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    if (kk < n_kt) {
+      int vj = kk * 16 + (lane & 15);
+      if (vj >= m) vj = m - 1;  // keys past m have P = 0
+      const int vrow = o + r * vj;
+      const uint32_t va = v_base + (uint32_t)vrow * 128u;
+      const int vsw = vrow & 7;
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {  // pairs of 8-dim tiles
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(va + ((uint32_t)((2 * dp + (lane >> 4)) ^ vsw) << 4), b0, b1, b2, b3);
+        mma16816(ov[2 * dp], pa[kk], b0, b1);
+        mma16816(ov[2 * dp + 1], pa[kk], b2, b3);
+      }
+    }
+  }
+  const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    ov[nt][0] *= inv0;
+    ov[nt][1] *= inv0;
+    ov[nt][2] *= inv1;
+    ov[nt][3] *= inv1;
+  }
+  lse0 = ms0 + __log2f(l0);
+  lse1 = ms1 + __log2f(l1);
+}
+
+__global__ void __launch_bounds__(kMaxPairs * 64, 1)
     smallseg_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -136,13 +269,14 @@ __global__ void __launch_bounds__(512, 1)
     return ok;
   };
 
-  const int W = P.W;
-  const int64_t H = P.pb.H, N = P.pb.N;
+  const int W = P.W, n_pat = P.pb.n_pat;
+  const int H = (int)P.pb.H;
+  const int64_t N = P.pb.N;
   const int n_seg = (int)(N / W);
+  const bool causal = P.pb.causal != 0;
   const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
   const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
   const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
-  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
   uint32_t phase = 0;
 
   for (int64_t item = (int64_t)blockIdx.x * P.n_pairs + pair; item < P.n_items;
@@ -164,161 +298,79 @@ __global__ void __launch_bounds__(512, 1)
       tma_load_4d(sK, &maps.m[1], bar, 0, h, seg * W, b);
       tma_load_4d(sV, &maps.m[2], bar, 0, h, seg * W, b);
     }
+    // per-item pattern table: head offset of every pattern, computed once
+    int oq[kMaxPat];
+#pragma unroll
+    for (int pi = 0; pi < kMaxPat; ++pi) oq[pi] = pi < n_pat ? h % P.r32[P.order[pi]] : 0;
+    const int64_t row0_pos = (int64_t)b * N + (int64_t)seg * W;  // position of the segment's row 0
     if (!mbar_wait(bar, phase, P.wait_limit_ns)) {
       record_status(P.pb.status, kStatusTimeout);
       return;
     }
 
     bool ok = true;
-    for (int pi = 0; pi < P.pb.n_pat; ++pi) {
+    for (int pi = 0; pi < n_pat; ++pi) {
       const int p = P.order[pi];
-      const bool last = pi == P.pb.n_pat - 1;
+      const bool last = pi == n_pat - 1;
       // the other warp's parked rows are complete before the merging pattern
       if (last && pi > 0 && !(ok = pair_sync())) break;
-      const int r = (int)P.pb.r[p];
-      const int o = h % r;
+      const int r = P.r32[p];
+      int o = 0;
+#pragma unroll
+      for (int q = 0; q < kMaxPat; ++q)
+        if (q == pi) o = oq[q];
       const int m = o >= W ? 0 : (W - o + r - 1) / r;  // kept rows of this head
       if (m == 0) continue;
       const int n_kt = (m + 15) >> 4;  // 16-key steps
+      const bool masked = causal || (m & 15) != 0;
       uint8_t* park = region + P.park_off[p];
       float* park_l = reinterpret_cast<float*>(park + P.park_rows[p] * 128);
-      for (int rc = wsub; rc < ((m + 15) >> 4); rc += 2) {
-        // ---- S = Q K^T for rows [16 rc, 16 rc + 16) of the sparsified segment
-        float acc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        {
-          // row (sparse index) this lane addresses for the A fragments
-          int qi = rc * 16 + (lane & 15);
-          if (qi >= m) qi = m - 1;
-          const int qrow = o + r * qi;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            uint32_t a[4];
-            ldsm_x4(sw_addr(q_base, qrow, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {  // pairs of 8-key tiles
-              if (np * 16 >= ((m + 15) & ~15)) break;
-              // matrices: keys [16np, 16np+8) d-chunk 2kk, same keys d-chunk 2kk+1,
-              // keys [16np+8, 16np+16) d-chunks 2kk, 2kk+1
-              int kj = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-              if (kj >= m) kj = m - 1;
-              const int krow = o + r * kj;
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4(sw_addr(k_base, krow, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
-              mma16816(acc[2 * np], a, b0, b1);
-              mma16816(acc[2 * np + 1], a, b2, b3);
-            }
-          }
-        }
-        // ---- softmax over the m keys (rows g and g + 8 of this chunk)
-        const int row0 = rc * 16 + g, row1 = row0 + 8;
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const int c0 = nt * 8 + 2 * t4;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = c0 + e;
-            const bool k_ok = c < m;
-            const bool ok0 = k_ok && (!P.pb.causal || c <= row0);
-            const bool ok1 = k_ok && (!P.pb.causal || c <= row1);
-            acc[nt][e] = ok0 ? acc[nt][e] * scale_log2 : -INFINITY;
-            acc[nt][2 + e] = ok1 ? acc[nt][2 + e] * scale_log2 : -INFINITY;
-            mx0 = fmaxf(mx0, acc[nt][e]);
-            mx1 = fmaxf(mx1, acc[nt][2 + e]);
-          }
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        if (mx0 == -INFINITY) mx0 = 0.f;  // padding rows past m
-        if (mx1 == -INFINITY) mx1 = 0.f;
-        float l0 = 0.f, l1 = 0.f;
-        uint32_t pa[4][4];  // P as A fragments, one per 16-key step
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const float p0 = ex2(acc[nt][0] - mx0), p1 = ex2(acc[nt][1] - mx0);
-          const float p2 = ex2(acc[nt][2] - mx1), p3 = ex2(acc[nt][3] - mx1);
-          l0 += p0 + p1;
-          l1 += p2 + p3;
-          const int kk = nt >> 1, hi = nt & 1;
-          pa[kk][hi * 2 + 0] = pack2(p0, p1);
-          pa[kk][hi * 2 + 1] = pack2(p2, p3);
-        }
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-        // ---- O = P V (16 rows x 64 dims)
+      for (int rc = wsub; rc < n_kt; rc += 2) {
         float ov[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) ov[nt][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          if (kk >= n_kt) break;
-          // the A fragment of step kk: (row g, keys 16kk+2t4..), (row g+8, ..),
-          // (row g, keys 16kk+8+2t4..), (row g+8, ..)
-          const uint32_t a[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
-          int vj = kk * 16 + (lane & 15);
-          if (vj >= m) vj = m - 1;  // masked keys have P = 0
-          const int vrow = o + r * vj;
-#pragma unroll
-          for (int dp = 0; dp < 4; ++dp) {  // pairs of 8-dim tiles
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(sw_addr(v_base, vrow, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
-            mma16816(ov[2 * dp], a, b0, b1);
-            mma16816(ov[2 * dp + 1], a, b2, b3);
-          }
-        }
-        // ---- normalise; park, or merge with the parked patterns and stage out
-        const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-        float lse0 = mx0 + __log2f(l0), lse1 = mx1 + __log2f(l1);  // log2 domain
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          ov[nt][0] *= inv0;
-          ov[nt][1] *= inv0;
-          ov[nt][2] *= inv1;
-          ov[nt][3] *= inv1;
-        }
+        float lse0, lse1;
+        if (masked)
+          attend_chunk<true>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
+        else
+          attend_chunk<false>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
+        const int row0 = rc * 16 + g, row1 = row0 + 8;
         if (!last) {
+          // ---- park the normalised rows (16-byte chunks rotated by row)
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const int row = half ? row1 : row0;
             if (row < m) {
+              uint8_t* pr = park + row * 128 + 4 * t4;
 #pragma unroll
               for (int nt = 0; nt < 8; ++nt)
-                *reinterpret_cast<uint32_t*>(park + row * 128 + ((nt ^ (row & 7)) << 4) + 4 * t4) =
+                *reinterpret_cast<uint32_t*>(pr + ((nt ^ (row & 7)) << 4)) =
                     pack2(ov[nt][2 * half], ov[nt][2 * half + 1]);
               if (t4 == 0) park_l[row] = half ? lse1 : lse0;
             }
           }
         } else {
+          // ---- merge with the parked patterns, stage over the row's own Q row
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const int row = half ? row1 : row0;  // sparse index = position in segment (r = 1)
             float lse = half ? lse1 : lse0;
             if (row < m) {
-              for (int qi = 0; qi < pi; ++qi) {
+#pragma unroll
+              for (int qi = 0; qi < kMaxPat - 1; ++qi) {
+                if (qi >= pi) break;
                 const int q = P.order[qi];
-                const int rq = (int)P.pb.r[q], oq = h % rq;
-                const int rel = row - oq;
-                if (rel < 0 || rel % rq) continue;
-                const int kq = rel / rq;
+                const int rq = P.r32[q];
+                const int rel = row - oq[qi];
+                const int kq = (int)(((uint32_t)rel * P.rcp16[q]) >> 16);  // rel / rq, exact for rel < 64
+                if (rel < 0 || kq * rq != rel) continue;
                 const uint8_t* pk = region + P.park_off[q];
                 const float lq = reinterpret_cast<const float*>(pk + P.park_rows[q] * 128)[kq];
                 const float mxl = fmaxf(lse, lq);
                 const float wa = ex2(lse - mxl), wb = ex2(lq - mxl);
                 const float iw = 1.f / (wa + wb);
+                const uint8_t* pq = pk + kq * 128 + 4 * t4;
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
-                  const __nv_bfloat162 pv =
-                      *reinterpret_cast<const __nv_bfloat162*>(pk + kq * 128 + ((nt ^ (kq & 7)) << 4) + 4 * t4);
+                  const __nv_bfloat162 pv = *reinterpret_cast<const __nv_bfloat162*>(pq + ((nt ^ (kq & 7)) << 4));
                   ov[nt][2 * half] = (wa * ov[nt][2 * half] + wb * __bfloat162float(pv.x)) * iw;
                   ov[nt][2 * half + 1] = (wa * ov[nt][2 * half + 1] + wb * __bfloat162float(pv.y)) * iw;
                 }
@@ -326,9 +378,10 @@ __global__ void __launch_bounds__(512, 1)
               }
               // stage the row over its own Q row (no longer read: later chunks
               // read other rows) in the same swizzled layout
+              uint8_t* sr = sQ + row * 128 + 4 * t4;
 #pragma unroll
               for (int nt = 0; nt < 8; ++nt)
-                *reinterpret_cast<uint32_t*>(sQ + sw_addr(0, row, nt) + 4 * t4) =
+                *reinterpret_cast<uint32_t*>(sr + ((nt ^ (row & 7)) << 4)) =
                     pack2(ov[nt][2 * half], ov[nt][2 * half + 1]);
               if (t4 == 0 && P.pb.lse)
                 P.pb.lse[((int64_t)b * H + h) * N + (int64_t)seg * W + row] = lse * 0.69314718055994531f;
@@ -342,12 +395,19 @@ __global__ void __launch_bounds__(512, 1)
     // ---- coalesced store of the rows this warp staged (its 16-row chunks):
     // 16-byte chunks, 8 per row
     __syncwarp();
-    for (int rc = wsub; rc * 16 < W; rc += 2) {
-      for (int idx = lane; idx < 16 * 8; idx += 32) {
-        const int row = rc * 16 + (idx >> 3), ch = idx & 7;
-        if (row >= W) break;
-        const uint4 u = *reinterpret_cast<const uint4*>(sQ + sw_addr(0, row, ch));
-        *reinterpret_cast<uint4*>(outp + (((int64_t)b * N + (int64_t)seg * W + row) * H + h) * kD + ch * 8) = u;
+    {
+      __nv_bfloat16* out_seg = static_cast<__nv_bfloat16*>(P.pb.out) + (row0_pos * H + h) * kD;
+      const int64_t row_stride = (int64_t)H * kD;
+      for (int rc = wsub; rc * 16 < W; rc += 2) {
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int idx = it * 32 + lane;
+          const int row = rc * 16 + (idx >> 3), ch = idx & 7;
+          if (row < W) {
+            const uint4 u = *reinterpret_cast<const uint4*>(sQ + sw_addr(0, row, ch));
+            *reinterpret_cast<uint4*>(out_seg + row * row_stride + ch * 8) = u;
+          }
+        }
       }
     }
     if (!pair_sync()) return;
@@ -413,6 +473,8 @@ bool smallseg_supports(const Problem& p) {
   for (int i = 0; i < p.n_pat; ++i)
     if (p.w[i] != W) return false;
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
+  for (int i = 0; i < p.n_pat; ++i)
+    if (p.r[i] < 1 || p.r[i] > (int64_t)INT32_MAX) return false;
   int off[kMaxPat], rows[kMaxPat], order[kMaxPat];
   const int pb = pair_bytes(p, off, rows, order);
   return pb > 0 && pb + 1024 <= kSmemLimit;
@@ -431,9 +493,13 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   P.W = (int)pb.w[0];
   P.wait_limit_ns = kWaitLimitNs;
   P.pair_bytes = pair_bytes(pb, P.park_off, P.park_rows, P.order);
+  for (int i = 0; i < pb.n_pat; ++i) {
+    P.r32[i] = (int)pb.r[i];
+    P.rcp16[i] = (uint32_t)((65536 + pb.r[i] - 1) / pb.r[i]);
+  }
   if (P.pair_bytes <= 0) return LONGNET_ERR_UNSUPPORTED;
   P.n_pairs = (kSmemLimit - 1024) / P.pair_bytes;
-  if (P.n_pairs > 8) P.n_pairs = 8;
+  if (P.n_pairs > kMaxPairs) P.n_pairs = kMaxPairs;
   if (P.n_pairs < 1) return LONGNET_ERR_UNSUPPORTED;
   P.n_items = pb.B * (pb.N / P.W) * pb.H;
   const void* bases[3] = {pb.q, pb.k, pb.v};

@@ -141,6 +141,27 @@ struct __align__(64) TmaMaps {
   CUtensorMap m[kMaxR][2][3];  // [distinct r][base / shifted][q, k, v]
 };
 
+// Exact division by a divisor d >= 1 fixed per launch, for dividends
+// 0 <= x < 2^31 (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with s = ceil(log2 d) and m = ceil(2^(31+s) / d),
+// x / d = (x * m) >> (31 + s).  m < 2^32 for every d, so one 32x32->64-bit
+// multiply and a shift replace the division.
+struct FastDiv {
+  uint32_t m;
+  int shift;
+};
+__host__ __device__ inline int fdiv(int x, FastDiv f) {
+  return (int)(((uint64_t)(uint32_t)x * f.m) >> f.shift);
+}
+inline FastDiv make_fastdiv(int64_t d) {
+  int sh = 0;
+  while (((int64_t)1 << sh) < d) ++sh;
+  FastDiv f;
+  f.m = (uint32_t)((((uint64_t)1 << (31 + sh)) + (uint64_t)d - 1) / (uint64_t)d);
+  f.shift = 31 + sh;
+  return f;
+}
+
 struct Params {
   Problem pb;
   int n_r;                    // distinct dilations
@@ -148,6 +169,8 @@ struct Params {
   int tail[kMaxR];            // N mod r
   int kfull[kMaxR];           // N div r
   int pat_r[kMaxPat];         // index into r_val of each pattern
+  FastDiv r_div[kMaxR];       // division by r_val
+  FastDiv w_div[kMaxPat];     // division by each pattern's w
   int range_len;              // R
   int n_ranges;
   int uncovered_possible;     // some position may be kept by no pattern
@@ -376,6 +399,24 @@ __host__ __device__ inline bool cover_pat(int w, int r, int o, int m, int A, int
   c.slot_row = (kq - lo) - t * kBM;
   return true;
 }
+// The same with the divisions by w and r done by multiply and shift.
+__host__ __device__ inline bool cover_pat_fd(int w, int r, int o, int m, int A, int x, FastDiv fw,
+                                             FastDiv fr, Cover& c) {
+  const int sq = fdiv(x, fw);
+  const int rel = x - sq * w - o;
+  if (rel < 0) return false;
+  const int kq = fdiv(rel, fr);
+  if (kq * r != rel) return false;
+  if (kq >= m) return false;
+  const int base = sq * w + o;
+  int lo = A - base;
+  lo = lo <= 0 ? 0 : fdiv(lo + r - 1, fr);
+  const int t = (kq - lo) >> 7;  // kq >= lo; / kBM
+  c.start = base + r * (lo + t * kBM);
+  c.slot_row = (kq - lo) - t * kBM;
+  return true;
+}
+static_assert(kBM == 128, "cover_pat_fd divides by kBM with a shift");
 __host__ __device__ inline bool cover_of(const TileWalker& tw, int q, int x, Cover& c) {
   return cover_pat(tw.w[q], tw.r[q], tw.o[q], tw.m[q], tw.A, x, c);
 }
@@ -428,16 +469,11 @@ __host__ __device__ inline TmaCoord tma_coord(const Params& P, int ri, int first
   const int r = P.r_val[ri];
   const int last_pos = first_pos + r * (need - 1);
   TmaCoord t;
-  if (last_pos >= r * P.kfull[ri]) {
-    const int x = first_pos - P.tail[ri];  // >= 0 by the host's shape check
-    t.map = 1;
-    t.c = (int)(x % r);
-    t.kk = (int)(x / r);
-  } else {
-    t.map = 0;
-    t.c = (int)(first_pos % r);
-    t.kk = (int)(first_pos / r);
-  }
+  const int x = last_pos >= r * P.kfull[ri] ? first_pos - P.tail[ri]  // >= 0 by the host's shape check
+                                            : first_pos;
+  t.map = last_pos >= r * P.kfull[ri] ? 1 : 0;
+  t.kk = fdiv(x, P.r_div[ri]);
+  t.c = x - t.kk * r;
   return t;
 }
 
@@ -1126,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q == tm.p) continue;
           const int4 pq = sPat[q];
           Cover cv;
-          if (!cover_pat(pq.x, pq.y, pq.z, pq.w, A, x, cv)) continue;
+          if (!cover_pat_fd(pq.x, pq.y, pq.z, pq.w, A, x, P.w_div[q], P.r_div[P.pat_r[q]], cv)) continue;
           if (!key_before(cv.start, pq.y, q, tm.start, pt.y, tm.p)) final_row = false;
         }
         if (final_row) {
@@ -1134,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q == tm.p) continue;
             const int4 pq = sPat[q];
             Cover cv;
-            if (!cover_pat(pq.x, pq.y, pq.z, pq.w, A, x, cv)) continue;
+            if (!cover_pat_fd(pq.x, pq.y, pq.z, pq.w, A, x, P.w_div[q], P.r_div[P.pat_r[q]], cv)) continue;
             const float lq = sSlotL[q * kBM + cv.slot_row];
             const float mxl = fmaxf(lse2, lq);
             const float wa = ex2(lse2 - mxl), wb = ex2(lq - mxl);
@@ -1290,6 +1326,9 @@ bool tcgen05_supports(const Problem& p) {
   static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
   if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 2) return false;
   if (p.H > 65535 || p.B > 65535) return false;
+  // positions and their sums stay below 2^31 (32-bit tile arithmetic, TMA
+  // coordinates, multiply-shift division)
+  if (p.N > ((int64_t)1 << 30)) return false;
   int n_r = 0;
   int64_t rv[kMaxR];
   for (int i = 0; i < p.n_pat; ++i) {
@@ -1326,9 +1365,11 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
       P.r_val[j] = pb.r[i];
       P.tail[j] = pb.N % pb.r[i];
       P.kfull[j] = pb.N / pb.r[i];
+      P.r_div[j] = make_fastdiv(pb.r[i]);
       ++P.n_r;
     }
     P.pat_r[i] = j;
+    P.w_div[i] = make_fastdiv(pb.w[i]);
   }
   bool has_r1 = false;
   for (int i = 0; i < pb.n_pat; ++i) has_r1 |= (pb.r[i] == 1);
