@@ -1151,44 +1151,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar_o_free + 2 * g + ob);
       if (row < tm.nrows) {
         const int4 pt = sPat[tm.p];  // (w, r, o, m) of this tile's pattern
-        const float inv = 1.f / st.y;
-#pragma unroll
-        for (int d = 0; d < kD; ++d) o[d] *= inv;
-        float lse2 = st.x + __log2f(st.y);  // log2 domain
         const int x = tm.start + pt.y * row;
-        // last tile covering x?  (all other covering tiles come earlier)
+        // The other patterns keeping x: their slot rows, and whether this is
+        // the last tile covering x (all other covering tiles come earlier).
+        int srow[kMaxPat];
+        uint32_t cov = 0;
         bool final_row = true;
-        for (int q = 0; q < n_pat && final_row; ++q) {
-          if (q == tm.p) continue;
-          const int4 pq = sPat[q];
-          Cover cv;
-          if (!cover_pat_fd(pq.x, pq.y, pq.z, pq.w, A, x, P.w_div[q], P.r_div[P.pat_r[q]], cv)) continue;
-          if (!key_before(cv.start, pq.y, q, tm.start, pt.y, tm.p)) final_row = false;
-        }
-        if (final_row) {
-          for (int q = 0; q < n_pat; ++q) {
-            if (q == tm.p) continue;
+#pragma unroll
+        for (int q = 0; q < kMaxPat; ++q) {
+          srow[q] = 0;
+          if (q < n_pat && q != tm.p) {
             const int4 pq = sPat[q];
             Cover cv;
-            if (!cover_pat_fd(pq.x, pq.y, pq.z, pq.w, A, x, P.w_div[q], P.r_div[P.pat_r[q]], cv)) continue;
-            const float lq = sSlotL[q * kBM + cv.slot_row];
-            const float mxl = fmaxf(lse2, lq);
-            const float wa = ex2(lse2 - mxl), wb = ex2(lq - mxl);
-            const float inv2 = 1.f / (wa + wb);
-            const uint4* src = reinterpret_cast<const uint4*>(sSlotO + q * kTileBytes + cv.slot_row * 128);
+            if (cover_pat_fd(pq.x, pq.y, pq.z, pq.w, A, x, P.w_div[q], P.r_div[P.pat_r[q]], cv)) {
+              if (!key_before(cv.start, pq.y, q, tm.start, pt.y, tm.p)) final_row = false;
+              cov |= 1u << q;
+              srow[q] = cv.slot_row;
+            }
+          }
+        }
+        const float l_inv = 1.f / st.y;
+        const float lse2 = st.x + __log2f(st.y);  // log2 domain
+        if (final_row) {
+          // out = sum_p 2^{lse_p} O_p / sum_p 2^{lse_p}: weights first, then one
+          // multiply-add per element and parked row
+          float mx = lse2;
+          float aq[kMaxPat];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 u = src[ch ^ (cv.slot_row & 7)];
-              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+          for (int q = 0; q < kMaxPat; ++q) {
+            aq[q] = -INFINITY;
+            if ((cov >> q) & 1u) {
+              aq[q] = sSlotL[q * kBM + srow[q]];
+              mx = fmaxf(mx, aq[q]);
+            }
+          }
+          const float a_self = ex2(lse2 - mx);
+          float wsum = a_self;
 #pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&wv[q2]);
-                const int d = ch * 8 + q2 * 2;
-                o[d] = (wa * o[d] + wb * __bfloat162float(pr.x)) * inv2;
-                o[d + 1] = (wa * o[d + 1] + wb * __bfloat162float(pr.y)) * inv2;
+          for (int q = 0; q < kMaxPat; ++q) {
+            aq[q] = ((cov >> q) & 1u) ? ex2(aq[q] - mx) : 0.f;
+            wsum += aq[q];
+          }
+          const float inv_w = 1.f / wsum;
+          const float c_self = a_self * inv_w * l_inv;
+#pragma unroll
+          for (int d = 0; d < kD; ++d) o[d] *= c_self;
+#pragma unroll
+          for (int q = 0; q < kMaxPat; ++q) {
+            if ((cov >> q) & 1u) {
+              const float cq = aq[q] * inv_w;
+              const uint4* src = reinterpret_cast<const uint4*>(sSlotO + q * kTileBytes + srow[q] * 128);
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {
+                const uint4 u = src[ch ^ (srow[q] & 7)];
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                  const int d = ch * 8 + q2 * 2;
+                  o[d] = fmaf(__uint_as_float(wv[q2] << 16), cq, o[d]);
+                  o[d + 1] = fmaf(__uint_as_float(wv[q2] & 0xffff0000u), cq, o[d + 1]);
+                }
               }
             }
-            lse2 = mxl + __log2f(wa + wb);
           }
           uint4* dst = reinterpret_cast<uint4*>(outp + ((b * P.pb.N + x) * P.pb.H + h) * kD);
 #pragma unroll
@@ -1200,16 +1224,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             u.w = pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]);
             dst[ch] = u;
           }
-          if (P.pb.lse) P.pb.lse[(b * P.pb.H + h) * P.pb.N + x] = lse2 * 0.69314718055994531f;
+          if (P.pb.lse) P.pb.lse[(b * P.pb.H + h) * P.pb.N + x] = (mx + __log2f(wsum)) * 0.69314718055994531f;
         } else {
           uint4* dst = reinterpret_cast<uint4*>(sSlotO + tm.p * kTileBytes + row * 128);
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             uint4 u;
-            u.x = pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]);
-            u.y = pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]);
-            u.z = pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]);
-            u.w = pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]);
+            u.x = pack_bf16(o[ch * 8 + 0] * l_inv, o[ch * 8 + 1] * l_inv);
+            u.y = pack_bf16(o[ch * 8 + 2] * l_inv, o[ch * 8 + 3] * l_inv);
+            u.z = pack_bf16(o[ch * 8 + 4] * l_inv, o[ch * 8 + 5] * l_inv);
+            u.w = pack_bf16(o[ch * 8 + 6] * l_inv, o[ch * 8 + 7] * l_inv);
             dst[ch ^ (row & 7)] = u;
           }
           sSlotL[tm.p * kBM + row] = lse2;
