@@ -680,13 +680,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sSlotO = smem + L.slot_o;
   float* sSlotL = reinterpret_cast<float*>(smem + L.slot_l);
   float2* sStats = reinterpret_cast<float2*>(smem + L.stats);
-  ElemMeta* sElemQ = reinterpret_cast<ElemMeta*>(smem + L.meta);     // [2][kQE]
+  ElemMeta* sElemQ = reinterpret_cast<ElemMeta*>(smem + L.meta);     // [2][kQE] tile descriptors per stream
   TileMeta* sTileQ = reinterpret_cast<TileMeta*>(sElemQ + 2 * kQE);   // [kQT]
   ElemMeta* sStageMeta = reinterpret_cast<ElemMeta*>(sTileQ + kQT);   // [2][kMaxStages]
   int4* sPat = reinterpret_cast<int4*>(sStageMeta + 2 * kMaxStages);  // [kMaxPat] (w, r, o, m)
   int* sCnt = reinterpret_cast<int*>(sPat + kMaxPat);
-  int* cnt_elem = sCnt + 0;       // [2] elements published per stream
-  int* cnt_soft = sCnt + 4;       // [2] elements consumed per stream
+  int* cnt_elem = sCnt + 0;       // [2] tile descriptors published per stream
+  int* cnt_soft = sCnt + 4;       // [2] tile descriptors consumed per stream
   int* cnt_epi = sCnt + 6;        // tiles consumed
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bar_q_full = bars + 0;        // [2]
@@ -857,10 +857,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         em.j = e.j;
         em.nkv = t.nkv;
         em.lim0 = causal ? t.k0 : pt.w - 1;
-        ok = wait_count(cnt_soft + g, ne - kQE);  // element queue has room
-        if (!ok) break;
-        sElemQ[g * kQE + (ne & (kQE - 1))] = em;
-        st_release(cnt_elem + g, ++ne);
+        if (e.j == 0) {
+          // the softmax warps take one descriptor per tile
+          ok = wait_count(cnt_soft + g, ne - kQE);  // queue has room
+          if (!ok) break;
+          sElemQ[g * kQE + (ne & (kQE - 1))] = em;
+          st_release(cnt_elem + g, ++ne);
+        }
         if (kv_it >= (uint32_t)NS) ok = sy.wait(kv_empty + st, st_par ^ 1);
         if (!ok) break;
         stage_meta[st] = em;
@@ -1013,7 +1016,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_cnt = 0, od_cnt = 0;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int i = 0; ok; ++i) {
+    for (int i = 0; ok; ++i) {  // this stream's tiles
       ok = wait_count(cnt_elem + g, i);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -1021,102 +1024,104 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if ((warp & 3) == 0 && lane == 0) {
         // Released by the first warp: the producer runs at most NS ring stages
-        // ahead of the MMA warp, which cannot pass this stream's next block
-        // before all four warps have arrived for this one, so slot i % kQE is
-        // not rewritten while another warp of this warpgroup may still read it.
+        // ahead of the MMA warp, which cannot start a block's S before all four
+        // warps have arrived for the block two before it; every tile has a
+        // block, so the producer is fewer than kQE tiles ahead of any warp of
+        // this warpgroup and slot i % kQE is not rewritten while one may still
+        // read it.
         st_release(cnt_soft + g, i + 1);
       }
       if (em.info & kInfoEnd) break;
       const int ob = (em.info >> 1) & 1;
-      if (em.j == 0) {
-        m_use = -INFINITY;
-        l_run = 0.f;
-      }
-      const int sb = s_cnt & 1;
-      ok = sy.wait_warp(bar_s_full + 2 * g + sb, (s_cnt >> 1) & 1);
-      if (!ok) break;
-      ++s_cnt;
-      tc_fence_after();
-      const uint32_t s_col = tmem + lane_base + col_s(g, sb);
-      const int lim = causal ? em.lim0 + row - em.j * kBN : em.lim0 - em.j * kBN;
-      uint32_t sr[kBN];
-      LN_TMEM_LD32(s_col + 0, (sr + 0));
-      LN_TMEM_LD32(s_col + 32, (sr + 32));
-      tmem_wait_ld();
-      if (lim < kBN - 1) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c > lim) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float pm[8];
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
-#pragma unroll
-      for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      const float m_blk = mx * scale_log2;
-      float corr = 1.f;
-      bool rescale = false;
-      if (m_blk > m_use + 8.f || m_use == -INFINITY) {
-        if (m_blk != -INFINITY) {
-          if (m_use != -INFINITY) {
-            corr = ex2(m_use - m_blk);
-            rescale = true;
+      m_use = -INFINITY;
+      l_run = 0.f;
+      for (int j = 0; j < em.nkv; ++j) {  // its 64-key blocks
+        const int sb = s_cnt & 1;
+        ok = sy.wait_warp(bar_s_full + 2 * g + sb, (s_cnt >> 1) & 1);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        const uint32_t s_col = tmem + lane_base + col_s(g, sb);
+        const int lim = causal ? em.lim0 + row - j * kBN : em.lim0 - j * kBN;
+        uint32_t sr[kBN];
+        LN_TMEM_LD32(s_col + 0, (sr + 0));
+        LN_TMEM_LD32(s_col + 32, (sr + 32));
+        tmem_wait_ld();
+        if (lim < kBN - 1) {
+  #pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float pm[8];
+  #pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
+  #pragma unroll
+        for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float m_blk = mx * scale_log2;
+        float corr = 1.f;
+        bool rescale = false;
+        if (m_blk > m_use + 8.f || m_use == -INFINITY) {
+          if (m_blk != -INFINITY) {
+            if (m_use != -INFINITY) {
+              corr = ex2(m_use - m_blk);
+              rescale = true;
+            }
+            m_use = m_blk;
           }
-          m_use = m_blk;
         }
-      }
-      // P = 2^(s*scale - m) as bf16 over the first 32 columns of this S buffer
-      float ps[8];
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float a = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, -m_use));
-          const float bq = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, -m_use));
-          ps[c & 7] += a + bq;
-          pk[c] = pack_bf16(a, bq);
+        // P = 2^(s*scale - m) as bf16 over the first 32 columns of this S buffer
+        float ps[8];
+  #pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+        {
+          uint32_t pk[32];
+  #pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float a = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, -m_use));
+            const float bq = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, -m_use));
+            ps[c & 7] += a + bq;
+            pk[c] = pack_bf16(a, bq);
+          }
+          LN_TMEM_ST32(s_col, pk);
         }
-        LN_TMEM_ST32(s_col, pk);
-      }
-      tmem_wait_st();
-      l_run = l_run * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
-      if (em.j > 0) {
-        // O may be rescaled only once the previous block's PV has completed.
-        // Every PV before that one has: this block's S, committed after them
-        // by the same thread, is complete.  So at most the o_done phase of
-        // the previous PV is pending, and its parity can be waited on
-        // without having waited on the phases before it; a warp with no row
-        // to rescale skips the wait (the lazy threshold makes that the rule).
-        const uint32_t ph = od_cnt++;
-        if (__any_sync(0xffffffffu, rescale)) {
-          ok = sy.wait_warp(bar_o_done + g, ph & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t o_col = tmem + lane_base + col_o(g, ob);
-          uint32_t rr[kD];
-          LN_TMEM_LD32(o_col, (rr + 0));
-          LN_TMEM_LD32(o_col + 32, (rr + 32));
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < kD; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
-          LN_TMEM_ST32(o_col, (rr + 0));
-          LN_TMEM_ST32(o_col + 32, (rr + 32));
-          tmem_wait_st();
+        tmem_wait_st();
+        l_run = l_run * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+        if (j > 0) {
+          // O may be rescaled only once the previous block's PV has completed.
+          // Every PV before that one has: this block's S, committed after them
+          // by the same thread, is complete.  So at most the o_done phase of
+          // the previous PV is pending, and its parity can be waited on
+          // without having waited on the phases before it; a warp with no row
+          // to rescale skips the wait (the lazy threshold makes that the rule).
+          const uint32_t ph = od_cnt++;
+          if (__any_sync(0xffffffffu, rescale)) {
+            ok = sy.wait_warp(bar_o_done + g, ph & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t o_col = tmem + lane_base + col_o(g, ob);
+            uint32_t rr[kD];
+            LN_TMEM_LD32(o_col, (rr + 0));
+            LN_TMEM_LD32(o_col + 32, (rr + 32));
+            tmem_wait_ld();
+  #pragma unroll
+            for (int c = 0; c < kD; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
+            LN_TMEM_ST32(o_col, (rr + 0));
+            LN_TMEM_ST32(o_col + 32, (rr + 32));
+            tmem_wait_st();
+          }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(bar_p_full + 2 * g + sb);
-      if (em.j == em.nkv - 1) {
-        // row statistics for the epilogue, then hand the tile over; indexed by
-        // use parity too: a one-block tile writes its statistics before
-        // anything orders it after the epilogue's read of the previous user
-        // of this O buffer, but always after the one before that
-        sStats[((2 * g + ob) * 2 + ((em.info >> 2) & 1)) * kBM + row] = make_float2(m_use, l_run);
-        mbar_arrive(bar_o_full + 2 * g + ob);
+        tc_fence_before();
+        mbar_arrive(bar_p_full + 2 * g + sb);
+        if (j == em.nkv - 1) {
+          // row statistics for the epilogue, then hand the tile over; indexed by
+          // use parity too: a one-block tile writes its statistics before
+          // anything orders it after the epilogue's read of the previous user
+          // of this O buffer, but always after the one before that
+          sStats[((2 * g + ob) * 2 + ((em.info >> 2) & 1)) * kBM + row] = make_float2(m_use, l_run);
+          mbar_arrive(bar_o_full + 2 * g + ob);
+        }
       }
     }
   } else {
