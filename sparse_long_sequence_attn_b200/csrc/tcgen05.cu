@@ -1048,14 +1048,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         LN_TMEM_LD32(s_col + 32, (sr + 32));
         tmem_wait_ld();
         if (lim < kBN - 1) {
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (c > lim) sr[c] = __float_as_uint(-INFINITY);
         }
         float pm[8];
-  #pragma unroll
+#pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
-  #pragma unroll
+#pragma unroll
         for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
         const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
@@ -1073,11 +1073,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P = 2^(s*scale - m) as bf16 over the first 32 columns of this S buffer
         float ps[8];
-  #pragma unroll
+#pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
         {
           uint32_t pk[32];
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float a = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, -m_use));
             const float bq = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, -m_use));
@@ -1105,7 +1105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             LN_TMEM_LD32(o_col, (rr + 0));
             LN_TMEM_LD32(o_col + 32, (rr + 32));
             tmem_wait_ld();
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < kD; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
             LN_TMEM_ST32(o_col, (rr + 0));
             LN_TMEM_ST32(o_col + 32, (rr + 32));
