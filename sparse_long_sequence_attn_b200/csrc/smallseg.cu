@@ -104,6 +104,26 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// Two fp32 values in one 64-bit register pair, for the packed f32x2 ops.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 // Byte address of the 16-byte chunk `ch` of row `row` in a 128-byte-swizzled
 // tile of 128-byte rows (the layout the TMA writes).
 __device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int ch) {
@@ -192,8 +212,10 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     if (nt < 2 * n_kt) {
-      const float p0 = ex2(fmaf(acc[nt][0], scale_log2, -ms0)), p1 = ex2(fmaf(acc[nt][1], scale_log2, -ms0));
-      const float p2 = ex2(fmaf(acc[nt][2], scale_log2, -ms1)), p3 = ex2(fmaf(acc[nt][3], scale_log2, -ms1));
+      float x0, x1, x2, x3;
+      f32x2_split(fma_f32x2(f32x2(acc[nt][0], acc[nt][1]), f32x2(scale_log2, scale_log2), f32x2(-ms0, -ms0)), x0, x1);
+      f32x2_split(fma_f32x2(f32x2(acc[nt][2], acc[nt][3]), f32x2(scale_log2, scale_log2), f32x2(-ms1, -ms1)), x2, x3);
+      const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
       l0 += p0 + p1;
       l1 += p2 + p3;
       const int kk = nt >> 1, hi = nt & 1;
@@ -230,10 +252,8 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
   const float inv0 = 1.f / l0, inv1 = 1.f / l1;
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
-    ov[nt][0] *= inv0;
-    ov[nt][1] *= inv0;
-    ov[nt][2] *= inv1;
-    ov[nt][3] *= inv1;
+    f32x2_split(mul_f32x2(f32x2(ov[nt][0], ov[nt][1]), f32x2(inv0, inv0)), ov[nt][0], ov[nt][1]);
+    f32x2_split(mul_f32x2(f32x2(ov[nt][2], ov[nt][3]), f32x2(inv1, inv1)), ov[nt][2], ov[nt][3]);
   }
   lse0 = ms0 + __log2f(l0);
   lse1 = ms1 + __log2f(l1);
@@ -367,12 +387,13 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
                 const float mxl = fmaxf(lse, lq);
                 const float wa = ex2(lse - mxl), wb = ex2(lq - mxl);
                 const float iw = 1.f / (wa + wb);
+                const float ca = wa * iw, cb = wb * iw;
                 const uint8_t* pq = pk + kq * 128 + 4 * t4;
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
-                  const __nv_bfloat162 pv = *reinterpret_cast<const __nv_bfloat162*>(pq + ((nt ^ (kq & 7)) << 4));
-                  ov[nt][2 * half] = (wa * ov[nt][2 * half] + wb * __bfloat162float(pv.x)) * iw;
-                  ov[nt][2 * half + 1] = (wa * ov[nt][2 * half + 1] + wb * __bfloat162float(pv.y)) * iw;
+                  const uint32_t pv = *reinterpret_cast<const uint32_t*>(pq + ((nt ^ (kq & 7)) << 4));
+                  ov[nt][2 * half] = fmaf(__uint_as_float(pv << 16), cb, ov[nt][2 * half] * ca);
+                  ov[nt][2 * half + 1] = fmaf(__uint_as_float(pv & 0xffff0000u), cb, ov[nt][2 * half + 1] * ca);
                 }
                 lse = mxl + __log2f(wa + wb);
               }
