@@ -391,10 +391,15 @@ def run_ours(args, wl):
     }
     if ws == 1 and not args.no_cpu_baseline:
         n = args.cpu_positions
-        if n <= 0:
+        calibrate = n <= 0
+        if calibrate:
             tps, dt, _, _ = oracle_cpu_sample(wl, 16, seed=1)
             n = int(max(16, min(wl.N, 10.0 * tps)))
         tps, dt, threads, desc = oracle_cpu_sample(wl, n, seed=2)
+        if calibrate and dt < 5.0 and n < wl.N:
+            # a small probe understates the threads' throughput: size again
+            n = int(min(wl.N, n * 10.0 / max(dt, 1e-3)))
+            tps, dt, threads, desc = oracle_cpu_sample(wl, n, seed=3)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc + f" ({dt:.1f} s)"}
     print(json.dumps(line), flush=True)
