@@ -273,6 +273,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+
+// Two fp32 values in one 64-bit register pair, for the packed f32x2 ops (one
+// instruction for two lanes' worth of multiply or multiply-add).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_bytes,
                                                     uint32_t sbo_bytes) {
@@ -1200,7 +1221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float inv_w = 1.f / wsum;
           const float c_self = a_self * inv_w * l_inv;
 #pragma unroll
-          for (int d = 0; d < kD; ++d) o[d] *= c_self;
+          for (int d = 0; d < kD; d += 2) f32x2_split(mul_f32x2(f32x2(o[d], o[d + 1]), f32x2(c_self, c_self)), o[d], o[d + 1]);
 #pragma unroll
           for (int q = 0; q < kMaxPat; ++q) {
             if ((cov >> q) & 1u) {
@@ -1213,8 +1234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
                   const int d = ch * 8 + q2 * 2;
-                  o[d] = fmaf(__uint_as_float(wv[q2] << 16), cq, o[d]);
-                  o[d + 1] = fmaf(__uint_as_float(wv[q2] & 0xffff0000u), cq, o[d + 1]);
+                  f32x2_split(fma_f32x2(f32x2(__uint_as_float(wv[q2] << 16), __uint_as_float(wv[q2] & 0xffff0000u)),
+                                        f32x2(cq, cq), f32x2(o[d], o[d + 1])), o[d], o[d + 1]);
                 }
               }
             }
@@ -1235,10 +1256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             uint4 u;
-            u.x = pack_bf16(o[ch * 8 + 0] * l_inv, o[ch * 8 + 1] * l_inv);
-            u.y = pack_bf16(o[ch * 8 + 2] * l_inv, o[ch * 8 + 3] * l_inv);
-            u.z = pack_bf16(o[ch * 8 + 4] * l_inv, o[ch * 8 + 5] * l_inv);
-            u.w = pack_bf16(o[ch * 8 + 6] * l_inv, o[ch * 8 + 7] * l_inv);
+            float t[8];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2)
+              f32x2_split(mul_f32x2(f32x2(o[ch * 8 + e], o[ch * 8 + e + 1]), f32x2(l_inv, l_inv)), t[e], t[e + 1]);
+            u.x = pack_bf16(t[0], t[1]);
+            u.y = pack_bf16(t[2], t[3]);
+            u.z = pack_bf16(t[4], t[5]);
+            u.w = pack_bf16(t[6], t[7]);
             dst[ch ^ (row & 7)] = u;
           }
           sSlotL[tm.p * kBM + row] = lse2;
