@@ -289,6 +289,11 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -1099,12 +1104,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           uint32_t pk[32];
 #pragma unroll
+          const uint64_t sc2 = f32x2(scale_log2, scale_log2), nm2 = f32x2(-m_use, -m_use);
+          uint64_t ls[4] = {0, 0, 0, 0};  // row sum of P in packed pairs
+#pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float a = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, -m_use));
-            const float bq = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, -m_use));
-            ps[c & 7] += a + bq;
+            float xa, xb;
+            f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sc2, nm2), xa, xb);
+            const float a = ex2(xa), bq = ex2(xb);
+            ls[c & 3] = add_f32x2(ls[c & 3], f32x2(a, bq));
             pk[c] = pack_bf16(a, bq);
           }
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) f32x2_split(ls[q4], ps[2 * q4], ps[2 * q4 + 1]);
           LN_TMEM_ST32(s_col, pk);
         }
         tmem_wait_st();
