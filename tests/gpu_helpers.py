@@ -43,10 +43,11 @@ def run_cuda(q, k, v, patterns, causal, impl, want_lse=True, stream=None):
     return o, l
 
 
-def compare_full(o, l, q, k, v, patterns, causal, dtype, label=""):
+def compare_full(o, l, q, k, v, patterns, causal, dtype, label="", tol_out=None):
     ro, rl = oracle.dilated_attn_fp64(q, k, v, patterns, causal)
     err = float(np.abs(o - ro).max())
-    assert err <= TOL_OUT[dtype], f"{label}: max|out - oracle| = {err}"
+    tol = TOL_OUT[dtype] if tol_out is None else tol_out
+    assert err <= tol, f"{label}: max|out - oracle| = {err} (tolerance {tol})"
     if l is not None:
         fin = np.isfinite(rl)
         assert np.array_equal(np.isfinite(l), fin), f"{label}: -inf pattern of lse differs"

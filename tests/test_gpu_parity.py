@@ -79,6 +79,34 @@ def test_specialised_families_vs_oracle(case, impl_name):
     gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
 
 
+@pytest.mark.parametrize("impl_name", ["auto", "tcgen05", "simt"])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("ramp", ["rising", "falling"])
+def test_scores_far_beyond_exp2_range(impl_name, causal, ramp):
+    """Keys scaled by a factor ramping between 1 and 40 along the sequence, so
+    that a row's scores differ by far more than exp2's range (over 100 in
+    log2 units).  Rising: later key blocks exceed the first block's maximum
+    and the softmax must move its exponent offset and rescale O; falling: the
+    first block dominates and later blocks underflow.  Compared with the fp64
+    oracle, which subtracts the exact maximum.
+
+    Attention this peaked makes |out| approach max|v| (about 4.5 here), so the
+    bf16 bound scales with it: the rounding of P to bf16 (2^-9 relative per
+    weight), of a parked pattern's partial row and of the output each add at
+    most 2^-9 max|v|; the test allows 3 * 2^-9 * max|v| (10 % margin), and
+    never less than the default 2e-2."""
+    B, N, H, D = 1, 2048, 4, 64
+    pats = ((512, 1), (1024, 2), (2048, 4))
+    q, k, v = wl.random_inputs(B, N, H, D, torch.float32, seed=4242 + causal)
+    f = torch.linspace(1.0, 40.0, N) if ramp == "rising" else torch.linspace(40.0, 1.0, N)
+    k = k * f.view(1, N, 1, 1)
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    o, l = gh.run_cuda(q, k, v, pats, causal, IMPLS[impl_name] if impl_name != "auto" else bd.LONGNET_IMPL_AUTO)
+    tol = max(gh.TOL_OUT[torch.bfloat16], 1.1 * 3 * 2.0 ** -9 * float(v.float().abs().max()))
+    gh.compare_full(o, l, q, k, v, pats, causal, torch.bfloat16, label=f"ramp_{ramp}_{causal}/{impl_name}",
+                    tol_out=tol)
+
+
 def test_named_tiny_workload_fp32():
     w = wl.WORKLOADS["tiny"]
     q, k, v = wl.make_inputs(w)
