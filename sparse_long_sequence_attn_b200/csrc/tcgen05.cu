@@ -48,6 +48,7 @@
 #include <algorithm>
 #include <mutex>
 #include <numeric>
+#include <queue>
 #include <type_traits>
 #include <vector>
 
@@ -172,13 +173,32 @@ struct Params {
   FastDiv r_div[kMaxR];       // division by r_val
   FastDiv w_div[kMaxPat];     // division by each pattern's w
   int range_len;              // R
-  int n_ranges;
+  int n_ranges;               // ceil(N / R)
+  int n_units;                // ranges, some of them split in halves
   int uncovered_possible;     // some position may be kept by no pattern
   int stages;                 // K/V ring depth
   int smem_bytes;             // dynamic shared memory requested
   uint64_t wait_limit_ns;
-  int range_order[kMaxRangeOrder];  // longest-first order of ranges (or -1: identity)
+  // Unit of each rank, longest first: (range << 2) | (half << 1) | split; or
+  // unit_code[0] = -1: rank r is whole range r.
+  int unit_code[kMaxRangeOrder];
 };
+
+// Positions [A, Bnd) of the unit a CTA of rank `rank` works on.
+__host__ __device__ inline void unit_bounds(const Params& P, int64_t rank, int& A, int& Bnd) {
+  const int R = P.range_len;
+  int i = (int)rank, len = R, off = 0;
+  if (P.unit_code[0] >= 0 && rank < kMaxRangeOrder) {
+    const int c = P.unit_code[rank];
+    i = c >> 2;
+    if (c & 1) {
+      len = R / 2;
+      off = ((c >> 1) & 1) * len;
+    }
+  }
+  A = i * R + off;
+  Bnd = (int64_t)A + len < P.pb.N ? A + len : (int)P.pb.N;
+}
 
 // ---------------------------------------------------------------- PTX bits
 
@@ -738,9 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t bh = blockIdx.x - rank * BH;
   const int64_t b = bh / P.pb.H;
   const int64_t h = bh - b * P.pb.H;
-  const int ri_range = (P.range_order[0] >= 0 && rank < kMaxRangeOrder) ? P.range_order[rank] : (int)rank;
-  const int A = ri_range * P.range_len;
-  const int Bnd = (int64_t)A + P.range_len < P.pb.N ? A + P.range_len : (int)P.pb.N;
+  int A, Bnd;
+  unit_bounds(P, rank, A, Bnd);
   const int n_pat = P.pb.n_pat;
   const bool causal = P.pb.causal != 0;
 
@@ -1412,7 +1431,7 @@ bool tcgen05_supports(const Problem& p) {
   }
   const int64_t R = kBM * r_max_of(p);
   const int64_t n_ranges = (p.N + R - 1) / R;
-  if (n_ranges * p.B * p.H > 0x7fffffffLL) return false;
+  if ((n_ranges + 8) * p.B * p.H > 0x7fffffffLL) return false;  // + ranges split in halves
   return true;
 }
 
@@ -1453,53 +1472,145 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     P.range_len /= 2;
     P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
   }
+  P.n_units = P.n_ranges;
+  P.unit_code[0] = -1;
   if (P.n_ranges <= kMaxRangeOrder) {
+    // Units launch longest first, so the block scheduler assigns them
+    // greedily (LPT).  The longest ranges may also be split in halves when a
+    // simulation of that greedy assignment over the SMs (with a per-unit
+    // overhead) says the last SM finishes earlier.
+    const int64_t R = P.range_len, N = pb.N, BH = pb.B * pb.H;
     std::vector<int64_t> cost(P.n_ranges);
-    for (int i = 0; i < P.n_ranges; ++i)
-      cost[i] = range_cost(pb, (int64_t)i * P.range_len, std::min<int64_t>(pb.N, (int64_t)(i + 1) * P.range_len));
+    for (int i = 0; i < P.n_ranges; ++i) cost[i] = range_cost(pb, i * R, std::min<int64_t>(N, (i + 1) * R));
     std::vector<int> idx(P.n_ranges);
     std::iota(idx.begin(), idx.end(), 0);
     std::stable_sort(idx.begin(), idx.end(), [&](int a, int c) { return cost[a] > cost[c]; });
-    for (int i = 0; i < P.n_ranges; ++i) P.range_order[i] = idx[i];
-  } else {
-    P.range_order[0] = -1;
+    struct Unit {
+      int64_t cost;
+      int code;
+    };
+    auto units_for = [&](int k) {
+      std::vector<Unit> u;
+      for (int t = 0; t < P.n_ranges; ++t) {
+        const int i = idx[t];
+        if (t < k) {
+          for (int hf = 0; hf < 2; ++hf) {
+            const int64_t a = i * R + hf * (R / 2);
+            if (a >= N) continue;
+            u.push_back({range_cost(pb, a, std::min<int64_t>(N, a + R / 2)), (i << 2) | (hf << 1) | 1});
+          }
+        } else {
+          u.push_back({cost[i], i << 2});
+        }
+      }
+      std::stable_sort(u.begin(), u.end(), [](const Unit& a, const Unit& c) { return a.cost > c.cost; });
+      return u;
+    };
+    auto makespan = [&](const std::vector<Unit>& u) {
+      constexpr int64_t kUnitOverhead = 16;  // fill and drain, in 64-key blocks
+      std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
+      for (int i = 0; i < n_sm; ++i) sm.push(0);
+      int64_t end = 0;
+      for (const Unit& x : u)
+        for (int64_t j = 0; j < BH; ++j) {
+          const int64_t t = sm.top() + x.cost + kUnitOverhead;
+          sm.pop();
+          sm.push(t);
+          end = std::max(end, t);
+        }
+      return end;
+    };
+    int best_k = 0;
+    const bool can_split = R % 2 == 0 && R / 2 >= kBM && (int64_t)P.n_ranges * BH <= 262144;
+    if (can_split) {
+      int64_t best = makespan(units_for(0));
+      for (int k = 1; k <= std::min(8, P.n_ranges); ++k) {
+        const std::vector<Unit> u = units_for(k);
+        if ((int64_t)u.size() > kMaxRangeOrder) break;
+        const int64_t m = makespan(u);
+        if (m * 100 < best * 99) {  // at least 1 % better
+          best = m;
+          best_k = k;
+        }
+      }
+    }
+    const std::vector<Unit> u = units_for(best_k);
+    P.n_units = (int)u.size();
+    for (int t = 0; t < P.n_units; ++t) P.unit_code[t] = u[t].code;
   }
 }
+
+namespace tc {
+// Host set-up of the last launch on a device: the unit plan and Params for a
+// shape, the tensor maps for a set of q, k, v pointers.  Repeated calls with
+// the same shape (and tensors) skip that work.
+struct LaunchCache {
+  bool valid = false;
+  Problem shape;
+  const void* q = nullptr;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  Params P;
+  TmaMaps maps;
+};
+inline bool same_shape(const Problem& a, const Problem& b) {
+  if (a.B != b.B || a.N != b.N || a.H != b.H || a.D != b.D || a.n_pat != b.n_pat ||
+      a.causal != b.causal || a.dtype != b.dtype)
+    return false;
+  for (int i = 0; i < a.n_pat; ++i)
+    if (a.w[i] != b.w[i] || a.r[i] != b.r[i]) return false;
+  return true;
+}
+}  // namespace tc
 
 int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
   using namespace tc;
   EncodeTiledFn enc = get_encoder();
   if (!enc) return LONGNET_ERR_CUDA;
-  static Params P;  // large; filled under a lock, copied into the launch
-  static TmaMaps maps;
   static std::mutex mu;
+  static LaunchCache* cache[64] = {nullptr};  // per device; kept for the process
   std::lock_guard<std::mutex> lock(mu);
-  int dev_sm = 0, n_sm = 148;
-  if (cudaGetDevice(&dev_sm) == cudaSuccess)
-    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev_sm);
-  fill_params(pb, P, n_sm);
-  const void* bases[3] = {pb.q, pb.k, pb.v};
-  for (int i = 0; i < P.n_r; ++i) {
-    for (int t = 0; t < 3; ++t) {
-      const int rows = t == 0 ? kBM : kBN;  // Q tiles 128 rows, K/V blocks 64 rows
-      if (!encode_map(enc, &maps.m[i][0][t], bases[t], pb, P.r_val[i], 0, P.kfull[i], rows))
-        return LONGNET_ERR_CUDA;
-      if (!encode_map(enc, &maps.m[i][1][t], bases[t], pb, P.r_val[i], P.tail[i], P.kfull[i], rows))
-        return LONGNET_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LONGNET_ERR_CUDA;
+  if (!cache[dev]) cache[dev] = new LaunchCache();
+  LaunchCache& c = *cache[dev];
+  if (!c.valid || !same_shape(c.shape, pb)) {
+    int n_sm = 148;
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    c.valid = false;
+    fill_params(pb, c.P, n_sm);
+    c.shape = pb;
+    c.q = c.k = c.v = nullptr;
+    c.valid = true;
+  }
+  Params& P = c.P;
+  P.pb = pb;  // this call's pointers and status word
+  if (c.q != pb.q || c.k != pb.k || c.v != pb.v) {
+    c.q = c.k = c.v = nullptr;
+    const void* bases[3] = {pb.q, pb.k, pb.v};
+    for (int i = 0; i < P.n_r; ++i) {
+      for (int t = 0; t < 3; ++t) {
+        const int rows = t == 0 ? kBM : kBN;  // Q tiles 128 rows, K/V blocks 64 rows
+        if (!encode_map(enc, &c.maps.m[i][0][t], bases[t], pb, P.r_val[i], 0, P.kfull[i], rows))
+          return LONGNET_ERR_CUDA;
+        if (!encode_map(enc, &c.maps.m[i][1][t], bases[t], pb, P.r_val[i], P.tail[i], P.kfull[i], rows))
+          return LONGNET_ERR_CUDA;
+      }
     }
+    c.q = pb.q;
+    c.k = pb.k;
+    c.v = pb.v;
   }
   const int smem_bytes = P.smem_bytes;
   static int attr_set[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LONGNET_ERR_CUDA;
   if (attr_set[dev] < smem_bytes) {
     if (cudaFuncSetAttribute(dilated_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
     attr_set[dev] = kSmemLimit;
   }
-  const int64_t grid = (int64_t)P.n_ranges * pb.B * pb.H;
-  dilated_fwd_kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, maps);
+  const int64_t grid = (int64_t)P.n_units * pb.B * pb.H;
+  dilated_fwd_kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, c.maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 

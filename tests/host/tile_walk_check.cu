@@ -60,10 +60,11 @@ void run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
   for (int64_t h = 0; h < H; ++h) {
     std::map<std::tuple<int, int64_t, int64_t>, int> seen;
     std::vector<int> finalized(N, 0);
-    for (int rank = 0; rank < P.n_ranges; ++rank) {
-      int64_t ri_range = P.range_order[0] >= 0 ? P.range_order[rank] : rank;
-      int64_t A = ri_range * P.range_len;
-      int64_t Bnd = std::min(N, A + P.range_len);
+    for (int rank = 0; rank < P.n_units; ++rank) {
+      int A32, B32;
+      unit_bounds(P, rank, A32, B32);
+      const int64_t A = A32, Bnd = B32;
+      CHECK(A < Bnd, "%s: empty unit %d\n", name, rank);
       TileWalker tw;
       tw.init(P, h, A, Bnd);
       Tile t;
@@ -148,7 +149,7 @@ void run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
       if (!covered) CHECK(P.uncovered_possible, "%s: uncovered position but flag off\n", name);
     }
   }
-  printf("%-28s ranges=%d R=%ld tiles/head=%.1f kv/head=%.1f %s\n", name, P.n_ranges, (long)P.range_len,
+  printf("%-28s ranges=%d units=%d R=%ld tiles/head=%.1f kv/head=%.1f %s\n", name, P.n_ranges, P.n_units, (long)P.range_len,
          (double)n_tiles / H, (double)n_kv / H, fails == f0 ? "OK" : "FAIL");
 }
 

@@ -107,6 +107,18 @@ def test_scores_far_beyond_exp2_range(impl_name, causal, ramp):
                     tol_out=tol)
 
 
+def test_repeated_shape_with_new_tensors():
+    """The launcher keeps the host set-up of the last shape and tensors: the
+    same shape with other tensors (and back) must still read the new ones."""
+    B, N, H, D = 1, 1024, 3, 64
+    pats = ((256, 1), (512, 2), (1024, 4))
+    sets = [wl.random_inputs(B, N, H, D, torch.bfloat16, seed=s) for s in (11, 12)]
+    for q, k, v in (sets[0], sets[1], sets[0], sets[1]):
+        for impl in (bd.LONGNET_IMPL_TCGEN05, bd.LONGNET_IMPL_AUTO):
+            o, l = gh.run_cuda(q, k, v, pats, True, impl)
+            gh.compare_full(o, l, q, k, v, pats, True, torch.bfloat16, label=f"repeat/{impl}")
+
+
 def test_named_tiny_workload_fp32():
     w = wl.WORKLOADS["tiny"]
     q, k, v = wl.make_inputs(w)
