@@ -21,7 +21,7 @@
  *
  * Conventions shared by every entry point
  *   - q, k, v, out: device pointers, contiguous [B, N, H, D] in the dtype
- *     given (LONGNET_DTYPE_F32 or LONGNET_DTYPE_BF16); 16-byte aligned.
+ *     given (LONGNET_DTYPE_F32, LONGNET_DTYPE_BF16 or LONGNET_DTYPE_F16); 16-byte aligned.
  *   - lse: device pointer to fp32 [B, H, N] (natural log, scale included),
  *     or NULL when not wanted.  4-byte aligned.
  *   - w, r: HOST arrays of n_pat pattern parameters, read during the call
@@ -64,15 +64,18 @@ enum longnet_status {
   LONGNET_ERR_NO_DEVICE = -7      /* no usable sm_100 device */
 };
 
-enum longnet_dtype { LONGNET_DTYPE_F32 = 0, LONGNET_DTYPE_BF16 = 1 };
+enum longnet_dtype { LONGNET_DTYPE_F32 = 0, LONGNET_DTYPE_BF16 = 1, LONGNET_DTYPE_F16 = 2 };
 
 /* Kernel families.  AUTO picks per shape; the others force one (tests). */
 enum longnet_impl {
   LONGNET_IMPL_AUTO = 0,
-  LONGNET_IMPL_SIMT = 1,     /* fp32 FMA, any D in {16,32,64,128}, both dtypes */
-  LONGNET_IMPL_TCGEN05 = 2,  /* bf16, D = 64: TMA + tcgen05/TMEM flash kernel,
-                                patterns fused in shared memory */
-  LONGNET_IMPL_SMALLSEG = 3  /* bf16, D = 64, w/r <= 128: memory-bound kernel */
+  LONGNET_IMPL_SIMT = 1,     /* fp32 FMA, any D in {16,32,64,128}, every dtype */
+  LONGNET_IMPL_TCGEN05 = 2,  /* bf16 or fp16, D = 64, <= 6 patterns: TMA +
+                                tcgen05/TMEM flash kernel, patterns fused in
+                                shared memory */
+  LONGNET_IMPL_SMALLSEG = 3  /* bf16 or fp16, D = 64, all patterns one segment
+                                length w <= 64 (a multiple of 8), one of them
+                                r = 1: memory-bound kernel */
 };
 
 /*

@@ -49,7 +49,7 @@ def load_library(path: str | None = None):
 
 
 def _f64(x) -> np.ndarray:
-    """Exact widening to a C-contiguous float64 array (bf16/fp32 -> fp64 is exact)."""
+    """Exact widening to a C-contiguous float64 array (bf16/fp16/fp32 -> fp64 is exact)."""
     try:
         import torch
 

@@ -27,6 +27,7 @@ LONGNET_MAX_PATTERNS = 16
 
 LONGNET_DTYPE_F32 = 0
 LONGNET_DTYPE_BF16 = 1
+LONGNET_DTYPE_F16 = 2
 
 LONGNET_IMPL_AUTO = 0
 LONGNET_IMPL_SIMT = 1
@@ -99,6 +100,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return LONGNET_DTYPE_F32
     if t.dtype == torch.bfloat16:
         return LONGNET_DTYPE_BF16
+    if t.dtype == torch.float16:
+        return LONGNET_DTYPE_F16
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -114,7 +117,7 @@ def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              impl: int = LONGNET_IMPL_AUTO, stream=None) -> None:
     """Enqueue the forward on `stream` (default: torch's current stream).
 
-    q, k, v, out: contiguous CUDA tensors [B, N, H, D] of one dtype (fp32/bf16);
+    q, k, v, out: contiguous CUDA tensors [B, N, H, D] of one dtype (fp32/bf16/fp16);
     lse: contiguous fp32 [B, H, N] or None.  Raises LongNetError on a non-zero
     status.
     """
@@ -153,7 +156,8 @@ def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def longnet_select_impl(B: int, N: int, H: int, D: int, patterns, causal: bool, dtype) -> int:
     """Kernel family AUTO would use (>= 1) or a negative status (host only)."""
     n, w, r = _patterns(patterns)
-    code = dtype if isinstance(dtype, int) else (LONGNET_DTYPE_F32 if dtype == torch.float32 else LONGNET_DTYPE_BF16)
+    code = dtype if isinstance(dtype, int) else {torch.float32: LONGNET_DTYPE_F32, torch.bfloat16: LONGNET_DTYPE_BF16,
+                                                 torch.float16: LONGNET_DTYPE_F16}[dtype]
     return int(load_library().longnet_select_impl(B, N, H, D, n, w, r, int(bool(causal)), code))
 
 

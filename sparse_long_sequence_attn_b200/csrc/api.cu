@@ -74,7 +74,8 @@ int check_args(const void* q, const void* k, const void* v, void* out, float* ls
     return LONGNET_ERR_INVALID_ARG;
   if (n_pat < 1 || n_pat > LONGNET_MAX_PATTERNS || !w || !r) return LONGNET_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return LONGNET_ERR_INVALID_ARG;
-  if (dtype != LONGNET_DTYPE_F32 && dtype != LONGNET_DTYPE_BF16) return LONGNET_ERR_INVALID_ARG;
+  if (dtype != LONGNET_DTYPE_F32 && dtype != LONGNET_DTYPE_BF16 && dtype != LONGNET_DTYPE_F16)
+    return LONGNET_ERR_INVALID_ARG;
   for (int i = 0; i < n_pat; ++i) {
     if (r[i] < 1 || w[i] < 1 || w[i] > N || N % w[i] != 0) return LONGNET_ERR_INVALID_ARG;
   }

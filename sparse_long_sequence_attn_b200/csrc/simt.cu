@@ -12,6 +12,7 @@
 // every pattern that keeps its row, and the combination needs no separate
 // step.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -26,8 +27,10 @@ constexpr int kWarps = 4;
 
 __device__ __forceinline__ float load_elem(const float* p) { return *p; }
 __device__ __forceinline__ float load_elem(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float load_elem(const __half* p) { return __half2float(*p); }
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void store_elem(__half* p, float x) { *p = __float2half_rn(x); }
 
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
@@ -149,6 +152,7 @@ int launch_typed(const Problem& p, cudaStream_t stream) {
 
 int launch_simt(const Problem& p, cudaStream_t stream) {
   if (p.dtype == LONGNET_DTYPE_F32) return launch_typed<float>(p, stream);
+  if (p.dtype == LONGNET_DTYPE_F16) return launch_typed<__half>(p, stream);
   return launch_typed<__nv_bfloat16>(p, stream);
 }
 

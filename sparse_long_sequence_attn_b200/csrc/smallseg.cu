@@ -1,6 +1,6 @@
 // Kernel family SMALLSEG: the multi-pattern dilated-attention forward when
 // every pattern's segments are short (all patterns share one segment length
-// W <= 64, bf16, D = 64).  Such shapes move far more bytes than they compute
+// W <= 64, bf16 or fp16, D = 64).  Such shapes move far more bytes than they compute
 // (the DilatedAttention usage example of the "LongNet" docs page: segment 64,
 // dilation 2), so this kernel is built for HBM bandwidth, not tensor peak.
 //
@@ -12,7 +12,7 @@
 //   * every pattern's sparsified segment (head offset o = h mod r, rows
 //     o + r*k < W) is read straight from shared memory by ldmatrix (the
 //     dilated gather is just a choice of row addresses) and attended with
-//     mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an fp32 softmax;
+//     mma.sync m16n8k16 (bf16 or fp16 in, fp32 accumulate) and an fp32 softmax;
 //   * patterns other than the r = 1 one park their normalised rows (16-byte
 //     chunks rotated by row, like the TMA swizzle, so a fragment's 8 rows hit
 //     distinct banks) and lse in the pair's shared memory;
@@ -27,6 +27,7 @@
 // own instantiation; six pairs leave 168 registers per thread.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -87,17 +88,47 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulators
+// Element formats of the 16-bit operands.
+constexpr int kFmtF16 = 0, kFmtBF16 = 1;
+// D += A * B, m16n8k16, 16-bit inputs (bf16 or f16), fp32 accumulators
+template <int kFmt>
 __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  if constexpr (kFmt == kFmtBF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
 }
+// Two floats rounded to the element format, lo in the low half.
+template <int kFmt>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+  if constexpr (kFmt == kFmtBF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+// The two elements of a packed pair as floats (exact).
+template <int kFmt>
+__device__ __forceinline__ void unpack2(uint32_t u, float& lo, float& hi) {
+  if constexpr (kFmt == kFmtBF16) {
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xffff0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    lo = f.x;
+    hi = f.y;
+  }
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -138,7 +169,7 @@ __device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int ch) {
 // the chunk; their O goes to ov and their lse (log2 domain) to lse0, lse1.
 // kMasked: some of the n_kt * 16 key columns are not keys of every row
 // (causal, or m not a multiple of 16).
-template <bool kMasked>
+template <int kFmt, bool kMasked>
 __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, uint32_t v_base, int o,
                                              int r, int m, int n_kt, int rc, bool causal,
                                              float scale_log2, int lane, float (&ov)[8][4],
@@ -177,8 +208,8 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
         if (np < n_kt) {
           uint32_t b0, b1, b2, b3;
           ldsm_x4(ka[np] + ((uint32_t)((2 * kk + ((lane >> 3) & 1)) ^ ksw[np]) << 4), b0, b1, b2, b3);
-          mma16816(acc[2 * np], a, b0, b1);
-          mma16816(acc[2 * np + 1], a, b2, b3);
+          mma16816<kFmt>(acc[2 * np], a, b0, b1);
+          mma16816<kFmt>(acc[2 * np + 1], a, b2, b3);
         }
       }
     }
@@ -219,8 +250,8 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
       l0 += p0 + p1;
       l1 += p2 + p3;
       const int kk = nt >> 1, hi = nt & 1;
-      pa[kk][hi * 2 + 0] = pack2(p0, p1);
-      pa[kk][hi * 2 + 1] = pack2(p2, p3);
+      pa[kk][hi * 2 + 0] = pack2<kFmt>(p0, p1);
+      pa[kk][hi * 2 + 1] = pack2<kFmt>(p2, p3);
     }
   }
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -244,8 +275,8 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
       for (int dp = 0; dp < 4; ++dp) {  // pairs of 8-dim tiles
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(va + ((uint32_t)((2 * dp + (lane >> 4)) ^ vsw) << 4), b0, b1, b2, b3);
-        mma16816(ov[2 * dp], pa[kk], b0, b1);
-        mma16816(ov[2 * dp + 1], pa[kk], b2, b3);
+        mma16816<kFmt>(ov[2 * dp], pa[kk], b0, b1);
+        mma16816<kFmt>(ov[2 * dp + 1], pa[kk], b2, b3);
       }
     }
   }
@@ -259,6 +290,7 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
   lse1 = ms1 + __log2f(l1);
 }
 
+template <int kFmt>
 __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     smallseg_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   extern __shared__ uint8_t smem_raw[];
@@ -349,9 +381,9 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
         float ov[8][4];
         float lse0, lse1;
         if (masked)
-          attend_chunk<true>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
+          attend_chunk<kFmt, true>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
         else
-          attend_chunk<false>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
+          attend_chunk<kFmt, false>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
         const int row0 = rc * 16 + g, row1 = row0 + 8;
         if (!last) {
           // ---- park the normalised rows (16-byte chunks rotated by row)
@@ -363,7 +395,7 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
 #pragma unroll
               for (int nt = 0; nt < 8; ++nt)
                 *reinterpret_cast<uint32_t*>(pr + ((nt ^ (row & 7)) << 4)) =
-                    pack2(ov[nt][2 * half], ov[nt][2 * half + 1]);
+                    pack2<kFmt>(ov[nt][2 * half], ov[nt][2 * half + 1]);
               if (t4 == 0) park_l[row] = half ? lse1 : lse0;
             }
           }
@@ -391,9 +423,10 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
                 const uint8_t* pq = pk + kq * 128 + 4 * t4;
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
-                  const uint32_t pv = *reinterpret_cast<const uint32_t*>(pq + ((nt ^ (kq & 7)) << 4));
-                  ov[nt][2 * half] = fmaf(__uint_as_float(pv << 16), cb, ov[nt][2 * half] * ca);
-                  ov[nt][2 * half + 1] = fmaf(__uint_as_float(pv & 0xffff0000u), cb, ov[nt][2 * half + 1] * ca);
+                  float plo, phi;
+                  unpack2<kFmt>(*reinterpret_cast<const uint32_t*>(pq + ((nt ^ (kq & 7)) << 4)), plo, phi);
+                  ov[nt][2 * half] = fmaf(plo, cb, ov[nt][2 * half] * ca);
+                  ov[nt][2 * half + 1] = fmaf(phi, cb, ov[nt][2 * half + 1] * ca);
                 }
                 lse = mxl + __log2f(wa + wb);
               }
@@ -403,7 +436,7 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
 #pragma unroll
               for (int nt = 0; nt < 8; ++nt)
                 *reinterpret_cast<uint32_t*>(sr + ((nt ^ (row & 7)) << 4)) =
-                    pack2(ov[nt][2 * half], ov[nt][2 * half + 1]);
+                    pack2<kFmt>(ov[nt][2 * half], ov[nt][2 * half + 1]);
               if (t4 == 0 && P.pb.lse)
                 P.pb.lse[((int64_t)b * H + h) * N + (int64_t)seg * W + row] = lse * 0.69314718055994531f;
             }
@@ -417,7 +450,7 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     // 16-byte chunks, 8 per row
     __syncwarp();
     {
-      __nv_bfloat16* out_seg = static_cast<__nv_bfloat16*>(P.pb.out) + (row0_pos * H + h) * kD;
+      uint16_t* out_seg = static_cast<uint16_t*>(P.pb.out) + (row0_pos * H + h) * kD;  // 16-bit elements
       const int64_t row_stride = (int64_t)H * kD;
       for (int rc = wsub; rc * 16 < W; rc += 2) {
 #pragma unroll
@@ -487,7 +520,7 @@ int pair_bytes(const Problem& p, int* park_off, int* park_rows, int* order) {
 
 bool smallseg_supports(const Problem& p) {
   using namespace ss;
-  if (p.dtype != LONGNET_DTYPE_BF16 || p.D != kD) return false;
+  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
   if (p.n_pat < 1 || p.n_pat > kMaxPat) return false;
   const int64_t W = p.w[0];
   if (W < 1 || W > kMaxW || W % 8 != 0) return false;
@@ -533,11 +566,11 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
     const void* q;
     const void* k;
     const void* v;
-    int64_t B, N, H, W;
+    int64_t B, N, H, W, dtype;
   };
   static MapKey last[64] = {};
   static Maps last_maps[64];
-  const MapKey key{pb.q, pb.k, pb.v, pb.B, pb.N, pb.H, P.W};
+  const MapKey key{pb.q, pb.k, pb.v, pb.B, pb.N, pb.H, P.W, pb.dtype};
   if (memcmp(&last[dev], &key, sizeof(key)) == 0) {
     maps = last_maps[dev];
   } else {
@@ -549,7 +582,7 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
                                (cuuint64_t)(pb.N * pb.H * kD * 2)};
       cuuint32_t box[4] = {(cuuint32_t)kD, 1, (cuuint32_t)P.W, 1};
       cuuint32_t estr[4] = {1, 1, 1, 1};
-      if (enc(&maps.m[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(bases[t]), dims, strides,
+      if (enc(&maps.m[t], pb.dtype == LONGNET_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(bases[t]), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return LONGNET_ERR_CUDA;
@@ -557,17 +590,18 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
     last_maps[dev] = maps;
     last[dev] = key;
   }
-  static int attr_set[64] = {0};
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(smallseg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
-        cudaSuccess)
+  const bool f16 = pb.dtype == LONGNET_DTYPE_F16;
+  auto kernel = f16 ? smallseg_kernel<kFmtF16> : smallseg_kernel<kFmtBF16>;
+  static bool attr_set[64][2] = {};
+  if (!attr_set[dev][f16]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
-    attr_set[dev] = 1;
+    attr_set[dev][f16] = true;
   }
   const int smem = P.n_pairs * P.pair_bytes + 1024;
   int64_t grid = (P.n_items + P.n_pairs - 1) / P.n_pairs;
   if (grid > n_sm) grid = n_sm;
-  smallseg_kernel<<<(unsigned)grid, P.n_pairs * 64, smem, stream>>>(P, maps);
+  kernel<<<(unsigned)grid, P.n_pairs * 64, smem, stream>>>(P, maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 

@@ -1,5 +1,5 @@
 // Kernel family TCGEN05: fused multi-pattern dilated flash-attention forward
-// for bf16, D = 64, on the 5th-generation tensor cores of sm_100a.
+// for bf16 or fp16, D = 64, on the 5th-generation tensor cores of sm_100a.
 //
 // What it computes ("LONGNET: Scaling Transformer to 1 billion tokens",
 // section "LongNet's attention allocation principle"; "LongNet论文精读",
@@ -22,8 +22,8 @@
 //    k at fixed (c, h, b) is exactly 128 kept rows, 128 B each, landing in
 //    shared memory with the 128-byte swizzle the tensor cores read.  A second
 //    map per r, shifted by N mod r positions, reaches the last few rows.
-//  * S = Q K^T and O += P V run as tcgen05.mma (bf16 in, fp32 accumulate in
-//    tensor memory).  S is double-buffered in TMEM; P (bf16) overwrites the
+//  * S = Q K^T and O += P V run as tcgen05.mma (bf16 or fp16 in, fp32 accumulate in
+//    tensor memory).  S is double-buffered in TMEM; P (the input format) overwrites the
 //    first half of its S buffer and is read from TMEM by the PV MMA.
 //  * Online softmax in fp32 by one warpgroup (thread i owns row i), exp2 on
 //    scaled scores, lazy rescaling of O (only when the row max grows by more
@@ -31,7 +31,7 @@
 //  * Cross-pattern combination without any HBM round trip: tiles are
 //    processed in order of (first position, larger r first, pattern index).
 //    Each tile's epilogue decides per row whether it is the last tile
-//    covering that position; if not, it parks the normalised row (bf16) and
+//    covering that position; if not, it parks the normalised row (input format) and
 //    its lse in a per-pattern shared-memory slot; the last one merges the
 //    parked rows of the other patterns and writes `out` / `lse` once.  With
 //    this order a pattern's slot is always fully consumed before that pattern's
@@ -40,6 +40,7 @@
 //    stops issuing work, drains what it issued and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -64,8 +65,8 @@ constexpr int kBN = 64;         // keys per KV block (MMA N of Q K^T)
 constexpr int kMaxPat = 6;      // patterns (and combination slots) supported
 constexpr int kMaxR = 8;        // distinct dilations supported
 constexpr int kThreads = 512;   // 16 warps: TMA, MMA, 2 idle, 2x4 softmax, 4 epilogue
-constexpr int kTileBytes = kBM * kD * 2;  // 16 KB per 128 x 64 bf16 Q tile
-constexpr int kKVBytes = kBN * kD * 2;    // 8 KB per 64 x 64 bf16 K or V block
+constexpr int kTileBytes = kBM * kD * 2;  // 16 KB per 128 x 64 Q tile (16-bit elements)
+constexpr int kKVBytes = kBN * kD * 2;    // 8 KB per 64 x 64 K or V block
 constexpr int kMaxRangeOrder = 4096;
 constexpr int kSmemLimit = 232448;       // dynamic shared memory per block on sm_100
 constexpr int kTileOverhead = 1;         // block-equivalents charged per tile (stream balance)
@@ -104,7 +105,7 @@ constexpr int kWalkerBytes = 512;  // per stream
 struct SmemLayout {
   int q;       // 2 Q tiles (one per stream)
   int kv;      // [stream][stages] x (K block, V block)
-  int slot_o;  // n_pat x 128 parked rows (bf16)
+  int slot_o;  // n_pat x 128 parked rows (input format)
   int slot_l;  // n_pat x 128 parked lse (fp32, log2 domain)
   int stats;   // [stream][O buffer][use parity][row] (m, l)
   int meta;    // element queues, tile queue, stage descriptors, pattern table, counters
@@ -288,9 +289,30 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
-  return *reinterpret_cast<uint32_t*>(&v);
+// Element formats of the 16-bit operands (the kind::f16 encoding).
+constexpr int kFmtF16 = 0, kFmtBF16 = 1;
+// Two floats rounded to the element format, lo in the low half.
+template <int kFmt>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (kFmt == kFmtBF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+// The two elements of a packed pair as floats (exact).
+template <int kFmt>
+__device__ __forceinline__ void unpack2(uint32_t u, float& lo, float& hi) {
+  if constexpr (kFmt == kFmtBF16) {
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xffff0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    lo = f.x;
+    hi = f.y;
+  }
 }
 
 
@@ -331,17 +353,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, given M, N, B major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+// Instruction descriptor, kind::f16: A, B in the element format (f16 or
+// bf16), D fp32, given M, N, B major.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool b_mn_major, int fmt) {
   return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
+         | ((uint32_t)fmt << 7)         // A format
+         | ((uint32_t)fmt << 10)        // B format
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
-constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false);  // S: 128 x 64
-constexpr uint32_t kIdescPV = idesc_bf16(kBM, kD, true);
+template <int kFmt>
+constexpr uint32_t kIdescQK = idesc_f16kind(kBM, kBN, false, kFmt);  // S: 128 x 64
+template <int kFmt>
+constexpr uint32_t kIdescPV = idesc_f16kind(kBM, kD, true, kFmt);
 
 // ---------------------------------------------------------------- tiles
 
@@ -714,6 +739,7 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   return v;
 }
 
+template <int kFmt>
 __global__ void __launch_bounds__(kThreads, 1)
     dilated_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ TmaMaps maps) {
   extern __shared__ uint8_t smem_raw[];
@@ -1005,7 +1031,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = ob ? o_tmem1 : o_tmem0;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, desc_from(v_lo + kk * 128, kDescHi), kIdescPV,
+          mma_ts(d_tmem, a_tmem + kk * 8, desc_from(v_lo + kk * 128, kDescHi), kIdescPV<kFmt>,
                  (pv_first && kk == 0) ? 0u : 1u);
         tc_commit(kv_empty + pv_st);
         tc_commit(pv_last ? bar_o_full + 2 * g + ob : bar_o_done + g);
@@ -1027,7 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
           mma_ss(sb ? s_tmem1 : s_tmem0, desc_from(q_lo + kk * 2, kDescHi),
-                 desc_from(k_lo + kk * 2, kDescHi), kIdescQK, kk > 0 ? 1u : 0u);
+                 desc_from(k_lo + kk * 2, kDescHi), kIdescQK<kFmt>, kk > 0 ? 1u : 0u);
         tc_commit(bar_s_full + 2 * g + sb);
         if (em.j == em.nkv - 1) tc_commit(bar_q_empty + g);
         if (have_prev) {
@@ -1116,7 +1142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_use = m_blk;
           }
         }
-        // P = 2^(s*scale - m) as bf16 over the first 32 columns of this S buffer
+        // P = 2^(s*scale - m) in the input format over the first 32 columns of this S buffer
         float ps[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
@@ -1131,7 +1157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sc2, nm2), xa, xb);
             const float a = ex2(xa), bq = ex2(xb);
             ls[c & 3] = add_f32x2(ls[c & 3], f32x2(a, bq));
-            pk[c] = pack_bf16(a, bq);
+            pk[c] = pack2<kFmt>(a, bq);
           }
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) f32x2_split(ls[q4], ps[2 * q4], ps[2 * q4 + 1]);
@@ -1180,7 +1206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (processing order)
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(P.pb.out);
+    uint16_t* outp = static_cast<uint16_t*>(P.pb.out);  // 16-bit elements
     bool ok = true;
     for (int i = 0; ok; ++i) {
       ok = wait_seq(&sTileQ[i % kQT].seq, i);
@@ -1264,8 +1290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
                   const int d = ch * 8 + q2 * 2;
-                  f32x2_split(fma_f32x2(f32x2(__uint_as_float(wv[q2] << 16), __uint_as_float(wv[q2] & 0xffff0000u)),
-                                        f32x2(cq, cq), f32x2(o[d], o[d + 1])), o[d], o[d + 1]);
+                  float plo, phi;
+                  unpack2<kFmt>(wv[q2], plo, phi);
+                  f32x2_split(fma_f32x2(f32x2(plo, phi), f32x2(cq, cq), f32x2(o[d], o[d + 1])), o[d], o[d + 1]);
                 }
               }
             }
@@ -1274,10 +1301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             uint4 u;
-            u.x = pack_bf16(o[ch * 8 + 0], o[ch * 8 + 1]);
-            u.y = pack_bf16(o[ch * 8 + 2], o[ch * 8 + 3]);
-            u.z = pack_bf16(o[ch * 8 + 4], o[ch * 8 + 5]);
-            u.w = pack_bf16(o[ch * 8 + 6], o[ch * 8 + 7]);
+            u.x = pack2<kFmt>(o[ch * 8 + 0], o[ch * 8 + 1]);
+            u.y = pack2<kFmt>(o[ch * 8 + 2], o[ch * 8 + 3]);
+            u.z = pack2<kFmt>(o[ch * 8 + 4], o[ch * 8 + 5]);
+            u.w = pack2<kFmt>(o[ch * 8 + 6], o[ch * 8 + 7]);
             dst[ch] = u;
           }
           if (P.pb.lse) P.pb.lse[(b * P.pb.H + h) * P.pb.N + x] = (mx + __log2f(wsum)) * 0.69314718055994531f;
@@ -1290,10 +1317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; e += 2)
               f32x2_split(mul_f32x2(f32x2(o[ch * 8 + e], o[ch * 8 + e + 1]), f32x2(l_inv, l_inv)), t[e], t[e + 1]);
-            u.x = pack_bf16(t[0], t[1]);
-            u.y = pack_bf16(t[2], t[3]);
-            u.z = pack_bf16(t[4], t[5]);
-            u.w = pack_bf16(t[6], t[7]);
+            u.x = pack2<kFmt>(t[0], t[1]);
+            u.y = pack2<kFmt>(t[2], t[3]);
+            u.z = pack2<kFmt>(t[4], t[5]);
+            u.w = pack2<kFmt>(t[6], t[7]);
             dst[ch ^ (row & 7)] = u;
           }
           sSlotL[tm.p * kBM + row] = lse2;
@@ -1355,7 +1382,7 @@ EncodeTiledFn get_encoder() {
   return fn;
 }
 
-// View [B, N, H, D] bf16 (starting `shift` positions in) as (d, h, c, k, b)
+// View [B, N, H, D] (16-bit elements, starting `shift` positions in) as (d, h, c, k, b)
 // with position = shift + r*k + c, k < kcount.
 bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem& p, int64_t r,
                 int64_t shift, int64_t kcount, int box_rows) {
@@ -1367,7 +1394,9 @@ bool encode_map(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Pro
                            (cuuint64_t)(r * p.H * kD * es), (cuuint64_t)(p.N * p.H * kD * es)};
   cuuint32_t box[5] = {(cuuint32_t)kD, 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult rc = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<char*>(ptr), dims, strides,
+  const CUtensorMapDataType ty =
+      p.dtype == LONGNET_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult rc = enc(map, ty, 5, const_cast<char*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return rc == CUDA_SUCCESS;
@@ -1406,7 +1435,7 @@ int64_t range_cost(const Problem& pb, int64_t A, int64_t Bnd) {
 
 bool tcgen05_supports(const Problem& p) {
   using namespace tc;
-  if (p.dtype != LONGNET_DTYPE_BF16 || p.D != kD) return false;
+  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
   static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
   if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 2) return false;
   if (p.H > 65535 || p.B > 65535) return false;
@@ -1602,15 +1631,16 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
     c.v = pb.v;
   }
   const int smem_bytes = P.smem_bytes;
-  static int attr_set[64] = {0};
-  if (attr_set[dev] < smem_bytes) {
-    if (cudaFuncSetAttribute(dilated_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemLimit) != cudaSuccess)
+  const bool f16 = pb.dtype == LONGNET_DTYPE_F16;
+  auto kernel = f16 ? dilated_fwd_kernel<kFmtF16> : dilated_fwd_kernel<kFmtBF16>;
+  static bool attr_set[64][2] = {};
+  if (!attr_set[dev][f16]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
-    attr_set[dev] = kSmemLimit;
+    attr_set[dev][f16] = true;
   }
   const int64_t grid = (int64_t)P.n_units * pb.B * pb.H;
-  dilated_fwd_kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, c.maps);
+  kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, c.maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 

@@ -13,7 +13,9 @@ from sparse_long_sequence_attn_b200 import binding as bd
 
 # Parity bar: max-abs error 1e-4 for fp32 inputs, 2e-2 for bf16 inputs (fp32
 # accumulation), lse within 1e-3.
-TOL_OUT = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+# fp16: P, a parked partial and the output are each rounded to 11 bits, at
+# most 3 * 2^-11 * max|v| ~ 7e-3 for the N(0,1) draws here; 1e-2 is allowed.
+TOL_OUT = {torch.float32: 1e-4, torch.bfloat16: 2e-2, torch.float16: 1e-2}
 TOL_LSE = 1e-3
 GUARD = 4096  # elements of NaN guard band on each side of every output
 

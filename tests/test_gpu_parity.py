@@ -51,6 +51,11 @@ SMALL_CASES = [
     ("bf16_d64_seg40_4pat", 1, 800, 5, 64, torch.bfloat16, True, ((40, 1), (40, 3), (40, 7), (40, 48))),
     ("bf16_d64_seg8_noncausal", 2, 256, 3, 64, torch.bfloat16, False, ((8, 1), (8, 2))),
     ("bf16_d64_seg56_r5", 1, 560, 6, 64, torch.bfloat16, False, ((56, 5), (56, 1), (56, 2))),
+    # fp16 inputs (every family)
+    ("f16_d64_lm_like", 2, 2048, 4, 64, torch.float16, True, ((512, 1), (1024, 2), (2048, 4))),
+    ("f16_d64_r_not_dividing", 1, 1536, 5, 64, torch.float16, True, ((384, 3), (768, 4), (1536, 8))),
+    ("f16_d64_seg64_r2_noncausal", 2, 1024, 4, 64, torch.float16, False, ((64, 1), (64, 2))),
+    ("f16_d32", 1, 512, 2, 32, torch.float16, True, ((128, 1), (512, 2))),
 ]
 
 
@@ -64,8 +69,8 @@ def test_small_cases_vs_oracle(case, impl_name):
     gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
 
 
-@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c[5] == torch.bfloat16 and c[4] == 64],
-                         ids=[c[0] for c in SMALL_CASES if c[5] == torch.bfloat16 and c[4] == 64])
+@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c[5] in (torch.bfloat16, torch.float16) and c[4] == 64],
+                         ids=[c[0] for c in SMALL_CASES if c[5] in (torch.bfloat16, torch.float16) and c[4] == 64])
 @pytest.mark.parametrize("impl_name", ["tcgen05", "smallseg"])
 def test_specialised_families_vs_oracle(case, impl_name):
     name, B, N, H, D, dtype, causal, pats = case
