@@ -25,9 +25,12 @@
  *   - lse: device pointer to fp32 [B, H, N] (natural log, scale included),
  *     or NULL when not wanted.  4-byte aligned.
  *   - w, r: HOST arrays of n_pat pattern parameters, read during the call
- *     and not kept.  1 <= n_pat <= LONGNET_MAX_PATTERNS, r >= 1,
- *     1 <= w <= N, N % w == 0.  Patterns may repeat and come in any order;
- *     a repeated pattern counts twice.
+ *     and not kept.  1 <= n_pat <= LONGNET_MAX_PATTERNS, r >= 1, w >= 1.
+ *     When w does not divide N the last segment is the shorter rest of the
+ *     sequence (no padding); w > N makes one segment of the whole sequence.
+ *     Patterns may repeat and come in any order; a repeated pattern counts
+ *     twice.  (The tcgen05 and small-segment kernels take N % w == 0 only;
+ *     LONGNET_IMPL_AUTO falls back to the SIMT kernel otherwise.)
  *   - causal: 1 = causal inside each sparsified segment, 0 = full.
  *   - stream: a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; the call returns before it finishes.

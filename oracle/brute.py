@@ -14,10 +14,11 @@ import math
 import numpy as np
 
 
-def keys_reaching(pos: int, h: int, patterns, causal: bool):
+def keys_reaching(pos: int, h: int, patterns, causal: bool, N: int | None = None):
     """List of key positions (with repeats across patterns) that row `pos` of
     head `h` attends to: for each pattern (w, r) that keeps the row, the kept
-    rows of its segment up to the row itself (all kept rows if not causal)."""
+    rows of its segment up to the row itself (all kept rows if not causal).
+    The last segment of a pattern ends with the sequence (length N mod w)."""
     keys = []
     for (w, r) in patterns:
         seg_start = (pos // w) * w
@@ -26,7 +27,7 @@ def keys_reaching(pos: int, h: int, patterns, causal: bool):
         if off < 0 or off % r:
             continue
         j = 0
-        while o + r * j < w:
+        while o + r * j < w and (N is None or seg_start + o + r * j < N):
             kp = seg_start + o + r * j
             if causal and kp > pos:
                 break
@@ -47,7 +48,7 @@ def dilated_attn_bruteforce(q, k, v, patterns, causal=True):
     for b in range(B):
         for h in range(H):
             for pos in range(N):
-                keys = keys_reaching(pos, h, patterns, causal)
+                keys = keys_reaching(pos, h, patterns, causal, N)
                 if not keys:
                     continue
                 s = np.array([float(np.dot(q[b, pos, h], k[b, kp, h])) * scale for kp in keys])

@@ -8,7 +8,9 @@
  * alone, plainly and slowly, in double precision.
  *
  * What it computes, in the order the pages describe it:
- *   1. split the sequence into segments of w tokens
+ *   1. split the sequence into segments of w tokens; when w does not divide
+ *      N the last segment is the shorter rest of the sequence (reading: no
+ *      padding, the pages only speak of equal segments)
  *      ("LongNet论文精读", section "Dilated Attention的工作原理", first step;
  *       "LONGNET: Scaling Transformer to 1 billion tokens", section
  *       "LongNet's attention allocation principle");
@@ -43,18 +45,26 @@
 #define ORACLE_BAD_ARG (-1)
 #define ORACLE_NO_MEMORY (-2)
 
-/* Number of rows head h keeps in one segment of pattern (w, r):
- * the offsets o + r*k that stay below w. */
-static int64_t rows_kept(int64_t w, int64_t r, int64_t o) {
-  if (o >= w) return 0;
-  return (w - o + r - 1) / r;
+/* Number of rows head h keeps in one segment of pattern (w, r) whose length
+ * is len (w, or less for a last segment cut by the end of the sequence): the
+ * offsets o + r*k that stay below len. */
+static int64_t rows_kept(int64_t len, int64_t r, int64_t o) {
+  if (o >= len) return 0;
+  return (len - o + r - 1) / r;
+}
+
+/* Length of segment seg of a pattern with segment length w: the sequence is
+ * cut into segments of w tokens and the last one ends with the sequence. */
+static int64_t seg_len(int64_t N, int64_t w, int64_t seg) {
+  const int64_t rest = N - seg * w;
+  return rest < w ? rest : w;
 }
 
 static int check_args(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
                       const int64_t* w, const int64_t* r) {
   if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || n_pat <= 0 || n_pat > 64) return ORACLE_BAD_ARG;
   for (int p = 0; p < n_pat; ++p) {
-    if (r[p] < 1 || w[p] < 1 || w[p] > N || N % w[p] != 0) return ORACLE_BAD_ARG;
+    if (r[p] < 1 || w[p] < 1) return ORACLE_BAD_ARG;
   }
   return ORACLE_OK;
 }
@@ -144,13 +154,14 @@ int oracle_dilated_attn_fp64(const double* q, const double* k, const double* v,
   int64_t task_base[64];
   for (int p = 0; p < n_pat; ++p) {
     task_base[p] = n_tasks_total;
-    n_tasks_total += B * H * (N / w[p]);
+    n_tasks_total += B * H * ((N + w[p] - 1) / w[p]);
   }
   int failed = 0;
 #pragma omp parallel
   {
     int64_t wmax = 0;
     for (int p = 0; p < n_pat; ++p) wmax = w[p] > wmax ? w[p] : wmax;
+    if (wmax > N) wmax = N; /* no segment is longer than the sequence */
     double* qs = (double*)malloc(sizeof(double) * (size_t)(wmax * D));
     double* ks = (double*)malloc(sizeof(double) * (size_t)(wmax * D));
     double* vs = (double*)malloc(sizeof(double) * (size_t)(wmax * D));
@@ -169,14 +180,14 @@ int oracle_dilated_attn_fp64(const double* q, const double* k, const double* v,
         }
         int p = 0;
         while (p + 1 < n_pat && t >= task_base[p + 1]) ++p;
-        const int64_t n_seg = N / w[p];
+        const int64_t n_seg = (N + w[p] - 1) / w[p];
         int64_t rem = t - task_base[p];
         const int64_t seg = rem % n_seg;
         rem /= n_seg;
         const int64_t h = rem % H;
         const int64_t b = rem / H;
         const int64_t o = h % r[p];
-        const int64_t m = rows_kept(w[p], r[p], o);
+        const int64_t m = rows_kept(seg_len(N, w[p], seg), r[p], o);
         /* step 1+2: gather the kept rows of this segment */
         for (int64_t i = 0; i < m; ++i) {
           const int64_t pos = seg * w[p] + o + r[p] * i;
@@ -251,6 +262,7 @@ int oracle_dilated_attn_rows_fp64(const double* q, const double* k, const double
   {
     int64_t wmax = 0;
     for (int p = 0; p < n_pat; ++p) wmax = w[p] > wmax ? w[p] : wmax;
+    if (wmax > N) wmax = N; /* no segment is longer than the sequence */
     double* sc = (double*)malloc(sizeof(double) * (size_t)wmax);
     double* orows = (double*)malloc(sizeof(double) * (size_t)(64 * D));
     const int have_buffers = sc && orows;
@@ -276,7 +288,7 @@ int oracle_dilated_attn_rows_fp64(const double* q, const double* k, const double
           const int64_t off = pos - seg * w[p] - o;
           if (off < 0 || off % r[p] != 0) continue; /* row not kept by p */
           const int64_t i = off / r[p];
-          const int64_t m = rows_kept(w[p], r[p], o);
+          const int64_t m = rows_kept(seg_len(N, w[p], seg), r[p], o);
           const int64_t n_keys = causal ? i + 1 : m;
           double mx = -INFINITY;
           for (int64_t j = 0; j < n_keys; ++j) {

@@ -89,7 +89,9 @@ __global__ void __launch_bounds__(kWarps * 32) simt_kernel(const Problem p) {
     const int64_t off = pos - seg_start - o;
     if (off < 0 || off % r != 0) continue;  // this pattern does not keep the row
     const int64_t kk = off / r;
-    const int64_t m = (w - o + r - 1) / r;
+    // the last segment ends with the sequence (shorter when w does not divide N)
+    const int64_t len = p.N - seg_start < w ? p.N - seg_start : w;
+    const int64_t m = (len - o + r - 1) / r;
     const int64_t n_keys = p.causal ? kk + 1 : m;
     const int64_t first = seg_start + o;
     for (int64_t j0 = 0; j0 < n_keys; j0 += 32) {

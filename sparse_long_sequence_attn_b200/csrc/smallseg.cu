@@ -526,6 +526,7 @@ bool smallseg_supports(const Problem& p) {
   if (W < 1 || W > kMaxW || W % 8 != 0) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.w[i] != W) return false;
+  if (W > p.N || p.N % W != 0) return false;  // whole segments only
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.r[i] < 1 || p.r[i] > (int64_t)INT32_MAX) return false;

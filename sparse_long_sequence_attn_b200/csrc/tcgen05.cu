@@ -1445,6 +1445,7 @@ bool tcgen05_supports(const Problem& p) {
   int n_r = 0;
   int64_t rv[kMaxR];
   for (int i = 0; i < p.n_pat; ++i) {
+    if (p.w[i] > p.N || p.N % p.w[i] != 0) return false;  // whole segments only
     bool found = false;
     for (int j = 0; j < n_r; ++j) found |= (rv[j] == p.r[i]);
     if (!found) {

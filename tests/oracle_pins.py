@@ -69,18 +69,22 @@ def check_dense_noncausal(lib):
 
 
 def check_block_diagonal(lib):
-    """r = 1 with w < N is block-diagonal attention (causal inside each block)."""
-    B, N, H, D, w = 1, 60, 2, 8, 12
+    """r = 1 with w < N is block-diagonal attention (causal inside each block);
+    when w does not divide N the last block is the shorter rest (N = 60 with
+    w = 16 or 25: last blocks of 12 and 10 positions), and w > N is one
+    block over the whole sequence."""
+    B, N, H, D = 1, 60, 2, 8
     q, k, v = (_rand((B, N, H, D), s) for s in (7, 8, 9))
-    for causal in (True, False):
-        out, _ = orc.dilated_attn_fp64(q, k, v, [(w, 1)], causal=causal, lib=lib)
-        blk = np.arange(N) // w
-        mask = blk[:, None] == blk[None, :]
-        if causal:
-            mask &= np.tril(np.ones((N, N), dtype=bool))
-        for h in range(H):
-            ref = _sdpa(q[0, :, h], k[0, :, h], v[0, :, h], mask=mask)
-            np.testing.assert_allclose(out[0, :, h], ref, atol=1e-12, rtol=0)
+    for w in (12, 16, 25, 80):
+        for causal in (True, False):
+            out, _ = orc.dilated_attn_fp64(q, k, v, [(w, 1)], causal=causal, lib=lib)
+            blk = np.arange(N) // w
+            mask = blk[:, None] == blk[None, :]
+            if causal:
+                mask &= np.tril(np.ones((N, N), dtype=bool))
+            for h in range(H):
+                ref = _sdpa(q[0, :, h], k[0, :, h], v[0, :, h], mask=mask)
+                np.testing.assert_allclose(out[0, :, h], ref, atol=1e-12, rtol=0)
 
 
 def read_selection_fixture():
@@ -162,6 +166,9 @@ def check_bruteforce_agreement(lib):
         (2, 30, 3, 6, [(10, 1), (15, 4), (30, 6)], True, 22),
         (1, 24, 4, 5, [(8, 3), (24, 5)], False, 23),
         (1, 32, 2, 8, [(16, 1), (16, 1)], True, 24),  # duplicated pattern
+        # w not dividing N (last segments of 10, 2 and 34 positions), w > N
+        (1, 34, 3, 4, [(12, 1), (8, 3), (40, 5)], True, 25),
+        (2, 26, 4, 4, [(8, 2), (11, 3), (26, 1)], False, 26),
     ]
     for (B, N, H, D, pats, causal, seed) in cases:
         q, k, v = (_rand((B, N, H, D), seed + 100 * i) for i in range(3))

@@ -47,7 +47,7 @@ def _call(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, ptr=Non
 
 @pytest.mark.parametrize("kw", [
     dict(B=0), dict(N=-1), dict(H=0), dict(D=0), dict(pats=()), dict(pats=((16, 0),)),
-    dict(pats=((0, 1),)), dict(pats=((128, 1),)), dict(pats=((24, 1),)), dict(causal=2),
+    dict(pats=((0, 1),)), dict(causal=2),
     dict(dtype=7), dict(pats=tuple((16, 1) for _ in range(17))), dict(impl=9),
 ])
 def test_invalid_arguments_rejected_on_host(kw):
@@ -67,6 +67,9 @@ def test_null_and_misaligned_pointers():
 def test_valid_call_without_device_reports_no_device():
     lib = bd.load_library()
     assert _call(lib) == bd.LONGNET_ERR_NO_DEVICE
+    # w not dividing N (a shorter last segment) and w > N are valid shapes
+    assert _call(lib, pats=((24, 1),)) == bd.LONGNET_ERR_NO_DEVICE
+    assert _call(lib, pats=((128, 1), (16, 2))) == bd.LONGNET_ERR_NO_DEVICE
     assert lib.longnet_last_device_status(None) == bd.LONGNET_ERR_NO_DEVICE
     assert lib.longnet_watchdog_selftest(1000, None) == bd.LONGNET_ERR_NO_DEVICE
 
@@ -75,6 +78,9 @@ def test_select_impl_host_logic():
     f32, bf16 = torch.float32, torch.bfloat16
     assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 1), (128, 2)), True, f32) == bd.LONGNET_IMPL_SIMT
     assert bd.longnet_select_impl(1, 256, 2, 48, ((64, 1),), True, f32) == bd.LONGNET_ERR_UNSUPPORTED
-    assert bd.longnet_select_impl(1, 255, 2, 16, ((64, 1),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
+    # a shorter last segment (255 = 3 * 64 + 63) goes to the general kernel
+    assert bd.longnet_select_impl(1, 255, 2, 16, ((64, 1),), True, f32) == bd.LONGNET_IMPL_SIMT
+    assert bd.longnet_select_impl(1, 4000, 4, 64, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_SIMT
+    assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 0),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
     impl = bd.longnet_select_impl(1, 32768, 12, 64, ((2048, 1), (4096, 2)), True, bf16)
     assert impl in (bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05)

@@ -56,6 +56,10 @@ SMALL_CASES = [
     ("f16_d64_r_not_dividing", 1, 1536, 5, 64, torch.float16, True, ((384, 3), (768, 4), (1536, 8))),
     ("f16_d64_seg64_r2_noncausal", 2, 1024, 4, 64, torch.float16, False, ((64, 1), (64, 2))),
     ("f16_d32", 1, 512, 2, 32, torch.float16, True, ((128, 1), (512, 2))),
+    # w not dividing N: the last segment is the shorter rest; w > N is one segment
+    ("fp32_d32_partial_segments", 1, 300, 3, 32, torch.float32, True, ((64, 1), (128, 3), (512, 5))),
+    ("bf16_d64_partial_noncausal", 2, 1000, 4, 64, torch.bfloat16, False, ((256, 1), (384, 2))),
+    ("f16_d64_partial_causal", 1, 777, 2, 64, torch.float16, True, ((128, 1), (256, 4))),
 ]
 
 

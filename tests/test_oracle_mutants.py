@@ -23,7 +23,10 @@ MUTANTS = [
     ("unweighted_merge", "const double wt = exp(lse_p[p] - mx);", "const double wt = 1.0;"),
     ("lse_without_max", "ls[i] = mx + log(denom);", "ls[i] = log(denom);"),
     ("transposed_qk", "s += qs[i * D + d] * ks[j * D + d];", "s += qs[j * D + d] * ks[i * D + d];"),
-    ("floor_row_count", "return (w - o + r - 1) / r;", "return (w - o) / r;"),
+    ("floor_row_count", "return (len - o + r - 1) / r;", "return (len - o) / r;"),
+    ("partial_segment_short", "return rest < w ? rest : w;", "return rest < w ? rest - 1 : w;"),
+    ("partial_segment_dropped", "n_tasks_total += B * H * ((N + w[p] - 1) / w[p]);",
+     "n_tasks_total += B * H * (N / w[p]);"),
     ("stride_dropped", "const int64_t pos = seg * w[p] + o + r[p] * i;\n          const int64_t src",
      "const int64_t pos = seg * w[p] + o + i;\n          const int64_t src"),
     ("v_from_query_row", "acc += scores[j] * vs[j * D + d];", "acc += scores[j] * vs[i * D + d];"),
