@@ -369,6 +369,11 @@ def run_ours(args, wl):
     roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
     roof["traffic"] = traffic_from_profiles(wl.name, kname)
     roof["algorithmic_flops_per_launch"] = flops
+    # secondary: the exact causal pair count (4*D flops per pair) instead of
+    # the nominal w/r formula
+    pairs = wlm.exact_pair_count(wl)
+    roof["exact_pairs_per_launch"] = pairs
+    roof["tflops_exact_pairs"] = 4.0 * wl.D * pairs / mean_step / 1e12
     roof["algorithmic_bytes_per_launch"] = wlm.algorithmic_bytes(wl)
     roof["frac_of_sustained_bf16"] = flops / mean_step / 1e12 / peaks.get("bf16_tflops_sustained", 1400.0)
     roof["frac_of_nominal_bf16"] = flops / mean_step / 1e12 / NOMINAL_BF16_TFLOPS

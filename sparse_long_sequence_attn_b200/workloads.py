@@ -128,6 +128,22 @@ def algorithmic_flops(wl: Workload) -> float:
     return tot
 
 
+def exact_pair_count(wl: Workload) -> int:
+    """Exact number of (query, key) score pairs the method evaluates: per
+    pattern, head and segment, m(m+1)/2 when causal or m^2 when not, with m the
+    rows the head keeps in that segment (the last segment may be shorter)."""
+    tot = 0
+    for (w, r) in wl.patterns:
+        n_seg = (wl.N + w - 1) // w
+        for h in range(wl.H):
+            o = h % r
+            for seg in range(n_seg):
+                ln = min(w, wl.N - seg * w)
+                m = 0 if o >= ln else (ln - o + r - 1) // r
+                tot += m * (m + 1) // 2 if wl.causal else m * m
+    return tot * wl.B
+
+
 def algorithmic_bytes(wl: Workload) -> float:
     """q, k, v read once, out written once, lse (fp32) written once."""
     es = 4 if wl.dtype == "fp32" else 2

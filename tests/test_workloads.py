@@ -36,3 +36,19 @@ def test_flops_formula_values():
     assert abs(wl.algorithmic_flops(wl.WORKLOADS["long32k"]) - 214.7e9) / 214.7e9 < 1e-3
     assert abs(wl.algorithmic_flops(wl.WORKLOADS["lm"]) - 180.4e9) / 180.4e9 < 1e-3
     assert abs(wl.algorithmic_flops(wl.WORKLOADS["smallseg"]) - 42.9e9) / 42.9e9 < 1e-2
+
+
+def test_exact_pair_count_matches_key_lists():
+    """The bench's exact pair count equals the number of (row, key) pairs the
+    brute-force formulation lists, on shapes with r not dividing w, w < r,
+    partial last segments and w > N."""
+    from oracle.brute import keys_reaching
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    cases = [(2, 36, 5, ((12, 5), (18, 3), (36, 7)), True),
+             (1, 34, 3, ((12, 1), (8, 3), (40, 5)), True),
+             (1, 26, 4, ((8, 2), (11, 3), (2, 3)), False)]
+    for B, N, H, pats, causal in cases:
+        w = wlm.Workload("pairs", 0, B=B, N=N, H=H, D=8, dtype="fp32", causal=causal, patterns=pats)
+        listed = B * sum(len(keys_reaching(pos, h, pats, causal, N)) for h in range(H) for pos in range(N))
+        assert wlm.exact_pair_count(w) == listed
