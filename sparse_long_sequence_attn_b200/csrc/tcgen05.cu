@@ -10,7 +10,9 @@
 // their softmax denominators.
 //
 // Design.
-//  * Work unit = (batch b, head h, position range [A, A + R)), R = 128 * r_max.
+//  * Work unit = (batch b, head h, position range [A, A + R)), R = 128 * r_max
+//    (halved while there are fewer units than SMs; the costliest ranges split
+//    in halves when a host simulation of the block schedule favours it).
 //    One CTA per unit; units are launched longest-first (host cost model), so
 //    the hardware block scheduler does greedy LPT balancing.
 //  * Inside a unit, every pattern's kept rows are cut into "natural" tiles of
@@ -25,9 +27,12 @@
 //  * S = Q K^T and O += P V run as tcgen05.mma (bf16 or fp16 in, fp32 accumulate in
 //    tensor memory).  S is double-buffered in TMEM; P (the input format) overwrites the
 //    first half of its S buffer and is read from TMEM by the PV MMA.
-//  * Online softmax in fp32 by one warpgroup (thread i owns row i), exp2 on
-//    scaled scores, lazy rescaling of O (only when the row max grows by more
-//    than 2^8).
+//  * The unit's tiles are dealt to two independent streams, each with its
+//    own TMA thread (Q per tile, a ring of 64-key K/V blocks), MMA thread and
+//    softmax warpgroup; one epilogue warpgroup takes the tiles of both in
+//    processing order.
+//  * Online softmax in fp32 (thread i owns row i), exp2 on scaled scores,
+//    lazy rescaling of O (only when the row max grows by more than 2^8).
 //  * Cross-pattern combination without any HBM round trip: tiles are
 //    processed in order of (first position, larger r first, pattern index).
 //    Each tile's epilogue decides per row whether it is the last tile
@@ -48,10 +53,7 @@
 
 #include <algorithm>
 #include <mutex>
-#include <numeric>
-#include <queue>
 #include <type_traits>
-#include <vector>
 
 #include "device_util.cuh"
 #include "params.h"
@@ -68,6 +70,7 @@ constexpr int kThreads = 512;   // 16 warps: TMA, MMA, 2 idle, 2x4 softmax, 4 ep
 constexpr int kTileBytes = kBM * kD * 2;  // 16 KB per 128 x 64 Q tile (16-bit elements)
 constexpr int kKVBytes = kBN * kD * 2;    // 8 KB per 64 x 64 K or V block
 constexpr int kMaxRangeOrder = 4096;
+constexpr int kMaxHeapSms = 1024;  // SMs the host schedule simulation models
 constexpr int kSmemLimit = 232448;       // dynamic shared memory per block on sm_100
 constexpr int kTileOverhead = 1;         // block-equivalents charged per tile (stream balance)
 
@@ -78,7 +81,7 @@ __host__ __device__ constexpr uint32_t col_s(int g, int sb) { return (uint32_t)(
 __host__ __device__ constexpr uint32_t col_o(int g, int ob) { return 256u + (uint32_t)(2 * g + ob) * 64u; }
 
 // Descriptors the TMA thread publishes for the other roles.
-constexpr int kQE = 16;  // element queue entries per softmax stream
+constexpr int kQE = 16;  // tile descriptor queue entries per softmax stream
 constexpr int kQT = 32;  // tile queue entries (epilogue)
 struct ElemMeta {        // one KV block of one tile
   int info;              // bit0 stream, bit1 O buffer, bit2 use parity, bit3 use > 0, bit4 end
@@ -95,7 +98,7 @@ struct TileMeta {        // one tile, in processing order
   int pad[3];
 };
 constexpr int kInfoEnd = 16;
-// element queues [2][kQE], tile queue [kQT], stage descriptors [kMaxStages],
+// softmax tile queues [2][kQE], epilogue tile queue [kQT], stage descriptors [kMaxStages],
 // pattern table [kMaxPat] (w, r, o, m), counters (16 ints)
 constexpr int kMaxStages = 4;   // K/V ring depth per stream (runtime, 2..4)
 constexpr int kMetaBytes = 2 * kQE * 16 + kQT * 32 + 2 * kMaxStages * 16 + kMaxPat * 16 + 64;
@@ -108,7 +111,7 @@ struct SmemLayout {
   int slot_o;  // n_pat x 128 parked rows (input format)
   int slot_l;  // n_pat x 128 parked lse (fp32, log2 domain)
   int stats;   // [stream][O buffer][use parity][row] (m, l)
-  int meta;    // element queues, tile queue, stage descriptors, pattern table, counters
+  int meta;    // tile queues, stage descriptors, pattern table, counters
   int walker;  // the TMA thread's block-sequence state (kept out of local memory)
   int bars;
   int misc;
@@ -1509,44 +1512,64 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     // greedily (LPT).  The longest ranges may also be split in halves when a
     // simulation of that greedy assignment over the SMs (with a per-unit
     // overhead) says the last SM finishes earlier.
-    const int64_t R = P.range_len, N = pb.N, BH = pb.B * pb.H;
-    std::vector<int64_t> cost(P.n_ranges);
-    for (int i = 0; i < P.n_ranges; ++i) cost[i] = range_cost(pb, i * R, std::min<int64_t>(N, (i + 1) * R));
-    std::vector<int> idx(P.n_ranges);
-    std::iota(idx.begin(), idx.end(), 0);
-    std::stable_sort(idx.begin(), idx.end(), [&](int a, int c) { return cost[a] > cost[c]; });
+    // Scratch in static storage (the library allocates nothing); callers
+    // serialise (the launcher holds its lock; the host tests are single
+    // threaded).
     struct Unit {
       int64_t cost;
       int code;
     };
-    auto units_for = [&](int k) {
-      std::vector<Unit> u;
+    static int64_t cost[kMaxRangeOrder];
+    static int idx[kMaxRangeOrder];
+    static Unit u[kMaxRangeOrder + 8];
+    static int64_t heap[kMaxHeapSms];
+    const int64_t R = P.range_len, N = pb.N, BH = pb.B * pb.H;
+    for (int i = 0; i < P.n_ranges; ++i) {
+      cost[i] = range_cost(pb, i * R, std::min<int64_t>(N, (i + 1) * R));
+      idx[i] = i;
+    }
+    // longest first; equal costs in range order
+    std::sort(idx, idx + P.n_ranges, [&](int a, int c) { return cost[a] != cost[c] ? cost[a] > cost[c] : a < c; });
+    auto units_for = [&](int k) -> int {
+      int n = 0;
       for (int t = 0; t < P.n_ranges; ++t) {
         const int i = idx[t];
         if (t < k) {
           for (int hf = 0; hf < 2; ++hf) {
             const int64_t a = i * R + hf * (R / 2);
             if (a >= N) continue;
-            u.push_back({range_cost(pb, a, std::min<int64_t>(N, a + R / 2)), (i << 2) | (hf << 1) | 1});
+            u[n++] = {range_cost(pb, a, std::min<int64_t>(N, a + R / 2)), (i << 2) | (hf << 1) | 1};
           }
         } else {
-          u.push_back({cost[i], i << 2});
+          u[n++] = {cost[i], i << 2};
         }
       }
-      std::stable_sort(u.begin(), u.end(), [](const Unit& a, const Unit& c) { return a.cost > c.cost; });
-      return u;
+      std::sort(u, u + n, [](const Unit& a, const Unit& c) { return a.cost != c.cost ? a.cost > c.cost : a.code < c.code; });
+      return n;
     };
-    auto makespan = [&](const std::vector<Unit>& u) {
+    // Greedy assignment of the n units (each B*H times) to the SMs: each goes
+    // to the SM that frees first (a binary min-heap of finish times).
+    const int n_heap = std::min(n_sm, kMaxHeapSms);
+    auto makespan = [&](int n) {
       constexpr int64_t kUnitOverhead = 16;  // fill and drain, in 64-key blocks
-      std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
-      for (int i = 0; i < n_sm; ++i) sm.push(0);
+      for (int i = 0; i < n_heap; ++i) heap[i] = 0;
       int64_t end = 0;
-      for (const Unit& x : u)
+      for (int x = 0; x < n; ++x)
         for (int64_t j = 0; j < BH; ++j) {
-          const int64_t t = sm.top() + x.cost + kUnitOverhead;
-          sm.pop();
-          sm.push(t);
+          const int64_t t = heap[0] + u[x].cost + kUnitOverhead;
           end = std::max(end, t);
+          int pos = 0;  // replace the root and sift it down
+          for (;;) {
+            const int l = 2 * pos + 1, r = l + 1;
+            int m = pos;
+            int64_t vm = t;
+            if (l < n_heap && heap[l] < vm) { m = l; vm = heap[l]; }
+            if (r < n_heap && heap[r] < vm) { m = r; vm = heap[r]; }
+            if (m == pos) break;
+            heap[pos] = heap[m];
+            pos = m;
+          }
+          heap[pos] = t;
         }
       return end;
     };
@@ -1555,17 +1578,16 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     if (can_split) {
       int64_t best = makespan(units_for(0));
       for (int k = 1; k <= std::min(8, P.n_ranges); ++k) {
-        const std::vector<Unit> u = units_for(k);
-        if ((int64_t)u.size() > kMaxRangeOrder) break;
-        const int64_t m = makespan(u);
+        const int n = units_for(k);
+        if (n > kMaxRangeOrder) break;
+        const int64_t m = makespan(n);
         if (m * 100 < best * 99) {  // at least 1 % better
           best = m;
           best_k = k;
         }
       }
     }
-    const std::vector<Unit> u = units_for(best_k);
-    P.n_units = (int)u.size();
+    P.n_units = units_for(best_k);
     for (int t = 0; t < P.n_units; ++t) P.unit_code[t] = u[t].code;
   }
 }
@@ -1598,12 +1620,11 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return LONGNET_ERR_CUDA;
   static std::mutex mu;
-  static LaunchCache* cache[64] = {nullptr};  // per device; kept for the process
+  static LaunchCache cache[64];  // per device, static storage (nothing is allocated)
   std::lock_guard<std::mutex> lock(mu);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LONGNET_ERR_CUDA;
-  if (!cache[dev]) cache[dev] = new LaunchCache();
-  LaunchCache& c = *cache[dev];
+  LaunchCache& c = cache[dev];
   if (!c.valid || !same_shape(c.shape, pb)) {
     int n_sm = 148;
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);

@@ -12,6 +12,7 @@
 #include "tcgen05.cu"
 
 #include <cstdio>
+#include <vector>
 #include <map>
 #include <set>
 #include <tuple>
