@@ -236,7 +236,10 @@ def main():
 
     from sparse_long_sequence_attn_b200 import workloads as wlm
 
-    wl = wlm.WORKLOADS[args.workload]
+    if args.workload.startswith("sweep") and args.workload[5:].isdigit():
+        wl = wlm.sweep_workload(int(args.workload[5:]))  # one sweep size, e.g. sweep65536
+    else:
+        wl = wlm.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
     if args.sweep:
