@@ -196,3 +196,48 @@ def test_watchdog_timeout_is_reported_and_context_survives():
     q, k, v = wl.make_inputs(w)
     o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
     gh.compare_full(o, l, q, k, v, w.patterns, w.causal, torch.float32, "after_watchdog")
+
+
+def _random_config(seed):
+    """A seeded random problem: dtype, D, B, H, N, 1..5 patterns (w may or may
+    not divide N, r may exceed w), causal or full; sized for the oracle."""
+    g = np.random.default_rng(1000 + seed)
+    dtype = [torch.float32, torch.bfloat16, torch.float16][seed % 3]
+    D = 64 if (dtype != torch.float32 and g.random() < 0.8) else int(g.choice([16, 32, 64, 128]))
+    B, H = int(g.integers(1, 3)), int(g.integers(1, 7))
+    n_pat = int(g.integers(1, 6))
+    if g.random() < 0.3:  # one shared short segment (the small-segment shape)
+        W = int(g.choice([8, 16, 24, 32, 40, 48, 56, 64]))
+        N = W * int(g.integers(2, 24))
+        rs = [1] + [int(g.integers(2, 9)) for _ in range(n_pat - 1)]
+        pats = tuple((W, r) for r in rs)
+    else:
+        N = int(g.choice([256, 384, 512, 640, 768, 1024, 1536, 2048]))
+        if g.random() < 0.2:
+            N += int(g.integers(1, 64))  # partial last segments
+        pats = []
+        for _ in range(n_pat):
+            r = int(g.choice([1, 1, 2, 3, 4, 5, 8, 12]))
+            w = int(g.choice([64, 128, 192, 256, 512, 1024, 2048]))
+            pats.append((min(w, max(N // 2, 64)) if g.random() < 0.5 else w, r))
+        pats = tuple(pats)
+    causal = bool(g.random() < 0.7)
+    return dtype, D, B, H, N, pats, causal
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_configurations_every_family(seed):
+    """Seeded random shapes through AUTO and through every family that takes
+    them; a family that declines returns UNSUPPORTED."""
+    dtype, D, B, H, N, pats, causal = _random_config(seed)
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=7000 + seed)
+    label = f"seed{seed} {dtype} D{D} B{B} H{H} N{N} {pats} causal={causal}"
+    ro, rl = None, None
+    for impl in (bd.LONGNET_IMPL_AUTO, bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05, bd.LONGNET_IMPL_SMALLSEG):
+        try:
+            o, l = gh.run_cuda(q, k, v, pats, causal, impl)
+        except bd.LongNetError as e:
+            assert impl not in (bd.LONGNET_IMPL_AUTO, bd.LONGNET_IMPL_SIMT) and e.code == bd.LONGNET_ERR_UNSUPPORTED, \
+                f"{label}: impl {impl} -> {e}"
+            continue
+        gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{label} impl={impl}")
