@@ -101,13 +101,16 @@ constexpr int kInfoEnd = 16;
 // softmax tile queues [2][kQE], epilogue tile queue [kQT], stage descriptors [kMaxStages],
 // pattern table [kMaxPat] (w, r, o, m), counters (16 ints)
 constexpr int kMaxStages = 4;   // K/V ring depth per stream (runtime, 2..4)
+// Ring depths of the two streams for a total of T stages: stream 0 takes the
+// odd one, so the shared memory left by the pattern slots is used in halves.
+__host__ __device__ constexpr int ring_stages(int total, int g) { return g == 0 ? (total + 1) >> 1 : total >> 1; }
 constexpr int kMetaBytes = 2 * kQE * 16 + kQT * 32 + 2 * kMaxStages * 16 + kMaxPat * 16 + 64;
 constexpr int kWalkerBytes = 512;  // per stream
 
 // Shared-memory carve-up, sized at run time from the pattern count.
 struct SmemLayout {
   int q;       // 2 Q tiles (one per stream)
-  int kv;      // [stream][stages] x (K block, V block)
+  int kv;      // stream 0's ring, then stream 1's: stages x (K block, V block)
   int slot_o;  // n_pat x 128 parked rows (input format)
   int slot_l;  // n_pat x 128 parked lse (fp32, log2 domain)
   int stats;   // [stream][O buffer][use parity][row] (m, l)
@@ -116,12 +119,12 @@ struct SmemLayout {
   int bars;
   int misc;
   int total;
-  int stages;
-  __host__ __device__ void make(int n_pat, int n_stages) {
-    stages = n_stages;
+  int stages;  // both streams' ring stages together
+  __host__ __device__ void make(int n_pat, int total_stages) {
+    stages = total_stages;
     q = 0;
     kv = q + 2 * kTileBytes;
-    slot_o = kv + 2 * stages * 2 * kKVBytes;
+    slot_o = kv + stages * 2 * kKVBytes;
     slot_l = slot_o + n_pat * kTileBytes;
     stats = slot_l + n_pat * kBM * 4;
     meta = stats + 2 * 2 * 2 * kBM * 8;
@@ -131,10 +134,11 @@ struct SmemLayout {
     total = misc + 64;
   }
 };
-// Largest per-stream K/V ring that fits with n_pat slots (>= 2: a stream's MMA
-// issues the S of its next block before the PV of the current one).
+// Most K/V ring stages (both streams together) that fit with n_pat slots;
+// each stream needs at least 2 (its MMA issues the S of its next block before
+// the PV of the current one).
 inline int pick_stages(int n_pat) {
-  for (int st = kMaxStages; st >= 2; --st) {
+  for (int st = 2 * kMaxStages; st >= 4; --st) {
     SmemLayout L;
     L.make(n_pat, st);
     if (L.total + 1024 <= kSmemLimit) return st;
@@ -749,9 +753,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SmemLayout L;
   L.make(P.pb.n_pat, P.stages);
-  const int NS = P.stages;
   uint8_t* sQ = smem + L.q;
-  uint8_t* sKV = smem + L.kv;  // stream g, stage s at (g*NS + s)*16K: K, then V at +8K
+  uint8_t* sKV = smem + L.kv;  // stream g's stage s at (g ? stages of stream 0 : 0) + s, x 16K: K, then V at +8K
   uint8_t* sSlotO = smem + L.slot_o;
   float* sSlotL = reinterpret_cast<float*>(smem + L.slot_l);
   float2* sStats = reinterpret_cast<float2*>(smem + L.stats);
@@ -893,7 +896,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       FastSeq seq;
       seq.init(twp);
       Elem e;
-      uint8_t* ring = sKV + g * NS * 2 * kKVBytes;
+      const int NS = ring_stages(P.stages, g);
+      uint8_t* ring = sKV + (g ? ring_stages(P.stages, 0) : 0) * 2 * kKVBytes;
       uint64_t* kv_full = bar_kv_full + g * kMaxStages;
       uint64_t* kv_empty = bar_kv_empty + g * kMaxStages;
       ElemMeta* stage_meta = sStageMeta + g * kMaxStages;
@@ -1004,7 +1008,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
     const int g = warp >> 1;
     if (lane == 0) {
-      uint8_t* ring = sKV + g * NS * 2 * kKVBytes;
+      const int NS = ring_stages(P.stages, g);
+      uint8_t* ring = sKV + (g ? ring_stages(P.stages, 0) : 0) * 2 * kKVBytes;
       uint64_t* kv_full = bar_kv_full + g * kMaxStages;
       uint64_t* kv_empty = bar_kv_empty + g * kMaxStages;
       const ElemMeta* stage_meta = sStageMeta + g * kMaxStages;
@@ -1440,7 +1445,7 @@ bool tcgen05_supports(const Problem& p) {
   using namespace tc;
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
   static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
-  if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 2) return false;
+  if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 4) return false;
   if (p.H > 65535 || p.B > 65535) return false;
   // positions and their sums stay below 2^31 (32-bit tile arithmetic, TMA
   // coordinates, multiply-shift division)
