@@ -103,6 +103,31 @@ int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
                                   int causal, int dtype, int impl,
                                   longnet_stream_t stream);
 
+/* Options of longnet_dilated_attn_fwd_ex (a bit set). */
+enum longnet_flags {
+  /* Scale every q row and every k row (over D) to unit L2 norm before the
+   * scores: x / max(|x|, 1e-12), computed in fp32 (the small-segment kernel
+   * then rounds the rows back to the input format, the SIMT kernel keeps them
+   * in fp32).  The reading adopted for the qk_norm
+   * option of the DilatedAttention module ("LongNet" docs page, usage
+   * example).  The SIMT and small-segment kernels take it; the tcgen05 kernel
+   * does not (LONGNET_IMPL_AUTO falls back). */
+  LONGNET_FLAG_QK_NORM = 1
+};
+
+/*
+ * longnet_dilated_attn_fwd_ex — the forward with options (flags, a
+ * longnet_flags bit set) and an explicit kernel family (impl, as in
+ * longnet_dilated_attn_fwd_impl).  Unknown flag bits: LONGNET_ERR_INVALID_ARG.
+ * The two entry points above are this call with flags = 0.
+ */
+int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
+                                void* out, float* lse,
+                                int64_t B, int64_t N, int64_t H, int64_t D,
+                                int n_pat, const int64_t* w, const int64_t* r,
+                                int causal, int dtype, int flags, int impl,
+                                longnet_stream_t stream);
+
 /*
  * longnet_select_impl — which family AUTO would run for these arguments
  * (a longnet_impl >= 1), or a negative longnet_status when the arguments

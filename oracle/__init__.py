@@ -9,5 +9,6 @@ from .oracle import (  # noqa: F401
     dilated_attn_fp64,
     dilated_attn_rows_fp64,
     num_threads,
+    qk_normalize_fp64,
 )
 from .brute import dilated_attn_bruteforce  # noqa: F401

@@ -64,13 +64,27 @@ def _ptr(a: np.ndarray, t=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(t))
 
 
-def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None):
+def qk_normalize_fp64(x) -> np.ndarray:
+    """Rows of x [B, N, H, D] scaled to unit L2 norm over D, x / max(|x|, 1e-12)
+    (a zero row stays zero), in fp64.  The reading adopted for the qk_norm
+    option of the DilatedAttention module ("LongNet" docs page, usage example):
+    the option is named there, not defined; L2 normalisation of every query and
+    key row is the plainest reading."""
+    x = _f64(x)
+    n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+    return x / np.maximum(n, 1e-12)
+
+
+def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None, qk_norm=False):
     """Full fp64 forward.  q, k, v: [B, N, H, D].  patterns: [(w, r), ...].
+    qk_norm: normalise q and k rows first (qk_normalize_fp64).
 
     Returns (out [B, N, H, D] float64, lse [B, H, N] float64).
     """
     lib = lib or load_library()
     q, k, v = _f64(q), _f64(k), _f64(v)
+    if qk_norm:
+        q, k = qk_normalize_fp64(q), qk_normalize_fp64(k)
     B, N, H, D = q.shape
     w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)
     r = np.ascontiguousarray([p[1] for p in patterns], dtype=np.int64)
@@ -84,13 +98,15 @@ def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None):
     return out, lse
 
 
-def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None):
+def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None, qk_norm=False):
     """fp64 forward of selected rows only.  rows_bph: int array [n, 3] of (b, pos, h).
 
     Returns (out_rows [n, D], lse_rows [n]).
     """
     lib = lib or load_library()
     q, k, v = _f64(q), _f64(k), _f64(v)
+    if qk_norm:
+        q, k = qk_normalize_fp64(q), qk_normalize_fp64(k)
     B, N, H, D = q.shape
     rows = np.ascontiguousarray(np.asarray(rows_bph, dtype=np.int64).reshape(-1, 3))
     w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)

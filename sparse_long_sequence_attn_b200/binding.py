@@ -28,6 +28,7 @@ LONGNET_MAX_PATTERNS = 16
 LONGNET_DTYPE_F32 = 0
 LONGNET_DTYPE_BF16 = 1
 LONGNET_DTYPE_F16 = 2
+LONGNET_FLAG_QK_NORM = 1
 
 LONGNET_IMPL_AUTO = 0
 LONGNET_IMPL_SIMT = 1
@@ -46,6 +47,10 @@ SIGNATURES = {
                                                      _i64, ctypes.c_int, _i64p, _i64p,
                                                      ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                      _vp]),
+    "longnet_dilated_attn_fwd_ex": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                   _i64, ctypes.c_int, _i64p, _i64p,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, _vp]),
     "longnet_select_impl": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
                                            ctypes.c_int, ctypes.c_int]),
     "longnet_last_device_status": (ctypes.c_int, [_vp]),
@@ -114,11 +119,12 @@ def _stream_handle(stream) -> int | None:
 def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              out: torch.Tensor, lse: torch.Tensor | None,
                              patterns: Sequence[Tuple[int, int]], causal: bool = True,
-                             impl: int = LONGNET_IMPL_AUTO, stream=None) -> None:
+                             impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False) -> None:
     """Enqueue the forward on `stream` (default: torch's current stream).
 
     q, k, v, out: contiguous CUDA tensors [B, N, H, D] of one dtype (fp32/bf16/fp16);
-    lse: contiguous fp32 [B, H, N] or None.  Raises LongNetError on a non-zero
+    lse: contiguous fp32 [B, H, N] or None.  qk_norm: scale q and k rows to unit
+    L2 norm first (LONGNET_FLAG_QK_NORM).  Raises LongNetError on a non-zero
     status.
     """
     lib = load_library()
@@ -134,22 +140,23 @@ def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if lse is not None and tuple(lse.shape) != (B, H, N):
         raise ValueError("lse must be [B, H, N]")
     n, w, r = _patterns(patterns)
-    rc = lib.longnet_dilated_attn_fwd_impl(
+    rc = lib.longnet_dilated_attn_fwd_ex(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
         None if lse is None else lse.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
-        _dtype_code(q), int(impl), _stream_handle(stream))
+        _dtype_code(q), LONGNET_FLAG_QK_NORM if qk_norm else 0, int(impl), _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_fwd")
 
 
 def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  patterns: Sequence[Tuple[int, int]], causal: bool = True,
-                 impl: int = LONGNET_IMPL_AUTO, want_lse: bool = True, stream=None):
+                 impl: int = LONGNET_IMPL_AUTO, want_lse: bool = True, stream=None,
+                 qk_norm: bool = False):
     """Allocate out (and lse) with torch and run the forward.  Returns (out, lse)."""
     B, N, H, D = q.shape
     out = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if want_lse else None
-    longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream)
+    longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream, qk_norm)
     return out, lse
 
 

@@ -131,15 +131,17 @@ __global__ void watchdog_selftest_kernel(int* status, uint64_t limit_ns) {
 
 using namespace longnet;
 
-extern "C" int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
-                                             void* out, float* lse, int64_t B, int64_t N,
-                                             int64_t H, int64_t D, int n_pat, const int64_t* w,
-                                             const int64_t* r, int causal, int dtype, int impl,
-                                             longnet_stream_t stream) {
+extern "C" int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
+                                           void* out, float* lse, int64_t B, int64_t N, int64_t H,
+                                           int64_t D, int n_pat, const int64_t* w, const int64_t* r,
+                                           int causal, int dtype, int flags, int impl,
+                                           longnet_stream_t stream) {
   if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
   int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
   if (rc) return rc;
+  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
   int dev = 0;
   rc = current_device_state(&dev, &pb.status);
   if (rc) return rc;
@@ -161,6 +163,15 @@ extern "C" int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const
     default:
       return LONGNET_ERR_INVALID_ARG;
   }
+}
+
+extern "C" int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
+                                             void* out, float* lse, int64_t B, int64_t N,
+                                             int64_t H, int64_t D, int n_pat, const int64_t* w,
+                                             const int64_t* r, int causal, int dtype, int impl,
+                                             longnet_stream_t stream) {
+  return longnet_dilated_attn_fwd_ex(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, 0,
+                                     impl, stream);
 }
 
 extern "C" int longnet_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out,

@@ -19,6 +19,7 @@ struct Problem {
   int n_pat;
   int causal;
   int dtype;
+  int qk_norm;  // 1: q and k rows are scaled to unit L2 norm first (LONGNET_FLAG_QK_NORM)
   int64_t w[LONGNET_MAX_PATTERNS];
   int64_t r[LONGNET_MAX_PATTERNS];
   int* status;  // device address of this device's status word

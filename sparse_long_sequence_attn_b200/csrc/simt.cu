@@ -52,6 +52,20 @@ __device__ __forceinline__ float dot_row(const float* qs, const T* krow) {
   return s;
 }
 
+// The same, also returning the key row's squared norm.
+template <typename T, int D>
+__device__ __forceinline__ float dot_row_norm(const float* qs, const T* krow, float& kk) {
+  float s = 0.f, n = 0.f;
+#pragma unroll 16
+  for (int d = 0; d < D; ++d) {
+    const float x = load_elem(krow + d);
+    s = fmaf(qs[d], x, s);
+    n = fmaf(x, x, n);
+  }
+  kk = n;
+  return s;
+}
+
 // One warp per (b, pos, h).  Lane l owns output dims l, l+32, ... (E of them);
 // within a block of 32 keys lane l scores key l, then the block's
 // probabilities are broadcast to accumulate V.
@@ -75,6 +89,15 @@ __global__ void __launch_bounds__(kWarps * 32) simt_kernel(const Problem p) {
 
   for (int d = lane; d < D; d += 32) qsh[warp][d] = load_elem(Q + base_b + pos * HD + h * D + d);
   __syncwarp();
+  if (p.qk_norm) {
+    // q / max(|q|, 1e-12) in fp32; each key row is scaled the same way below
+    float ss = 0.f;
+    for (int d = lane; d < D; d += 32) ss = fmaf(qsh[warp][d], qsh[warp][d], ss);
+    const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
+    __syncwarp();
+    for (int d = lane; d < D; d += 32) qsh[warp][d] *= inv;
+    __syncwarp();
+  }
 
   const float scale = rsqrtf((float)D);
   float m_run = -INFINITY, l_run = 0.f;
@@ -99,7 +122,13 @@ __global__ void __launch_bounds__(kWarps * 32) simt_kernel(const Problem p) {
       float s = -INFINITY;
       if (j < n_keys) {
         const int64_t kp = first + r * j;
-        s = dot_row<T, D>(qsh[warp], K + base_b + kp * HD + h * D) * scale;
+        if (p.qk_norm) {
+          float kk;
+          s = dot_row_norm<T, D>(qsh[warp], K + base_b + kp * HD + h * D, kk);
+          s *= scale / fmaxf(sqrtf(kk), 1e-12f);
+        } else {
+          s = dot_row<T, D>(qsh[warp], K + base_b + kp * HD + h * D) * scale;
+        }
       }
       const float m_new = fmaxf(m_run, warp_max(s));
       const float corr = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);

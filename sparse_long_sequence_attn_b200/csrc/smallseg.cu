@@ -359,6 +359,40 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
       record_status(P.pb.status, kStatusTimeout);
       return;
     }
+    if (P.pb.qk_norm) {
+      // q and k rows to unit L2 norm (x / max(|x|, 1e-12), fp32), rounded back
+      // to the input format in place; the pair splits the 2W rows
+      for (int rr = wsub * 32 + lane; rr < 2 * W; rr += 64) {
+        uint8_t* tile = rr < W ? sQ : sK;
+        const int row = rr < W ? rr : rr - W;
+        uint4 u[8];
+        float ss = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          u[ch] = *reinterpret_cast<const uint4*>(tile + sw_addr(0, row, ch));
+          const uint32_t wv[4] = {u[ch].x, u[ch].y, u[ch].z, u[ch].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float lo, hi;
+            unpack2<kFmt>(wv[e], lo, hi);
+            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+          }
+        }
+        const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t wv[4] = {u[ch].x, u[ch].y, u[ch].z, u[ch].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float lo, hi;
+            unpack2<kFmt>(wv[e], lo, hi);
+            wv[e] = pack2<kFmt>(lo * inv, hi * inv);
+          }
+          *reinterpret_cast<uint4*>(tile + sw_addr(0, row, ch)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+      if (!pair_sync()) return;  // every row is normalised before any is read
+    }
 
     bool ok = true;
     for (int pi = 0; pi < n_pat; ++pi) {
@@ -446,6 +480,9 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
       }
     }
     if (!ok) return;
+    // rows this thread wrote with ordinary stores (normalised q and k, staged
+    // output) may next be overwritten by the async proxy (the next item's TMA)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     // ---- coalesced store of the rows this warp staged (its 16-row chunks):
     // 16-byte chunks, 8 per row
     __syncwarp();

@@ -1444,6 +1444,7 @@ int64_t range_cost(const Problem& pb, int64_t A, int64_t Bnd) {
 bool tcgen05_supports(const Problem& p) {
   using namespace tc;
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
+  if (p.qk_norm) return false;  // no normalisation pass on this path
   static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
   if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 4) return false;
   if (p.H > 65535 || p.B > 65535) return false;

@@ -20,7 +20,7 @@ TOL_LSE = 1e-3
 GUARD = 4096  # elements of NaN guard band on each side of every output
 
 
-def run_cuda(q, k, v, patterns, causal, impl, want_lse=True, stream=None):
+def run_cuda(q, k, v, patterns, causal, impl, want_lse=True, stream=None, qk_norm=False):
     """Copy inputs to cuda:0, run the forward into guarded NaN-filled buffers,
     check the guards and the device status word, return CPU (out, lse)."""
     dev = torch.device("cuda:0")
@@ -31,7 +31,7 @@ def run_cuda(q, k, v, patterns, causal, impl, want_lse=True, stream=None):
     out = obuf[GUARD:GUARD + n_out].view(B, N, H, D)
     lbuf = torch.full((B * H * N + 2 * GUARD,), float("nan"), dtype=torch.float32, device=dev)
     lse = lbuf[GUARD:GUARD + B * H * N].view(B, H, N) if want_lse else None
-    bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, patterns, causal, impl, stream)
+    bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, patterns, causal, impl, stream, qk_norm)
     st = bd.longnet_last_device_status(stream)
     assert st == 0, f"device status word: {bd.status_string(st)}"
     assert torch.isnan(obuf[:GUARD].float()).all() and torch.isnan(obuf[-GUARD:].float()).all(), \
@@ -45,8 +45,8 @@ def run_cuda(q, k, v, patterns, causal, impl, want_lse=True, stream=None):
     return o, l
 
 
-def compare_full(o, l, q, k, v, patterns, causal, dtype, label="", tol_out=None):
-    ro, rl = oracle.dilated_attn_fp64(q, k, v, patterns, causal)
+def compare_full(o, l, q, k, v, patterns, causal, dtype, label="", tol_out=None, qk_norm=False):
+    ro, rl = oracle.dilated_attn_fp64(q, k, v, patterns, causal, qk_norm=qk_norm)
     err = float(np.abs(o - ro).max())
     tol = TOL_OUT[dtype] if tol_out is None else tol_out
     assert err <= tol, f"{label}: max|out - oracle| = {err} (tolerance {tol})"

@@ -280,8 +280,42 @@ def check_rows_function_direct(lib):
         assert abs(lrow[t] - math.log(len(keys))) < 1e-14
 
 
+def check_qk_norm(lib):
+    """qk_norm: rows are scaled to unit L2 norm (torch's F.normalize in fp64 on
+    the same rows, a zero row stays zero); attention with qk_norm equals plain
+    attention on rows normalised by F.normalize; and it does not change when
+    every q and k row is scaled by its own positive factor."""
+    B, N, H, D = 1, 48, 3, 8
+    q, k, v = (_rand((B, N, H, D), s) for s in (61, 62, 63))
+    q[0, 5, 1] = 0.0  # a zero row
+    nq = orc.qk_normalize_fp64(q)
+    ref = F.normalize(torch.from_numpy(q), dim=-1, eps=1e-12).numpy()
+    np.testing.assert_allclose(nq, ref, atol=1e-15, rtol=0)
+    norms = np.linalg.norm(nq, axis=-1)
+    assert np.allclose(np.delete(norms.reshape(-1), 5 * H + 1), 1.0, atol=1e-14, rtol=0)
+    assert not nq[0, 5, 1].any()
+    pats = [(12, 1), (24, 3), (48, 5)]
+    for causal in (True, False):
+        o1, l1 = orc.dilated_attn_fp64(q, k, v, pats, causal=causal, lib=lib, qk_norm=True)
+        qn = F.normalize(torch.from_numpy(q), dim=-1, eps=1e-12).numpy()
+        kn = F.normalize(torch.from_numpy(k), dim=-1, eps=1e-12).numpy()
+        o2, l2 = orc.dilated_attn_fp64(qn, kn, v, pats, causal=causal, lib=lib)
+        np.testing.assert_allclose(o1, o2, atol=1e-13, rtol=0)
+        np.testing.assert_allclose(l1, l2, atol=1e-13, rtol=0)
+        g = np.random.default_rng(64)
+        cq = g.uniform(0.1, 10.0, size=(B, N, H, 1))
+        ck = g.uniform(0.1, 10.0, size=(B, N, H, 1))
+        o3, l3 = orc.dilated_attn_fp64(q * cq, k * ck, v, pats, causal=causal, lib=lib, qk_norm=True)
+        np.testing.assert_allclose(o3, o1, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(l3, l1, atol=1e-12, rtol=0)
+        # without the option the scaled rows give another result
+        o4, _ = orc.dilated_attn_fp64(q * cq, k * ck, v, pats, causal=causal, lib=lib)
+        assert np.abs(o4 - o1).max() > 1e-3
+
+
 ALL_CHECKS = [
     check_rows_function_direct,
+    check_qk_norm,
     check_dense_causal,
     check_dense_noncausal,
     check_block_diagonal,

@@ -56,6 +56,17 @@ def test_invalid_arguments_rejected_on_host(kw):
     assert rc == bd.LONGNET_ERR_INVALID_ARG, rc
 
 
+def test_unknown_flag_bits_rejected_on_host():
+    lib = bd.load_library()
+    buf = ctypes.c_void_p(0x1000)
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+    for flags in (2, 4, -1):
+        rc = lib.longnet_dilated_attn_fwd_ex(buf, buf, buf, buf, None, 1, 64, 2, 16, 1, w, r, 1, 0,
+                                             flags, 0, None)
+        assert rc == bd.LONGNET_ERR_INVALID_ARG, (flags, rc)
+
+
 def test_null_and_misaligned_pointers():
     lib = bd.load_library()
     assert _call(lib, ptr=ctypes.c_void_p(0)) == bd.LONGNET_ERR_INVALID_ARG
