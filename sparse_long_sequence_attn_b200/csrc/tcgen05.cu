@@ -913,6 +913,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 pt = sPat[t.p];  // (w, r, o, m)
         const int seg_base = t.seg * pt.x + pt.z;
         const int info = g | (e.ob << 1) | ((e.use & 1) << 2) | ((e.use > 0) << 3);
+        ElemMeta em;
+        em.info = info;
+        em.j = e.j;
+        em.nkv = t.nkv;
+        em.lim0 = causal ? t.k0 : pt.w - 1;
         if (e.j == 0) {
           ok = wait_count(cnt_epi, e.tile_idx - kQT);  // tile queue entry is free
           if (!ok) break;
@@ -922,6 +927,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tm.start = t.start;
           tm.nrows = t.nrows;
           st_release(&tm.seq, e.tile_idx);
+          // the softmax warps take one descriptor per tile; it goes out before
+          // the wait for the Q buffer, which it does not depend on
+          ok = wait_count(cnt_soft + g, ne - kQE);  // queue has room
+          if (!ok) break;
+          sElemQ[g * kQE + (ne & (kQE - 1))] = em;
+          st_release(cnt_elem + g, ++ne);
           if (qc > 0) ok = sy.wait(bar_q_empty + g, (qc - 1) & 1);
           if (!ok) break;
           const TmaCoord c = tma_coord(P, ri, seg_base + pt.y * t.k0, t.nrows);
@@ -929,18 +940,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_5d(sQ + g * kTileBytes, &maps.m[ri][c.map][0], bar_q_full + g, 0, (int)h, c.c, c.kk,
                       (int)b);
           ++qc;
-        }
-        ElemMeta em;
-        em.info = info;
-        em.j = e.j;
-        em.nkv = t.nkv;
-        em.lim0 = causal ? t.k0 : pt.w - 1;
-        if (e.j == 0) {
-          // the softmax warps take one descriptor per tile
-          ok = wait_count(cnt_soft + g, ne - kQE);  // queue has room
-          if (!ok) break;
-          sElemQ[g * kQE + (ne & (kQE - 1))] = em;
-          st_release(cnt_elem + g, ++ne);
         }
         if (kv_it >= (uint32_t)NS) ok = sy.wait(kv_empty + st, st_par ^ 1);
         if (!ok) break;
