@@ -47,12 +47,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources a kernel family's device code is built from: its own file and
+# the shared headers.  A change anywhere else leaves its counters valid.
+_FAMILY_SOURCES = ("device_util.cuh", "params.h")
+
+
+def kernel_source_hash(family: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_long_sequence_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in (f"{family}.cu",) + _FAMILY_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    with open(os.path.join(ROOT, "include", "longnet.h"), "rb") as f:
+        h.update(b"longnet.h" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -65,7 +72,7 @@ def traffic_from_profiles(workload: str, impl_name: str):
     with open(path) as f:
         d = json.load(f)
     ent = d.get(f"{impl_name}:{workload}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(impl_name):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -6,6 +6,8 @@ no code with the CUDA library (see oracle.c for the method it restates).
 """
 from .oracle import (  # noqa: F401
     build_oracle,
+    dilated_attn_bwd_fp64,
+    dilated_attn_bwd_rows_fp64,
     dilated_attn_fp64,
     dilated_attn_rows_fp64,
     num_threads,

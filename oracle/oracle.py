@@ -42,6 +42,13 @@ def load_library(path: str | None = None):
     lib.oracle_dilated_attn_rows_fp64.argtypes = [dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
                                                   ip, ip, ctypes.c_int, i64, ip, dp, dp]
     lib.oracle_dilated_attn_rows_fp64.restype = ctypes.c_int
+    lib.oracle_dilated_attn_bwd_fp64.argtypes = [dp, dp, dp, dp, dp, dp, dp, i64, i64, i64, i64,
+                                                 ctypes.c_int, ip, ip, ctypes.c_int]
+    lib.oracle_dilated_attn_bwd_fp64.restype = ctypes.c_int
+    lib.oracle_dilated_attn_bwd_rows_fp64.argtypes = [dp, dp, dp, dp, i64, i64, i64, i64,
+                                                      ctypes.c_int, ip, ip, ctypes.c_int, i64, ip,
+                                                      dp, dp, dp]
+    lib.oracle_dilated_attn_bwd_rows_fp64.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -120,6 +127,52 @@ def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None, q
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (code {rc})")
     return out, lse
+
+
+def _patterns(patterns):
+    w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)
+    r = np.ascontiguousarray([p[1] for p in patterns], dtype=np.int64)
+    return w, r
+
+
+def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None):
+    """Full fp64 backward: the gradients of sum(dout * out) with respect to
+    q, k and v, where out is the forward's output.  All tensors [B, N, H, D].
+
+    Returns (dq, dk, dv) as float64 arrays.
+    """
+    lib = lib or load_library()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, H, D = q.shape
+    w, r = _patterns(patterns)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = lib.oracle_dilated_attn_bwd_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
+                                          _ptr(dk), _ptr(dv), B, N, H, D, len(patterns),
+                                          _ptr(w, ctypes.c_int64), _ptr(r, ctypes.c_int64),
+                                          int(bool(causal)))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return dq, dk, dv
+
+
+def dilated_attn_bwd_rows_fp64(q, k, v, dout, patterns, rows_bph, causal=True, lib=None):
+    """fp64 backward of selected rows only.  rows_bph: int array [n, 3] of
+    (b, pos, h).  Returns (dq_rows, dk_rows, dv_rows), each [n, D]."""
+    lib = lib or load_library()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, H, D = q.shape
+    rows = np.ascontiguousarray(np.asarray(rows_bph, dtype=np.int64).reshape(-1, 3))
+    w, r = _patterns(patterns)
+    n = rows.shape[0]
+    dq, dk, dv = (np.empty((n, D), dtype=np.float64) for _ in range(3))
+    rc = lib.oracle_dilated_attn_bwd_rows_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, N, H, D,
+                                               len(patterns), _ptr(w, ctypes.c_int64),
+                                               _ptr(r, ctypes.c_int64), int(bool(causal)), n,
+                                               _ptr(rows, ctypes.c_int64), _ptr(dq), _ptr(dk),
+                                               _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (code {rc})")
+    return dq, dk, dv
 
 
 def num_threads(lib=None) -> int:

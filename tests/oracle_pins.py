@@ -313,6 +313,145 @@ def check_qk_norm(lib):
         assert np.abs(o4 - o1).max() > 1e-3
 
 
+# ---------------------------------------------------------------- backward
+
+
+def _brute_autograd(q, k, v, dout, patterns, causal):
+    """Gradients of sum(dout * out) by torch autograd through the multiset
+    formulation of brute.py: one softmax per row over the (pattern, key) pairs
+    that reach it, written as a dense masked softmax in which a key reached
+    c times gets the logit s + log c.  A different formulation from the
+    oracle's, differentiated by the library."""
+    from oracle.brute import keys_reaching
+
+    B, N, H, D = q.shape
+    tq, tk, tv = (torch.from_numpy(np.array(x)).requires_grad_(True) for x in (q, k, v))
+    bias = np.full((H, N, N), -math.inf)
+    for h in range(H):
+        for pos in range(N):
+            keys = keys_reaching(pos, h, patterns, causal, N)
+            cnt = np.bincount(keys, minlength=N) if keys else np.zeros(N)
+            nz = cnt > 0
+            bias[h, pos, nz] = np.log(cnt[nz])
+    tb = torch.from_numpy(bias)
+    rows_out = []
+    for b in range(B):
+        per_h = []
+        for h in range(H):
+            s = tq[b, :, h] @ tk[b, :, h].T / math.sqrt(D) + tb[h]
+            kept = torch.isfinite(tb[h]).any(dim=-1)
+            p = torch.softmax(torch.where(kept[:, None], s, torch.zeros_like(s)), dim=-1)
+            o = (p @ tv[b, :, h]) * kept[:, None]
+            per_h.append(o)
+        rows_out.append(torch.stack(per_h, dim=1))
+    outs = torch.stack(rows_out, dim=0)
+    (outs * torch.from_numpy(np.array(dout))).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def check_bwd_dense_autograd(lib):
+    """One pattern with w = N, r = 1 is ordinary softmax attention: its
+    gradients equal torch autograd through scaled_dot_product_attention in
+    fp64, causal and not."""
+    B, N, H, D = 1, 40, 2, 8
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (81, 82, 83, 84))
+    for causal in (True, False):
+        dq, dk, dv = orc.dilated_attn_bwd_fp64(q, k, v, do, [(N, 1)], causal=causal, lib=lib)
+        for h in range(H):
+            tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x[0, :, h]))[None, None]
+                          .requires_grad_(True) for x in (q, k, v))
+            o = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+            (o[0, 0] * torch.from_numpy(np.ascontiguousarray(do[0, :, h]))).sum().backward()
+            np.testing.assert_allclose(dq[0, :, h], tq.grad[0, 0].numpy(), atol=1e-12, rtol=0)
+            np.testing.assert_allclose(dk[0, :, h], tk.grad[0, 0].numpy(), atol=1e-12, rtol=0)
+            np.testing.assert_allclose(dv[0, :, h], tv.grad[0, 0].numpy(), atol=1e-12, rtol=0)
+
+
+def check_bwd_bruteforce_autograd(lib):
+    """Several overlapping patterns (rows reached by 1..3 patterns, r not
+    dividing w, partial last segments, w > N, a duplicated pattern): the
+    oracle's gradients equal torch autograd through the multiset-softmax
+    formulation."""
+    cases = [
+        (1, 36, 5, 4, [(12, 5), (18, 3), (36, 7)], True, 91),
+        (2, 26, 4, 4, [(8, 2), (11, 3), (26, 1)], False, 92),
+        (1, 34, 3, 4, [(12, 1), (8, 3), (40, 5)], True, 93),
+        (1, 32, 2, 8, [(16, 1), (16, 1)], True, 94),
+        (1, 24, 4, 5, [(12, 3), (24, 4)], True, 95),  # rows kept by no pattern
+    ]
+    for (B, N, H, D, pats, causal, seed) in cases:
+        q, k, v, do = (_rand((B, N, H, D), seed + 100 * i) for i in range(4))
+        got = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib)
+        ref = _brute_autograd(q, k, v, do, pats, causal)
+        for g, r_ in zip(got, ref):
+            np.testing.assert_allclose(g, r_, atol=1e-12, rtol=0)
+
+
+def check_bwd_finite_differences(lib):
+    """Central differences of the oracle's own forward, sum(dout * out), on a
+    handful of coordinates of q, k and v: the backward is the forward's
+    derivative."""
+    B, N, H, D = 1, 30, 3, 4
+    pats = [(10, 1), (15, 2), (30, 4)]
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (101, 102, 103, 104))
+    eps = 1e-5
+    for causal in (True, False):
+        grads = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib)
+        g = np.random.default_rng(105)
+        for which in range(3):
+            for _ in range(6):
+                idx = (0, int(g.integers(N)), int(g.integers(H)), int(g.integers(D)))
+                vals = []
+                for sgn in (1.0, -1.0):
+                    args = [q.copy(), k.copy(), v.copy()]
+                    args[which][idx] += sgn * eps
+                    o, _ = orc.dilated_attn_fp64(*args, pats, causal=causal, lib=lib)
+                    vals.append(float((o * do).sum()))
+                fd = (vals[0] - vals[1]) / (2 * eps)
+                assert abs(fd - grads[which][idx]) < 1e-7 * max(1.0, abs(fd)), (which, idx)
+
+
+def check_bwd_invariants(lib):
+    """Each row's probabilities sum to one over its pairs, so per (b, h) the
+    dv rows add up to the sum of dout over the rows some pattern keeps; the
+    score cotangents of a row sum to zero, so the dk rows add up to zero; a
+    row kept by no pattern gets dq = dk = dv = 0; scaling dout scales every
+    gradient."""
+    B, N, H, D = 2, 24, 4, 5
+    pats = [(12, 3), (24, 4)]
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (111, 112, 113, 114))
+    for causal in (True, False):
+        dq, dk, dv = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib)
+        _, lse = orc.dilated_attn_fp64(q, k, v, pats, causal=causal, lib=lib)
+        kept = np.isfinite(lse).transpose(0, 2, 1)  # [B, N, H]
+        assert (~kept).any()
+        np.testing.assert_allclose(dv.sum(axis=1), (do * kept[..., None]).sum(axis=1),
+                                   atol=1e-12, rtol=0)
+        np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12, rtol=0)
+        for g_ in (dq, dk, dv):
+            assert not g_[~kept].any()
+        d2 = orc.dilated_attn_bwd_fp64(q, k, v, 2.5 * do, pats, causal=causal, lib=lib)
+        for a_, b_ in zip(d2, (dq, dk, dv)):
+            np.testing.assert_allclose(a_, 2.5 * b_, atol=1e-12, rtol=0)
+
+
+def check_bwd_rows_function(lib):
+    """The per-row backward returns the full backward's rows, and on its own
+    agrees with autograd through the multiset formulation."""
+    B, N, H, D = 2, 36, 3, 4
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (121, 122, 123, 124))
+    pats = [(12, 1), (18, 4), (40, 5)]
+    rows = [(b, pos, h) for b in range(B) for pos in range(0, N, 5) for h in range(H)]
+    for causal in (True, False):
+        full = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib)
+        got = orc.dilated_attn_bwd_rows_fp64(q, k, v, do, pats, rows, causal=causal, lib=lib)
+        ref = _brute_autograd(q, k, v, do, pats, causal)
+        for t, (b, pos, h) in enumerate(rows):
+            for which in range(3):
+                np.testing.assert_allclose(got[which][t], full[which][b, pos, h], atol=1e-13, rtol=0)
+                np.testing.assert_allclose(got[which][t], ref[which][b, pos, h], atol=1e-12, rtol=0)
+
+
 ALL_CHECKS = [
     check_rows_function_direct,
     check_qk_norm,
@@ -326,4 +465,9 @@ ALL_CHECKS = [
     check_invariants,
     check_uncovered_rows,
     check_rows_function,
+    check_bwd_dense_autograd,
+    check_bwd_bruteforce_autograd,
+    check_bwd_finite_differences,
+    check_bwd_invariants,
+    check_bwd_rows_function,
 ]

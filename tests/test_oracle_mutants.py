@@ -31,6 +31,22 @@ MUTANTS = [
      "const int64_t pos = seg * w[p] + o + i;\n          const int64_t src"),
     ("v_from_query_row", "acc += scores[j] * vs[j * D + d];", "acc += scores[j] * vs[i * D + d];"),
     ("merge_lse_no_log", "*lse = mx + log(wsum);", "*lse = mx + wsum;"),
+    # backward: a dropped term, a wrong operand, a missing weight, a sign, a bound
+    ("bwd_no_delta", "const double ds = pij * (dp - delta + dls[i]);",
+     "const double ds = pij * (dp + dls[i]);"),
+    ("bwd_no_dlse", "const double ds = pij * (dp - delta + dls[i]);",
+     "const double ds = pij * (dp - delta);"),
+    ("bwd_dk_from_k", "dks[j * D + d] += scale * ds * qs[i * D + d];",
+     "dks[j * D + d] += scale * ds * ks[i * D + d];"),
+    ("bwd_dv_without_prob", "dvs[j * D + d] += pij * dos[i * D + d];",
+     "dvs[j * D + d] += dos[i * D + d];"),
+    ("bwd_unweighted_cotangent", "do_p[p][d] = a * dout[d];", "do_p[p][d] = dout[d];"),
+    ("bwd_combine_sign", "dot += dout[d] * (o_p[p][d] - out[d]);",
+     "dot += dout[d] * (out[d] - o_p[p][d]);"),
+    ("bwd_rows_causal_start", "for (int64_t i = causal ? j : 0; i < m; ++i) {",
+     "for (int64_t i = causal ? j + 1 : 0; i < m; ++i) {"),
+    ("bwd_rows_dq_scale", "for (int64_t d = 0; d < D; ++d) dq_r[d] += scale * ds * kj[d];",
+     "for (int64_t d = 0; d < D; ++d) dq_r[d] += ds * kj[d];"),
 ]
 
 
