@@ -34,8 +34,11 @@ if ROOT not in sys.path:
 
 METRIC = "Dilated-attn fwd tokens/s @32K, 5 patterns; % of bf16 tensor-core peak"
 UNIT = "tokens/s"
+METRIC_BWD = "Dilated-attn bwd (dq, dk, dv) tokens/s; % of fp32 ALU peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_BF16_TFLOPS = 2250.0
+# fp32 FMA peak: 148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz (clocks.max.sm)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def load_peaks():
@@ -237,6 +240,8 @@ def main():
                     help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="linear-scaling sweep instead")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=("fwd", "bwd"),
+                    help="fwd: the forward (default); bwd: the backward (dq, dk, dv)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -248,9 +253,13 @@ def main():
     else:
         wl = wlm.WORKLOADS[args.workload]
     if args.impl == "reference":
+        if args.pass_ == "bwd":
+            return run_reference_bwd(args, wl)
         return run_reference(args, wl)
     if args.sweep:
         return run_sweep(args)
+    if args.pass_ == "bwd":
+        return run_backward(args, wl)
     return run_ours(args, wl)
 
 
@@ -415,6 +424,180 @@ def run_ours(args, wl):
             # a small probe understates the threads' throughput: size again
             n = int(min(wl.N, n * 10.0 / max(dt, 1e-3)))
             tps, dt, threads, desc = oracle_cpu_sample(wl, n, seed=3)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc + f" ({dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def oracle_bwd_sample(wl, n_positions: int, seed: int):
+    """Time the fp64 oracle's per-row backward (as it stands) on n_positions
+    random positions, all heads each.  Returns (tokens/s, seconds, threads,
+    description)."""
+    import numpy as np
+
+    import oracle
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    key = ("bwd", wl.name, wl.N)
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE.clear()
+        q, k, v = wlm.make_inputs(wl)
+        _INPUT_CACHE[key] = (q, k, v, wlm.random_cotangent(wl.B, wl.N, wl.H, wl.D,
+                                                           wl.torch_dtype, seed=wl.seed))
+    q, k, v, dout = _INPUT_CACHE[key]
+    g = np.random.default_rng(seed)
+    pos = g.choice(wl.N, size=n_positions, replace=False)
+    bs = g.integers(0, wl.B, size=n_positions)
+    rows = np.array([(b, p, h) for b, p in zip(bs, pos) for h in range(wl.H)], dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.dilated_attn_bwd_rows_fp64(q, k, v, dout, wl.patterns, rows, wl.causal)
+    dt = time.perf_counter() - t0
+    desc = (f"{n_positions} random positions (all {wl.H} heads each) of workload {wl.name}, "
+            f"fp64 oracle per-row backward (dq, dk, dv of each row)")
+    return n_positions / dt, dt, oracle.num_threads(), desc
+
+
+def run_reference_bwd(args, wl):
+    """Reference arm of the backward: the fp64 oracle's per-row backward on a
+    bounded sample of positions per step, on the host cores."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    n_pos = max(1, args.ref_positions // 16)
+    times, threads, desc = [], None, None
+    for i in range(args.warmup + args.steps):
+        _, dt, threads, desc = oracle_bwd_sample(wl, n_pos, seed=1000 + i)
+        if i >= args.warmup:
+            times.append(dt)
+    mean_dt = sum(times) / len(times)
+    value = n_pos / mean_dt
+    line = {
+        "impl": "reference", "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "pass": "bwd", "B": wl.B, "N": wl.N, "H": wl.H,
+                   "D": wl.D, "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
+                   "sample_positions_per_step": n_pos},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_backward(args, wl):
+    """The backward (dq, dk, dv) of the workload: the CUDA forward runs once
+    before timing to give out and lse; a step is one longnet_dilated_attn_bwd
+    call (two kernels)."""
+    import torch
+    import torch.distributed as dist
+
+    from sparse_long_sequence_attn_b200 import binding as bd
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+    from sparse_long_sequence_attn_b200.replicas import max_over_ranks, replica_seed, weak_scaling_rate
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    bd.load_library()
+    seed = replica_seed(wl.seed, rank)
+    q, k, v = wlm.make_inputs(wl, seed=seed)
+    dout = wlm.random_cotangent(wl.B, wl.N, wl.H, wl.D, wl.torch_dtype, seed=seed)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, dout))
+    out, lse = bd.dilated_attn(qd, kd, vd, wl.patterns, wl.causal)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, wl.patterns, wl.causal,
+                                    stream)
+
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    per_step = time_steps(step, args.steps, args.warmup, stream, flush)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    sampler.stop()
+    st = bd.longnet_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after the timed region: {bd.status_string(st)}")
+    mean_step = max_over_ranks(sum(per_step), dev) / args.steps
+
+    # end to end: pinned H2D of q, k, v, out, lse, dout; the backward; D2H of
+    # dq, dk, dv
+    hosts = [x.cpu().pin_memory() for x in (qd, kd, vd, out, lse, dod)]
+    devs = (qd, kd, vd, out, lse, dod)
+    grads_h = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (dq, dk, dv)]
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, wl.patterns,
+                                        wl.causal, stream)
+            for h_, d_ in zip(grads_h, (dq, dk, dv)):
+                h_.copy_(d_, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    if ws > 1:
+        dist.barrier()
+    per_e2e = time_steps(e2e_step, e2e_steps, 2, stream, flush)
+    e2e_total = max_over_ranks(sum(per_e2e), dev)
+    h2d = sum(x.numel() * x.element_size() for x in hosts)
+    d2h = sum(x.numel() * x.element_size() for x in grads_h)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    tokens = wl.B * wl.N
+    pairs = wlm.exact_pair_count(wl)
+    # 10*D flops per pair: the score and dP products and the dq, dk, dv sums
+    flops = 10.0 * wl.D * pairs
+    achieved = flops / mean_step / 1e12
+    roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+            "frac": achieved / FP32_ALU_TFLOPS,
+            "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz",
+            "traffic": traffic_from_profiles(wl.name + ":bwd", "backward"),
+            "kernel": "bwd_dq_kernel + bwd_dkv_kernel (one call)",
+            "exact_pairs_per_launch": pairs, "algorithmic_flops_per_launch": flops}
+    line = {
+        "metric": METRIC_BWD, "value": weak_scaling_rate(tokens, ws, mean_step), "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (bf16 in/out)" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic: seeded N(0,1) q/k/v/dout at the workload's shape (no dataset)",
+        "config": {"workload": wl.name, "pass": "bwd", "B": wl.B, "N": wl.N, "H": wl.H,
+                   "D": wl.D, "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
+                   "global_batch": wl.B * ws, "seq_len": wl.N,
+                   "parallelism": f"independent replicas x{ws}" if ws > 1 else "single GPU",
+                   "kernel": "simt backward",
+                   "l2": "512 MiB flush between timed steps (outside events)"},
+        "roofline": roof,
+        "e2e": {"value": weak_scaling_rate(tokens * e2e_steps, ws, e2e_total), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        tps, dt, _, _ = oracle_bwd_sample(wl, 1, seed=1)
+        n = int(max(1, min(wl.N, 10.0 * tps)))
+        tps, dt, threads, desc = oracle_bwd_sample(wl, n, seed=2)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc + f" ({dt:.1f} s)"}
     print(json.dumps(line), flush=True)

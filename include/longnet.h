@@ -129,6 +129,39 @@ int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
                                 longnet_stream_t stream);
 
 /*
+ * longnet_dilated_attn_bwd — the backward of the forward above: the gradients
+ * of sum(dout * out) with respect to q, k and v.  The pages present LongNet
+ * as a model that is trained ("LONGNET: Scaling Transformer to 1 billion
+ * tokens", section "Distributed training"; "LongNet" docs page, features);
+ * they give no formula for the gradient, so it is the exact derivative of the
+ * forward's function.  Since the combination weighted by e^{lse_p} is one
+ * softmax over all (pattern, key) pairs reaching a row, with
+ * P_ij = e^{s_ij - lse_i}, delta_i = <dout_i, out_i> and
+ * ds_ij = P_ij (<dout_i, v_j> - delta_i):
+ *   dq_i = sum_j ds_ij k_j / sqrt(D), dk_j = sum_i ds_ij q_i / sqrt(D),
+ *   dv_j = sum_i P_ij dout_i   (sums over the pairs of every pattern).
+ *   - q, k, v, w, r, B, N, H, D, n_pat, causal, dtype: as given to the
+ *     forward (same conventions).
+ *   - out, lse: the forward's results for these inputs (device, out
+ *     [B, N, H, D] in dtype, 16-byte aligned; lse fp32 [B, H, N], required,
+ *     4-byte aligned).  lse is the combined one the forward writes.
+ *   - dout: device [B, N, H, D] in dtype, the cotangent of out.
+ *   - dq, dk, dv: device [B, N, H, D] in dtype, written (every row; a row
+ *     no pattern keeps gets zeros).  Must not alias the inputs.
+ *   - flags: 0 (LONGNET_FLAG_QK_NORM: LONGNET_ERR_UNSUPPORTED; other bits:
+ *     LONGNET_ERR_INVALID_ARG).  D in {16, 32, 64, 128}, else UNSUPPORTED.
+ *   - Computed in fp32 by two SIMT kernels (dq; dk and dv), enqueued on
+ *     stream; allocates nothing.  Returns a longnet_status.
+ */
+int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
+                             const void* out, const float* lse, const void* dout,
+                             void* dq, void* dk, void* dv,
+                             int64_t B, int64_t N, int64_t H, int64_t D,
+                             int n_pat, const int64_t* w, const int64_t* r,
+                             int causal, int dtype, int flags,
+                             longnet_stream_t stream);
+
+/*
  * longnet_select_impl — which family AUTO would run for these arguments
  * (a longnet_impl >= 1), or a negative longnet_status when the arguments
  * are invalid.  Host-only; touches no device.

@@ -51,6 +51,10 @@ SIGNATURES = {
                                                    _i64, ctypes.c_int, _i64p, _i64p,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, _vp]),
+    "longnet_dilated_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                _i64, _i64, _i64, _i64, ctypes.c_int, _i64p,
+                                                _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                _vp]),
     "longnet_select_impl": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
                                            ctypes.c_int, ctypes.c_int]),
     "longnet_last_device_status": (ctypes.c_int, [_vp]),
@@ -158,6 +162,63 @@ def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if want_lse else None
     longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream, qk_norm)
     return out, lse
+
+
+def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                             out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                             dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
+                             patterns: Sequence[Tuple[int, int]], causal: bool = True,
+                             stream=None) -> None:
+    """Enqueue the backward on `stream`: dq, dk, dv receive the gradients of
+    sum(dout * out).  out and lse are the forward's results for q, k, v.  All
+    tensors contiguous CUDA [B, N, H, D] of q's dtype, lse fp32 [B, H, N].
+    Raises LongNetError on a non-zero status."""
+    lib = load_library()
+    B, N, H, D = q.shape
+    for t in (q, k, v, out, dout, dq, dk, dv):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out, dout, dq, dk, dv must be contiguous CUDA tensors "
+                             "of one shape and dtype")
+    if not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
+            and tuple(lse.shape) == (B, H, N)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), 0, _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_bwd")
+
+
+def dilated_attn_bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, stream=None):
+    """Allocate dq, dk, dv with torch and run the backward.  Returns (dq, dk, dv)."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    longnet_dilated_attn_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal,
+                             stream)
+    return dq, dk, dv
+
+
+class DilatedAttnFunction(torch.autograd.Function):
+    """The forward and backward entry points as one torch autograd op."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, patterns, causal):
+        out, lse = dilated_attn(q, k, v, patterns, causal)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.patterns, ctx.causal = list(patterns), causal
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout, ctx.patterns, ctx.causal)
+        return dq, dk, dv, None, None
+
+
+def dilated_attention(q, k, v, patterns, causal: bool = True):
+    """Differentiable forward: out [B, N, H, D], gradients through the backward."""
+    return DilatedAttnFunction.apply(q, k, v, patterns, causal)
 
 
 def longnet_select_impl(B: int, N: int, H: int, D: int, patterns, causal: bool, dtype) -> int:

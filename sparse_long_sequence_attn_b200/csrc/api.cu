@@ -182,6 +182,36 @@ extern "C" int longnet_dilated_attn_fwd(const void* q, const void* k, const void
                                        LONGNET_IMPL_AUTO, stream);
 }
 
+extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
+                                        const void* out, const float* lse, const void* dout,
+                                        void* dq, void* dk, void* dv, int64_t B, int64_t N,
+                                        int64_t H, int64_t D, int n_pat, const int64_t* w,
+                                        const int64_t* r, int causal, int dtype, int flags,
+                                        longnet_stream_t stream) {
+  if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
+  if (!out || !lse || !dout || !dq || !dk || !dv) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  // the forward's checks on q, k, v and the shape (dq stands in the output's
+  // place, the gradients go through BwdArgs); lse is read, not written
+  int rc = check_args(q, k, v, dq, const_cast<float*>(lse), B, N, H, D, n_pat, w, r, causal, dtype,
+                      &pb);
+  if (rc) return rc;
+  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+    return LONGNET_ERR_MISALIGNED;
+  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
+  if (!backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+  int dev = 0;
+  rc = current_device_state(&dev, &pb.status);
+  if (rc) return rc;
+  BwdArgs g;
+  g.out = out;
+  g.dout = dout;
+  g.dq = dq;
+  g.dk = dk;
+  g.dv = dv;
+  return launch_backward(pb, g, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
                                    const int64_t* w, const int64_t* r, int causal, int dtype) {
   // Stand-in pointers: only their alignment is looked at here.

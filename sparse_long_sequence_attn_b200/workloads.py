@@ -119,6 +119,14 @@ def random_inputs(B: int, N: int, H: int, D: int, dtype, seed: int, scale: float
     return tuple(out)
 
 
+def random_cotangent(B: int, N: int, H: int, D: int, dtype, seed: int):
+    """Seeded N(0, 1) dout [B, N, H, D] for the backward (drawn after a
+    distinct seed offset so it never repeats q, k or v)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 1000003)
+    return torch.randn(B, N, H, D, generator=g, dtype=torch.float32).to(dtype)
+
+
 def algorithmic_flops(wl: Workload) -> float:
     """sum_p 2*2*B*H*(N/r)*(w/r)*D, halved when causal (sparse work only)."""
     tot = 0.0

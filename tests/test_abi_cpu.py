@@ -95,3 +95,38 @@ def test_select_impl_host_logic():
     assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 0),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
     impl = bd.longnet_select_impl(1, 32768, 12, 64, ((2048, 1), (4096, 2)), True, bf16)
     assert impl in (bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05)
+
+
+def _call_bwd(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, flags=0,
+              ptrs=None):
+    buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    p = dict(q=buf, k=buf, v=buf, out=buf, lse=buf, dout=buf, dq=buf, dk=buf, dv=buf)
+    p.update(ptrs or {})
+    n = len(pats)
+    w = (ctypes.c_int64 * max(n, 1))(*[x[0] for x in pats])
+    r = (ctypes.c_int64 * max(n, 1))(*[x[1] for x in pats])
+    return lib.longnet_dilated_attn_bwd(p["q"], p["k"], p["v"], p["out"], p["lse"], p["dout"],
+                                        p["dq"], p["dk"], p["dv"], B, N, H, D, n, w, r, causal,
+                                        dtype, flags, None)
+
+
+def test_backward_argument_checks_on_host():
+    lib = bd.load_library()
+    null = ctypes.c_void_p(0)
+    for name in ("q", "out", "lse", "dout", "dq", "dk", "dv"):
+        assert _call_bwd(lib, ptrs={name: null}) == bd.LONGNET_ERR_INVALID_ARG, name
+    for name in ("out", "dout", "dk", "dv", "q"):
+        assert _call_bwd(lib, ptrs={name: ctypes.c_void_p(0x1008)}) == bd.LONGNET_ERR_MISALIGNED, name
+    assert _call_bwd(lib, ptrs={"lse": ctypes.c_void_p(0x1002)}) == bd.LONGNET_ERR_MISALIGNED
+    assert _call_bwd(lib, flags=2) == bd.LONGNET_ERR_INVALID_ARG
+    assert _call_bwd(lib, flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_UNSUPPORTED
+    assert _call_bwd(lib, D=48) == bd.LONGNET_ERR_UNSUPPORTED
+    assert _call_bwd(lib, pats=((16, 0),)) == bd.LONGNET_ERR_INVALID_ARG
+    assert _call_bwd(lib, causal=3) == bd.LONGNET_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_backward_valid_call_without_device_reports_no_device():
+    lib = bd.load_library()
+    for dtype in (0, 1, 2):
+        assert _call_bwd(lib, dtype=dtype, pats=((24, 1), (64, 4))) == bd.LONGNET_ERR_NO_DEVICE

@@ -1,0 +1,157 @@
+"""GPU parity of the backward (dq, dk, dv) through the C ABI against the fp64
+oracle's backward on the same seeded inputs (needs a B200).
+
+The CUDA backward takes the CUDA forward's out and lse, as a training step
+would; the oracle recomputes its own forward in fp64, so nothing from the
+CUDA path enters the reference.  Tolerance, per gradient, on
+max|g - ref| / max(1, max|ref|): the result is rounded once to the input
+format (2^-9 relative for bf16, 2^-12 for fp16) and delta_i = <dout_i, out_i>
+uses the forward's rounded out (again 2^-9 or 2^-12); fp32 accumulation over
+the pairs adds ~1e-6.  1e-2 (bf16), 2e-3 (fp16) and 1e-4 (fp32) hold these
+with a margin of about 3."""
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_sequence_attn_b200 import binding as bd
+from sparse_long_sequence_attn_b200 import workloads as wl
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+TOL_GRAD = {torch.float32: 1e-4, torch.bfloat16: 1e-2, torch.float16: 2e-3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    bd.load_library()
+    yield
+
+
+def run_cuda_bwd(q, k, v, dout, patterns, causal):
+    """CUDA forward (AUTO family) then the backward into NaN-guarded buffers;
+    checks the guards and the status word; returns CPU float64 (dq, dk, dv)."""
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (x.to(dev).contiguous() for x in (q, k, v, dout))
+    out, lse = bd.dilated_attn(qd, kd, vd, patterns, causal)
+    n = q.numel()
+    G = gh.GUARD
+    bufs = [torch.full((n + 2 * G,), float("nan"), dtype=q.dtype, device=dev) for _ in range(3)]
+    views = [b[G:G + n].view(q.shape) for b in bufs]
+    bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, *views, patterns, causal)
+    st = bd.longnet_last_device_status(None)
+    assert st == 0, f"device status word: {bd.status_string(st)}"
+    for b in bufs:
+        assert torch.isnan(b[:G].float()).all() and torch.isnan(b[-G:].float()).all(), \
+            "write outside a gradient"
+    res = [x.double().cpu().numpy() for x in views]
+    for x in res:
+        assert not np.isnan(x).any(), "some gradient rows were never written"
+    return res
+
+
+def check(got, ref, dtype, label):
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        err = float(np.abs(g - r).max())
+        bound = TOL_GRAD[dtype] * max(1.0, float(np.abs(r).max()))
+        assert err <= bound, f"{label} {name}: max err {err} > {bound}"
+
+
+# name, B, N, H, D, dtype, causal, patterns
+CASES = [
+    ("tiny_cfg", 1, 256, 2, 16, torch.float32, True, ((64, 1), (128, 2), (256, 4))),
+    ("fp32_d32_rdivw", 2, 384, 3, 32, torch.float32, True, ((96, 1), (192, 5), (384, 7))),
+    ("fp32_d64_noncausal", 1, 512, 2, 64, torch.float32, False, ((128, 1), (256, 3))),
+    ("fp32_d128_uncovered", 1, 240, 3, 128, torch.float32, True, ((48, 3), (240, 4))),
+    ("fp32_partial_segments", 1, 300, 3, 32, torch.float32, True, ((64, 1), (128, 3), (512, 5))),
+    ("bf16_d64_lm_like", 2, 1024, 4, 64, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
+    ("bf16_d64_paper_like", 1, 1536, 6, 64, torch.bfloat16, True,
+     ((128, 1), (256, 2), (512, 4), (768, 6), (1536, 12))),
+    ("bf16_d64_dup_unordered", 1, 512, 3, 64, torch.bfloat16, True, ((512, 4), (128, 1), (128, 1))),
+    ("bf16_d64_smallseg_noncausal", 2, 1024, 4, 64, torch.bfloat16, False, ((64, 1), (64, 2))),
+    ("bf16_d32_partial", 1, 700, 2, 32, torch.bfloat16, False, ((128, 1), (300, 2))),
+    ("f16_d64_r_not_dividing", 1, 768, 5, 64, torch.float16, True, ((192, 3), (384, 4), (768, 8))),
+    ("f16_d128", 1, 256, 2, 128, torch.float16, True, ((64, 1), (256, 2))),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(case):
+    name, B, N, H, D, dtype, causal, pats = case
+    seed = zlib.crc32(name.encode()) % 100000
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=seed)
+    dout = wl.random_cotangent(B, N, H, D, dtype, seed=seed)
+    got = run_cuda_bwd(q, k, v, dout, pats, causal)
+    ref = oracle.dilated_attn_bwd_fp64(q, k, v, dout, pats, causal)
+    check(got, ref, dtype, name)
+
+
+def test_uncovered_rows_get_zero_gradients():
+    B, N, H, D = 1, 240, 3, 64
+    pats = ((48, 3), (240, 4))
+    q, k, v = wl.random_inputs(B, N, H, D, torch.bfloat16, seed=5)
+    dout = wl.random_cotangent(B, N, H, D, torch.bfloat16, seed=5)
+    got = run_cuda_bwd(q, k, v, dout, pats, True)
+    _, lse = oracle.dilated_attn_fp64(q, k, v, pats, True)
+    kept = np.isfinite(lse).transpose(0, 2, 1)
+    assert (~kept).any()
+    for g in got:
+        assert not g[~kept].any()
+
+
+def test_autograd_function_matches_direct_calls():
+    B, N, H, D = 1, 512, 4, 64
+    pats = ((128, 1), (256, 2), (512, 4))
+    q, k, v = (x.cuda().requires_grad_(True)
+               for x in wl.random_inputs(B, N, H, D, torch.bfloat16, seed=17))
+    dout = wl.random_cotangent(B, N, H, D, torch.bfloat16, seed=17).cuda()
+    out = bd.dilated_attention(q, k, v, pats, True)
+    (out.float() * dout.float()).sum().backward()
+    with torch.no_grad():
+        o2, l2 = bd.dilated_attn(q.detach(), k.detach(), v.detach(), pats, True)
+        dq, dk, dv = bd.dilated_attn_bwd(q.detach(), k.detach(), v.detach(), o2, l2, dout, pats, True)
+    assert torch.equal(out.detach(), o2)
+    for a, b in ((q.grad, dq), (k.grad, dk), (v.grad, dv)):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["lm", "long32k"])
+def test_backward_full_size_sampled_rows(name):
+    """The bench workloads at full size: the gradients of sampled rows against
+    the oracle's per-row backward.  Rows at the ends of every pattern's first
+    segment (many keys as queries, few queries as keys), rows at the starts of
+    segments (every query of the segment reaches them) and random rows near the
+    end of the sequence."""
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.make_inputs(w)
+    dout = wl.random_cotangent(w.B, w.N, w.H, w.D, w.torch_dtype, seed=w.seed)
+    got = run_cuda_bwd(q, k, v, dout, w.patterns, w.causal)
+    g = np.random.default_rng(w.seed)
+    rows = []
+    for h in (0, w.H - 1):
+        for (wp, rp) in w.patterns:
+            o = h % rp
+            last = wp - 1 - ((wp - 1 - o) % rp)  # last kept row of segment 0
+            rows.append((w.B - 1, last, h))
+    for _ in range(4):
+        rows.append((int(g.integers(w.B)), int(w.N - 1 - g.integers(256)), int(g.integers(w.H))))
+    # first kept row of a segment of the densest pattern: every query of the
+    # segment reaches it as a key
+    w0, r0 = w.patterns[0]
+    rows.append((0, w0, 0))
+    rows.append((w.B - 1, w.N - w0 + (w.H - 1) % r0, w.H - 1))
+    rows = np.array(sorted(set(rows)), dtype=np.int64)
+    ref = oracle.dilated_attn_bwd_rows_fp64(q, k, v, dout, w.patterns, rows, w.causal)
+    b, pos, h = rows[:, 0], rows[:, 1], rows[:, 2]
+    for nm, full, r in zip(("dq", "dk", "dv"), got, ref):
+        err = float(np.abs(full[b, pos, h] - r).max())
+        bound = TOL_GRAD[w.torch_dtype] * max(1.0, float(np.abs(r).max()))
+        assert err <= bound, f"{name} {nm}: max err {err} > {bound} over {len(rows)} rows"
