@@ -234,7 +234,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", help="ours | reference")
-    ap.add_argument("--kernel", default="auto", help="auto | simt | tcgen05 | smallseg")
+    ap.add_argument("--kernel", default="auto",
+                    help="auto | simt | tcgen05 | smallseg (forward); auto | simt | tiles (--pass bwd)")
     ap.add_argument("--ref-positions", type=int, default=48)
     ap.add_argument("--cpu-positions", type=int, default=0,
                     help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
@@ -511,14 +512,18 @@ def run_backward(args, wl):
     dout = wlm.random_cotangent(wl.B, wl.N, wl.H, wl.D, wl.torch_dtype, seed=seed)
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, dout))
     out, lse = bd.dilated_attn(qd, kd, vd, wl.patterns, wl.causal)
-    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    dq, dk, dv = (torch.empty(qd.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    impl = {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT,
+            "tiles": bd.LONGNET_IMPL_TILES}[args.kernel]
+    tiles = impl == bd.LONGNET_IMPL_TILES or (
+        impl == bd.LONGNET_IMPL_AUTO and wl.D == 64 and wl.dtype != "fp32")
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
 
     def step():
         bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, wl.patterns, wl.causal,
-                                    stream)
+                                    impl, stream)
 
     sampler = ClockSampler(dev.index)
     sampler.start()
@@ -548,7 +553,7 @@ def run_backward(args, wl):
             for d_, h_ in zip(devs, hosts):
                 d_.copy_(h_, non_blocking=True)
             bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, wl.patterns,
-                                        wl.causal, stream)
+                                        wl.causal, impl, stream)
             for h_, d_ in zip(grads_h, (dq, dk, dv)):
                 h_.copy_(d_, non_blocking=True)
 
@@ -568,25 +573,37 @@ def run_backward(args, wl):
     tokens = wl.B * wl.N
     pairs = wlm.exact_pair_count(wl)
     # 10*D flops per pair: the score and dP products and the dq, dk, dv sums
+    # (the tile kernels execute 14*D: S and dP are computed in both kernels)
     flops = 10.0 * wl.D * pairs
     achieved = flops / mean_step / 1e12
-    roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-            "frac": achieved / FP32_ALU_TFLOPS,
-            "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz",
-            "traffic": traffic_from_profiles(wl.name + ":bwd", "backward"),
-            "kernel": "bwd_dq_kernel + bwd_dkv_kernel (one call)",
-            "exact_pairs_per_launch": pairs, "algorithmic_flops_per_launch": flops}
+    peaks, peak_kind = load_peaks()
+    if tiles:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peak_kind} bf16 GEMM "
+                               f"({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
+                "traffic": traffic_from_profiles(wl.name + ":bwd", "backward"),
+                "kernel": "bwd_dkv_tile_kernel + bwd_dq_tile_kernel (one call)",
+                "executed_flops_per_launch": 14.0 * wl.D * pairs}
+    else:
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_ALU_TFLOPS,
+                "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz",
+                "traffic": None, "kernel": "bwd_dkv_kernel + bwd_dq_kernel (one call)"}
+    roof["exact_pairs_per_launch"] = pairs
+    roof["algorithmic_flops_per_launch"] = flops
     line = {
         "metric": METRIC_BWD, "value": weak_scaling_rate(tokens, ws, mean_step), "unit": UNIT,
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": mean_step * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 (bf16 in/out)" if wl.dtype == "bf16" else "f32",
+        "vs_baseline": None, "dtype": ("bf16 (fp32 accumulate, fp32 gradients)" if tiles else
+                                       "f32") if wl.dtype == "bf16" else "f32",
         "data": "synthetic: seeded N(0,1) q/k/v/dout at the workload's shape (no dataset)",
         "config": {"workload": wl.name, "pass": "bwd", "B": wl.B, "N": wl.N, "H": wl.H,
                    "D": wl.D, "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
                    "global_batch": wl.B * ws, "seq_len": wl.N,
                    "parallelism": f"independent replicas x{ws}" if ws > 1 else "single GPU",
-                   "kernel": "simt backward",
+                   "kernel": "tiles (mma.sync)" if tiles else "simt",
                    "l2": "512 MiB flush between timed steps (outside events)"},
         "roofline": roof,
         "e2e": {"value": weak_scaling_rate(tokens * e2e_steps, ws, e2e_total), "unit": UNIT,

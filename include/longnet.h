@@ -76,9 +76,12 @@ enum longnet_impl {
   LONGNET_IMPL_TCGEN05 = 2,  /* bf16 or fp16, D = 64, <= 6 patterns: TMA +
                                 tcgen05/TMEM flash kernel, patterns fused in
                                 shared memory */
-  LONGNET_IMPL_SMALLSEG = 3  /* bf16 or fp16, D = 64, all patterns one segment
+  LONGNET_IMPL_SMALLSEG = 3, /* bf16 or fp16, D = 64, all patterns one segment
                                 length w <= 64 (a multiple of 8), one of them
                                 r = 1: memory-bound kernel */
+  LONGNET_IMPL_TILES = 4     /* backward only: bf16 or fp16, D = 64, any
+                                patterns: 64-row tiles of the sparsified
+                                segments on mma.sync tensor cores */
 };
 
 /*
@@ -146,19 +149,27 @@ int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
  *     [B, N, H, D] in dtype, 16-byte aligned; lse fp32 [B, H, N], required,
  *     4-byte aligned).  lse is the combined one the forward writes.
  *   - dout: device [B, N, H, D] in dtype, the cotangent of out.
- *   - dq, dk, dv: device [B, N, H, D] in dtype, written (every row; a row
- *     no pattern keeps gets zeros).  Must not alias the inputs.
+ *   - dq, dk, dv: device fp32 [B, N, H, D] (fp32 whatever dtype is, the
+ *     precision gradients are accumulated in), 16-byte aligned, written in
+ *     full (a row no pattern keeps gets zeros).  Must not alias the inputs.
  *   - flags: 0 (LONGNET_FLAG_QK_NORM: LONGNET_ERR_UNSUPPORTED; other bits:
- *     LONGNET_ERR_INVALID_ARG).  D in {16, 32, 64, 128}, else UNSUPPORTED.
- *   - Computed in fp32 by two SIMT kernels (dq; dk and dv), enqueued on
- *     stream; allocates nothing.  Returns a longnet_status.
+ *     LONGNET_ERR_INVALID_ARG).
+ *   - impl: LONGNET_IMPL_AUTO (the tile kernels where they apply, else
+ *     SIMT), LONGNET_IMPL_SIMT (fp32 FMA, D in {16, 32, 64, 128}, every
+ *     dtype) or LONGNET_IMPL_TILES (bf16/fp16, D = 64: tensor cores).  A
+ *     family that does not cover the call: LONGNET_ERR_UNSUPPORTED.
+ *   - Enqueued on stream; allocates nothing.  The tile kernels zero dq, dk
+ *     and dv on the stream first, then add each pattern's share with fp32
+ *     atomics, so the summation order of a row's patterns (at most n_pat
+ *     terms) may vary between runs in the last bits.  Returns a
+ *     longnet_status.
  */
 int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
                              const void* out, const float* lse, const void* dout,
-                             void* dq, void* dk, void* dv,
+                             float* dq, float* dk, float* dv,
                              int64_t B, int64_t N, int64_t H, int64_t D,
                              int n_pat, const int64_t* w, const int64_t* r,
-                             int causal, int dtype, int flags,
+                             int causal, int dtype, int flags, int impl,
                              longnet_stream_t stream);
 
 /*

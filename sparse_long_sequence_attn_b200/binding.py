@@ -34,6 +34,7 @@ LONGNET_IMPL_AUTO = 0
 LONGNET_IMPL_SIMT = 1
 LONGNET_IMPL_TCGEN05 = 2
 LONGNET_IMPL_SMALLSEG = 3
+LONGNET_IMPL_TILES = 4
 
 # Every symbol include/longnet.h declares, with its ctypes signature.
 _i64 = ctypes.c_int64
@@ -54,7 +55,7 @@ SIGNATURES = {
     "longnet_dilated_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _i64, _i64, _i64, _i64, ctypes.c_int, _i64p,
                                                 _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                                _vp]),
+                                                ctypes.c_int, _vp]),
     "longnet_select_impl": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
                                            ctypes.c_int, ctypes.c_int]),
     "longnet_last_device_status": (ctypes.c_int, [_vp]),
@@ -168,17 +169,21 @@ def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
                              dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
                              patterns: Sequence[Tuple[int, int]], causal: bool = True,
-                             stream=None) -> None:
-    """Enqueue the backward on `stream`: dq, dk, dv receive the gradients of
-    sum(dout * out).  out and lse are the forward's results for q, k, v.  All
-    tensors contiguous CUDA [B, N, H, D] of q's dtype, lse fp32 [B, H, N].
-    Raises LongNetError on a non-zero status."""
+                             impl: int = LONGNET_IMPL_AUTO, stream=None) -> None:
+    """Enqueue the backward on `stream`: dq, dk, dv (fp32) receive the
+    gradients of sum(dout * out).  out and lse are the forward's results for
+    q, k, v.  q, k, v, out, dout: contiguous CUDA [B, N, H, D] of one dtype;
+    dq, dk, dv: contiguous fp32 [B, N, H, D]; lse fp32 [B, H, N].  impl:
+    LONGNET_IMPL_AUTO, LONGNET_IMPL_SIMT or LONGNET_IMPL_TILES.  Raises
+    LongNetError on a non-zero status."""
     lib = load_library()
     B, N, H, D = q.shape
-    for t in (q, k, v, out, dout, dq, dk, dv):
+    for t in (q, k, v, out, dout):
         if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
-            raise ValueError("q, k, v, out, dout, dq, dk, dv must be contiguous CUDA tensors "
-                             "of one shape and dtype")
+            raise ValueError("q, k, v, out, dout must be contiguous CUDA tensors of one shape and dtype")
+    for t in (dq, dk, dv):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != torch.float32:
+            raise ValueError("dq, dk, dv must be contiguous fp32 CUDA tensors [B, N, H, D]")
     if not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
             and tuple(lse.shape) == (B, H, N)):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
@@ -186,16 +191,17 @@ def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     rc = lib.longnet_dilated_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
-        _dtype_code(q), 0, _stream_handle(stream))
+        _dtype_code(q), 0, int(impl), _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_bwd")
 
 
-def dilated_attn_bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, stream=None):
-    """Allocate dq, dk, dv with torch and run the backward.  Returns (dq, dk, dv)."""
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+def dilated_attn_bwd(q, k, v, out, lse, dout, patterns, causal: bool = True,
+                     impl: int = LONGNET_IMPL_AUTO, stream=None):
+    """Allocate fp32 dq, dk, dv with torch and run the backward.  Returns (dq, dk, dv)."""
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
     longnet_dilated_attn_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal,
-                             stream)
+                             impl, stream)
     return dq, dk, dv
 
 
@@ -212,8 +218,9 @@ class DilatedAttnFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
-        dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout, ctx.patterns, ctx.causal)
-        return dq, dk, dv, None, None
+        dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout.to(q.dtype), ctx.patterns, ctx.causal)
+        # autograd wants each gradient in its input's dtype
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None
 
 
 def dilated_attention(q, k, v, patterns, causal: bool = True):

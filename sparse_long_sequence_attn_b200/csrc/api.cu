@@ -184,11 +184,13 @@ extern "C" int longnet_dilated_attn_fwd(const void* q, const void* k, const void
 
 extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
                                         const void* out, const float* lse, const void* dout,
-                                        void* dq, void* dk, void* dv, int64_t B, int64_t N,
+                                        float* dq, float* dk, float* dv, int64_t B, int64_t N,
                                         int64_t H, int64_t D, int n_pat, const int64_t* w,
                                         const int64_t* r, int causal, int dtype, int flags,
-                                        longnet_stream_t stream) {
+                                        int impl, longnet_stream_t stream) {
   if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
+  if (impl != LONGNET_IMPL_AUTO && impl != LONGNET_IMPL_SIMT && impl != LONGNET_IMPL_TILES)
+    return LONGNET_ERR_INVALID_ARG;
   if (!out || !lse || !dout || !dq || !dk || !dv) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
   // the forward's checks on q, k, v and the shape (dq stands in the output's
@@ -199,7 +201,10 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
   if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dk, 16) || !aligned(dv, 16))
     return LONGNET_ERR_MISALIGNED;
   pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
-  if (!backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_AUTO && !backward_supports(pb) && !tile_backward_supports(pb))
+    return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_SIMT && !backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_TILES && !tile_backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
   int dev = 0;
   rc = current_device_state(&dev, &pb.status);
   if (rc) return rc;
@@ -209,7 +214,7 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
   g.dq = dq;
   g.dk = dk;
   g.dv = dv;
-  return launch_backward(pb, g, reinterpret_cast<cudaStream_t>(stream));
+  return launch_backward(pb, g, impl, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,

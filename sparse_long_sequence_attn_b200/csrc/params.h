@@ -25,14 +25,15 @@ struct Problem {
   int* status;  // device address of this device's status word
 };
 
-// The backward's extra arguments (device pointers, [B, N, H, D] in the
-// problem's dtype): the forward's output and its cotangent, and the gradients.
+// The backward's extra arguments (device pointers, [B, N, H, D]): the
+// forward's output and its cotangent in the problem's dtype, and the
+// gradients in fp32.
 struct BwdArgs {
   const void* out;
   const void* dout;
-  void* dq;
-  void* dk;
-  void* dv;
+  float* dq;
+  float* dk;
+  float* dv;
 };
 
 // Status codes written into the device status word (first error wins).
@@ -46,11 +47,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 int launch_simt(const Problem& p, cudaStream_t stream);
 int launch_tcgen05(const Problem& p, cudaStream_t stream);
 int launch_smallseg(const Problem& p, cudaStream_t stream);
-int launch_backward(const Problem& p, const BwdArgs& g, cudaStream_t stream);
+int launch_backward(const Problem& p, const BwdArgs& g, int impl, cudaStream_t stream);
 
 // Shape checks of the specialised families (host only, no device access).
 bool tcgen05_supports(const Problem& p);
 bool smallseg_supports(const Problem& p);
-bool backward_supports(const Problem& p);
+bool backward_supports(const Problem& p);       // the SIMT backward
+bool tile_backward_supports(const Problem& p);  // the mma.sync tile backward
 
 }  // namespace longnet

@@ -98,7 +98,7 @@ def test_select_impl_host_logic():
 
 
 def _call_bwd(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, flags=0,
-              ptrs=None):
+              ptrs=None, impl=0):
     buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
     p = dict(q=buf, k=buf, v=buf, out=buf, lse=buf, dout=buf, dq=buf, dk=buf, dv=buf)
     p.update(ptrs or {})
@@ -107,7 +107,7 @@ def _call_bwd(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, fla
     r = (ctypes.c_int64 * max(n, 1))(*[x[1] for x in pats])
     return lib.longnet_dilated_attn_bwd(p["q"], p["k"], p["v"], p["out"], p["lse"], p["dout"],
                                         p["dq"], p["dk"], p["dv"], B, N, H, D, n, w, r, causal,
-                                        dtype, flags, None)
+                                        dtype, flags, impl, None)
 
 
 def test_backward_argument_checks_on_host():
@@ -123,6 +123,17 @@ def test_backward_argument_checks_on_host():
     assert _call_bwd(lib, D=48) == bd.LONGNET_ERR_UNSUPPORTED
     assert _call_bwd(lib, pats=((16, 0),)) == bd.LONGNET_ERR_INVALID_ARG
     assert _call_bwd(lib, causal=3) == bd.LONGNET_ERR_INVALID_ARG
+    for impl in (2, 3, 5, -1):
+        assert _call_bwd(lib, impl=impl) == bd.LONGNET_ERR_INVALID_ARG, impl
+    # the tile family: bf16/fp16 and D = 64 only
+    assert _call_bwd(lib, impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_UNSUPPORTED
+    assert _call_bwd(lib, impl=bd.LONGNET_IMPL_TILES, dtype=1, D=32) == bd.LONGNET_ERR_UNSUPPORTED
+    # the forward has no tile family
+    buf = ctypes.c_void_p(0x1000)
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+    assert lib.longnet_dilated_attn_fwd_ex(buf, buf, buf, buf, None, 1, 64, 2, 16, 1, w, r, 1, 0, 0,
+                                           bd.LONGNET_IMPL_TILES, None) == bd.LONGNET_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
@@ -130,3 +141,4 @@ def test_backward_valid_call_without_device_reports_no_device():
     lib = bd.load_library()
     for dtype in (0, 1, 2):
         assert _call_bwd(lib, dtype=dtype, pats=((24, 1), (64, 4))) == bd.LONGNET_ERR_NO_DEVICE
+    assert _call_bwd(lib, dtype=1, D=64, impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
