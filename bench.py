@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "Dilated-attn fwd tokens/s @32K, 5 patterns; % of bf16 tensor-core peak"
 UNIT = "tokens/s"
-METRIC_BWD = "Dilated-attn bwd (dq, dk, dv) tokens/s; % of fp32 ALU peak"
+METRIC_BWD = "Dilated-attn bwd (dq, dk, dv) tokens/s; % of the kernel's roofline peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_BF16_TFLOPS = 2250.0
 # fp32 FMA peak: 148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz (clocks.max.sm)

@@ -456,7 +456,7 @@ constexpr int kKvSmem = kKvDelta + 256 + 1024;
 // dk, dv: CTA (unit = blockIdx.x, key tile jt = blockIdx.y); four warps, warp
 // w owns key rows 16 w .. 16 w + 15 of the tile.
 template <int kFmt>
-__global__ void __launch_bounds__(128) bwd_dkv_tile_kernel(const __grid_constant__ TileParams P) {
+__global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_constant__ TileParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const SegRef s = decode_unit(P, blockIdx.x);
