@@ -11,6 +11,7 @@ from .oracle import (  # noqa: F401
     dilated_attn_fp64,
     dilated_attn_rows_fp64,
     num_threads,
+    qk_normalize_bwd_fp64,
     qk_normalize_fp64,
 )
 from .brute import dilated_attn_bruteforce  # noqa: F401

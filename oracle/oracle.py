@@ -135,12 +135,31 @@ def _patterns(patterns):
     return w, r
 
 
-def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None):
+def qk_normalize_bwd_fp64(x, dxhat) -> np.ndarray:
+    """Chain rule through x -> x / max(|x|, 1e-12) (qk_normalize_fp64), per
+    row over D: with a = 1 / max(|x|, 1e-12) and xhat = a x, the Jacobian is
+    a (I - xhat xhat^T) where |x| > 1e-12 and a I elsewhere.  Returns
+    the cotangent of x given dxhat, the cotangent of xhat."""
+    x, dxhat = _f64(x), _f64(dxhat)
+    n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+    a = 1.0 / np.maximum(n, 1e-12)
+    xhat = x * a
+    proj = dxhat - xhat * (xhat * dxhat).sum(axis=-1, keepdims=True)
+    return np.where(n > 1e-12, a * proj, a * dxhat)
+
+
+def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None, qk_norm=False):
     """Full fp64 backward: the gradients of sum(dout * out) with respect to
     q, k and v, where out is the forward's output.  All tensors [B, N, H, D].
+    qk_norm: the forward normalised q and k rows first (qk_normalize_fp64);
+    the gradients then go back through that normalisation.
 
     Returns (dq, dk, dv) as float64 arrays.
     """
+    if qk_norm:
+        qh, kh = qk_normalize_fp64(q), qk_normalize_fp64(k)
+        dqh, dkh, dv = dilated_attn_bwd_fp64(qh, kh, v, dout, patterns, causal, lib)
+        return qk_normalize_bwd_fp64(q, dqh), qk_normalize_bwd_fp64(k, dkh), dv
     lib = lib or load_library()
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, N, H, D = q.shape
@@ -155,9 +174,18 @@ def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None):
     return dq, dk, dv
 
 
-def dilated_attn_bwd_rows_fp64(q, k, v, dout, patterns, rows_bph, causal=True, lib=None):
+def dilated_attn_bwd_rows_fp64(q, k, v, dout, patterns, rows_bph, causal=True, lib=None,
+                               qk_norm=False):
     """fp64 backward of selected rows only.  rows_bph: int array [n, 3] of
-    (b, pos, h).  Returns (dq_rows, dk_rows, dv_rows), each [n, D]."""
+    (b, pos, h).  qk_norm as in dilated_attn_bwd_fp64.  Returns (dq_rows,
+    dk_rows, dv_rows), each [n, D]."""
+    if qk_norm:
+        rows = np.asarray(rows_bph, dtype=np.int64).reshape(-1, 3)
+        qh, kh = qk_normalize_fp64(q), qk_normalize_fp64(k)
+        dqh, dkh, dv = dilated_attn_bwd_rows_fp64(qh, kh, v, dout, patterns, rows, causal, lib)
+        b, pos, h = rows[:, 0], rows[:, 1], rows[:, 2]
+        qr, kr = _f64(q)[b, pos, h], _f64(k)[b, pos, h]
+        return qk_normalize_bwd_fp64(qr, dqh), qk_normalize_bwd_fp64(kr, dkh), dv
     lib = lib or load_library()
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, N, H, D = q.shape

@@ -452,6 +452,51 @@ def check_bwd_rows_function(lib):
                 np.testing.assert_allclose(got[which][t], ref[which][b, pos, h], atol=1e-12, rtol=0)
 
 
+def check_bwd_qk_norm(lib):
+    """The backward with qk_norm: central differences of the qk_norm forward,
+    torch autograd through F.normalize and the multiset formulation, a zero
+    row (the 1/eps branch of the normalisation), and the per-row entry point
+    against the full backward."""
+    B, N, H, D = 1, 36, 3, 4
+    pats = [(12, 1), (18, 3), (36, 4)]
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (131, 132, 133, 134))
+    q[0, 7, 1] = 0.0  # a zero query row
+    for causal in (True, False):
+        grads = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib, qk_norm=True)
+        # autograd through F.normalize, then the multiset formulation
+        tq, tk = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k))
+        qn = F.normalize(tq, dim=-1, eps=1e-12)
+        kn = F.normalize(tk, dim=-1, eps=1e-12)
+        gq, gk, gv = _brute_autograd(qn.detach().numpy(), kn.detach().numpy(), v, do, pats, causal)
+        torch.autograd.backward([qn, kn], [torch.from_numpy(gq), torch.from_numpy(gk)])
+        # the zero row's gradient is dqhat / 1e-12 (~1e12): compare it relatively
+        np.testing.assert_allclose(grads[0], tq.grad.numpy(), atol=1e-11, rtol=1e-12)
+        assert np.abs(grads[0][0, 7, 1]).max() > 1e9
+        np.testing.assert_allclose(grads[1], tk.grad.numpy(), atol=1e-11, rtol=0)
+        np.testing.assert_allclose(grads[2], gv, atol=1e-12, rtol=0)
+        # central differences of the qk_norm forward (away from the zero row)
+        eps = 1e-6
+        g = np.random.default_rng(135)
+        for which in range(3):
+            for _ in range(5):
+                idx = (0, int(g.integers(8, N)), int(g.integers(H)), int(g.integers(D)))
+                vals = []
+                for sgn in (1.0, -1.0):
+                    args = [q.copy(), k.copy(), v.copy()]
+                    args[which][idx] += sgn * eps
+                    o, _ = orc.dilated_attn_fp64(*args, pats, causal=causal, lib=lib, qk_norm=True)
+                    vals.append(float((o * do).sum()))
+                fd = (vals[0] - vals[1]) / (2 * eps)
+                assert abs(fd - grads[which][idx]) < 1e-6 * max(1.0, abs(fd)), (which, idx)
+        rows = [(0, pos, h) for pos in range(0, N, 5) for h in range(H)] + [(0, 7, 1)]
+        got = orc.dilated_attn_bwd_rows_fp64(q, k, v, do, pats, rows, causal=causal, lib=lib,
+                                             qk_norm=True)
+        for t, (b, pos, h) in enumerate(rows):
+            for which in range(3):
+                np.testing.assert_allclose(got[which][t], grads[which][b, pos, h], atol=1e-12,
+                                           rtol=1e-12)
+
+
 ALL_CHECKS = [
     check_rows_function_direct,
     check_qk_norm,
@@ -470,4 +515,5 @@ ALL_CHECKS = [
     check_bwd_finite_differences,
     check_bwd_invariants,
     check_bwd_rows_function,
+    check_bwd_qk_norm,
 ]

@@ -72,3 +72,35 @@ def test_pins_catch_mutant(tmp_path, name, old, new):
         except (AssertionError, ValueError, FloatingPointError):
             caught.append(check.__name__)
     assert caught, f"no pin caught mutant {name}"
+
+
+# The chain rule through the qk normalisation lives in oracle.py: planted
+# mistakes there are swapped in for the duration of the check.
+def _no_projection(x, dxhat):
+    import numpy as np
+
+    from oracle.oracle import _f64
+
+    x, dxhat = _f64(x), _f64(dxhat)
+    return dxhat / np.maximum(np.sqrt((x * x).sum(axis=-1, keepdims=True)), 1e-12)
+
+
+def _squared_norm_scale(x, dxhat):
+    import numpy as np
+
+    from oracle.oracle import _f64
+
+    x, dxhat = _f64(x), _f64(dxhat)
+    n2 = np.maximum((x * x).sum(axis=-1, keepdims=True), 1e-24)
+    xhat = x / np.sqrt(n2)
+    return (dxhat - xhat * (xhat * dxhat).sum(axis=-1, keepdims=True)) / n2
+
+
+@pytest.mark.parametrize("mutant", [_no_projection, _squared_norm_scale],
+                         ids=lambda f: f.__name__.strip("_"))
+def test_pins_catch_python_mutant(monkeypatch, oracle_lib, mutant):
+    import oracle.oracle as orc
+
+    monkeypatch.setattr(orc, "qk_normalize_bwd_fp64", mutant)
+    with pytest.raises(AssertionError):
+        pins.check_bwd_qk_norm(oracle_lib)
