@@ -152,8 +152,11 @@ int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
  *   - dq, dk, dv: device fp32 [B, N, H, D] (fp32 whatever dtype is, the
  *     precision gradients are accumulated in), 16-byte aligned, written in
  *     full (a row no pattern keeps gets zeros).  Must not alias the inputs.
- *   - flags: 0 (LONGNET_FLAG_QK_NORM: LONGNET_ERR_UNSUPPORTED; other bits:
- *     LONGNET_ERR_INVALID_ARG).
+ *   - flags: 0 or LONGNET_FLAG_QK_NORM, as given to the forward: the scores
+ *     then use q / max(|q|, 1e-12) and k / max(|k|, 1e-12), and dq, dk are
+ *     taken back through that normalisation (a (g - xhat <xhat, g>) per row,
+ *     a = 1 / max(|x|, 1e-12); a g for a row with |x| <= 1e-12).  Other bits:
+ *     LONGNET_ERR_INVALID_ARG.
  *   - impl: LONGNET_IMPL_AUTO (the tile kernels where they apply, else
  *     SIMT), LONGNET_IMPL_SIMT (fp32 FMA, D in {16, 32, 64, 128}, every
  *     dtype) or LONGNET_IMPL_TILES (bf16/fp16, D = 64: tensor cores).  A

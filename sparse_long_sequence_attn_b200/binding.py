@@ -169,13 +169,14 @@ def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
                              dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
                              patterns: Sequence[Tuple[int, int]], causal: bool = True,
-                             impl: int = LONGNET_IMPL_AUTO, stream=None) -> None:
+                             impl: int = LONGNET_IMPL_AUTO, stream=None,
+                             qk_norm: bool = False) -> None:
     """Enqueue the backward on `stream`: dq, dk, dv (fp32) receive the
     gradients of sum(dout * out).  out and lse are the forward's results for
-    q, k, v.  q, k, v, out, dout: contiguous CUDA [B, N, H, D] of one dtype;
-    dq, dk, dv: contiguous fp32 [B, N, H, D]; lse fp32 [B, H, N].  impl:
-    LONGNET_IMPL_AUTO, LONGNET_IMPL_SIMT or LONGNET_IMPL_TILES.  Raises
-    LongNetError on a non-zero status."""
+    q, k, v (with the same qk_norm).  q, k, v, out, dout: contiguous CUDA
+    [B, N, H, D] of one dtype; dq, dk, dv: contiguous fp32 [B, N, H, D]; lse
+    fp32 [B, H, N].  impl: LONGNET_IMPL_AUTO, LONGNET_IMPL_SIMT or
+    LONGNET_IMPL_TILES.  Raises LongNetError on a non-zero status."""
     lib = load_library()
     B, N, H, D = q.shape
     for t in (q, k, v, out, dout):
@@ -191,17 +192,17 @@ def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     rc = lib.longnet_dilated_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
-        _dtype_code(q), 0, int(impl), _stream_handle(stream))
+        _dtype_code(q), LONGNET_FLAG_QK_NORM if qk_norm else 0, int(impl), _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_bwd")
 
 
 def dilated_attn_bwd(q, k, v, out, lse, dout, patterns, causal: bool = True,
-                     impl: int = LONGNET_IMPL_AUTO, stream=None):
+                     impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False):
     """Allocate fp32 dq, dk, dv with torch and run the backward.  Returns (dq, dk, dv)."""
     dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
     longnet_dilated_attn_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal,
-                             impl, stream)
+                             impl, stream, qk_norm)
     return dq, dk, dv
 
 
@@ -209,23 +210,24 @@ class DilatedAttnFunction(torch.autograd.Function):
     """The forward and backward entry points as one torch autograd op."""
 
     @staticmethod
-    def forward(ctx, q, k, v, patterns, causal):
-        out, lse = dilated_attn(q, k, v, patterns, causal)
+    def forward(ctx, q, k, v, patterns, causal, qk_norm=False):
+        out, lse = dilated_attn(q, k, v, patterns, causal, qk_norm=qk_norm)
         ctx.save_for_backward(q, k, v, out, lse)
-        ctx.patterns, ctx.causal = list(patterns), causal
+        ctx.patterns, ctx.causal, ctx.qk_norm = list(patterns), causal, qk_norm
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
-        dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout.to(q.dtype), ctx.patterns, ctx.causal)
+        dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout.to(q.dtype), ctx.patterns, ctx.causal,
+                                      qk_norm=ctx.qk_norm)
         # autograd wants each gradient in its input's dtype
-        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None
 
 
-def dilated_attention(q, k, v, patterns, causal: bool = True):
+def dilated_attention(q, k, v, patterns, causal: bool = True, qk_norm: bool = False):
     """Differentiable forward: out [B, N, H, D], gradients through the backward."""
-    return DilatedAttnFunction.apply(q, k, v, patterns, causal)
+    return DilatedAttnFunction.apply(q, k, v, patterns, causal, qk_norm)
 
 
 def longnet_select_impl(B: int, N: int, H: int, D: int, patterns, causal: bool, dtype) -> int:

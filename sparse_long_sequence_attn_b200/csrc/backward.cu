@@ -59,6 +59,29 @@ __device__ __forceinline__ float warp_sum32(float x) {
   return x;
 }
 
+// Back through the qk_norm normalisation xhat = a x, a = 1 / max(|x|, 1e-12):
+// given the cotangent g of xhat (lane l holds dims l, l + 32, ...), the
+// cotangent of x is a (g - xhat <xhat, g>) where |x| > 1e-12, else a g.
+// xhat: the normalised row in shared memory; xx = |x|^2.
+template <int D>
+__device__ __forceinline__ void project_row(float (&g)[(D + 31) / 32], const float* xhat, float a,
+                                            float xx, int lane) {
+  constexpr int E = (D + 31) / 32;
+  float dot = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int d = lane + 32 * e;
+    if (d < D) dot = fmaf(xhat[d], g[e], dot);
+  }
+  dot = warp_sum32(dot);
+  const bool proj = sqrtf(xx) > 1e-12f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int d = lane + 32 * e;
+    if (d < D) g[e] = a * (proj ? g[e] - xhat[d] * dot : g[e]);
+  }
+}
+
 // Where row pos of head h sits in pattern (w, r): its index in the sparsified
 // segment (-1 when the pattern does not keep it), the segment's first kept
 // position and its number of kept rows (the last segment ends with the
@@ -103,15 +126,24 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(const Problem p,
   const int64_t base_b = b * p.N * HD;
   const int64_t me = base_b + pos * HD + h * D;
 
-  float delta = 0.f;
+  float delta = 0.f, qq = 0.f;
   for (int d = lane; d < D; d += 32) {
-    qsh[warp][d] = ld(Q + me + d);
+    const float xq = ld(Q + me + d);
+    qsh[warp][d] = xq;
+    qq = fmaf(xq, xq, qq);
     const float x = ld(dO + me + d);
     dosh[warp][d] = x;
     delta = fmaf(x, ld(O + me + d), delta);
   }
   delta = warp_sum32(delta);
+  qq = warp_sum32(qq);
   __syncwarp();
+  // qk_norm: the scores use qhat = a_q q, a_q = 1 / max(|q|, 1e-12)
+  const float a_q = p.qk_norm ? 1.f / fmaxf(sqrtf(qq), 1e-12f) : 1.f;
+  if (p.qk_norm) {
+    for (int d = lane; d < D; d += 32) qsh[warp][d] *= a_q;
+    __syncwarp();
+  }
   const float lse_i = p.lse[(b * p.H + h) * p.N + pos];
   const float scale = rsqrtf((float)D);
   float acc[E];
@@ -129,13 +161,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(const Problem p,
         float ds = 0.f;
         if (j < n_keys) {
           const int64_t off = base_b + (kp.first + r * j) * HD + h * D;
-          float s = 0.f, dp = 0.f;
+          float s = 0.f, dp = 0.f, kk = 0.f;
 #pragma unroll 16
           for (int d = 0; d < D; ++d) {
-            s = fmaf(qsh[warp][d], ld(K + off + d), s);
+            const float xk = ld(K + off + d);
+            s = fmaf(qsh[warp][d], xk, s);
+            kk = fmaf(xk, xk, kk);
             dp = fmaf(dosh[warp][d], ld(V + off + d), dp);
           }
-          ds = expf(s * scale - lse_i) * (dp - delta);
+          // qk_norm: khat = a_k k, so dqhat gets ds * a_k * k
+          const float a_k = p.qk_norm ? 1.f / fmaxf(sqrtf(kk), 1e-12f) : 1.f;
+          ds = expf(s * a_k * scale - lse_i) * (dp - delta) * a_k;
         }
         const int cnt = (n_keys - j0 < 32) ? (int)(n_keys - j0) : 32;
         for (int t = 0; t < cnt; ++t) {
@@ -151,9 +187,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dq_kernel(const Problem p,
     }
   }
 #pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] *= scale;
+  if (p.qk_norm) project_row<D>(acc, qsh[warp], a_q, qq, lane);
+#pragma unroll
   for (int e = 0; e < E; ++e) {
     const int d = lane + 32 * e;
-    if (d < D) g.dq[me + d] = acc[e] * scale;
+    if (d < D) g.dq[me + d] = acc[e];
   }
 }
 
@@ -183,11 +222,21 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkv_kernel(const Problem p
   const int64_t me = base_b + pos * HD + h * D;
   const float* lse_bh = p.lse + (b * p.H + h) * p.N;
 
+  float kk = 0.f;
   for (int d = lane; d < D; d += 32) {
-    ksh[warp][d] = ld(K + me + d);
+    const float xk = ld(K + me + d);
+    ksh[warp][d] = xk;
+    kk = fmaf(xk, xk, kk);
     vsh[warp][d] = ld(V + me + d);
   }
+  kk = warp_sum32(kk);
   __syncwarp();
+  // qk_norm: the scores use khat = a_k k
+  const float a_k = p.qk_norm ? 1.f / fmaxf(sqrtf(kk), 1e-12f) : 1.f;
+  if (p.qk_norm) {
+    for (int d = lane; d < D; d += 32) ksh[warp][d] *= a_k;
+    __syncwarp();
+  }
   const float scale = rsqrtf((float)D);
   float acc_k[E], acc_v[E];
 #pragma unroll
@@ -204,16 +253,20 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkv_kernel(const Problem p
       if (i < kp.m) {
         const int64_t qpos = kp.first + r * i;
         const int64_t off = base_b + qpos * HD + h * D;
-        float s = 0.f, dp = 0.f, delta = 0.f;
+        float s = 0.f, dp = 0.f, delta = 0.f, qq = 0.f;
 #pragma unroll 16
         for (int d = 0; d < D; ++d) {
           const float x = ld(dO + off + d);
-          s = fmaf(ld(Q + off + d), ksh[warp][d], s);
+          const float xq = ld(Q + off + d);
+          s = fmaf(xq, ksh[warp][d], s);
+          qq = fmaf(xq, xq, qq);
           dp = fmaf(x, vsh[warp][d], dp);
           delta = fmaf(x, ld(O + off + d), delta);
         }
-        pr = expf(s * scale - lse_bh[qpos]);
-        ds = pr * (dp - delta);
+        // qk_norm: qhat = a_q q, so dkhat gets ds * a_q * q
+        const float a_q = p.qk_norm ? 1.f / fmaxf(sqrtf(qq), 1e-12f) : 1.f;
+        pr = expf(s * a_q * scale - lse_bh[qpos]);
+        ds = pr * (dp - delta) * a_q;
       }
       const int cnt = (kp.m - i0 < 32) ? (int)(kp.m - i0) : 32;
       for (int t = 0; t < cnt; ++t) {
@@ -232,10 +285,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkv_kernel(const Problem p
     }
   }
 #pragma unroll
+  for (int e = 0; e < E; ++e) acc_k[e] *= scale;
+  if (p.qk_norm) project_row<D>(acc_k, ksh[warp], a_k, kk, lane);
+#pragma unroll
   for (int e = 0; e < E; ++e) {
     const int d = lane + 32 * e;
     if (d < D) {
-      g.dk[me + d] = acc_k[e] * scale;
+      g.dk[me + d] = acc_k[e];
       g.dv[me + d] = acc_v[e];
     }
   }
@@ -445,17 +501,96 @@ __device__ __forceinline__ void tile_delta(uint32_t s_do, uint32_t s_o, float* l
   }
 }
 
+// qk_norm: the 64 rows of a swizzled tile scaled in place to xhat = a x,
+// a = 1 / max(|x|, 1e-12) (rounded back to the 16-bit format, so every
+// product sees |xhat| <= 1), and a of each row into a[].  Thread pairs share
+// a row; no thread touches another pair's row.
+constexpr float kInvNormEps = 1e12f;  // 1 / 1e-12: a row with |x| <= 1e-12 has this a
+template <int kFmt>
+__device__ __forceinline__ void tile_normalize(uint32_t s_x, float* a, int tid) {
+  const int row = tid >> 1, half = tid & 1;
+  uint32_t x[4][4];
+  float n = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(x[c][0]), "=r"(x[c][1]), "=r"(x[c][2]), "=r"(x[c][3])
+                 : "r"(tile_addr(s_x, row, 4 * half + c)));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float x0, x1;
+      unpack2<kFmt>(x[c][e], x0, x1);
+      n = fmaf(x0, x0, n);
+      n = fmaf(x1, x1, n);
+    }
+  }
+  n += __shfl_xor_sync(0xffffffffu, n, 1);
+  const float ar = 1.f / fmaxf(sqrtf(n), 1e-12f);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float x0, x1;
+      unpack2<kFmt>(x[c][e], x0, x1);
+      y[e] = pack2<kFmt>(x0 * ar, x1 * ar);
+    }
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(tile_addr(s_x, row, 4 * half + c)),
+                 "r"(y[0]), "r"(y[1]), "r"(y[2]), "r"(y[3])
+                 : "memory");
+  }
+  if (half == 0) a[row] = ar;
+}
+
+// qk_norm, at the end of a tile kernel: this lane's gradient g[nt][2 half ..]
+// of xhat (rows row0 + 8 half of the normalised tile in s_x, dims
+// nt * 8 + 2 t4 + {0, 1}) turned into the gradient of x:
+// a (g - xhat <xhat, g>), or a g for a row with |x| <= 1e-12.  The four lanes
+// of a row add up <xhat, g>.
+template <int kFmt>
+__device__ __forceinline__ void tile_project(float (&gr)[8][4], uint32_t s_x, int row0, int t4,
+                                             const float (&a)[2]) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float xh[8][2];
+    float dot = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      uint32_t u;
+      asm volatile("ld.shared.u32 %0, [%1];"
+                   : "=r"(u)
+                   : "r"(tile_addr(s_x, row0 + 8 * half, nt) + 4u * t4));
+      unpack2<kFmt>(u, xh[nt][0], xh[nt][1]);
+      dot = fmaf(xh[nt][0], gr[nt][2 * half], dot);
+      dot = fmaf(xh[nt][1], gr[nt][2 * half + 1], dot);
+    }
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    const bool proj = a[half] < kInvNormEps;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = gr[nt][2 * half + e];
+        gr[nt][2 * half + e] = a[half] * (proj ? v - xh[nt][e] * dot : v);
+      }
+    }
+  }
+}
+
 // Shared memory of the dk/dv kernel (bytes from a 1024-aligned base): K and V
 // tiles, then two stages of (Q, dout, out) tiles, two stages of lse, delta.
 constexpr int kKvK = 0, kKvV = kTileBytes, kKvStage = 2 * kTileBytes;
 constexpr int kKvStageBytes = 3 * kTileBytes;
 constexpr int kKvLse = kKvStage + 2 * kKvStageBytes;
 constexpr int kKvDelta = kKvLse + 2 * 256;
-constexpr int kKvSmem = kKvDelta + 256 + 1024;
+constexpr int kKvNormK = kKvDelta + 256;  // qk_norm: a of the key rows
+constexpr int kKvNormQ = kKvNormK + 256;  // qk_norm: a of the current query rows
+constexpr int kKvSmem = kKvNormQ + 256 + 1024;
 
 // dk, dv: CTA (unit = blockIdx.x, key tile jt = blockIdx.y); four warps, warp
 // w owns key rows 16 w .. 16 w + 15 of the tile.
-template <int kFmt>
+template <int kFmt, bool kNorm>
 __global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_constant__ TileParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -468,6 +603,11 @@ __global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_const
   const uint32_t sb = smem_u32(smem);
   float* sLse = reinterpret_cast<float*>(smem + kKvLse);
   float* sDelta = reinterpret_cast<float*>(smem + kKvDelta);
+  float* sAk = reinterpret_cast<float*>(smem + kKvNormK);
+  float* sAq = reinterpret_cast<float*>(smem + kKvNormQ);
+  float aK[2] = {1.f, 1.f};  // qk_norm: a of this lane's key rows
+  (void)sAk;  // sAk, sAq: the qk_norm instantiation only
+  (void)sAq;
   const uint16_t* Q = static_cast<const uint16_t*>(P.pb.q);
   const uint16_t* K = static_cast<const uint16_t*>(P.pb.k);
   const uint16_t* V = static_cast<const uint16_t*>(P.pb.v);
@@ -511,7 +651,17 @@ __global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_const
     const uint32_t sdO = sQ + kTileBytes;
     float* lse = sLse + stage * 64;
     tile_delta<kFmt>(sdO, sQ + 2 * kTileBytes, lse, sDelta, tid);
+    if constexpr (kNorm) {  // q rows, and once the key rows, to unit norm
+      tile_normalize<kFmt>(sQ, sAq, tid);
+      if (it == it0) tile_normalize<kFmt>(k_row, sAk, tid);
+    }
     __syncthreads();
+    if constexpr (kNorm) {
+      if (it == it0) {
+        aK[0] = sAk[16 * warp + g];
+        aK[1] = sAk[16 * warp + g + 8];
+      }
+    }
 
 #pragma unroll
     for (int hq = 0; hq < 2; ++hq) {  // 32 queries at a time
@@ -577,6 +727,14 @@ __global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_const
     __syncthreads();  // the stage is refilled two iterations on
   }
   cp_async_wait<0>();
+  if constexpr (kNorm) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dk[nt][e] *= P.scale;
+    tile_project<kFmt>(dk, k_row, 16 * warp + g, t4, aK);
+  }
+  const float dk_scale = kNorm ? 1.f : P.scale;
 
   // one fp32 add per pattern into the caller's gradients
 #pragma unroll
@@ -588,7 +746,7 @@ __global__ void __launch_bounds__(128, 3) bwd_dkv_tile_kernel(const __grid_const
       for (int nt = 0; nt < 8; ++nt) {
         const int d = nt * 8 + 2 * t4;
         atomicAdd(reinterpret_cast<float2*>(P.g.dk + off + d),
-                  make_float2(dk[nt][2 * half] * P.scale, dk[nt][2 * half + 1] * P.scale));
+                  make_float2(dk[nt][2 * half] * dk_scale, dk[nt][2 * half + 1] * dk_scale));
         atomicAdd(reinterpret_cast<float2*>(P.g.dv + off + d),
                   make_float2(dv[nt][2 * half], dv[nt][2 * half + 1]));
       }
@@ -602,11 +760,13 @@ constexpr int kQQ = 0, kQdO = kTileBytes, kQO = 2 * kTileBytes, kQStage = 3 * kT
 constexpr int kQStageBytes = 2 * kTileBytes;
 constexpr int kQLse = kQStage + 2 * kQStageBytes;
 constexpr int kQDelta = kQLse + 256;
-constexpr int kQSmem = kQDelta + 256 + 1024;
+constexpr int kQNormQ = kQDelta + 256;  // qk_norm: a of the query rows
+constexpr int kQNormK = kQNormQ + 256;  // qk_norm: a of the current key rows
+constexpr int kQSmem = kQNormK + 256 + 1024;
 
 // dq: CTA (unit = blockIdx.x, query tile it = T - 1 - blockIdx.y, the
 // costliest first when causal); warp w owns query rows 16 w .. 16 w + 15.
-template <int kFmt>
+template <int kFmt, bool kNorm>
 __global__ void __launch_bounds__(128) bwd_dq_tile_kernel(const __grid_constant__ TileParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -619,6 +779,11 @@ __global__ void __launch_bounds__(128) bwd_dq_tile_kernel(const __grid_constant_
   const uint32_t sb = smem_u32(smem);
   float* sLse = reinterpret_cast<float*>(smem + kQLse);
   float* sDelta = reinterpret_cast<float*>(smem + kQDelta);
+  float* sAq = reinterpret_cast<float*>(smem + kQNormQ);
+  float* sAk = reinterpret_cast<float*>(smem + kQNormK);
+  float aQ[2] = {1.f, 1.f};  // qk_norm: a of this lane's query rows
+  (void)sAq;  // sAq, sAk: the qk_norm instantiation only
+  (void)sAk;
   const uint16_t* Q = static_cast<const uint16_t*>(P.pb.q);
   const uint16_t* K = static_cast<const uint16_t*>(P.pb.k);
   const uint16_t* V = static_cast<const uint16_t*>(P.pb.v);
@@ -653,16 +818,22 @@ __global__ void __launch_bounds__(128) bwd_dq_tile_kernel(const __grid_constant_
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
+    const uint32_t sK = sb + kQStage + stage * kQStageBytes;
     if (jt == 0) {
       tile_delta<kFmt>(sb + kQdO, sb + kQO, sLse, sDelta, tid);
+      if constexpr (kNorm) tile_normalize<kFmt>(sb + kQQ, sAq, tid);
       __syncthreads();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         lse2[half] = sLse[16 * warp + g + 8 * half];
         dlt[half] = sDelta[16 * warp + g + 8 * half];
+        if constexpr (kNorm) aQ[half] = sAq[16 * warp + g + 8 * half];
       }
     }
-    const uint32_t sK = sb + kQStage + stage * kQStageBytes;
+    if constexpr (kNorm) {  // the key rows to unit norm
+      tile_normalize<kFmt>(sK, sAk, tid);
+      __syncthreads();
+    }
     const uint32_t sV = sK + kTileBytes;
 #pragma unroll
     for (int hk = 0; hk < 2; ++hk) {  // 32 keys at a time
@@ -720,6 +891,14 @@ __global__ void __launch_bounds__(128) bwd_dq_tile_kernel(const __grid_constant_
     __syncthreads();
   }
   cp_async_wait<0>();
+  if constexpr (kNorm) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dq[nt][e] *= P.scale;
+    tile_project<kFmt>(dq, sb + kQQ, 16 * warp + g, t4, aQ);
+  }
+  const float dq_scale = kNorm ? 1.f : P.scale;
 
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -730,7 +909,7 @@ __global__ void __launch_bounds__(128) bwd_dq_tile_kernel(const __grid_constant_
       for (int nt = 0; nt < 8; ++nt) {
         const int d = nt * 8 + 2 * t4;
         atomicAdd(reinterpret_cast<float2*>(P.g.dq + off + d),
-                  make_float2(dq[nt][2 * half] * P.scale, dq[nt][2 * half + 1] * P.scale));
+                  make_float2(dq[nt][2 * half] * dq_scale, dq[nt][2 * half + 1] * dq_scale));
       }
     }
   }
@@ -757,7 +936,7 @@ bool tile_geometry(const Problem& p, TileParams* tp, int64_t* t_max) {
   return units > 0 && units <= 0x7fffffffLL && tm >= 1 && tm <= 65535;
 }
 
-template <int kFmt>
+template <int kFmt, bool kNorm>
 int launch_tile_bwd_fmt(const TileParams& tp, int64_t units, int64_t t_max, cudaStream_t stream) {
   static bool attr_set[64] = {false};  // per device: the attribute is set once on each
   int dev = 0;
@@ -766,19 +945,19 @@ int launch_tile_bwd_fmt(const TileParams& tp, int64_t units, int64_t t_max, cuda
     return LONGNET_ERR_CUDA;
   }
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(bwd_dkv_tile_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kKvSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dq_tile_kernel<kFmt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kQSmem) != cudaSuccess) {
+    if (cudaFuncSetAttribute(bwd_dkv_tile_kernel<kFmt, kNorm>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dq_tile_kernel<kFmt, kNorm>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
     attr_set[dev] = true;
   }
   const dim3 grid((unsigned)units, (unsigned)t_max);
-  bwd_dq_tile_kernel<kFmt><<<grid, 128, kQSmem, stream>>>(tp);
+  bwd_dq_tile_kernel<kFmt, kNorm><<<grid, 128, kQSmem, stream>>>(tp);
   if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
-  bwd_dkv_tile_kernel<kFmt><<<grid, 128, kKvSmem, stream>>>(tp);
+  bwd_dkv_tile_kernel<kFmt, kNorm><<<grid, 128, kKvSmem, stream>>>(tp);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 
@@ -798,19 +977,23 @@ int launch_tile_bwd(const Problem& p, const BwdArgs& g, cudaStream_t stream) {
     return LONGNET_ERR_CUDA;
   }
   const int64_t units = tp.unit_base[p.n_pat];
-  if (p.dtype == LONGNET_DTYPE_F16) return launch_tile_bwd_fmt<kFmtF16>(tp, units, t_max, stream);
-  return launch_tile_bwd_fmt<kFmtBF16>(tp, units, t_max, stream);
+  if (p.qk_norm) {
+    if (p.dtype == LONGNET_DTYPE_F16) return launch_tile_bwd_fmt<kFmtF16, true>(tp, units, t_max, stream);
+    return launch_tile_bwd_fmt<kFmtBF16, true>(tp, units, t_max, stream);
+  }
+  if (p.dtype == LONGNET_DTYPE_F16) return launch_tile_bwd_fmt<kFmtF16, false>(tp, units, t_max, stream);
+  return launch_tile_bwd_fmt<kFmtBF16, false>(tp, units, t_max, stream);
 }
 
 }  // namespace
 
 bool backward_supports(const Problem& p) {
-  return !p.qk_norm && (p.D == 16 || p.D == 32 || p.D == 64 || p.D == 128);
+  return p.D == 16 || p.D == 32 || p.D == 64 || p.D == 128;
 }
 
 bool tile_backward_supports(const Problem& p) {
   int64_t t_max = 0;
-  return !p.qk_norm && p.D == 64 &&
+  return p.D == 64 &&
          (p.dtype == LONGNET_DTYPE_BF16 || p.dtype == LONGNET_DTYPE_F16) &&
          tile_geometry(p, nullptr, &t_max);
 }

@@ -119,7 +119,6 @@ def test_backward_argument_checks_on_host():
         assert _call_bwd(lib, ptrs={name: ctypes.c_void_p(0x1008)}) == bd.LONGNET_ERR_MISALIGNED, name
     assert _call_bwd(lib, ptrs={"lse": ctypes.c_void_p(0x1002)}) == bd.LONGNET_ERR_MISALIGNED
     assert _call_bwd(lib, flags=2) == bd.LONGNET_ERR_INVALID_ARG
-    assert _call_bwd(lib, flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_UNSUPPORTED
     assert _call_bwd(lib, D=48) == bd.LONGNET_ERR_UNSUPPORTED
     assert _call_bwd(lib, pats=((16, 0),)) == bd.LONGNET_ERR_INVALID_ARG
     assert _call_bwd(lib, causal=3) == bd.LONGNET_ERR_INVALID_ARG
@@ -142,3 +141,7 @@ def test_backward_valid_call_without_device_reports_no_device():
     for dtype in (0, 1, 2):
         assert _call_bwd(lib, dtype=dtype, pats=((24, 1), (64, 4))) == bd.LONGNET_ERR_NO_DEVICE
     assert _call_bwd(lib, dtype=1, D=64, impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
+    # qk_norm is taken by both families
+    assert _call_bwd(lib, flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_NO_DEVICE
+    assert _call_bwd(lib, dtype=2, D=64, flags=bd.LONGNET_FLAG_QK_NORM,
+                     impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE

@@ -39,18 +39,19 @@ def _cuda():
     yield
 
 
-def run_cuda_bwd(q, k, v, dout, patterns, causal, impl=bd.LONGNET_IMPL_AUTO):
+def run_cuda_bwd(q, k, v, dout, patterns, causal, impl=bd.LONGNET_IMPL_AUTO, qk_norm=False):
     """CUDA forward (AUTO family) then the backward into NaN-guarded fp32
     buffers; checks the guards and the status word; returns CPU float64
     (dq, dk, dv)."""
     dev = torch.device("cuda:0")
     qd, kd, vd, dod = (x.to(dev).contiguous() for x in (q, k, v, dout))
-    out, lse = bd.dilated_attn(qd, kd, vd, patterns, causal)
+    out, lse = bd.dilated_attn(qd, kd, vd, patterns, causal, qk_norm=qk_norm)
     n = q.numel()
     G = gh.GUARD
     bufs = [torch.full((n + 2 * G,), float("nan"), dtype=torch.float32, device=dev) for _ in range(3)]
     views = [b[G:G + n].view(q.shape) for b in bufs]
-    bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, *views, patterns, causal, impl)
+    bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, *views, patterns, causal, impl,
+                                qk_norm=qk_norm)
     st = bd.longnet_last_device_status(None)
     assert st == 0, f"device status word: {bd.status_string(st)}"
     for b in bufs:
@@ -201,3 +202,32 @@ def test_backward_full_size_sampled_rows(name):
         err = float(np.abs(full[b, pos, h] - r).max())
         bound = TOL_GRAD[w.torch_dtype] * max(1.0, float(np.abs(r).max()))
         assert err <= bound, f"{name} {nm}: max err {err} > {bound} over {len(rows)} rows"
+
+
+# qk_norm: q and k rows scaled to unit L2 norm before the scores, gradients
+# taken back through the normalisation.  Inputs are drawn at scale 3 so the
+# norms are far from 1; one zero key row takes the 1/eps branch (its dk is
+# compared relatively: it is dkhat / 1e-12).
+QK_NORM_CASES = [
+    ("qkn_bf16_lm_like", 1, 512, 3, 64, torch.bfloat16, True, ((128, 1), (256, 2), (512, 4))),
+    ("qkn_f16_noncausal_small", 2, 256, 4, 64, torch.float16, False, ((64, 1), (64, 2))),
+    ("qkn_fp32_d32_partial", 1, 300, 3, 32, torch.float32, True, ((64, 1), (128, 3), (512, 5))),
+]
+QKN_PARAMS = [(c, nm, code) for c in QK_NORM_CASES for (nm, code) in _impls(c[5], c[4])]
+
+
+@pytest.mark.parametrize("case,impl_name,impl", QKN_PARAMS,
+                         ids=[f"{c[0]}-{nm}" for (c, nm, _) in QKN_PARAMS])
+def test_backward_qk_norm(case, impl_name, impl):
+    name, B, N, H, D, dtype, causal, pats = case
+    seed = zlib.crc32(name.encode()) % 100000
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=seed, scale=3.0)
+    dout = wl.random_cotangent(B, N, H, D, dtype, seed=seed)
+    k[0, 5, 1] = 0.0  # a zero key row
+    got = run_cuda_bwd(q, k, v, dout, pats, causal, impl, qk_norm=True)
+    ref = oracle.dilated_attn_bwd_fp64(q, k, v, dout, pats, causal, qk_norm=True)
+    zero = got[1][0, 5, 1].copy(), ref[1][0, 5, 1].copy()
+    got[1][0, 5, 1] = ref[1][0, 5, 1] = 0.0
+    check(got, ref, dtype, f"{name} ({impl_name})")
+    bound = 10 * TOL_GRAD[dtype] * max(1.0, float(np.abs(zero[1]).max()))
+    assert np.abs(zero[0] - zero[1]).max() <= bound, "zero key row (1/eps branch)"
