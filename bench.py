@@ -51,18 +51,29 @@ def load_peaks():
 
 
 # The sources a kernel family's device code is built from: its own file and
-# the shared headers.  A change anywhere else leaves its counters valid.
+# the shared headers (code only: comments and layout are ignored).  A change
+# anywhere else leaves its counters valid.
 _FAMILY_SOURCES = ("device_util.cuh", "params.h")
+
+
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed: the part
+    a comment or layout edit does not change."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
 
 
 def kernel_source_hash(family: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_long_sequence_attn_b200", "csrc")
-    for name in (f"{family}.cu",) + _FAMILY_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    with open(os.path.join(ROOT, "include", "longnet.h"), "rb") as f:
-        h.update(b"longnet.h" + f.read())
+    paths = [os.path.join(csrc, n) for n in (f"{family}.cu",) + _FAMILY_SOURCES]
+    paths.append(os.path.join(ROOT, "include", "longnet.h"))
+    for path in paths:
+        with open(path, encoding="utf-8") as f:
+            h.update(os.path.basename(path).encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
