@@ -1,4 +1,5 @@
-"""B200 (sm_100a) multi-pattern dilated-attention forward of LongNet.
+"""B200 (sm_100a) multi-pattern dilated-attention forward of LongNet, and its
+backward.
 
 The product is the C-ABI library liblongnet.so (include/longnet.h); this
 package holds its CUDA sources (csrc/), the build script, a thin ctypes
@@ -9,9 +10,14 @@ from .binding import (  # noqa: F401
     LONGNET_IMPL_SIMT,
     LONGNET_IMPL_SMALLSEG,
     LONGNET_IMPL_TCGEN05,
+    LONGNET_IMPL_TILES,
+    DilatedAttnFunction,
     LongNetError,
+    dilated_attention,
     dilated_attn,
+    dilated_attn_bwd,
     load_library,
+    longnet_dilated_attn_bwd,
     longnet_dilated_attn_fwd,
     longnet_last_device_status,
     longnet_select_impl,
