@@ -35,8 +35,11 @@
  *   - stream: a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; the call returns before it finishes.
  *   - Memory: every pointer is owned by the caller.  The library allocates
- *     no device or host memory in any call.  Its only global state is one
- *     status word per device (see longnet_last_device_status).
+ *     no device or host memory in any call.  Its global state is one status
+ *     word per device (see longnet_last_device_status) and, on the host,
+ *     small per-device caches in static storage (the launch set-up of the
+ *     last shapes and pointers, kernel attributes), guarded for concurrent
+ *     callers.
  *   - Errors: every entry point returns LONGNET_OK (0) or a negative code,
  *     never aborts, traps or exits.  Arguments are checked before anything is
  *     enqueued: a rejected call enqueues nothing.

@@ -41,6 +41,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "device_util.cuh"
 #include "params.h"
 
@@ -938,13 +940,15 @@ bool tile_geometry(const Problem& p, TileParams* tp, int64_t* t_max) {
 
 template <int kFmt, bool kNorm>
 int launch_tile_bwd_fmt(const TileParams& tp, int64_t units, int64_t t_max, cudaStream_t stream) {
-  static bool attr_set[64] = {false};  // per device: the attribute is set once on each
+  // per device: the attribute is set once on each (setting it twice, from two
+  // threads at once, is harmless)
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return LONGNET_ERR_CUDA;
   }
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(bwd_dkv_tile_kernel<kFmt, kNorm>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_dq_tile_kernel<kFmt, kNorm>,
@@ -952,7 +956,7 @@ int launch_tile_bwd_fmt(const TileParams& tp, int64_t units, int64_t t_max, cuda
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const dim3 grid((unsigned)units, (unsigned)t_max);
   bwd_dq_tile_kernel<kFmt, kNorm><<<grid, 128, kQSmem, stream>>>(tp);
