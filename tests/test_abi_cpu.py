@@ -145,3 +145,23 @@ def test_backward_valid_call_without_device_reports_no_device():
     assert _call_bwd(lib, flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_NO_DEVICE
     assert _call_bwd(lib, dtype=2, D=64, flags=bd.LONGNET_FLAG_QK_NORM,
                      impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
+
+
+def test_backward_tile_grid_limit_on_host():
+    """A segment of more than 65535 tiles (2^22 + rows at r = 1) is beyond the
+    tile kernels' grid: a forced tile call is UNSUPPORTED before any device
+    access, while SIMT (and AUTO, which falls back to it) get as far as the
+    device check."""
+    lib = bd.load_library()
+    N = 65536 * 64 + 64
+    assert _call_bwd(lib, N=N, D=64, dtype=1, pats=((N, 1),),
+                     impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        for impl in (bd.LONGNET_IMPL_AUTO, bd.LONGNET_IMPL_SIMT):
+            assert _call_bwd(lib, N=N, D=64, dtype=1, pats=((N, 1),),
+                             impl=impl) == bd.LONGNET_ERR_NO_DEVICE
+    # one tile fewer is inside the limit
+    N2 = 65535 * 64
+    if not torch.cuda.is_available():
+        assert _call_bwd(lib, N=N2, D=64, dtype=1, pats=((N2, 1),),
+                         impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
