@@ -46,15 +46,19 @@ void check_tma(const Params& P, int ri, int64_t first, int64_t need, int64_t r) 
   }
 }
 
-void run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std::pair<int64_t, int64_t>> pats, int causal) {
+bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std::pair<int64_t, int64_t>> pats, int causal,
+              int sms = 148, bool quiet = false) {
   Problem pb;
   memset(&pb, 0, sizeof(pb));
   pb.B = B; pb.N = N; pb.H = H; pb.D = 64; pb.n_pat = (int)pats.size(); pb.causal = causal;
   pb.dtype = LONGNET_DTYPE_BF16;
   for (int i = 0; i < pb.n_pat; ++i) { pb.w[i] = pats[i].first; pb.r[i] = pats[i].second; }
-  if (!tcgen05_supports(pb)) { printf("%s: not supported\n", name); return; }
+  if (!tcgen05_supports(pb)) {
+    if (!quiet) printf("%s: not supported\n", name);
+    return false;
+  }
   static Params P;
-  fill_params(pb, P, 148);
+  fill_params(pb, P, sms);
   int f0 = fails;
   long n_tiles = 0, n_kv = 0;
   // coverage: (p, h, seg, k) -> count
@@ -150,8 +154,44 @@ void run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
       if (!covered) CHECK(P.uncovered_possible, "%s: uncovered position but flag off\n", name);
     }
   }
-  printf("%-28s ranges=%d units=%d R=%ld tiles/head=%.1f kv/head=%.1f %s\n", name, P.n_ranges, P.n_units, (long)P.range_len,
-         (double)n_tiles / H, (double)n_kv / H, fails == f0 ? "OK" : "FAIL");
+  if (!quiet || fails != f0)
+    printf("%-28s ranges=%d units=%d R=%ld tiles/head=%.1f kv/head=%.1f %s\n", name, P.n_ranges, P.n_units,
+           (long)P.range_len, (double)n_tiles / H, (double)n_kv / H, fails == f0 ? "OK" : "FAIL");
+  return true;
+}
+
+// Seeded random shapes the kernel takes: N a multiple of 64 up to 16384,
+// 1..6 patterns whose w divides N, r up to 16 (r > w allowed), 1..12 heads,
+// causal or not, and SM counts that change the unit plan.
+void random_cases(int count) {
+  uint64_t st = 0x9e3779b97f4a7c15ull;
+  auto next = [&]() { st ^= st << 13; st ^= st >> 7; st ^= st << 17; return st; };
+  const int64_t rs[] = {1, 1, 2, 3, 4, 5, 6, 7, 8, 12, 16};
+  const int sms[] = {148, 132, 16, 1};
+  int ran = 0, f0 = fails;
+  for (int c = 0; c < count; ++c) {
+    const int64_t N = 64 * (int64_t)(2 + next() % 255);
+    std::vector<int64_t> divs;
+    for (int64_t w = 2; w <= N; ++w)
+      if (N % w == 0) divs.push_back(w);
+    const int n_pat = 1 + (int)(next() % 6);
+    std::vector<std::pair<int64_t, int64_t>> pats;
+    for (int i = 0; i < n_pat; ++i)
+      pats.push_back({divs[next() % divs.size()], rs[next() % (sizeof(rs) / sizeof(rs[0]))]});
+    const int64_t H = 1 + (int64_t)(next() % 12);
+    const int causal = (int)(next() & 1);
+    char name[64];
+    snprintf(name, sizeof(name), "random%d", c);
+    const int f1 = fails;
+    if (!run_case(name, 1, N, H, pats, causal, sms[next() % 4], true)) continue;
+    if (fails != f1) {
+      printf("  N=%ld H=%ld causal=%d patterns:", (long)N, (long)H, causal);
+      for (auto& pr : pats) printf(" (%ld,%ld)", (long)pr.first, (long)pr.second);
+      printf("\n");
+    }
+    ++ran;
+  }
+  printf("random cases: %d of %d taken by the kernel, %s\n", ran, count, fails == f0 ? "OK" : "FAIL");
 }
 
 // Multiply-shift division against plain division: every divisor up to 4100
@@ -193,6 +233,7 @@ int main() {
   run_case("odd_mix", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 1);
   run_case("odd_mix_nc", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 0);
   run_case("sweep1M_part", 1, 1048576, 1, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 8}, {32768, 16}, {65536, 32}}, 1);
+  random_cases(300);
   printf("fails=%d\n", fails);
   return fails ? 1 : 0;
 }

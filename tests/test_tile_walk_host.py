@@ -2,8 +2,9 @@
 
 The kernel source is compiled with nvcc for sm_100a, but only its host code
 runs: the tile walk and combination order, the parking-slot lifetimes, the TMA
-coordinates, and the multiply-shift divider against integer division.  Every
-case prints OK and the program exits 0.
+coordinates, and the multiply-shift divider against integer division, on the
+named shapes and 300 seeded random ones (with SM counts that change the unit
+plan).  Every case prints OK and the program exits 0.
 """
 import os
 import shutil
@@ -32,3 +33,6 @@ def test_tile_walk_host_checks():
     assert "fails=0" in res.stdout
     assert "fastdiv OK" in res.stdout
     assert "FAIL" not in res.stdout
+    # the seeded random shapes: most of them must be ones the kernel takes
+    line = [l for l in res.stdout.splitlines() if l.startswith("random cases:")][0]
+    assert int(line.split()[2]) >= 200, line
