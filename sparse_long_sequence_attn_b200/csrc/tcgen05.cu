@@ -30,7 +30,9 @@
 //  * The unit's tiles are dealt to two independent streams, each with its
 //    own TMA thread (Q per tile, a ring of 64-key K/V blocks), MMA thread and
 //    softmax warpgroup; one epilogue warpgroup takes the tiles of both in
-//    processing order.
+//    processing order.  The ring stages that fit next to the pattern slots
+//    are split between the streams (the first gets the odd one), and the
+//    softmax warps take one descriptor per tile, not per block.
 //  * Online softmax in fp32 (thread i owns row i), exp2 on scaled scores,
 //    lazy rescaling of O (only when the row max grows by more than 2^8).
 //  * Cross-pattern combination without any HBM round trip: tiles are
@@ -43,6 +45,9 @@
 //    next tile overwrites it, so one 16 KB slot per pattern is enough.
 //  * Every wait is bounded; on a timeout the kernel records the status word,
 //    stops issuing work, drains what it issued and returns.
+//  * Host side: the launch set-up (tensor maps, unit plan) is cached per
+//    device for the last shapes and pointers; the device-side walk divides by
+//    per-launch constants with multiply-shift dividers (FastDiv).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
