@@ -19,6 +19,7 @@ synchronize around the timed region, max over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -316,7 +317,9 @@ def run_ours(args, wl):
     ws, rank, local = dist_env()
     if ws > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+        # a short timeout: a rank left waiting for a dead peer ends with an error
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(dev)
     bd.load_library()
@@ -514,7 +517,9 @@ def run_backward(args, wl):
     ws, rank, local = dist_env()
     if ws > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+        # a short timeout: a rank left waiting for a dead peer ends with an error
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(dev)
     bd.load_library()
