@@ -37,7 +37,8 @@
  *
  * Layouts: q, k, v, out are [B, N, H, D] contiguous doubles; lse is [B, H, N]
  * (natural log, scale included).  Every pin against which this file is
- * checked lives in tests/test_oracle_pins.py.
+ * checked lives in tests/oracle_pins.py (run by tests/test_oracle_pins.py;
+ * tests/test_oracle_mutants.py runs them against planted mistakes).
  */
 #include <math.h>
 #include <omp.h>

@@ -38,7 +38,7 @@ class Workload:
     N: int
     H: int
     D: int
-    dtype: str  # "fp32" or "bf16"
+    dtype: str  # "fp32", "bf16" or "fp16"
     causal: bool
     patterns: Tuple[Pattern, ...]
     qk_norm: bool = False
@@ -51,7 +51,7 @@ class Workload:
 
     @property
     def torch_dtype(self):
-        return torch.float32 if self.dtype == "fp32" else torch.bfloat16
+        return {"fp32": torch.float32, "bf16": torch.bfloat16, "fp16": torch.float16}[self.dtype]
 
     def with_n(self, N: int) -> "Workload":
         """Same workload at another length, patterns truncated to w <= N."""
