@@ -415,7 +415,7 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": mean_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": {"bf16": "bf16", "fp16": "f16", "fp32": "f32"}[wl.dtype],
         "data": "synthetic: seeded N(0,1) q/k/v at the workload's shape (no dataset)",
         "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
                    "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
@@ -612,8 +612,8 @@ def run_backward(args, wl):
         "metric": METRIC_BWD, "value": weak_scaling_rate(tokens, ws, mean_step), "unit": UNIT,
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": mean_step * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": ("bf16 (fp32 accumulate, fp32 gradients)" if tiles else
-                                       "f32") if wl.dtype == "bf16" else "f32",
+        "vs_baseline": None,
+        "dtype": (f"{wl.dtype} (fp32 accumulate, fp32 gradients)" if tiles else "f32"),
         "data": "synthetic: seeded N(0,1) q/k/v/dout at the workload's shape (no dataset)",
         "config": {"workload": wl.name, "pass": "bwd", "B": wl.B, "N": wl.N, "H": wl.H,
                    "D": wl.D, "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
