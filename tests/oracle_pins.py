@@ -452,6 +452,35 @@ def check_bwd_rows_function(lib):
                 np.testing.assert_allclose(got[which][t], ref[which][b, pos, h], atol=1e-12, rtol=0)
 
 
+def check_bwd_closed_form(lib):
+    """N = 2, D = 1, one pattern (2, 1), causal: row 0 sees key 0 only
+    (out0 = v0), row 1 sees keys 0 and 1 with p0 = 1 / (1 + e^{q1 (k1 - k0)}).
+    With L = g0 out0 + g1 out1, by hand: dv0 = g0 + g1 p0, dv1 = g1 p1,
+    ds10 = g1 p0 p1 (v0 - v1) = -ds11, dq0 = 0, dq1 = ds10 (k0 - k1),
+    dk0 = ds10 q1, dk1 = -ds10 q1.  And duplicating every pattern leaves out,
+    hence every gradient, unchanged."""
+    q0, q1, k0, k1, v0, v1, g0, g1 = 0.5, 1.0, 2.0, -1.0, 3.0, 1.0, 0.25, 2.0
+    q = np.array([q0, q1]).reshape(1, 2, 1, 1)
+    k = np.array([k0, k1]).reshape(1, 2, 1, 1)
+    v = np.array([v0, v1]).reshape(1, 2, 1, 1)
+    do = np.array([g0, g1]).reshape(1, 2, 1, 1)
+    dq, dk, dv = orc.dilated_attn_bwd_fp64(q, k, v, do, [(2, 1)], causal=True, lib=lib)
+    p0 = 1.0 / (1.0 + math.exp(q1 * (k1 - k0)))
+    p1 = 1.0 - p0
+    ds10 = g1 * p0 * p1 * (v0 - v1)
+    np.testing.assert_allclose(dq.ravel(), [0.0, ds10 * (k0 - k1)], atol=1e-15, rtol=0)
+    np.testing.assert_allclose(dk.ravel(), [ds10 * q1, -ds10 * q1], atol=1e-15, rtol=0)
+    np.testing.assert_allclose(dv.ravel(), [g0 + g1 * p0, g1 * p1], atol=1e-15, rtol=0)
+    B, N, H, D = 1, 36, 3, 4
+    pats = [(12, 1), (18, 3), (36, 5)]
+    qr, kr, vr, dor = (_rand((B, N, H, D), s) for s in (141, 142, 143, 144))
+    for causal in (True, False):
+        once = orc.dilated_attn_bwd_fp64(qr, kr, vr, dor, pats, causal=causal, lib=lib)
+        twice = orc.dilated_attn_bwd_fp64(qr, kr, vr, dor, pats + pats, causal=causal, lib=lib)
+        for a_, b_ in zip(once, twice):
+            np.testing.assert_allclose(b_, a_, atol=1e-13, rtol=0)
+
+
 def check_bwd_qk_norm(lib):
     """The backward with qk_norm: central differences of the qk_norm forward,
     torch autograd through F.normalize and the multiset formulation, a zero
@@ -515,5 +544,6 @@ ALL_CHECKS = [
     check_bwd_finite_differences,
     check_bwd_invariants,
     check_bwd_rows_function,
+    check_bwd_closed_form,
     check_bwd_qk_norm,
 ]
