@@ -58,30 +58,37 @@ def compare_full(o, l, q, k, v, patterns, causal, dtype, label="", tol_out=None,
     return err
 
 
-def sample_rows(B, N, H, patterns, n_random, seed):
-    """(b, pos, h) rows: first and last row of every segment of every pattern
-    for every head (the edges of the tiles), plus seeded random rows."""
+def sample_rows(B, N, H, patterns, n_random, seed, boundary=0, boundary_heads=None):
+    """(b, pos, h) rows to compare at full size, all kept (no subsampling of
+    the structured ones):
+      * the first and last kept row of every segment of every pattern, for
+        every head and for the first and last batch (the tile edges);
+      * with boundary > 0, the rows on both sides of every multiple of
+        `boundary` positions and of its half (the kernel's range and split
+        points), for the heads in boundary_heads (default: all);
+      * n_random seeded random rows."""
     rows = set()
     g = np.random.default_rng(seed)
-    for b in {0, B - 1}:
+    for b in sorted({0, B - 1}):
         for h in range(H):
             for (w, r) in patterns:
                 o = h % r
-                for seg in range(0, N // w):
-                    if o < w:
-                        first = seg * w + o
-                        last = seg * w + o + r * ((w - o - 1) // r)
-                        rows.add((b, first, h))
-                        rows.add((b, last, h))
-                    if len(rows) > 20000:
-                        break
+                for seg in range((N + w - 1) // w):
+                    ln = min(w, N - seg * w)
+                    if o < ln:
+                        rows.add((b, seg * w + o, h))
+                        rows.add((b, seg * w + o + r * ((ln - o - 1) // r), h))
+        if boundary > 0:
+            heads = range(H) if boundary_heads is None else boundary_heads
+            half = max(1, boundary // 2)
+            for x in range(0, N + 1, half):
+                for pos in (x - 1, x):
+                    if 0 <= pos < N:
+                        for h in heads:
+                            rows.add((b, pos, h))
     for _ in range(n_random):
         rows.add((int(g.integers(B)), int(g.integers(N)), int(g.integers(H))))
-    rows = sorted(rows)
-    if len(rows) > 6000:
-        idx = g.choice(len(rows), 6000, replace=False)
-        rows = [rows[i] for i in sorted(idx)]
-    return np.array(rows, dtype=np.int64)
+    return np.array(sorted(rows), dtype=np.int64)
 
 
 def compare_rows(o, l, q, k, v, patterns, causal, dtype, rows, label=""):
