@@ -101,7 +101,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.period = period_s
         self._stop = threading.Event()
@@ -253,6 +253,10 @@ def main():
                     help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="linear-scaling sweep instead")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave the linear-scaling sweep out of the default line")
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="seconds of repeated steps after the timed region, for the clock record")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=("fwd", "bwd"),
                     help="fwd: the forward (default); bwd: the backward (dq, dk, dv)")
     args = ap.parse_args()
@@ -359,6 +363,25 @@ def run_ours(args, wl):
     total = max_over_ranks(sum(per_step), dev)
     mean_step = total / args.steps
 
+    # clock soak (after the timed region, not part of `value`): the same step
+    # repeated for at least a second, with the clocks sampled throughout, so
+    # the clock record is a distribution even when the timed region is short
+    soak = None
+    if args.soak_s > 0:
+        soak_sampler = ClockSampler(dev.index)
+        soak_sampler.start()
+        torch.cuda.synchronize()
+        s0 = time.time()
+        n_soak, soak_dev_s = 0, 0.0
+        while time.time() - s0 < args.soak_s:
+            per = time_steps(step, 50, 0, stream, flush)
+            n_soak += len(per)
+            soak_dev_s += sum(per)
+        s1 = time.time()
+        soak_sampler.stop()
+        soak = {"steps": n_soak, "ms_per_step": soak_dev_s / n_soak * 1e3,
+                "clocks": soak_sampler.summary(s0, s1)}
+
     # end-to-end through the public API with host buffers: pinned H2D of the
     # inputs, the forward, D2H of out and lse, every step
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
@@ -428,6 +451,11 @@ def run_ours(args, wl):
         "gpu_launches": args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
+    if soak is not None:
+        line["clock_soak"] = soak
+    if ws == 1 and wl.name == "long32k" and not args.no_sweep:
+        line["sweep"] = sweep_lines(args.steps, args.warmup, args.kernel, dev.index)
+        line["sweep_linear_1M_vs_64K"] = line["sweep"][-1]["tokens_per_s_vs_65536"]
     if ws == 1 and not args.no_cpu_baseline:
         n = args.cpu_positions
         calibrate = n <= 0
@@ -637,24 +665,26 @@ def run_backward(args, wl):
     return 0
 
 
-def run_sweep(args):
-    """Linear-scaling sweep: tokens/s at N = 65536, 262144, 1048576."""
+def sweep_lines(steps, warmup, kernel="auto", dev_index=0):
+    """Linear-scaling sweep: the forward at N = 65536, 262144, 1048576 (B 1,
+    H 8, six patterns of sparse length 2048), each timed over `steps` steps
+    with CUDA events and an L2 flush between steps.  Inputs are drawn on the
+    device (the sweep measures speed; its parity is tested separately)."""
     import torch
 
     from sparse_long_sequence_attn_b200 import binding as bd
     from sparse_long_sequence_attn_b200 import workloads as wlm
 
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
+    dev = torch.device("cuda", dev_index)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    impl = _impl_code(args.kernel)
+    impl = _impl_code(kernel)
+    peaks, _ = load_peaks()
     res = []
     for N in wlm.SWEEP_NS:
         wl = wlm.sweep_workload(N)
         g = torch.Generator(device=dev)
         g.manual_seed(wl.seed)
-        # device-side draws: the sweep measures speed only (parity is tested separately)
         qd, kd, vd = (torch.randn(wl.B, N, wl.H, wl.D, device=dev, generator=g,
                                   dtype=torch.float32).to(torch.bfloat16) for _ in range(3))
         out = torch.empty_like(qd)
@@ -663,16 +693,31 @@ def run_sweep(args):
         def step():
             bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, wl.patterns, wl.causal, impl, stream)
 
-        per = time_steps(step, args.steps, args.warmup, stream, flush)
+        per = time_steps(step, steps, warmup, stream, flush)
+        st = bd.longnet_last_device_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status after the sweep at N={N}: {bd.status_string(st)}")
         t = sum(per) / len(per)
-        res.append({"N": N, "ms": t * 1e3, "tokens_per_s": N / t,
-                    "tflops": wlm.algorithmic_flops(wl) / t / 1e12})
+        tf = wlm.algorithmic_flops(wl) / t / 1e12
+        res.append({"N": N, "ms": t * 1e3, "tokens_per_s": N / t, "tflops": tf,
+                    "frac": tf / peaks["bf16_tflops"]})
         del qd, kd, vd, out, lse
         torch.cuda.empty_cache()
     base = res[0]["tokens_per_s"]
     for r in res:
         r["tokens_per_s_vs_65536"] = r["tokens_per_s"] / base
-    print(json.dumps({"sweep": res}), flush=True)
+    return res
+
+
+def run_sweep(args):
+    """Linear-scaling sweep alone: one JSON line {"sweep": [...]}."""
+    import torch
+
+    torch.cuda.set_device(0)
+    from sparse_long_sequence_attn_b200 import binding as bd
+
+    bd.load_library()
+    print(json.dumps({"sweep": sweep_lines(args.steps, args.warmup, args.kernel)}), flush=True)
     return 0
 
 

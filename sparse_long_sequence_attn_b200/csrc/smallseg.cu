@@ -357,6 +357,9 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     const int64_t row0_pos = (int64_t)b * N + (int64_t)seg * W;  // position of the segment's row 0
     if (!mbar_wait(bar, phase, P.wait_limit_ns)) {
       record_status(P.pb.status, kStatusTimeout);
+      // the segment's loads may still be in flight into this pair's shared
+      // memory: wait for them once more (bounded) before the warps leave
+      mbar_wait(bar, phase, P.wait_limit_ns);
       return;
     }
     if (P.pb.qk_norm) {
