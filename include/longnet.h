@@ -66,7 +66,7 @@ enum longnet_status {
   LONGNET_ERR_MISALIGNED = -3,    /* a pointer misses its alignment */
   LONGNET_ERR_CUDA = -4,          /* a CUDA call failed (launch, config) */
   LONGNET_ERR_DEVICE_TIMEOUT = -5,/* a kernel wait ran out of time (status word) */
-  LONGNET_ERR_DEVICE_BOUNDS = -6, /* reserved: a kernel index check failed */
+  LONGNET_ERR_DEVICE_BOUNDS = -6, /* a kernel index check failed (status word) */
   LONGNET_ERR_NO_DEVICE = -7      /* no usable sm_100 device */
 };
 
@@ -135,6 +135,57 @@ int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
                                 longnet_stream_t stream);
 
 /*
+ * longnet_dilated_attn_fwd_part — the forward with options and a family (as
+ * longnet_dilated_attn_fwd_ex), computing only part of the output: positions
+ * [q_begin, q_end) and heads [h_begin, h_end) of out and lse; every other
+ * element of out and lse is left untouched.  q, k, v are full-length
+ * [B, N, H, D] tensors.  The caller provides q at the part's positions and
+ * heads, and k and v wherever the part's rows need keys (the kept rows of
+ * the same segments, before each row when causal).  Other rows of q may hold
+ * anything (rows are computed independently).  Other rows of k and v may be
+ * read too, and masked: they must hold finite values, since a masked row's
+ * weight, 0, multiplies its v row (zero is the natural fill).
+ * This is the step a device takes when the sequence is split over devices
+ * ("LONGNET: Scaling Transformer to 1 billion tokens", section "Token
+ * expansion reaches 1 billion+": each device attends for its own shard,
+ * the keys and values of longer segments coming from the other devices), and
+ * the step of a split by heads.  0 <= q_begin < q_end <= N and
+ * 0 <= h_begin < h_end <= H, else LONGNET_ERR_INVALID_ARG.  The small-segment
+ * kernel takes parts made of whole segments only (AUTO then picks another
+ * family).  The other conventions are those of the full forward.
+ */
+int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,
+                                  void* out, float* lse,
+                                  int64_t B, int64_t N, int64_t H, int64_t D,
+                                  int n_pat, const int64_t* w, const int64_t* r,
+                                  int causal, int dtype, int flags, int impl,
+                                  int64_t q_begin, int64_t q_end,
+                                  int64_t h_begin, int64_t h_end,
+                                  longnet_stream_t stream);
+
+/*
+ * longnet_gather_rows / longnet_scatter_rows — the data movement of the
+ * sequence-parallel exchange (same pages and sections as
+ * longnet_dilated_attn_fwd_part): the kept rows of one device's shard that
+ * other devices need are packed into a contiguous buffer, exchanged by a
+ * collective, and written back at their positions on the receiving device.
+ *   gather:  dst[i] = src[idx[i]] for i < n (dst holds n rows);
+ *   scatter: dst[idx[i]] = src[i] for i < n (src holds n rows).
+ * A row is row_bytes bytes (a positive multiple of 16, at most 1 MiB); for a
+ * [B, N, H, D] tensor the row of (b, x, h) is (b N + x) H + h and
+ * row_bytes = D times the element size.  src, dst: device pointers,
+ * 16-byte aligned; idx: a device array of n int64, 8-byte aligned, caller
+ * owned.  src_rows / dst_rows: rows the indexed buffer holds; an index
+ * outside [0, rows) is not accessed and records LONGNET_ERR_DEVICE_BOUNDS in
+ * the status word (see longnet_last_device_status).  n = 0 does nothing.
+ * Enqueued on stream; returns a longnet_status.
+ */
+int longnet_gather_rows(const void* src, int64_t src_rows, const int64_t* idx, int64_t n,
+                        void* dst, int64_t row_bytes, longnet_stream_t stream);
+int longnet_scatter_rows(const void* src, int64_t n, const int64_t* idx, void* dst,
+                         int64_t dst_rows, int64_t row_bytes, longnet_stream_t stream);
+
+/*
  * longnet_dilated_attn_bwd — the backward of the forward above: the gradients
  * of sum(dout * out) with respect to q, k and v.  The pages present LongNet
  * as a model that is trained ("LONGNET: Scaling Transformer to 1 billion
@@ -189,13 +240,13 @@ int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
 
 /*
  * longnet_last_device_status — synchronises `stream`, then returns and
- * clears the current device's status word: LONGNET_OK, or
+ * clears the current device's status word: LONGNET_OK,
  * LONGNET_ERR_DEVICE_TIMEOUT when a kernel's bounded wait gave up (its
- * outputs are then undefined).  LONGNET_ERR_DEVICE_BOUNDS is reserved for a
- * kernel-side index check: the kernels of this version carry none (their
- * index arithmetic is checked on the host by the tests' walk restatements)
- * and never report it.  LONGNET_ERR_CUDA if the synchronisation itself
- * failed.
+ * outputs are then undefined), or LONGNET_ERR_DEVICE_BOUNDS when a row index
+ * given to longnet_gather_rows / longnet_scatter_rows was out of range (that
+ * row was skipped; the attention kernels' index arithmetic is checked on the
+ * host by the tests' walk restatements and carries no device-side check).
+ * LONGNET_ERR_CUDA if the synchronisation itself failed.
  */
 int longnet_last_device_status(longnet_stream_t stream);
 

@@ -3,7 +3,8 @@ backward.
 
 The product is the C-ABI library liblongnet.so (include/longnet.h); this
 package holds its CUDA sources (csrc/), the build script, a thin ctypes
-binding and the named synthetic workloads.
+binding, the named synthetic workloads and the sequence-parallel
+forward (seqpar).
 """
 from .binding import (  # noqa: F401
     LONGNET_IMPL_AUTO,
@@ -19,7 +20,10 @@ from .binding import (  # noqa: F401
     load_library,
     longnet_dilated_attn_bwd,
     longnet_dilated_attn_fwd,
+    longnet_dilated_attn_fwd_part,
+    longnet_gather_rows,
     longnet_last_device_status,
+    longnet_scatter_rows,
     longnet_select_impl,
     longnet_watchdog_selftest,
     status_string,

@@ -52,6 +52,12 @@ SIGNATURES = {
                                                    _i64, ctypes.c_int, _i64p, _i64p,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, _vp]),
+    "longnet_dilated_attn_fwd_part": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                     _i64, ctypes.c_int, _i64p, _i64p,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_int, _i64, _i64, _i64, _i64, _vp]),
+    "longnet_gather_rows": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp]),
+    "longnet_scatter_rows": (ctypes.c_int, [_vp, _i64, _vp, _vp, _i64, _i64, _vp]),
     "longnet_dilated_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _i64, _i64, _i64, _i64, ctypes.c_int, _i64p,
                                                 _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -151,6 +157,73 @@ def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         _dtype_code(q), LONGNET_FLAG_QK_NORM if qk_norm else 0, int(impl), _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_fwd")
+
+
+def longnet_dilated_attn_fwd_part(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  out: torch.Tensor, lse: torch.Tensor | None,
+                                  patterns: Sequence[Tuple[int, int]], causal: bool,
+                                  q_range: Tuple[int, int], h_range: Tuple[int, int] | None = None,
+                                  impl: int = LONGNET_IMPL_AUTO, stream=None,
+                                  qk_norm: bool = False) -> None:
+    """Enqueue the forward for part of the output: positions q_range = (begin,
+    end) and heads h_range (default all) of out and lse; the rest of out and
+    lse is left as it is.  Tensors as in longnet_dilated_attn_fwd (full
+    length).  Raises LongNetError on a non-zero status."""
+    lib = load_library()
+    B, N, H, D = q.shape
+    for t in (q, k, v, out):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must be contiguous CUDA tensors of one shape and dtype")
+    if lse is not None and not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
+                                and tuple(lse.shape) == (B, H, N)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    h0, h1 = (0, H) if h_range is None else h_range
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_fwd_part(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        None if lse is None else lse.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), LONGNET_FLAG_QK_NORM if qk_norm else 0, int(impl), int(q_range[0]),
+        int(q_range[1]), int(h0), int(h1), _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_fwd_part")
+
+
+def _rows_view(t: torch.Tensor, row_elems: int):
+    if not (t.is_cuda and t.is_contiguous()) or t.numel() % row_elems != 0:
+        raise ValueError("row buffers must be contiguous CUDA tensors of whole rows")
+    return t.numel() // row_elems
+
+
+def longnet_gather_rows(src: torch.Tensor, idx: torch.Tensor, dst: torch.Tensor, row_elems: int,
+                        stream=None) -> None:
+    """dst row i = src row idx[i] (rows of row_elems elements of src's dtype);
+    idx: int64 CUDA tensor.  Raises LongNetError on a non-zero status."""
+    if idx.dtype != torch.int64 or not (idx.is_cuda and idx.is_contiguous()):
+        raise ValueError("idx must be a contiguous int64 CUDA tensor")
+    src_rows, dst_rows = _rows_view(src, row_elems), _rows_view(dst, row_elems)
+    if dst_rows != idx.numel() or src.dtype != dst.dtype:
+        raise ValueError("dst must hold one row per index, in src's dtype")
+    rc = load_library().longnet_gather_rows(src.data_ptr(), src_rows, idx.data_ptr(), idx.numel(),
+                                            dst.data_ptr(), row_elems * src.element_size(),
+                                            _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_gather_rows")
+
+
+def longnet_scatter_rows(src: torch.Tensor, idx: torch.Tensor, dst: torch.Tensor, row_elems: int,
+                         stream=None) -> None:
+    """dst row idx[i] = src row i; idx: int64 CUDA tensor.  Raises
+    LongNetError on a non-zero status."""
+    if idx.dtype != torch.int64 or not (idx.is_cuda and idx.is_contiguous()):
+        raise ValueError("idx must be a contiguous int64 CUDA tensor")
+    src_rows, dst_rows = _rows_view(src, row_elems), _rows_view(dst, row_elems)
+    if src_rows != idx.numel() or src.dtype != dst.dtype:
+        raise ValueError("src must hold one row per index, in dst's dtype")
+    rc = load_library().longnet_scatter_rows(src.data_ptr(), idx.numel(), idx.data_ptr(),
+                                             dst.data_ptr(), dst_rows, row_elems * src.element_size(),
+                                             _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_scatter_rows")
 
 
 def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -99,6 +99,10 @@ int check_args(const void* q, const void* k, const void* v, void* out, float* ls
     pb->w[i] = w[i];
     pb->r[i] = r[i];
   }
+  pb->q0 = 0;
+  pb->q1 = N;
+  pb->h0 = 0;
+  pb->h1 = H;
   return LONGNET_OK;
 }
 
@@ -131,16 +135,21 @@ __global__ void watchdog_selftest_kernel(int* status, uint64_t limit_ns) {
 
 using namespace longnet;
 
-extern "C" int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
-                                           void* out, float* lse, int64_t B, int64_t N, int64_t H,
-                                           int64_t D, int n_pat, const int64_t* w, const int64_t* r,
-                                           int causal, int dtype, int flags, int impl,
-                                           longnet_stream_t stream) {
+namespace longnet {
+namespace {
+int forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
+            int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
+            int flags, int impl, int64_t q0, int64_t q1, int64_t h0, int64_t h1, longnet_stream_t stream) {
   if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
   if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
   int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
   if (rc) return rc;
+  if (q0 < 0 || q1 > N || q0 >= q1 || h0 < 0 || h1 > H || h0 >= h1) return LONGNET_ERR_INVALID_ARG;
+  pb.q0 = q0;
+  pb.q1 = q1;
+  pb.h0 = h0;
+  pb.h1 = h1;
   pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
   int dev = 0;
   rc = current_device_state(&dev, &pb.status);
@@ -163,6 +172,60 @@ extern "C" int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const v
     default:
       return LONGNET_ERR_INVALID_ARG;
   }
+}
+}  // namespace
+}  // namespace longnet
+
+extern "C" int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
+                                           void* out, float* lse, int64_t B, int64_t N, int64_t H,
+                                           int64_t D, int n_pat, const int64_t* w, const int64_t* r,
+                                           int causal, int dtype, int flags, int impl,
+                                           longnet_stream_t stream) {
+  return forward(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, flags, impl, 0, N, 0, H,
+                 stream);
+}
+
+extern "C" int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,
+                                             void* out, float* lse, int64_t B, int64_t N,
+                                             int64_t H, int64_t D, int n_pat, const int64_t* w,
+                                             const int64_t* r, int causal, int dtype, int flags,
+                                             int impl, int64_t q_begin, int64_t q_end,
+                                             int64_t h_begin, int64_t h_end,
+                                             longnet_stream_t stream) {
+  return forward(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, flags, impl, q_begin,
+                 q_end, h_begin, h_end, stream);
+}
+
+namespace longnet {
+namespace {
+int move_rows(const void* src, const int64_t* src_idx, int64_t src_rows, void* dst, const int64_t* dst_idx,
+              int64_t dst_rows, int64_t n, int64_t row_bytes, longnet_stream_t stream) {
+  if (n < 0 || src_rows < 0 || dst_rows < 0 || row_bytes <= 0 || row_bytes % 16 != 0 ||
+      row_bytes > ((int64_t)1 << 20))
+    return LONGNET_ERR_INVALID_ARG;
+  if (n == 0) return LONGNET_OK;
+  if (!src || !dst || (!src_idx && !dst_idx)) return LONGNET_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(dst, 16) || (src_idx && !aligned(src_idx, 8)) ||
+      (dst_idx && !aligned(dst_idx, 8)))
+    return LONGNET_ERR_MISALIGNED;
+  int dev = 0;
+  int* status = nullptr;
+  int rc = current_device_state(&dev, &status);
+  if (rc) return rc;
+  return launch_move_rows(src, src_idx, src_rows, dst, dst_idx, dst_rows, n, row_bytes, status,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+}  // namespace
+}  // namespace longnet
+
+extern "C" int longnet_gather_rows(const void* src, int64_t src_rows, const int64_t* idx, int64_t n,
+                                   void* dst, int64_t row_bytes, longnet_stream_t stream) {
+  return move_rows(src, idx, src_rows, dst, nullptr, n, n, row_bytes, stream);
+}
+
+extern "C" int longnet_scatter_rows(const void* src, int64_t n, const int64_t* idx, void* dst,
+                                    int64_t dst_rows, int64_t row_bytes, longnet_stream_t stream) {
+  return move_rows(src, nullptr, n, dst, idx, dst_rows, n, row_bytes, stream);
 }
 
 extern "C" int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,

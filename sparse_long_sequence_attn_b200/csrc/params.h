@@ -20,6 +20,10 @@ struct Problem {
   int causal;
   int dtype;
   int qk_norm;  // 1: q and k rows are scaled to unit L2 norm first (LONGNET_FLAG_QK_NORM)
+  // The part of the output computed: positions [q0, q1) and heads [h0, h1)
+  // (the whole output: 0, N, 0, H).  Keys and values are read wherever the
+  // method needs them, inside or outside the part.
+  int64_t q0, q1, h0, h1;
   int64_t w[LONGNET_MAX_PATTERNS];
   int64_t r[LONGNET_MAX_PATTERNS];
   int* status;  // device address of this device's status word
@@ -48,6 +52,13 @@ int launch_simt(const Problem& p, cudaStream_t stream);
 int launch_tcgen05(const Problem& p, cudaStream_t stream);
 int launch_smallseg(const Problem& p, cudaStream_t stream);
 int launch_backward(const Problem& p, const BwdArgs& g, int impl, cudaStream_t stream);
+
+// Row moves of the sequence-parallel exchange: dst[dst_idx[i]] = src[src_idx[i]]
+// for i < n (a null index array is the identity), rows of row_bytes (a
+// multiple of 16) bytes; indices checked against src_rows / dst_rows.
+int launch_move_rows(const void* src, const int64_t* src_idx, int64_t src_rows, void* dst,
+                     const int64_t* dst_idx, int64_t dst_rows, int64_t n, int64_t row_bytes, int* status,
+                     cudaStream_t stream);
 
 // Shape checks of the specialised families (host only, no device access).
 bool tcgen05_supports(const Problem& p);

@@ -75,12 +75,14 @@ __global__ void __launch_bounds__(kWarps * 32) simt_kernel(const Problem p) {
   __shared__ float qsh[kWarps][D];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  // rows of the computed part: positions [q0, q1), heads [h0, h1)
   const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
-  const int64_t n_rows = p.B * p.N * p.H;
+  const int64_t Hr = p.h1 - p.h0, Nr = p.q1 - p.q0;
+  const int64_t n_rows = p.B * Nr * Hr;
   if (row >= n_rows) return;
-  const int64_t h = row % p.H;
-  const int64_t pos = (row / p.H) % p.N;
-  const int64_t b = row / (p.H * p.N);
+  const int64_t h = p.h0 + row % Hr;
+  const int64_t pos = p.q0 + (row / Hr) % Nr;
+  const int64_t b = row / (Hr * Nr);
   const T* Q = static_cast<const T*>(p.q);
   const T* K = static_cast<const T*>(p.k);
   const T* V = static_cast<const T*>(p.v);
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kWarps * 32) simt_kernel(const Problem p) {
 
 template <typename T>
 int launch_typed(const Problem& p, cudaStream_t stream) {
-  const int64_t n_rows = p.B * p.N * p.H;
+  const int64_t n_rows = p.B * (p.q1 - p.q0) * (p.h1 - p.h0);
   const int64_t blocks = (n_rows + kWarps - 1) / kWarps;
   if (blocks > 0x7fffffffLL) return LONGNET_ERR_UNSUPPORTED;
   dim3 grid((unsigned)blocks), block(kWarps * 32);

@@ -58,7 +58,7 @@ struct Params {
   uint32_t rcp16[kMaxPat];  // ceil(2^16 / r): (x * rcp16) >> 16 = x / r for 0 <= x < 64
   int pair_bytes;           // shared memory per warp pair (1024-aligned)
   int n_pairs;
-  int64_t n_items;          // B * (N / W) * H
+  int64_t n_items;          // B * (segments of the part) * (heads of the part)
   uint64_t wait_limit_ns;
 };
 
@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
   const int W = P.W, n_pat = P.pb.n_pat;
   const int H = (int)P.pb.H;
   const int64_t N = P.pb.N;
-  const int n_seg = (int)(N / W);
+  const int seg0 = (int)(P.pb.q0 / W), n_seg = (int)((P.pb.q1 - P.pb.q0) / W);
+  const int h0 = (int)P.pb.h0, Hr = (int)(P.pb.h1 - P.pb.h0);
   const bool causal = P.pb.causal != 0;
   const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
   const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
@@ -333,9 +334,9 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
 
   for (int64_t item = (int64_t)blockIdx.x * P.n_pairs + pair; item < P.n_items;
        item += (int64_t)gridDim.x * P.n_pairs, phase ^= 1) {
-    const int h = (int)(item % H);
-    const int64_t bs = item / H;
-    const int seg = (int)(bs % n_seg);
+    const int h = h0 + (int)(item % Hr);
+    const int64_t bs = item / Hr;
+    const int seg = seg0 + (int)(bs % n_seg);
     const int b = (int)(bs / n_seg);
     // ---- load the segment's rows of this head (both warps are done with the
     // previous item: the pair synchronised at its end)
@@ -567,6 +568,7 @@ bool smallseg_supports(const Problem& p) {
   for (int i = 0; i < p.n_pat; ++i)
     if (p.w[i] != W) return false;
   if (W > p.N || p.N % W != 0) return false;  // whole segments only
+  if (p.q0 % W != 0 || p.q1 % W != 0) return false;  // a part of whole segments
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.r[i] < 1 || p.r[i] > (int64_t)INT32_MAX) return false;
@@ -596,7 +598,9 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   P.n_pairs = (kSmemLimit - 1024) / P.pair_bytes;
   if (P.n_pairs > kMaxPairs) P.n_pairs = kMaxPairs;
   if (P.n_pairs < 1) return LONGNET_ERR_UNSUPPORTED;
-  P.n_items = pb.B * (pb.N / P.W) * pb.H;
+  // items of the computed part: (b, segment, head) with segments in
+  // [q0 / W, q1 / W) and heads in [h0, h1)
+  P.n_items = pb.B * ((pb.q1 - pb.q0) / P.W) * (pb.h1 - pb.h0);
   int dev = 0, n_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
       cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

@@ -186,7 +186,8 @@ struct Params {
   FastDiv r_div[kMaxR];       // division by r_val
   FastDiv w_div[kMaxPat];     // division by each pattern's w
   int range_len;              // R
-  int n_ranges;               // ceil(N / R)
+  int range_first;            // first range of the computed part: floor(q0 / R)
+  int n_ranges;               // ranges meeting the part [q0, q1)
   int n_units;                // ranges, some of them split in halves
   int uncovered_possible;     // some position may be kept by no pattern
   int stages;                 // K/V ring depth
@@ -197,20 +198,24 @@ struct Params {
   int unit_code[kMaxRangeOrder];
 };
 
-// Positions [A, Bnd) of the unit a CTA of rank `rank` works on.
+// Positions [A, Bnd) of the unit a CTA of rank `rank` works on: range i
+// covers [i R, (i + 1) R), a split unit one half of it, both clipped to the
+// computed part [q0, q1) (so a unit may be empty).
 __host__ __device__ inline void unit_bounds(const Params& P, int64_t rank, int& A, int& Bnd) {
   const int R = P.range_len;
-  int i = (int)rank, len = R, off = 0;
+  int i = P.range_first + (int)rank, len = R, off = 0;
   if (P.unit_code[0] >= 0 && rank < kMaxRangeOrder) {
     const int c = P.unit_code[rank];
-    i = c >> 2;
+    i = P.range_first + (c >> 2);
     if (c & 1) {
       len = R / 2;
       off = ((c >> 1) & 1) * len;
     }
   }
-  A = i * R + off;
-  Bnd = (int64_t)A + len < P.pb.N ? A + len : (int)P.pb.N;
+  const int64_t a = (int64_t)i * R + off, e = a + len;
+  A = (int)(a > P.pb.q0 ? a : P.pb.q0);
+  Bnd = (int)(e < P.pb.q1 ? e : P.pb.q1);
+  if (Bnd < A) Bnd = A;
 }
 
 // ---------------------------------------------------------------- PTX bits
@@ -789,12 +794,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // unit -> (b, h, range)
-  const int64_t BH = P.pb.B * P.pb.H;
+  // unit -> (b, h, range), h among the part's heads [h0, h1)
+  const int64_t Hr = P.pb.h1 - P.pb.h0;
+  const int64_t BH = P.pb.B * Hr;
   const int64_t rank = blockIdx.x / BH;
   const int64_t bh = blockIdx.x - rank * BH;
-  const int64_t b = bh / P.pb.H;
-  const int64_t h = bh - b * P.pb.H;
+  const int64_t b = bh / Hr;
+  const int64_t h = P.pb.h0 + (bh - b * Hr);
   int A, Bnd;
   unit_bounds(P, rank, A, Bnd);
   const int n_pat = P.pb.n_pat;
@@ -1509,12 +1515,16 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
   }
   // A unit spans 128 * r_max positions, so the coarsest pattern's tiles are
   // full; while that leaves SMs idle, halve it (its tiles are then partial).
-  P.range_len = kBM * r_max_of(pb);
-  P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
-  while ((int64_t)P.n_ranges * pb.B * pb.H < n_sm && P.range_len >= 2 * kBM && P.range_len % 2 == 0) {
-    P.range_len /= 2;
-    P.n_ranges = (int)((pb.N + P.range_len - 1) / P.range_len);
-  }
+  // Ranges are aligned to multiples of R and clipped to the computed part.
+  const int64_t Hr = pb.h1 - pb.h0;
+  auto set_ranges = [&](int64_t R) {
+    P.range_len = (int)R;
+    P.range_first = (int)(pb.q0 / R);
+    P.n_ranges = (int)((pb.q1 + R - 1) / R - pb.q0 / R);
+  };
+  set_ranges(kBM * r_max_of(pb));
+  while ((int64_t)P.n_ranges * pb.B * Hr < n_sm && P.range_len >= 2 * kBM && P.range_len % 2 == 0)
+    set_ranges(P.range_len / 2);
   P.n_units = P.n_ranges;
   P.unit_code[0] = -1;
   if (P.n_ranges <= kMaxRangeOrder) {
@@ -1533,9 +1543,16 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     static int idx[kMaxRangeOrder];
     static Unit u[kMaxRangeOrder + 8];
     static int64_t heap[kMaxHeapSms];
-    const int64_t R = P.range_len, N = pb.N, BH = pb.B * pb.H;
+    const int64_t R = P.range_len, BH = pb.B * Hr;
+    // range i of the plan covers [(range_first + i) R, ...) clipped to the part
+    auto clip_cost = [&](int64_t a, int64_t e) -> int64_t {
+      a = std::max<int64_t>(a, pb.q0);
+      e = std::min<int64_t>(e, pb.q1);
+      return a < e ? range_cost(pb, a, e) : 0;
+    };
     for (int i = 0; i < P.n_ranges; ++i) {
-      cost[i] = range_cost(pb, i * R, std::min<int64_t>(N, (i + 1) * R));
+      const int64_t a = (P.range_first + (int64_t)i) * R;
+      cost[i] = clip_cost(a, a + R);
       idx[i] = i;
     }
     // longest first; equal costs in range order
@@ -1546,9 +1563,9 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
         const int i = idx[t];
         if (t < k) {
           for (int hf = 0; hf < 2; ++hf) {
-            const int64_t a = i * R + hf * (R / 2);
-            if (a >= N) continue;
-            u[n++] = {range_cost(pb, a, std::min<int64_t>(N, a + R / 2)), (i << 2) | (hf << 1) | 1};
+            const int64_t a = (P.range_first + (int64_t)i) * R + hf * (R / 2);
+            if (std::max<int64_t>(a, pb.q0) >= std::min<int64_t>(a + R / 2, pb.q1)) continue;
+            u[n++] = {clip_cost(a, a + R / 2), (i << 2) | (hf << 1) | 1};
           }
         } else {
           u[n++] = {cost[i], i << 2};
@@ -1617,7 +1634,8 @@ struct LaunchCache {
 };
 inline bool same_shape(const Problem& a, const Problem& b) {
   if (a.B != b.B || a.N != b.N || a.H != b.H || a.D != b.D || a.n_pat != b.n_pat ||
-      a.causal != b.causal || a.dtype != b.dtype)
+      a.causal != b.causal || a.dtype != b.dtype || a.q0 != b.q0 || a.q1 != b.q1 || a.h0 != b.h0 ||
+      a.h1 != b.h1)
     return false;
   for (int i = 0; i < a.n_pat; ++i)
     if (a.w[i] != b.w[i] || a.r[i] != b.r[i]) return false;
@@ -1671,7 +1689,7 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
       return LONGNET_ERR_CUDA;
     attr_set[dev][f16] = true;
   }
-  const int64_t grid = (int64_t)P.n_units * pb.B * pb.H;
+  const int64_t grid = (int64_t)P.n_units * pb.B * (pb.h1 - pb.h0);
   kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, c.maps);
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }

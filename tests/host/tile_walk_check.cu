@@ -47,12 +47,16 @@ void check_tma(const Params& P, int ri, int64_t first, int64_t need, int64_t r) 
 }
 
 bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std::pair<int64_t, int64_t>> pats, int causal,
-              int sms = 148, bool quiet = false) {
+              int sms = 148, bool quiet = false, int64_t q0 = 0, int64_t q1 = -1, int64_t h0 = 0, int64_t h1 = -1) {
   Problem pb;
   memset(&pb, 0, sizeof(pb));
   pb.B = B; pb.N = N; pb.H = H; pb.D = 64; pb.n_pat = (int)pats.size(); pb.causal = causal;
   pb.dtype = LONGNET_DTYPE_BF16;
   for (int i = 0; i < pb.n_pat; ++i) { pb.w[i] = pats[i].first; pb.r[i] = pats[i].second; }
+  pb.q0 = q0;
+  pb.q1 = q1 < 0 ? N : q1;
+  pb.h0 = h0;
+  pb.h1 = h1 < 0 ? H : h1;
   if (!tcgen05_supports(pb)) {
     if (!quiet) printf("%s: not supported\n", name);
     return false;
@@ -62,14 +66,14 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
   int f0 = fails;
   long n_tiles = 0, n_kv = 0;
   // coverage: (p, h, seg, k) -> count
-  for (int64_t h = 0; h < H; ++h) {
+  for (int64_t h = pb.h0; h < pb.h1; ++h) {
     std::map<std::tuple<int, int64_t, int64_t>, int> seen;
     std::vector<int> finalized(N, 0);
     for (int rank = 0; rank < P.n_units; ++rank) {
       int A32, B32;
       unit_bounds(P, rank, A32, B32);
       const int64_t A = A32, Bnd = B32;
-      CHECK(A < Bnd, "%s: empty unit %d\n", name, rank);
+      CHECK(A >= pb.q0 && Bnd <= pb.q1, "%s: unit [%ld, %ld) outside the part\n", name, (long)A, (long)Bnd);
       TileWalker tw;
       tw.init(P, h, A, Bnd);
       Tile t;
@@ -139,6 +143,8 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
       int64_t m = o >= w ? 0 : (w - o + r - 1) / r;
       for (int64_t seg = 0; seg < N / w; ++seg)
         for (int64_t k = 0; k < m; ++k) {
+          const int64_t xk = seg * w + o + r * k;
+          if (xk < pb.q0 || xk >= pb.q1) continue;  // outside the computed part
           auto it = seen.find(std::make_tuple(p, seg, k));
           CHECK(it != seen.end() && it->second == 1, "%s: row p=%d seg=%ld k=%ld seen %d times\n", name, p, (long)seg, (long)k, it == seen.end() ? 0 : it->second);
         }
@@ -150,7 +156,8 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
         int64_t rel = x - (x / w) * w - o;
         if (rel >= 0 && rel % r == 0) covered = true;
       }
-      CHECK(finalized[x] == (covered ? 1 : 0), "%s: position %ld finalized %d times (covered %d)\n", name, (long)x, finalized[x], covered);
+      const bool in_part = x >= pb.q0 && x < pb.q1;
+      CHECK(finalized[x] == (covered && in_part ? 1 : 0), "%s: position %ld finalized %d times (covered %d)\n", name, (long)x, finalized[x], covered);
       if (!covered) CHECK(P.uncovered_possible, "%s: uncovered position but flag off\n", name);
     }
   }
@@ -233,6 +240,13 @@ int main() {
   run_case("odd_mix", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 1);
   run_case("odd_mix_nc", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 0);
   run_case("sweep1M_part", 1, 1048576, 1, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 8}, {32768, 16}, {65536, 32}}, 1);
+  // computed parts: a sequence shard (positions), a head range, unaligned bounds
+  run_case("long32k_shard1of2", 1, 32768, 12, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 6}, {32768, 12}}, 1, 148,
+           false, 16384, 32768);
+  run_case("long32k_shard3of4_heads", 1, 32768, 12, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 6}, {32768, 12}}, 1,
+           148, false, 16384, 24576, 3, 9);
+  run_case("lm_unaligned_part", 1, 8192, 12, {{2048, 1}, {4096, 2}, {8192, 4}}, 1, 148, false, 1000, 7001, 5, 6);
+  run_case("noncausal_part", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 0, 132, false, 777, 4321, 1, 7);
   random_cases(300);
   printf("fails=%d\n", fails);
   return fails ? 1 : 0;

@@ -165,3 +165,44 @@ def test_backward_tile_grid_limit_on_host():
     if not torch.cuda.is_available():
         assert _call_bwd(lib, N=N2, D=64, dtype=1, pats=((N2, 1),),
                          impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
+
+
+def _call_part(lib, q_range=(0, 64), h_range=(0, 2), N=64, H=2):
+    buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+    return lib.longnet_dilated_attn_fwd_part(buf, buf, buf, buf, None, 1, N, H, 16, 1, w, r, 1, 0, 0, 0,
+                                             q_range[0], q_range[1], h_range[0], h_range[1], None)
+
+
+@pytest.mark.parametrize("q_range,h_range", [
+    ((-1, 64), (0, 2)), ((0, 65), (0, 2)), ((32, 32), (0, 2)), ((40, 8), (0, 2)),
+    ((0, 64), (-1, 2)), ((0, 64), (0, 3)), ((0, 64), (1, 1)),
+])
+def test_part_ranges_checked_on_host(q_range, h_range):
+    assert _call_part(bd.load_library(), q_range, h_range) == bd.LONGNET_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_part_valid_ranges_reach_the_device_check():
+    lib = bd.load_library()
+    for qr, hr in (((0, 64), (0, 2)), ((17, 33), (1, 2)), ((63, 64), (0, 1))):
+        assert _call_part(lib, qr, hr) == bd.LONGNET_ERR_NO_DEVICE
+
+
+def test_row_moves_checked_on_host():
+    lib = bd.load_library()
+    buf, idx = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000)
+    g, s = lib.longnet_gather_rows, lib.longnet_scatter_rows
+    assert g(buf, 10, idx, 0, buf, 128, None) == bd.LONGNET_OK  # nothing to move
+    assert g(buf, 10, idx, -1, buf, 128, None) == bd.LONGNET_ERR_INVALID_ARG
+    assert g(buf, 10, idx, 4, buf, 24, None) == bd.LONGNET_ERR_INVALID_ARG  # not whole 16-byte words
+    assert g(buf, 10, idx, 4, buf, 0, None) == bd.LONGNET_ERR_INVALID_ARG
+    assert g(buf, 10, None, 4, buf, 128, None) == bd.LONGNET_ERR_INVALID_ARG
+    assert g(ctypes.c_void_p(0x1008), 10, idx, 4, buf, 128, None) == bd.LONGNET_ERR_MISALIGNED
+    assert g(buf, 10, ctypes.c_void_p(0x2004), 4, buf, 128, None) == bd.LONGNET_ERR_MISALIGNED
+    assert s(buf, 4, idx, ctypes.c_void_p(0x1004), 10, 128, None) == bd.LONGNET_ERR_MISALIGNED
+    assert s(buf, 4, idx, buf, -1, 128, None) == bd.LONGNET_ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        assert g(buf, 10, idx, 4, buf, 128, None) == bd.LONGNET_ERR_NO_DEVICE
+        assert s(buf, 4, idx, buf, 10, 128, None) == bd.LONGNET_ERR_NO_DEVICE
