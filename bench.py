@@ -255,6 +255,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="linear-scaling sweep instead")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave the linear-scaling sweep out of the default line")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="leave the one-change variants of the 32K shape out of the default line")
     ap.add_argument("--soak-s", type=float, default=1.0,
                     help="seconds of repeated steps after the timed region, for the clock record")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=("fwd", "bwd"),
@@ -456,6 +458,8 @@ def run_ours(args, wl):
     if ws == 1 and wl.name == "long32k" and not args.no_sweep:
         line["sweep"] = sweep_lines(args.steps, args.warmup, args.kernel, dev.index)
         line["sweep_linear_1M_vs_64K"] = line["sweep"][-1]["tokens_per_s_vs_65536"]
+    if ws == 1 and wl.name == "long32k" and not args.no_variants:
+        line["variants"] = variant_lines(args.steps, args.warmup, dev.index)
     if ws == 1 and not args.no_cpu_baseline:
         n = args.cpu_positions
         calibrate = n <= 0
@@ -706,6 +710,72 @@ def sweep_lines(steps, warmup, kernel="auto", dev_index=0):
     base = res[0]["tokens_per_s"]
     for r in res:
         r["tokens_per_s_vs_65536"] = r["tokens_per_s"] / base
+    return res
+
+
+def variant_lines(steps, warmup, dev_index=0):
+    """The 32K-token shape (B 1, H 12, D 64, five patterns, causal) with one
+    thing changed at a time, each timed like the main line (CUDA events, L2
+    flush between steps): the input options through the prologue pass
+    (longnet_dilated_attn_fwd_ws: qk_norm, XPOS), qk_norm inside the kernel
+    (longnet_dilated_attn_fwd_ex, which AUTO sends to the family that takes
+    it), a sequence 64 tokens short (a partial last segment) and D = 128
+    (H 6).  Reports the family AUTO picked for each.  Inputs drawn on the
+    device; parity of each variant is tested separately."""
+    import torch
+
+    from sparse_long_sequence_attn_b200 import binding as bd
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    dev = torch.device("cuda", dev_index)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    base = wlm.WORKLOADS["long32k"]
+    res = []
+    cases = [("plain", base.N, base.H, base.D, "plain"), ("qk_norm_prologue", base.N, base.H, base.D, "ws_norm"),
+             ("xpos_prologue", base.N, base.H, base.D, "ws_xpos"),
+             ("qk_norm_in_kernel", base.N, base.H, base.D, "ex_norm"),
+             ("partial_last_segment", base.N - 64, base.H, base.D, "plain"),
+             ("d128", base.N, base.H // 2, 128, "plain")]
+    for name, N, H, D, mode in cases:
+        g = torch.Generator(device=dev)
+        g.manual_seed(base.seed)
+        qd, kd, vd = (torch.randn(base.B, N, H, D, device=dev, generator=g,
+                                  dtype=torch.float32).to(torch.bfloat16) for _ in range(3))
+        out = torch.empty_like(qd)
+        lse = torch.empty((base.B, H, N), device=dev, dtype=torch.float32)
+        qk_norm = mode in ("ws_norm", "ex_norm")
+        xpos = mode == "ws_xpos"
+        ws = None
+        if mode.startswith("ws"):
+            ws = torch.empty(bd.longnet_fwd_workspace_bytes(base.B, N, H, D, torch.bfloat16, qk_norm, xpos),
+                             dtype=torch.uint8, device=dev)
+
+        def step():
+            if ws is not None:
+                bd.longnet_dilated_attn_fwd_ws(qd, kd, vd, out, lse, base.patterns, base.causal, ws,
+                                               bd.LONGNET_IMPL_AUTO, stream, qk_norm, xpos)
+            else:
+                bd.longnet_dilated_attn_fwd(qd, kd, vd, out, lse, base.patterns, base.causal,
+                                            bd.LONGNET_IMPL_AUTO, stream, qk_norm)
+
+        # one untimed call to see how long a step takes; slow families get fewer steps
+        t0 = time.time()
+        step()
+        torch.cuda.synchronize()
+        n = steps if time.time() - t0 < 0.05 else 3
+        per = time_steps(step, n, min(warmup, 3), stream, flush)
+        st = bd.longnet_last_device_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status after variant {name}: {bd.status_string(st)}")
+        fam = _impl_name(bd.longnet_select_impl(base.B, N, H, D, base.patterns, base.causal, torch.bfloat16))
+        if mode == "ex_norm":
+            fam = "simt or smallseg (the families that apply qk_norm in the kernel)"
+        t = sum(per) / len(per)
+        res.append({"variant": name, "N": N, "H": H, "D": D, "family": fam, "steps": n,
+                    "ms": t * 1e3, "tokens_per_s": base.B * N / t})
+        del qd, kd, vd, out, lse, ws
+        torch.cuda.empty_cache()
     return res
 
 

@@ -109,22 +109,40 @@ int longnet_dilated_attn_fwd_impl(const void* q, const void* k, const void* v,
                                   int causal, int dtype, int impl,
                                   longnet_stream_t stream);
 
-/* Options of longnet_dilated_attn_fwd_ex (a bit set). */
+/* Options of the forward (a bit set). */
 enum longnet_flags {
   /* Scale every q row and every k row (over D) to unit L2 norm before the
-   * scores: x / max(|x|, 1e-12), computed in fp32 (the small-segment kernel
-   * then rounds the rows back to the input format, the SIMT kernel keeps them
-   * in fp32).  The reading adopted for the qk_norm
-   * option of the DilatedAttention module ("LongNet" docs page, usage
-   * example).  The SIMT and small-segment kernels take it; the tcgen05 kernel
-   * does not (LONGNET_IMPL_AUTO falls back). */
-  LONGNET_FLAG_QK_NORM = 1
+   * scores: x / max(|x|, 1e-12), computed in fp32.  The reading adopted for
+   * the qk_norm option of the DilatedAttention module ("LongNet" docs page,
+   * usage example).  Through longnet_dilated_attn_fwd_ex the SIMT and
+   * small-segment kernels apply it inside the attention (the small-segment
+   * kernel then rounds the rows back to the input format, the SIMT kernel
+   * keeps them in fp32) and the tcgen05 kernel declines it (AUTO falls
+   * back); through longnet_dilated_attn_fwd_ws a prologue pass applies it
+   * and every family takes the result. */
+  LONGNET_FLAG_QK_NORM = 1,
+  /* XPOS on q and k, the rotary position encoding with exponential scaling
+   * that the use_xpos option names ("LongNet论文精读", section "Dilated
+   * Attention的核心参数解析"; the pages give no formula, the published XPOS
+   * definition of Sun et al., "A Length-Extrapolatable Transformer", is
+   * taken).  For the element pair (2i, 2i+1) of a row at position n:
+   * theta_i = 10000^(-2i/D), zeta_i = (2i + 0.4 D) / (1.4 D),
+   * s = zeta_i^((n - floor(N/2)) / 512); queries become
+   * s (x0 cos(n theta_i) - x1 sin(n theta_i), x1 cos(n theta_i) + x0 sin(n theta_i))
+   * and keys the same with 1/s, so a score depends on the positions' difference
+   * only.  Applied after the norm when both flags are set, computed in fp32
+   * and rounded to the input format.  longnet_dilated_attn_fwd_ws only.  The
+   * scales must stay in the input format's range: |log2 s| <= 100 (fp32,
+   * bf16: N <= 56,000 or so) or <= 8 (fp16: N <= 4,500 or so), else
+   * LONGNET_ERR_UNSUPPORTED. */
+  LONGNET_FLAG_XPOS = 2
 };
 
 /*
  * longnet_dilated_attn_fwd_ex — the forward with options (flags, a
  * longnet_flags bit set) and an explicit kernel family (impl, as in
- * longnet_dilated_attn_fwd_impl).  Unknown flag bits: LONGNET_ERR_INVALID_ARG.
+ * longnet_dilated_attn_fwd_impl).  flags: LONGNET_FLAG_QK_NORM or 0; any
+ * other bit (LONGNET_FLAG_XPOS included): LONGNET_ERR_INVALID_ARG.
  * The two entry points above are this call with flags = 0.
  */
 int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
@@ -132,6 +150,42 @@ int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const void* v,
                                 int64_t B, int64_t N, int64_t H, int64_t D,
                                 int n_pat, const int64_t* w, const int64_t* r,
                                 int causal, int dtype, int flags, int impl,
+                                longnet_stream_t stream);
+
+/*
+ * longnet_fwd_workspace_bytes — device workspace, in bytes, that
+ * longnet_dilated_attn_fwd_ws needs for these sizes, dtype and flags: 0 for
+ * flags = 0, else two tensors of B*N*H*D elements of dtype (the transformed
+ * q and k), each rounded up to 256 bytes.  Invalid sizes, dtype or flag
+ * bits: LONGNET_ERR_INVALID_ARG (negative).
+ */
+int64_t longnet_fwd_workspace_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int dtype, int flags);
+
+/*
+ * longnet_dilated_attn_fwd_ws — the forward with the input-side options
+ * (flags: LONGNET_FLAG_QK_NORM, LONGNET_FLAG_XPOS, or both) applied by a
+ * prologue pass: q and k are read once, transformed (norm first, then
+ * XPOS) and written to the caller's workspace, and the attention (family
+ * impl, AUTO picking as for the plain forward) runs on the workspace's q
+ * and k and the caller's v, both launches on `stream` in that order.  The
+ * options of the DilatedAttention module ("LongNet" docs page, usage
+ * example; "LongNet论文精读", section "Dilated Attention的核心参数解析").
+ *   workspace: device memory owned by the caller, 256-byte aligned
+ *     (else LONGNET_ERR_MISALIGNED), at least longnet_fwd_workspace_bytes
+ *     bytes (else LONGNET_ERR_INVALID_ARG), overlapping none of q, k, v, out,
+ *     lse; its contents on entry do not matter and on return are the
+ *     transformed q and k.  Unused when flags = 0 (the call is then
+ *     longnet_dilated_attn_fwd_ex with flags 0; workspace may be null).
+ *   D a multiple of 16, at most 128, for the prologue; XPOS range limits as
+ *   stated at LONGNET_FLAG_XPOS (LONGNET_ERR_UNSUPPORTED).  The other
+ *   arguments, results and errors are those of longnet_dilated_attn_fwd_ex.
+ */
+int longnet_dilated_attn_fwd_ws(const void* q, const void* k, const void* v,
+                                void* out, float* lse,
+                                int64_t B, int64_t N, int64_t H, int64_t D,
+                                int n_pat, const int64_t* w, const int64_t* r,
+                                int causal, int dtype, int flags, int impl,
+                                void* workspace, int64_t workspace_bytes,
                                 longnet_stream_t stream);
 
 /*

@@ -82,16 +82,59 @@ def qk_normalize_fp64(x) -> np.ndarray:
     return x / np.maximum(n, 1e-12)
 
 
-def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None, qk_norm=False):
+def xpos_fp64(x, downscale=False) -> np.ndarray:
+    """XPOS applied to x [B, N, H, D] (D even) by absolute position n = 0..N-1,
+    in fp64.  The use_xpos option is named by "LongNet论文精读" (section
+    "Dilated Attention的核心参数解析") without a formula; this is the
+    published XPOS definition (Sun et al., "A Length-Extrapolatable
+    Transformer"), element pairs (2i, 2i+1):
+        theta_i = 10000^(-2i/D)           rotation frequency of pair i
+        zeta_i  = (2i + 0.4 D) / (1.4 D)  decay base of pair i
+        s(n)    = zeta_i^((n - c) / 512), c = floor(N / 2)
+        pair at n -> s(n) * R(n theta_i) (x_2i, x_2i+1)
+    with R(a) the rotation by angle a; keys (downscale=True) use 1 / s(n).
+    The centring c cancels in every query-key product; it keeps the scales
+    near 1."""
+    x = _f64(x)
+    B, N, H, D = x.shape
+    if D % 2:
+        raise ValueError("XPOS needs an even head dimension")
+    n = np.arange(N, dtype=np.float64)[:, None]            # [N, 1]
+    i = np.arange(D // 2, dtype=np.float64)[None, :]       # [1, D/2]
+    theta = 10000.0 ** (-2.0 * i / D)
+    zeta = (2.0 * i + 0.4 * D) / (1.4 * D)
+    s = zeta ** ((n - (N // 2)) / 512.0)                   # [N, D/2]
+    if downscale:
+        s = 1.0 / s
+    ang = n * theta
+    cos = (np.cos(ang) * s)[None, :, None, :]
+    sin = (np.sin(ang) * s)[None, :, None, :]
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = x0 * cos - x1 * sin
+    y[..., 1::2] = x1 * cos + x0 * sin
+    return y
+
+
+def _prologue(q, k, qk_norm, xpos):
+    """The input-side options in their order: the norm, then XPOS."""
+    if qk_norm:
+        q, k = qk_normalize_fp64(q), qk_normalize_fp64(k)
+    if xpos:
+        q, k = xpos_fp64(q), xpos_fp64(k, downscale=True)
+    return q, k
+
+
+def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None, qk_norm=False, xpos=False):
     """Full fp64 forward.  q, k, v: [B, N, H, D].  patterns: [(w, r), ...].
-    qk_norm: normalise q and k rows first (qk_normalize_fp64).
+    qk_norm: normalise q and k rows first (qk_normalize_fp64); xpos: then
+    apply XPOS to them (xpos_fp64).
 
     Returns (out [B, N, H, D] float64, lse [B, H, N] float64).
     """
     lib = lib or load_library()
     q, k, v = _f64(q), _f64(k), _f64(v)
-    if qk_norm:
-        q, k = qk_normalize_fp64(q), qk_normalize_fp64(k)
+    q, k = _prologue(q, k, qk_norm, xpos)
     B, N, H, D = q.shape
     w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)
     r = np.ascontiguousarray([p[1] for p in patterns], dtype=np.int64)
@@ -105,15 +148,16 @@ def dilated_attn_fp64(q, k, v, patterns, causal=True, lib=None, qk_norm=False):
     return out, lse
 
 
-def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None, qk_norm=False):
+def dilated_attn_rows_fp64(q, k, v, patterns, rows_bph, causal=True, lib=None, qk_norm=False,
+                           xpos=False):
     """fp64 forward of selected rows only.  rows_bph: int array [n, 3] of (b, pos, h).
+    qk_norm, xpos: as in dilated_attn_fp64.
 
     Returns (out_rows [n, D], lse_rows [n]).
     """
     lib = lib or load_library()
     q, k, v = _f64(q), _f64(k), _f64(v)
-    if qk_norm:
-        q, k = qk_normalize_fp64(q), qk_normalize_fp64(k)
+    q, k = _prologue(q, k, qk_norm, xpos)
     B, N, H, D = q.shape
     rows = np.ascontiguousarray(np.asarray(rows_bph, dtype=np.int64).reshape(-1, 3))
     w = np.ascontiguousarray([p[0] for p in patterns], dtype=np.int64)

@@ -21,6 +21,8 @@ from .binding import (  # noqa: F401
     longnet_dilated_attn_bwd,
     longnet_dilated_attn_fwd,
     longnet_dilated_attn_fwd_part,
+    longnet_dilated_attn_fwd_ws,
+    longnet_fwd_workspace_bytes,
     longnet_gather_rows,
     longnet_last_device_status,
     longnet_scatter_rows,

@@ -29,6 +29,7 @@ LONGNET_DTYPE_F32 = 0
 LONGNET_DTYPE_BF16 = 1
 LONGNET_DTYPE_F16 = 2
 LONGNET_FLAG_QK_NORM = 1
+LONGNET_FLAG_XPOS = 2
 
 LONGNET_IMPL_AUTO = 0
 LONGNET_IMPL_SIMT = 1
@@ -56,6 +57,11 @@ SIGNATURES = {
                                                      _i64, ctypes.c_int, _i64p, _i64p,
                                                      ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                      ctypes.c_int, _i64, _i64, _i64, _i64, _vp]),
+    "longnet_fwd_workspace_bytes": (ctypes.c_int64, [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int]),
+    "longnet_dilated_attn_fwd_ws": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                                   ctypes.c_int, _i64p, _i64p, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _i64,
+                                                   _vp]),
     "longnet_gather_rows": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp]),
     "longnet_scatter_rows": (ctypes.c_int, [_vp, _i64, _vp, _vp, _i64, _i64, _vp]),
     "longnet_dilated_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -159,6 +165,51 @@ def longnet_dilated_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise LongNetError(rc, "longnet_dilated_attn_fwd")
 
 
+def _flags(qk_norm: bool, xpos: bool) -> int:
+    return (LONGNET_FLAG_QK_NORM if qk_norm else 0) | (LONGNET_FLAG_XPOS if xpos else 0)
+
+
+def longnet_fwd_workspace_bytes(B: int, N: int, H: int, D: int, dtype: torch.dtype, qk_norm: bool = False,
+                                xpos: bool = False) -> int:
+    """Device workspace bytes longnet_dilated_attn_fwd_ws needs (0 without options)."""
+    code = {torch.float32: LONGNET_DTYPE_F32, torch.bfloat16: LONGNET_DTYPE_BF16,
+            torch.float16: LONGNET_DTYPE_F16}[dtype]
+    n = load_library().longnet_fwd_workspace_bytes(B, N, H, D, code, _flags(qk_norm, xpos))
+    if n < 0:
+        raise LongNetError(n, "longnet_fwd_workspace_bytes")
+    return int(n)
+
+
+def longnet_dilated_attn_fwd_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                out: torch.Tensor, lse: torch.Tensor | None,
+                                patterns: Sequence[Tuple[int, int]], causal: bool,
+                                workspace: torch.Tensor | None, impl: int = LONGNET_IMPL_AUTO,
+                                stream=None, qk_norm: bool = False, xpos: bool = False) -> None:
+    """Enqueue the prologue (qk_norm, then XPOS) into `workspace` (a CUDA
+    tensor of at least longnet_fwd_workspace_bytes bytes, 256-byte aligned)
+    and the forward on its result.  Tensors as in longnet_dilated_attn_fwd.
+    Raises LongNetError on a non-zero status."""
+    lib = load_library()
+    B, N, H, D = q.shape
+    for t in (q, k, v, out):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must be contiguous CUDA tensors of one shape and dtype")
+    if lse is not None and not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
+                                and tuple(lse.shape) == (B, H, N)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    if workspace is not None and not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_ptr = None if workspace is None else workspace.data_ptr()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_fwd_ws(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        None if lse is None else lse.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), _flags(qk_norm, xpos), int(impl), ws_ptr, ws_bytes, _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_fwd_ws")
+
+
 def longnet_dilated_attn_fwd_part(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                   out: torch.Tensor, lse: torch.Tensor | None,
                                   patterns: Sequence[Tuple[int, int]], causal: bool,
@@ -229,12 +280,20 @@ def longnet_scatter_rows(src: torch.Tensor, idx: torch.Tensor, dst: torch.Tensor
 def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  patterns: Sequence[Tuple[int, int]], causal: bool = True,
                  impl: int = LONGNET_IMPL_AUTO, want_lse: bool = True, stream=None,
-                 qk_norm: bool = False):
-    """Allocate out (and lse) with torch and run the forward.  Returns (out, lse)."""
+                 qk_norm: bool = False, xpos: bool = False):
+    """Allocate out (and lse) with torch and run the forward.  Returns (out,
+    lse).  xpos (and qk_norm with it) goes through the prologue pass, with a
+    workspace allocated by torch; qk_norm alone is applied inside the
+    attention kernel."""
     B, N, H, D = q.shape
     out = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if want_lse else None
-    longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream, qk_norm)
+    if xpos:
+        ws = torch.empty(longnet_fwd_workspace_bytes(B, N, H, D, q.dtype, qk_norm, True),
+                         dtype=torch.uint8, device=q.device)
+        longnet_dilated_attn_fwd_ws(q, k, v, out, lse, patterns, causal, ws, impl, stream, qk_norm, True)
+    else:
+        longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream, qk_norm)
     return out, lse
 
 

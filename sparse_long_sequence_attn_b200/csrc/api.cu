@@ -137,22 +137,10 @@ using namespace longnet;
 
 namespace longnet {
 namespace {
-int forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
-            int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
-            int flags, int impl, int64_t q0, int64_t q1, int64_t h0, int64_t h1, longnet_stream_t stream) {
-  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
-  if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
-  Problem pb;
-  int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
-  if (rc) return rc;
-  if (q0 < 0 || q1 > N || q0 >= q1 || h0 < 0 || h1 > H || h0 >= h1) return LONGNET_ERR_INVALID_ARG;
-  pb.q0 = q0;
-  pb.q1 = q1;
-  pb.h0 = h0;
-  pb.h1 = h1;
-  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
+// Launch the attention of a checked problem with the family impl (AUTO picks).
+int run(Problem& pb, int impl, longnet_stream_t stream) {
   int dev = 0;
-  rc = current_device_state(&dev, &pb.status);
+  int rc = current_device_state(&dev, &pb.status);
   if (rc) return rc;
   if (impl == LONGNET_IMPL_AUTO) {
     impl = choose_impl(pb);
@@ -173,6 +161,58 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
       return LONGNET_ERR_INVALID_ARG;
   }
 }
+
+int check_part(Problem& pb, int64_t q0, int64_t q1, int64_t h0, int64_t h1) {
+  if (q0 < 0 || q1 > pb.N || q0 >= q1 || h0 < 0 || h1 > pb.H || h0 >= h1) return LONGNET_ERR_INVALID_ARG;
+  pb.q0 = q0;
+  pb.q1 = q1;
+  pb.h0 = h0;
+  pb.h1 = h1;
+  return LONGNET_OK;
+}
+
+int forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
+            int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
+            int flags, int impl, int64_t q0, int64_t q1, int64_t h0, int64_t h1, longnet_stream_t stream) {
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
+  if (rc) return rc;
+  rc = check_part(pb, q0, q1, h0, h1);
+  if (rc) return rc;
+  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
+  return run(pb, impl, stream);
+}
+
+// The forward with the q/k prologue into a caller-provided workspace.
+int forward_ws(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
+               int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
+               int flags, int impl, void* workspace, int64_t workspace_bytes, longnet_stream_t stream) {
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  if (flags & ~(LONGNET_FLAG_QK_NORM | LONGNET_FLAG_XPOS)) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
+  if (rc) return rc;
+  if (flags == 0) return run(pb, impl, stream);
+  if (!workspace || workspace_bytes < prologue_workspace_bytes(B, N, H, D, dtype))
+    return LONGNET_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return LONGNET_ERR_MISALIGNED;
+  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
+  const int xpos = (flags & LONGNET_FLAG_XPOS) ? 1 : 0;
+  if (!prologue_supports(pb, xpos)) return LONGNET_ERR_UNSUPPORTED;
+  int dev = 0;
+  rc = current_device_state(&dev, &pb.status);
+  if (rc) return rc;
+  char* qo = static_cast<char*>(workspace);
+  char* ko = qo + prologue_workspace_bytes(B, N, H, D, dtype) / 2;
+  rc = launch_prologue(pb, xpos, qo, ko, reinterpret_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  pb.q = qo;
+  pb.k = ko;
+  pb.qk_norm = 0;
+  return run(pb, impl, stream);
+}
 }  // namespace
 }  // namespace longnet
 
@@ -183,6 +223,26 @@ extern "C" int longnet_dilated_attn_fwd_ex(const void* q, const void* k, const v
                                            longnet_stream_t stream) {
   return forward(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, flags, impl, 0, N, 0, H,
                  stream);
+}
+
+extern "C" int64_t longnet_fwd_workspace_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int dtype,
+                                               int flags) {
+  if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || B * N > ((int64_t)1 << 40) || H > 65535 || D > 65535 ||
+      B * N * H * D > ((int64_t)1 << 50))
+    return LONGNET_ERR_INVALID_ARG;
+  if (dtype != LONGNET_DTYPE_F32 && dtype != LONGNET_DTYPE_BF16 && dtype != LONGNET_DTYPE_F16)
+    return LONGNET_ERR_INVALID_ARG;
+  if (flags & ~(LONGNET_FLAG_QK_NORM | LONGNET_FLAG_XPOS)) return LONGNET_ERR_INVALID_ARG;
+  return flags ? prologue_workspace_bytes(B, N, H, D, dtype) : 0;
+}
+
+extern "C" int longnet_dilated_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
+                                           float* lse, int64_t B, int64_t N, int64_t H, int64_t D,
+                                           int n_pat, const int64_t* w, const int64_t* r, int causal,
+                                           int dtype, int flags, int impl, void* workspace,
+                                           int64_t workspace_bytes, longnet_stream_t stream) {
+  return forward_ws(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, flags, impl, workspace,
+                    workspace_bytes, stream);
 }
 
 extern "C" int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,

@@ -53,6 +53,12 @@ int launch_tcgen05(const Problem& p, cudaStream_t stream);
 int launch_smallseg(const Problem& p, cudaStream_t stream);
 int launch_backward(const Problem& p, const BwdArgs& g, int impl, cudaStream_t stream);
 
+// The q/k prologue (qk_norm and XPOS) into a workspace of
+// prologue_workspace_bytes: q rows first, k rows from half of it on.
+int64_t prologue_workspace_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int dtype);
+bool prologue_supports(const Problem& p, int xpos);
+int launch_prologue(const Problem& p, int xpos, void* qo, void* ko, cudaStream_t stream);
+
 // Row moves of the sequence-parallel exchange: dst[dst_idx[i]] = src[src_idx[i]]
 // for i < n (a null index array is the identity), rows of row_bytes (a
 // multiple of 16) bytes; indices checked against src_rows / dst_rows.

@@ -313,6 +313,59 @@ def check_qk_norm(lib):
         assert np.abs(o4 - o1).max() > 1e-3
 
 
+def _xpos_score(xpos, qv, m, kv, n, N):
+    """xpos(q) at position m dotted with xpos_down(k) at position n, one head."""
+    D = len(qv)
+    Q = np.zeros((1, N, 1, D))
+    K = np.zeros((1, N, 1, D))
+    Q[0, m, 0] = qv
+    K[0, n, 0] = kv
+    return float(np.dot(xpos(Q)[0, m, 0], xpos(K, downscale=True)[0, n, 0]))
+
+
+def check_xpos(lib, xpos=None):
+    """XPOS (the published definition; the pages name the option only):
+      * two hand-derived scores.  D = 2 (one pair, theta_0 = 1, zeta_0 =
+        0.8 / 2.8 = 2/7), q = (1, 0) at m = 600, k = (0, 1) at n = 88: the
+        rotated q is s_m (cos 600, sin 600), the rotated k is
+        (-sin 88, cos 88) / s_n, so the score is (s_m / s_n) sin(600 - 88) =
+        (2/7)^(512/512) sin(512).  D = 4, q = k = (0, 0, 1, 0) at m = 1100,
+        n = 76: only pair 1 (theta_1 = 10000^(-1/2) = 0.01, zeta_1 = 3.6 / 5.6
+        = 9/14) is non-zero, score (9/14)^(1024/512) cos(1024 * 0.01);
+      * every pair's length scales by zeta_i^((n - c) / 512) (c = N // 2) for
+        queries and by its inverse for keys;
+      * a score depends on the positions' difference only (shift both by t).
+    """
+    xpos = xpos or orc.xpos_fp64
+    got = _xpos_score(xpos, [1.0, 0.0], 600, [0.0, 1.0], 88, 1024)
+    assert abs(got - (2.0 / 7.0) * math.sin(512.0)) < 1e-12, got
+    got = _xpos_score(xpos, [0.0, 0.0, 1.0, 0.0], 1100, [0.0, 0.0, 1.0, 0.0], 76, 2048)
+    assert abs(got - (9.0 / 14.0) ** 2 * math.cos(10.24)) < 1e-12, got
+    B, N, H, D = 2, 300, 3, 8
+    x = _rand((B, N, H, D), 71)
+    zeta = np.array([(2 * i + 0.4 * D) / (1.4 * D) for i in range(D // 2)])
+    rel = (np.arange(N) - N // 2)[:, None] / 512.0
+    pair_len = lambda a: np.sqrt(a[..., 0::2] ** 2 + a[..., 1::2] ** 2)  # noqa: E731
+    for down, sgn in ((False, 1.0), (True, -1.0)):
+        want = pair_len(x) * (zeta[None, :] ** (sgn * rel))[None, :, None, :]
+        np.testing.assert_allclose(pair_len(xpos(x, downscale=down)), want, rtol=1e-12, atol=0)
+    g = np.random.default_rng(72)
+    qv, kv = g.standard_normal(16), g.standard_normal(16)
+    for (m, n, t) in ((700, 100, 1500), (64, 2000, 333), (3000, 3000, -2900)):
+        a = _xpos_score(xpos, qv, m, kv, n, 4096)
+        b = _xpos_score(xpos, qv, m + t, kv, n + t, 4096)
+        assert abs(a - b) < 1e-9 * max(1.0, abs(a)), (m, n, t, a, b)
+    # the option reaches the attention: it changes the result, and the
+    # attention on pre-encoded rows is the same
+    q, k, v = (_rand((1, 64, 2, 8), s) for s in (73, 74, 75))
+    pats = [(16, 1), (64, 2)]
+    o1, l1 = orc.dilated_attn_fp64(q, k, v, pats, lib=lib, xpos=True)
+    o2, l2 = orc.dilated_attn_fp64(orc.xpos_fp64(q), orc.xpos_fp64(k, downscale=True), v, pats, lib=lib)
+    np.testing.assert_allclose(o1, o2, atol=1e-13, rtol=0)
+    o3, _ = orc.dilated_attn_fp64(q, k, v, pats, lib=lib)
+    assert np.abs(o3 - o1).max() > 1e-3
+
+
 # ---------------------------------------------------------------- backward
 
 
@@ -529,6 +582,7 @@ def check_bwd_qk_norm(lib):
 ALL_CHECKS = [
     check_rows_function_direct,
     check_qk_norm,
+    check_xpos,
     check_dense_causal,
     check_dense_noncausal,
     check_block_diagonal,

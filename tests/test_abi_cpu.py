@@ -206,3 +206,38 @@ def test_row_moves_checked_on_host():
     if not torch.cuda.is_available():
         assert g(buf, 10, idx, 4, buf, 128, None) == bd.LONGNET_ERR_NO_DEVICE
         assert s(buf, 4, idx, buf, 10, 128, None) == bd.LONGNET_ERR_NO_DEVICE
+
+
+def test_workspace_bytes_on_host():
+    lib = bd.load_library()
+    f = lib.longnet_fwd_workspace_bytes
+    assert f(1, 1000, 3, 64, 1, 0) == 0  # no options, no workspace
+    one = 1000 * 3 * 64 * 2
+    assert f(1, 1000, 3, 64, 1, 1) == 2 * ((one + 255) // 256 * 256)
+    assert f(1, 1000, 3, 64, 0, 3) == 2 * ((2 * one + 255) // 256 * 256)
+    assert f(0, 1000, 3, 64, 1, 1) == bd.LONGNET_ERR_INVALID_ARG
+    assert f(1, 1000, 3, 64, 7, 1) == bd.LONGNET_ERR_INVALID_ARG
+    assert f(1, 1000, 3, 64, 1, 4) == bd.LONGNET_ERR_INVALID_ARG
+
+
+def _call_ws(lib, flags, ws=0x10000, ws_bytes=1 << 30, D=64, N=64, dtype=1):
+    buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+    return lib.longnet_dilated_attn_fwd_ws(buf, buf, buf, buf, None, 1, N, 2, D, 1, w, r, 1, dtype, flags, 0,
+                                           None if ws is None else ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_workspace_entry_checked_on_host():
+    lib = bd.load_library()
+    assert _call_ws(lib, 4) == bd.LONGNET_ERR_INVALID_ARG           # unknown option
+    assert _call_ws(lib, 1, ws=None) == bd.LONGNET_ERR_INVALID_ARG   # options need a workspace
+    assert _call_ws(lib, 2, ws_bytes=100) == bd.LONGNET_ERR_INVALID_ARG
+    assert _call_ws(lib, 3, ws=0x10010) == bd.LONGNET_ERR_MISALIGNED
+    assert _call_ws(lib, 1, D=24) == bd.LONGNET_ERR_UNSUPPORTED       # the prologue's D
+    # fp16 XPOS: |log2 s| reaches 1.807 * 4096 / 512 > 8 at N = 8192
+    assert _call_ws(lib, 2, N=8192, dtype=2) == bd.LONGNET_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert _call_ws(lib, 3) == bd.LONGNET_ERR_NO_DEVICE
+        assert _call_ws(lib, 0, ws=None, ws_bytes=0) == bd.LONGNET_ERR_NO_DEVICE
+        assert _call_ws(lib, 2, N=4096, dtype=2) == bd.LONGNET_ERR_NO_DEVICE  # within fp16's range

@@ -104,3 +104,56 @@ def test_pins_catch_python_mutant(monkeypatch, oracle_lib, mutant):
     monkeypatch.setattr(orc, "qk_normalize_bwd_fp64", mutant)
     with pytest.raises(AssertionError):
         pins.check_bwd_qk_norm(oracle_lib)
+
+
+def _xpos_variant(sin_sign=1.0, halves=False, invert_keys=True, gamma=0.4, freq_step=2.0, base=512.0):
+    """An XPOS with one planted mistake (the parameters name it)."""
+    import numpy as np
+
+    from oracle.oracle import _f64
+
+    def xp(x, downscale=False):
+        x = _f64(x)
+        B, N, H, D = x.shape
+        n = np.arange(N, dtype=np.float64)[:, None]
+        i = np.arange(D // 2, dtype=np.float64)[None, :]
+        theta = 10000.0 ** (-freq_step * i / D)
+        zeta = (2.0 * i + gamma * D) / ((1.0 + gamma) * D)
+        s = zeta ** ((n - N // 2) / base)
+        if downscale and invert_keys:
+            s = 1.0 / s
+        cos = (np.cos(n * theta) * s)[None, :, None, :]
+        sin = (sin_sign * np.sin(n * theta) * s)[None, :, None, :]
+        if halves:
+            a, b = x[..., : D // 2], x[..., D // 2:]
+        else:
+            a, b = x[..., 0::2], x[..., 1::2]
+        y = np.empty_like(x)
+        ya, yb = a * cos - b * sin, b * cos + a * sin
+        if halves:
+            y[..., : D // 2], y[..., D // 2:] = ya, yb
+        else:
+            y[..., 0::2], y[..., 1::2] = ya, yb
+        return y
+
+    return xp
+
+
+XPOS_MUTANTS = {
+    "sin_sign": dict(sin_sign=-1.0),
+    "half_split_pairs": dict(halves=True),
+    "keys_not_inverted": dict(invert_keys=False),
+    "gamma_0p5": dict(gamma=0.5),
+    "freq_step_1": dict(freq_step=1.0),
+    "scale_base_256": dict(base=256.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(XPOS_MUTANTS))
+def test_xpos_pins_catch_mutant(oracle_lib, name):
+    with pytest.raises(AssertionError):
+        pins.check_xpos(oracle_lib, xpos=_xpos_variant(**XPOS_MUTANTS[name]))
+
+
+def test_xpos_unmutated_variant_passes(oracle_lib):
+    pins.check_xpos(oracle_lib, xpos=_xpos_variant())
