@@ -67,7 +67,9 @@ enum longnet_status {
   LONGNET_ERR_CUDA = -4,          /* a CUDA call failed (launch, config) */
   LONGNET_ERR_DEVICE_TIMEOUT = -5,/* a kernel wait ran out of time (status word) */
   LONGNET_ERR_DEVICE_BOUNDS = -6, /* a kernel index check failed (status word) */
-  LONGNET_ERR_NO_DEVICE = -7      /* no usable sm_100 device */
+  LONGNET_ERR_NO_DEVICE = -7,     /* no usable sm_100 device */
+  LONGNET_ERR_SCRATCH_LIMIT = -8  /* longnet_dilated_attn_fwd_noalloc: the problem
+                                     needs more than the fixed scratch holds */
 };
 
 enum longnet_dtype { LONGNET_DTYPE_F32 = 0, LONGNET_DTYPE_BF16 = 1, LONGNET_DTYPE_F16 = 2 };
@@ -187,6 +189,44 @@ int longnet_dilated_attn_fwd_ws(const void* q, const void* k, const void* v,
                                 int causal, int dtype, int flags, int impl,
                                 void* workspace, int64_t workspace_bytes,
                                 longnet_stream_t stream);
+
+/* Size of the fixed device scratch of longnet_dilated_attn_fwd_noalloc, per
+ * device: 32 MiB. */
+#define LONGNET_NOALLOC_SCRATCH_BYTES (32 << 20)
+
+/*
+ * longnet_dilated_attn_fwd_noalloc — longnet_dilated_attn_fwd_ws with its
+ * workspace taken from a fixed array of LONGNET_NOALLOC_SCRATCH_BYTES in the
+ * library's own device memory (one per device) instead of from the caller.
+ * The pages have no counterpart: the method says nothing about who owns
+ * memory.  It is for callers that cannot allocate device memory when they
+ * call: a C host with no device allocator of its own, or a serving process
+ * whose device memory is planned up front (handed to its caches), where an
+ * allocation at call time fails or must first free cached blocks.  The call
+ * allocates nothing (no cudaMalloc or cudaFree, directly or through torch).
+ *   Limit: longnet_fwd_workspace_bytes(B, N, H, D, dtype, flags) must not
+ *     exceed LONGNET_NOALLOC_SCRATCH_BYTES (for bf16: B*N*H*D up to 8 Mi
+ *     elements), else LONGNET_ERR_SCRATCH_LIMIT and nothing is launched.
+ *     flags = 0 needs no scratch (the call is the plain forward).
+ *   Contents: nothing in the scratch has to start at zero or at any value:
+ *     the prologue writes every byte of it that the attention then reads.
+ *   First call on a device: it looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current), which may load the
+ *     library's device code; make that first call before any stream capture
+ *     begins.  A failed lookup returns LONGNET_ERR_CUDA.
+ *   Calls that overlap race: every call on a device uses the same array, so
+ *     two calls whose work may run at the same time (different streams, or
+ *     different host threads, without an ordering between them) corrupt each
+ *     other's q and k.  Order them (one stream, or events).
+ * The other arguments, results and errors are those of
+ * longnet_dilated_attn_fwd_ws.
+ */
+int longnet_dilated_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                     void* out, float* lse,
+                                     int64_t B, int64_t N, int64_t H, int64_t D,
+                                     int n_pat, const int64_t* w, const int64_t* r,
+                                     int causal, int dtype, int flags, int impl,
+                                     longnet_stream_t stream);
 
 /*
  * longnet_dilated_attn_fwd_part — the forward with options and a family (as

@@ -23,6 +23,8 @@ LONGNET_ERR_CUDA = -4
 LONGNET_ERR_DEVICE_TIMEOUT = -5
 LONGNET_ERR_DEVICE_BOUNDS = -6
 LONGNET_ERR_NO_DEVICE = -7
+LONGNET_ERR_SCRATCH_LIMIT = -8
+LONGNET_NOALLOC_SCRATCH_BYTES = 32 << 20
 LONGNET_MAX_PATTERNS = 16
 
 LONGNET_DTYPE_F32 = 0
@@ -62,6 +64,9 @@ SIGNATURES = {
                                                    ctypes.c_int, _i64p, _i64p, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _i64,
                                                    _vp]),
+    "longnet_dilated_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                                        ctypes.c_int, _i64p, _i64p, ctypes.c_int,
+                                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]),
     "longnet_gather_rows": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp]),
     "longnet_scatter_rows": (ctypes.c_int, [_vp, _i64, _vp, _vp, _i64, _i64, _vp]),
     "longnet_dilated_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -208,6 +213,33 @@ def longnet_dilated_attn_fwd_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
         _dtype_code(q), _flags(qk_norm, xpos), int(impl), ws_ptr, ws_bytes, _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_fwd_ws")
+
+
+def longnet_dilated_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                     out: torch.Tensor, lse: torch.Tensor | None,
+                                     patterns: Sequence[Tuple[int, int]], causal: bool,
+                                     impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False,
+                                     xpos: bool = False) -> None:
+    """longnet_dilated_attn_fwd_ws with the library's fixed device scratch
+    (LONGNET_NOALLOC_SCRATCH_BYTES per device) as the workspace: nothing is
+    allocated.  Calls that may run at the same time on one device race on
+    that scratch.  Raises LongNetError on a non-zero status
+    (LONGNET_ERR_SCRATCH_LIMIT when the problem needs more scratch)."""
+    lib = load_library()
+    B, N, H, D = q.shape
+    for t in (q, k, v, out):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out must be contiguous CUDA tensors of one shape and dtype")
+    if lse is not None and not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
+                                and tuple(lse.shape) == (B, H, N)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_fwd_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        None if lse is None else lse.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), _flags(qk_norm, xpos), int(impl), _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_fwd_noalloc")
 
 
 def longnet_dilated_attn_fwd_part(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -245,6 +245,53 @@ extern "C" int longnet_dilated_attn_fwd_ws(const void* q, const void* k, const v
                     workspace_bytes, stream);
 }
 
+namespace longnet {
+namespace {
+// The fixed workspace of longnet_dilated_attn_fwd_noalloc, for callers that
+// cannot allocate device memory at the call (a C host without a device
+// allocator, a process whose device memory is planned up front): part of the
+// library's own device memory, so the call allocates nothing.  Its device
+// address is looked up once per device, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LONGNET_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+int noalloc_scratch(void** addr) {
+  int dev = 0;
+  int* status = nullptr;
+  int rc = current_device_state(&dev, &status);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return LONGNET_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return LONGNET_OK;
+}
+}  // namespace
+}  // namespace longnet
+
+extern "C" int longnet_dilated_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                                float* lse, int64_t B, int64_t N, int64_t H, int64_t D,
+                                                int n_pat, const int64_t* w, const int64_t* r, int causal,
+                                                int dtype, int flags, int impl, longnet_stream_t stream) {
+  void* scratch = nullptr;
+  if (flags != 0) {
+    const int64_t need = longnet_fwd_workspace_bytes(B, N, H, D, dtype, flags);
+    if (need < 0) return (int)need;
+    if (need > (int64_t)LONGNET_NOALLOC_SCRATCH_BYTES) return LONGNET_ERR_SCRATCH_LIMIT;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+  }
+  return forward_ws(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, flags, impl, scratch,
+                    LONGNET_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 extern "C" int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,
                                              void* out, float* lse, int64_t B, int64_t N,
                                              int64_t H, int64_t D, int n_pat, const int64_t* w,
@@ -396,6 +443,8 @@ extern "C" const char* longnet_status_string(int status) {
     case LONGNET_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case LONGNET_ERR_DEVICE_BOUNDS: return "device index check failed";
     case LONGNET_ERR_NO_DEVICE: return "no usable sm_100 device";
+    case LONGNET_ERR_SCRATCH_LIMIT:
+      return "problem too large for the fixed scratch of longnet_dilated_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }

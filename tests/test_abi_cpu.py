@@ -241,3 +241,22 @@ def test_workspace_entry_checked_on_host():
         assert _call_ws(lib, 3) == bd.LONGNET_ERR_NO_DEVICE
         assert _call_ws(lib, 0, ws=None, ws_bytes=0) == bd.LONGNET_ERR_NO_DEVICE
         assert _call_ws(lib, 2, N=4096, dtype=2) == bd.LONGNET_ERR_NO_DEVICE  # within fp16's range
+
+
+def test_noalloc_entry_checked_on_host():
+    lib = bd.load_library()
+    buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+
+    def call(N, H, flags):
+        return lib.longnet_dilated_attn_fwd_noalloc(buf, buf, buf, buf, None, 1, N, H, 64, 1, w, r, 1, 1,
+                                                    flags, 0, None)
+
+    assert call(1024, 2, 4) == bd.LONGNET_ERR_INVALID_ARG
+    # 2 x 32768 x 8 x 64 bf16 = 64 MiB of workspace > the 32 MiB scratch
+    assert call(32768, 8, 1) == bd.LONGNET_ERR_SCRATCH_LIMIT
+    assert "fixed scratch" in bd.status_string(bd.LONGNET_ERR_SCRATCH_LIMIT)
+    if not torch.cuda.is_available():
+        assert call(1024, 2, 1) == bd.LONGNET_ERR_NO_DEVICE
+        assert call(32768, 8, 0) == bd.LONGNET_ERR_NO_DEVICE  # no options: no scratch needed
