@@ -392,13 +392,15 @@ struct Tile {
   int seg;    // segment index
   int k0;     // first kept row (sparse index within the segment)
   int nrows;      // rows in this tile (<= 128)
-  int nkv;        // KV blocks of 128 keys
+  int nkv;        // KV blocks of 64 keys
+  int nkeys;      // keys the tile attends to (the last block may be partial)
   int start;  // position of the first row
 };
 
 // Walks the unit's tiles in processing order.  All roles run identical copies.
 struct TileWalker {
   int n_pat;
+  int N;       // sequence length (the last segment of a pattern may be shorter than w)
   int A, Bnd;  // range [A, Bnd)
   int w[kMaxPat], r[kMaxPat], o[kMaxPat], m[kMaxPat];
   int seg[kMaxPat], k0[kMaxPat], khi[kMaxPat], seg_last[kMaxPat];
@@ -423,6 +425,7 @@ struct TileWalker {
   }
   __host__ __device__ void init(const Params& P, int h, int a, int bnd) {
     n_pat = P.pb.n_pat;
+    N = (int)P.pb.N;
     A = a;
     Bnd = bnd;
     causal = P.pb.causal != 0;
@@ -456,7 +459,14 @@ struct TileWalker {
     const int n = khi[p] - k0[p];
     t.nrows = (int)(n < kBM ? n : kBM);
     t.start = best_start;
-    const int nkeys = causal ? k0[p] + t.nrows : m[p];
+    // causal: the segment's kept rows up to the tile's last row; otherwise all
+    // of them, fewer in a last segment cut short by the sequence's end
+    int nkeys = k0[p] + t.nrows;
+    if (!causal) {
+      const int seg_len = N - seg[p] * w[p] < w[p] ? N - seg[p] * w[p] : w[p];
+      nkeys = o[p] >= seg_len ? 0 : (seg_len - o[p] + r[p] - 1) / r[p];
+    }
+    t.nkeys = nkeys;
     t.nkv = (int)((nkeys + kBN - 1) / kBN);
     k0[p] += t.nrows;
     advance_to_nonempty(p);
@@ -928,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         em.info = info;
         em.j = e.j;
         em.nkv = t.nkv;
-        em.lim0 = causal ? t.k0 : pt.w - 1;
+        em.lim0 = causal ? t.k0 : t.nkeys - 1;
         if (e.j == 0) {
           ok = wait_count(cnt_epi, e.tile_idx - kQT);  // tile queue entry is free
           if (!ok) break;
@@ -955,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kv_it >= (uint32_t)NS) ok = sy.wait(kv_empty + st, st_par ^ 1);
         if (!ok) break;
         stage_meta[st] = em;
-        const int n_keys_total = causal ? t.k0 + t.nrows : pt.w;
+        const int n_keys_total = t.nkeys;
         const int kstart = e.j * kBN;
         const int need = n_keys_total - kstart < kBN ? n_keys_total - kstart : kBN;
         const TmaCoord c = tma_coord(P, ri, seg_base + pt.y * kstart, need);
@@ -1431,9 +1441,9 @@ int64_t range_cost(const Problem& pb, int64_t A, int64_t Bnd) {
   int64_t cost = 0;
   for (int p = 0; p < pb.n_pat; ++p) {
     const int64_t w = pb.w[p], r = pb.r[p], o = 0;
-    const int64_t m = (w - o + r - 1) / r;
     for (int64_t seg = A / w; seg <= (Bnd - 1) / w; ++seg) {
       const int64_t base = seg * w + o;
+      const int64_t m = (std::min(w, pb.N - seg * w) - o + r - 1) / r;
       int64_t lo = A - base;
       lo = lo <= 0 ? 0 : (lo + r - 1) / r;
       int64_t hi = Bnd - base;
@@ -1464,7 +1474,8 @@ bool tcgen05_supports(const Problem& p) {
   int n_r = 0;
   int64_t rv[kMaxR];
   for (int i = 0; i < p.n_pat; ++i) {
-    if (p.w[i] > p.N || p.N % p.w[i] != 0) return false;  // whole segments only
+    // w need not divide N (the last segment is the shorter rest) and may
+    // exceed it (one segment); fill_params works with min(w, N)
     bool found = false;
     for (int j = 0; j < n_r; ++j) found |= (rv[j] == p.r[i]);
     if (!found) {
@@ -1490,6 +1501,9 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
   using namespace tc;
   memset(&P, 0, sizeof(P));
   P.pb = pb;
+  // a segment longer than the sequence is the sequence: same kept rows
+  for (int i = 0; i < pb.n_pat; ++i)
+    if (P.pb.w[i] > pb.N) P.pb.w[i] = pb.N;
   P.wait_limit_ns = kWaitLimitNs;
   for (int i = 0; i < pb.n_pat; ++i) {
     int j = 0;
@@ -1502,7 +1516,7 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
       ++P.n_r;
     }
     P.pat_r[i] = j;
-    P.w_div[i] = make_fastdiv(pb.w[i]);
+    P.w_div[i] = make_fastdiv(P.pb.w[i]);
   }
   bool has_r1 = false;
   for (int i = 0; i < pb.n_pat; ++i) has_r1 |= (pb.r[i] == 1);
@@ -1548,7 +1562,7 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     auto clip_cost = [&](int64_t a, int64_t e) -> int64_t {
       a = std::max<int64_t>(a, pb.q0);
       e = std::min<int64_t>(e, pb.q1);
-      return a < e ? range_cost(pb, a, e) : 0;
+      return a < e ? range_cost(P.pb, a, e) : 0;
     };
     for (int i = 0; i < P.n_ranges; ++i) {
       const int64_t a = (P.range_first + (int64_t)i) * R;

@@ -89,7 +89,14 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
         const int64_t r = tw.r[t.p];
         const int64_t base = t.seg * tw.w[t.p] + tw.o[t.p];
         CHECK(t.start == base + r * t.k0, "start mismatch\n");
-        int64_t nkeys = causal ? t.k0 + t.nrows : tw.m[t.p];
+        // keys: the kept rows of the segment (before the sequence's end), up
+        // to the tile's last row when causal
+        const int64_t seg_end = std::min<int64_t>((t.seg + 1) * (int64_t)tw.w[t.p], N);
+        int64_t seg_kept = 0;
+        for (int64_t xk = base; xk < seg_end; xk += r) ++seg_kept;
+        int64_t nkeys = causal ? t.k0 + t.nrows : seg_kept;
+        CHECK(t.k0 + t.nrows <= seg_kept, "%s: tile rows past the segment's kept rows\n", name);
+        CHECK(t.nkeys == nkeys, "%s: nkeys %d, expected %ld\n", name, t.nkeys, (long)nkeys);
         CHECK(t.nkv == (nkeys + kBN - 1) / kBN, "nkv\n");
         // TMA coords
         check_tma(P, P.pat_r[t.p], t.start, t.nrows, r);
@@ -141,9 +148,10 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
     for (int p = 0; p < pb.n_pat; ++p) {
       int64_t w = pb.w[p], r = pb.r[p], o = h % r;
       int64_t m = o >= w ? 0 : (w - o + r - 1) / r;
-      for (int64_t seg = 0; seg < N / w; ++seg)
+      for (int64_t seg = 0; seg * w < N; ++seg)
         for (int64_t k = 0; k < m; ++k) {
           const int64_t xk = seg * w + o + r * k;
+          if (xk >= N) break;  // a last segment cut short by the sequence's end
           if (xk < pb.q0 || xk >= pb.q1) continue;  // outside the computed part
           auto it = seen.find(std::make_tuple(p, seg, k));
           CHECK(it != seen.end() && it->second == 1, "%s: row p=%d seg=%ld k=%ld seen %d times\n", name, p, (long)seg, (long)k, it == seen.end() ? 0 : it->second);
@@ -168,7 +176,8 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
 }
 
 // Seeded random shapes the kernel takes: N a multiple of 64 up to 16384,
-// 1..6 patterns whose w divides N, r up to 16 (r > w allowed), 1..12 heads,
+// 1..6 patterns, w dividing N or (one in three) any length up to 1.5 N,
+// r up to 16 (r > w allowed), 1..12 heads,
 // causal or not, and SM counts that change the unit plan.
 void random_cases(int count) {
   uint64_t st = 0x9e3779b97f4a7c15ull;
@@ -183,8 +192,11 @@ void random_cases(int count) {
       if (N % w == 0) divs.push_back(w);
     const int n_pat = 1 + (int)(next() % 6);
     std::vector<std::pair<int64_t, int64_t>> pats;
-    for (int i = 0; i < n_pat; ++i)
-      pats.push_back({divs[next() % divs.size()], rs[next() % (sizeof(rs) / sizeof(rs[0]))]});
+    for (int i = 0; i < n_pat; ++i) {
+      // every third pattern: any w up to 1.5 N (a shorter last segment, or w > N)
+      const int64_t w = next() % 3 == 0 ? 2 + (int64_t)(next() % (uint64_t)(N + N / 2)) : divs[next() % divs.size()];
+      pats.push_back({w, rs[next() % (sizeof(rs) / sizeof(rs[0]))]});
+    }
     const int64_t H = 1 + (int64_t)(next() % 12);
     const int causal = (int)(next() & 1);
     char name[64];
@@ -247,6 +259,14 @@ int main() {
            148, false, 16384, 24576, 3, 9);
   run_case("lm_unaligned_part", 1, 8192, 12, {{2048, 1}, {4096, 2}, {8192, 4}}, 1, 148, false, 1000, 7001, 5, 6);
   run_case("noncausal_part", 1, 6000, 7, {{600, 1}, {1200, 7}, {3000, 5}, {6000, 9}}, 0, 132, false, 777, 4321, 1, 7);
+  // partial last segments (w not dividing N) and w > N
+  run_case("long32k_minus64", 1, 32704, 12, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 6}, {32768, 12}}, 1);
+  run_case("long32k_minus64_nc", 1, 32704, 12, {{2048, 1}, {4096, 2}, {8192, 4}, {16384, 6}, {32768, 12}}, 0);
+  run_case("partial_odd", 1, 5000, 5, {{768, 1}, {1536, 3}, {4096, 7}, {9000, 5}}, 1);
+  run_case("partial_odd_nc", 1, 5000, 5, {{768, 1}, {1536, 3}, {4096, 7}, {9000, 5}}, 0);
+  run_case("partial_777", 1, 777, 2, {{128, 1}, {256, 4}}, 1);
+  run_case("partial_1000_nc", 2, 1000, 4, {{256, 1}, {384, 2}}, 0);
+  run_case("partial_part", 1, 10000, 6, {{3000, 1}, {7000, 3}}, 0, 148, false, 2999, 9001, 2, 5);
   random_cases(300);
   printf("fails=%d\n", fails);
   return fails ? 1 : 0;

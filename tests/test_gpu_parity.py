@@ -191,6 +191,26 @@ def test_sweep_sampled_rows(N):
     print(f"sweep{N}: max|out - oracle| = {err:.3e} over {len(rows)} rows")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_partial_last_segments_full_size(causal):
+    """The 32K-token shape 64 positions short, so every pattern's last segment
+    is cut by the sequence's end (and the longest segment exceeds it), in the
+    benchmark's launch configuration (AUTO): sampled rows, including every
+    segment's first and last kept row and all rows of the last 2048
+    positions, against the oracle."""
+    w = wl.WORKLOADS["long32k"]
+    N = w.N - 64
+    assert bd.longnet_select_impl(w.B, N, w.H, w.D, w.patterns, causal, torch.bfloat16) == \
+        bd.LONGNET_IMPL_TCGEN05
+    q, k, v = wl.make_inputs(w, N=N)
+    o, l = gh.run_cuda(q, k, v, w.patterns, causal, bd.LONGNET_IMPL_AUTO)
+    rows = gh.sample_rows(w.B, N, w.H, w.patterns, n_random=1000, seed=17, boundary=4096)
+    tail = np.array([(0, x, h) for x in range(N - 2048, N) for h in range(w.H)], dtype=np.int64)
+    rows = np.unique(np.concatenate([rows, tail]), axis=0)
+    err = gh.compare_rows(o, l, q, k, v, w.patterns, causal, torch.bfloat16, rows, label=f"long32k-64/{causal}")
+    print(f"long32k-64 causal={causal}: max|out - oracle| = {err:.3e} over {len(rows)} rows")
+
+
 def test_lse_optional_and_deterministic():
     pats = ((256, 1), (512, 2), (1024, 4))
     q, k, v = wl.random_inputs(1, 1024, 4, 64, torch.bfloat16, seed=5)
