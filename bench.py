@@ -54,7 +54,7 @@ def load_peaks():
 # The sources a kernel family's device code is built from: its own file and
 # the shared headers (code only: comments and layout are ignored).  A change
 # anywhere else leaves its counters valid.
-_FAMILY_SOURCES = ("device_util.cuh", "params.h")
+_FAMILY_SOURCES = ("device_util.cuh", "params.h", "tc_ptx.cuh")
 
 
 def _code_only(text: str) -> str:
@@ -247,7 +247,7 @@ def main():
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", help="ours | reference")
     ap.add_argument("--kernel", default="auto",
-                    help="auto | simt | tcgen05 | smallseg (forward); auto | simt | tiles (--pass bwd)")
+                    help="auto | simt | tcgen05 | smallseg (forward); auto | simt | tiles | tcgen05 (--pass bwd)")
     ap.add_argument("--ref-positions", type=int, default=48)
     ap.add_argument("--cpu-positions", type=int, default=0,
                     help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
@@ -561,10 +561,23 @@ def run_backward(args, wl):
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, dout))
     out, lse = bd.dilated_attn(qd, kd, vd, wl.patterns, wl.causal)
     dq, dk, dv = (torch.empty(qd.shape, dtype=torch.float32, device=dev) for _ in range(3))
-    impl = {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT,
-            "tiles": bd.LONGNET_IMPL_TILES}[args.kernel]
-    tiles = impl == bd.LONGNET_IMPL_TILES or (
-        impl == bd.LONGNET_IMPL_AUTO and wl.D == 64 and wl.dtype != "fp32")
+    impl = {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT, "tiles": bd.LONGNET_IMPL_TILES,
+            "tcgen05": bd.LONGNET_IMPL_TCGEN05}[args.kernel]
+    # the family AUTO runs: the first of tcgen05, tiles that takes the call
+    # (one untimed probe call each), else SIMT
+    family = {bd.LONGNET_IMPL_SIMT: "simt", bd.LONGNET_IMPL_TILES: "tiles",
+              bd.LONGNET_IMPL_TCGEN05: "tcgen05"}.get(impl)
+    if family is None:
+        family = "simt"
+        for name, code in (("tcgen05", bd.LONGNET_IMPL_TCGEN05), ("tiles", bd.LONGNET_IMPL_TILES)):
+            try:
+                bd.longnet_dilated_attn_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, wl.patterns, wl.causal, code)
+                family = name
+                break
+            except bd.LongNetError as e:
+                if e.code != bd.LONGNET_ERR_UNSUPPORTED:
+                    raise
+    tiles = family in ("tiles", "tcgen05")  # tensor cores
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
@@ -630,8 +643,10 @@ def run_backward(args, wl):
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                 "peak_source": f"{peak_kind} bf16 GEMM "
                                f"({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
-                "traffic": traffic_from_profiles(wl.name + ":bwd", "backward"),
-                "kernel": "bwd_dkv_tile_kernel + bwd_dq_tile_kernel (one call)",
+                "traffic": traffic_from_profiles(wl.name + ":bwd", "backward" if family == "tiles"
+                                                 else "bwd_tcgen05"),
+                "kernel": ("bwd_dkv_tile_kernel + bwd_dq_tile_kernel (one call)" if family == "tiles" else
+                           "bwd_delta_kernel + bwd_tc_kernel keys (dk, dv) + bwd_tc_kernel queries (dq)"),
                 "executed_flops_per_launch": 14.0 * wl.D * pairs}
     else:
         roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
@@ -651,12 +666,12 @@ def run_backward(args, wl):
                    "D": wl.D, "patterns": [list(p) for p in wl.patterns], "causal": wl.causal,
                    "global_batch": wl.B * ws, "seq_len": wl.N,
                    "parallelism": f"independent replicas x{ws}" if ws > 1 else "single GPU",
-                   "kernel": "tiles (mma.sync)" if tiles else "simt",
+                   "kernel": {"tiles": "tiles (mma.sync)", "tcgen05": "tcgen05 (TMA, TMEM)"}.get(family, "simt"),
                    "l2": "512 MiB flush between timed steps (outside events)"},
         "roofline": roof,
         "e2e": {"value": weak_scaling_rate(tokens * e2e_steps, ws, e2e_total), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (3 if family == "tcgen05" else 2) * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
     if ws == 1 and not args.no_cpu_baseline:

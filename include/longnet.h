@@ -305,15 +305,18 @@ int longnet_scatter_rows(const void* src, int64_t n, const int64_t* idx, void* d
  *     taken back through that normalisation (a (g - xhat <xhat, g>) per row,
  *     a = 1 / max(|x|, 1e-12); a g for a row with |x| <= 1e-12).  Other bits:
  *     LONGNET_ERR_INVALID_ARG.
- *   - impl: LONGNET_IMPL_AUTO (the tile kernels where they apply, else
- *     SIMT), LONGNET_IMPL_SIMT (fp32 FMA, D in {16, 32, 64, 128}, every
- *     dtype) or LONGNET_IMPL_TILES (bf16/fp16, D = 64: tensor cores).  A
- *     family that does not cover the call: LONGNET_ERR_UNSUPPORTED.
- *   - Enqueued on stream; allocates nothing.  The tile kernels zero dq, dk
- *     and dv on the stream first, then add each pattern's share with fp32
- *     atomics, so the summation order of a row's patterns (at most n_pat
- *     terms) may vary between runs in the last bits.  Returns a
- *     longnet_status.
+ *   - impl: LONGNET_IMPL_AUTO (tcgen05 where it applies, else the tile
+ *     kernels, else SIMT), LONGNET_IMPL_TCGEN05 (bf16/fp16, D = 64, no
+ *     qk_norm, up to 6 patterns: TMA-fed tcgen05 tensor cores with TMEM
+ *     accumulators), LONGNET_IMPL_TILES (bf16/fp16, D = 64: mma.sync tensor
+ *     cores) or LONGNET_IMPL_SIMT (fp32 FMA, D in {16, 32, 64, 128}, every
+ *     dtype).  A family that does not cover the call: LONGNET_ERR_UNSUPPORTED.
+ *   - Enqueued on stream; allocates nothing.  The tcgen05 and tile kernels
+ *     zero dq, dk and dv on the stream first, then add each pattern's share
+ *     with fp32 atomics, so the summation order of a row's patterns (at most
+ *     n_pat terms) may vary between runs in the last bits; the tcgen05
+ *     family also uses dq as scratch for delta before it computes dq.
+ *     Returns a longnet_status.
  */
 int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
                              const void* out, const float* lse, const void* dout,

@@ -359,7 +359,8 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
                                         const int64_t* r, int causal, int dtype, int flags,
                                         int impl, longnet_stream_t stream) {
   if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
-  if (impl != LONGNET_IMPL_AUTO && impl != LONGNET_IMPL_SIMT && impl != LONGNET_IMPL_TILES)
+  if (impl != LONGNET_IMPL_AUTO && impl != LONGNET_IMPL_SIMT && impl != LONGNET_IMPL_TILES &&
+      impl != LONGNET_IMPL_TCGEN05)
     return LONGNET_ERR_INVALID_ARG;
   if (!out || !lse || !dout || !dq || !dk || !dv) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
@@ -375,6 +376,7 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
     return LONGNET_ERR_UNSUPPORTED;
   if (impl == LONGNET_IMPL_SIMT && !backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
   if (impl == LONGNET_IMPL_TILES && !tile_backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_TCGEN05 && !tcgen05_backward_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
   int dev = 0;
   rc = current_device_state(&dev, &pb.status);
   if (rc) return rc;

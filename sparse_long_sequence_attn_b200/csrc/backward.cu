@@ -1003,7 +1003,10 @@ bool tile_backward_supports(const Problem& p) {
 }
 
 int launch_backward(const Problem& p, const BwdArgs& g, int impl, cudaStream_t stream) {
-  if (impl == LONGNET_IMPL_AUTO) impl = tile_backward_supports(p) ? LONGNET_IMPL_TILES : LONGNET_IMPL_SIMT;
+  if (impl == LONGNET_IMPL_AUTO)
+    impl = tcgen05_backward_supports(p) ? LONGNET_IMPL_TCGEN05
+                                        : tile_backward_supports(p) ? LONGNET_IMPL_TILES : LONGNET_IMPL_SIMT;
+  if (impl == LONGNET_IMPL_TCGEN05) return launch_tcgen05_backward(p, g, stream);
   if (impl == LONGNET_IMPL_TILES) {
     if (!tile_backward_supports(p)) return LONGNET_ERR_UNSUPPORTED;
     return launch_tile_bwd(p, g, stream);

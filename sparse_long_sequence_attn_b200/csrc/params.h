@@ -71,5 +71,7 @@ bool tcgen05_supports(const Problem& p);
 bool smallseg_supports(const Problem& p);
 bool backward_supports(const Problem& p);       // the SIMT backward
 bool tile_backward_supports(const Problem& p);  // the mma.sync tile backward
+bool tcgen05_backward_supports(const Problem& p);  // the tcgen05 backward
+int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t stream);
 
 }  // namespace longnet
