@@ -18,7 +18,9 @@
 // Design.
 //  * Work is cut per pattern, batch, head and segment (a "unit": the
 //    sparsified segment of that pattern, kept row t at position
-//    first + r t), and per 128-row tile of it: one CTA per (unit, tile).
+//    first + r t), and per 128-row tile of it: one CTA per (unit, tile), the
+//    tiles of a unit launched together (longest first) so the blocks they
+//    all stream are read from L2.
 //  * Two kernels, so no tile pair needs atomics:
 //      key-centric (dk, dv): the CTA holds a tile of 128 keys (K, V) and
 //      streams 64-query blocks (Q, dout, lse, delta) through a 3-stage ring:
@@ -87,7 +89,8 @@ struct PatGeo {
   int kfull, tail;    // N div r, N mod r (TMA maps)
   FastDiv r_div;
   int n_seg;
-  int64_t unit_base;  // first unit of this pattern
+  int tiles;          // 128-row tiles of the pattern's fullest segment
+  int64_t cta_base;   // first CTA of this pattern
 };
 
 struct Params {
@@ -95,7 +98,7 @@ struct Params {
   BwdArgs g;
   const float* delta;  // [B, H, N] <dout_i, out_i> (key-centric kernel)
   PatGeo pat[kMaxPat];
-  int64_t n_units;
+  int64_t n_ctas;
   float scale, scale_log2;
   uint64_t wait_limit_ns;
 };
@@ -105,16 +108,26 @@ struct __align__(64) Maps {
   CUtensorMap m[kMaxPat][2][4];
 };
 
-// One sparsified segment: kept row t (t < m) at position first + r t.
+// One sparsified segment: kept row t (t < m) at position first + r t, and
+// the CTA's tile of it.
 struct Unit {
-  int p, b, h, first, m;
+  int p, b, h, first, m, tile;
 };
-__device__ __forceinline__ Unit decode_unit(const Params& P, int64_t x) {
+// CTA x -> (pattern, batch, head, segment, tile).  Within a pattern the
+// tiles of one segment are consecutive CTAs (they share the streamed blocks,
+// which then stay in L2), longest first: the key-centric kernel's first tile
+// (it meets every later query when causal) and the query-centric kernel's
+// last one.
+template <bool kKeys>
+__device__ __forceinline__ Unit decode_cta(const Params& P, int64_t x) {
   Unit u;
   int p = 0;
-  while (p + 1 < P.pb.n_pat && x >= P.pat[p + 1].unit_base) ++p;
+  while (p + 1 < P.pb.n_pat && x >= P.pat[p + 1].cta_base) ++p;
   const PatGeo& g = P.pat[p];
-  int64_t rem = x - g.unit_base;
+  int64_t rem = x - g.cta_base;
+  const int t = (int)(rem % g.tiles);
+  rem /= g.tiles;
+  u.tile = kKeys ? t : g.tiles - 1 - t;
   const int seg = (int)(rem % g.n_seg);
   rem /= g.n_seg;
   u.p = p;
@@ -189,14 +202,62 @@ __device__ __forceinline__ float row_dot(const uint16_t* a, const uint16_t* b) {
   return d;
 }
 
+// P and dS of 32 streamed rows for this thread's tile row (tr), packed in
+// pairs: P = 2^(s scale log2(e) - lse log2(e)), dS = P (dP - delta).
+// Key-centric: the row is a key, the columns are queries (their -lse, -delta
+// from shared memory, nl and nd); query-centric: the row is a query with its
+// own lse2 and delta.  kMask: zero P outside the segment and, when causal,
+// outside the lower triangle.
+template <int kFmt, bool kKeys, bool kMask>
+__device__ __forceinline__ void p_ds_half(const uint32_t (&sr)[32], const uint32_t (&dr)[32], const float* nl_col,
+                                          const float* nd_col, float lse2, float delta, uint64_t sc2, int c0, int m,
+                                          int tr, bool causal, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+  const uint64_t nl_row = f32x2(-lse2, -lse2), nd_row = f32x2(-delta, -delta);
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    uint64_t nl[2], nd[2];
+    if (kKeys) {
+      const float4 l4 = *reinterpret_cast<const float4*>(nl_col + c);
+      const float4 d4 = *reinterpret_cast<const float4*>(nd_col + c);
+      nl[0] = f32x2(l4.x, l4.y);
+      nl[1] = f32x2(l4.z, l4.w);
+      nd[0] = f32x2(d4.x, d4.y);
+      nd[1] = f32x2(d4.z, d4.w);
+    } else {
+      nl[0] = nl[1] = nl_row;
+      nd[0] = nd[1] = nd_row;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      float x0, x1;
+      f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[c + e]), __uint_as_float(sr[c + e + 1])), sc2, nl[e / 2]), x0,
+                  x1);
+      float p0 = ex2(x0), p1 = ex2(x1);
+      if (kMask) {
+        const int col = c0 + c + e;
+        const bool v0 = col < m && (!causal || (kKeys ? col >= tr : col <= tr));
+        const bool v1 = col + 1 < m && (!causal || (kKeys ? col + 1 >= tr : col + 1 <= tr));
+        p0 = v0 ? p0 : 0.f;
+        p1 = v1 ? p1 : 0.f;
+      }
+      float d0, d1;
+      f32x2_split(mul_f32x2(f32x2(p0, p1),
+                            add_f32x2(f32x2(__uint_as_float(dr[c + e]), __uint_as_float(dr[c + e + 1])), nd[e / 2])),
+                  d0, d1);
+      pk[(c + e) / 2] = pack2<kFmt>(p0, p1);
+      dk[(c + e) / 2] = pack2<kFmt>(d0, d1);
+    }
+  }
+}
+
 // kKeys: the key-centric kernel (dk, dv); else the query-centric one (dq).
 template <int kFmt, bool kKeys>
 __global__ void __launch_bounds__(kThreads, 2)
     bwd_tc_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Unit u = decode_unit(P, blockIdx.x);
-  const int t0 = (int)blockIdx.y * kTile;  // first sparse row of this CTA's tile
+  const Unit u = decode_cta<kKeys>(P, blockIdx.x);
+  const int t0 = u.tile * kTile;  // first sparse row of this CTA's tile
   if (t0 >= u.m) return;                   // whole CTA, before any barrier or TMEM use
   const int nrows = u.m - t0 < kTile ? u.m - t0 : kTile;
   const bool causal = P.pb.causal != 0;
@@ -273,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int b0 = s0 + j * kBlk;
       const int need = s1 - b0 < kBlk ? s1 - b0 : kBlk;
       if (kKeys) {
-        // lse (log2 domain) and delta of the block's queries; zero past the segment
+        // -lse (log2 domain) and -delta of the block's queries; zero past the segment
         float* sl = reinterpret_cast<float*>(stage + 2 * kBlkBytes);
         float* sd = sl + kBlk;
 #pragma unroll
@@ -281,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int i = lane + 32 * e;
           const bool in = i < need;
           const int64_t pos = (int64_t)u.first + (int64_t)geo.r * (b0 + (in ? i : 0));
-          sl[i] = in ? P.pb.lse[bhN + pos] * kLog2e : 0.f;
-          sd[i] = in ? P.delta[bhN + pos] : 0.f;
+          sl[i] = in ? -P.pb.lse[bhN + pos] * kLog2e : 0.f;  // negated: the exponent's addend
+          sd[i] = in ? -P.delta[bhN + pos] : 0.f;
         }
       }
       if (lane == 0) {
@@ -371,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       delta = row_dot<kFmt>(static_cast<const uint16_t*>(P.g.dout) + elem,
                             static_cast<const uint16_t*>(P.g.out) + elem);
     }
+    const uint64_t sc2 = f32x2(P.scale_log2, P.scale_log2);
     bool ok = true;
     for (int j = 0; j < nblk && ok; ++j) {
       const int st = j % kStages;
@@ -381,6 +443,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!ok) break;
       tc_fence_after();
       const int b0 = s0 + j * kBlk;
+      // every (row, column) pair of the block real: no masking needed
+      const bool full = b0 + kBlk <= u.m && (!causal || (kKeys ? b0 >= tr : b0 + kBlk - 1 <= tr));
       // two halves of 32 streamed rows: scores and dP in, P and dS (packed
       // pairs) out over the first columns of the same TMEM buffers, which the
       // first half has already read when the second half is written
@@ -391,30 +455,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         LN_TMEM_LD32(tmem + lane_base + kColDP + 32 * hf, dr);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = b0 + 32 * hf + c + e;  // sparse index of the streamed row
-            bool valid;
-            float l2, dl;
-            if (kKeys) {  // row = key tr, column = query col
-              valid = col < u.m && (!causal || col >= tr);
-              l2 = sl[32 * hf + c + e];
-              dl = sd[32 * hf + c + e];
-            } else {      // row = query tr, column = key col
-              valid = col < u.m && (!causal || col <= tr);
-              l2 = lse2;
-              dl = delta;
-            }
-            const float p = valid ? ex2(fmaf(__uint_as_float(sr[c + e]), P.scale_log2, -l2)) : 0.f;
-            pv[e] = p;
-            dv[e] = p * (__uint_as_float(dr[c + e]) - dl);
-          }
-          pk[c / 2] = pack2<kFmt>(pv[0], pv[1]);
-          dk[c / 2] = pack2<kFmt>(dv[0], dv[1]);
-        }
+        const int c0 = b0 + 32 * hf;  // sparse index of the half's first streamed row
+        if (full)
+          p_ds_half<kFmt, kKeys, false>(sr, dr, sl + 32 * hf, sd + 32 * hf, lse2, delta, sc2, c0, u.m, tr, causal, pk, dk);
+        else
+          p_ds_half<kFmt, kKeys, true>(sr, dr, sl + 32 * hf, sd + 32 * hf, lse2, delta, sc2, c0, u.m, tr, causal, pk, dk);
         if (kKeys) LN_TMEM_ST16(tmem + lane_base + kColS + 16 * hf, pk);
         LN_TMEM_ST16(tmem + lane_base + kColDP + 16 * hf, dk);
       }
@@ -484,12 +529,12 @@ bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Units, tiles per segment and the per-pattern geometry; false when the
-// shape is outside this family.
-bool geometry(const Problem& p, Params* P, int64_t* t_max) {
+// CTAs and the per-pattern geometry; false when the shape is outside this
+// family.
+bool geometry(const Problem& p, Params* P) {
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD || p.qk_norm) return false;
   if (p.n_pat > kMaxPat || p.N > ((int64_t)1 << 30) || p.H > 65535 || p.B > 65535) return false;
-  int64_t units = 0, tm = 0;
+  int64_t ctas = 0;
   for (int i = 0; i < p.n_pat; ++i) {
     const int64_t w = p.w[i] < p.N ? p.w[i] : p.N, r = p.r[i];
     if (r > 4096) return false;
@@ -498,8 +543,7 @@ bool geometry(const Problem& p, Params* P, int64_t* t_max) {
     if (tail > 0 && p.N < kTile * r + 2 * tail) return false;
     if (p.N / r < 1) return false;
     const int64_t n_seg = (p.N + w - 1) / w;
-    const int64_t t = ((w + r - 1) / r + kTile - 1) / kTile;
-    if (t > tm) tm = t;
+    const int64_t tiles = ((w + r - 1) / r + kTile - 1) / kTile;
     if (P) {
       PatGeo& g = P->pat[i];
       g.w = (int)w;
@@ -508,20 +552,20 @@ bool geometry(const Problem& p, Params* P, int64_t* t_max) {
       g.tail = (int)tail;
       g.r_div = make_fastdiv(r);
       g.n_seg = (int)n_seg;
-      g.unit_base = units;
+      g.tiles = (int)tiles;
+      g.cta_base = ctas;
     }
-    units += p.B * p.H * n_seg;
+    ctas += p.B * p.H * n_seg * tiles;
+    if (ctas > 0x7fffffffLL) return false;
   }
-  if (P) P->n_units = units;
-  *t_max = tm;
-  return units > 0 && units <= 0x7fffffffLL && tm >= 1 && tm <= 65535;
+  if (P) P->n_ctas = ctas;
+  return ctas > 0;
 }
 
 }  // namespace tb
 
 bool tcgen05_backward_supports(const Problem& p) {
-  int64_t t_max = 0;
-  return tb::geometry(p, nullptr, &t_max);
+  return tb::geometry(p, nullptr);
 }
 
 int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t stream) {
@@ -531,8 +575,7 @@ int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t str
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   memset(&P, 0, sizeof(P));
-  int64_t t_max = 0;
-  if (!geometry(p, &P, &t_max)) return LONGNET_ERR_UNSUPPORTED;
+  if (!geometry(p, &P)) return LONGNET_ERR_UNSUPPORTED;
   EncodeTiledFn enc = get_encoder();
   if (!enc) return LONGNET_ERR_CUDA;
   P.pb = p;
@@ -589,7 +632,7 @@ int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t str
     cudaGetLastError();
     return LONGNET_ERR_CUDA;
   }
-  const dim3 grid((unsigned)P.n_units, (unsigned)t_max);
+  const dim3 grid((unsigned)P.n_ctas);
   kern_k<<<grid, kThreads, kSmemBytes, stream>>>(P, mk);
   if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
   if (cudaMemsetAsync(g.dq, 0, bytes, stream) != cudaSuccess) {
