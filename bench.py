@@ -460,6 +460,7 @@ def run_ours(args, wl):
         line["sweep_linear_1M_vs_64K"] = line["sweep"][-1]["tokens_per_s_vs_65536"]
     if ws == 1 and wl.name == "long32k" and not args.no_variants:
         line["variants"] = variant_lines(args.steps, args.warmup, dev.index)
+        line["backward"] = backward_line(wl, args.steps, args.warmup, dev.index)
     if ws == 1 and not args.no_cpu_baseline:
         n = args.cpu_positions
         calibrate = n <= 0
@@ -725,6 +726,50 @@ def sweep_lines(steps, warmup, kernel="auto", dev_index=0):
     base = res[0]["tokens_per_s"]
     for r in res:
         r["tokens_per_s_vs_65536"] = r["tokens_per_s"] / base
+    return res
+
+
+def backward_line(wl, steps, warmup, dev_index=0):
+    """The backward (dq, dk, dv) of the same workload after its forward, timed
+    like the main line: ms per call, the family AUTO ran, and the algorithmic
+    rate (10 D flops per attended pair) against the bf16 peak."""
+    import torch
+
+    from sparse_long_sequence_attn_b200 import binding as bd
+    from sparse_long_sequence_attn_b200 import workloads as wlm
+
+    dev = torch.device("cuda", dev_index)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    q, k, v = (x.to(dev) for x in wlm.make_inputs(wl))
+    dout = wlm.random_cotangent(wl.B, wl.N, wl.H, wl.D, wl.torch_dtype, seed=wl.seed).to(dev)
+    out, lse = bd.dilated_attn(q, k, v, wl.patterns, wl.causal)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    family = "tiles or simt"
+    try:
+        bd.longnet_dilated_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, wl.patterns, wl.causal,
+                                    bd.LONGNET_IMPL_TCGEN05)
+        family = "tcgen05"
+    except bd.LongNetError as e:
+        if e.code != bd.LONGNET_ERR_UNSUPPORTED:
+            raise
+
+    def step():
+        bd.longnet_dilated_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, wl.patterns, wl.causal,
+                                    bd.LONGNET_IMPL_AUTO, stream)
+
+    per = time_steps(step, steps, warmup, stream, flush)
+    st = bd.longnet_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after the backward: {bd.status_string(st)}")
+    t = sum(per) / len(per)
+    flops = 10.0 * wl.D * wlm.exact_pair_count(wl)
+    peaks, peak_kind = load_peaks()
+    tf = flops / t / 1e12
+    res = {"ms": t * 1e3, "steps": steps, "family": family, "tokens_per_s": wl.B * wl.N / t,
+           "tflops_algorithmic": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "peak_source": peak_kind}
+    del q, k, v, dout, out, lse, dq, dk, dv
+    torch.cuda.empty_cache()
     return res
 
 
