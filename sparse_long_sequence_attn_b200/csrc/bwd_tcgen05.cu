@@ -80,7 +80,7 @@ constexpr uint32_t kColS = 0, kColDP = 64, kColAcc0 = 128, kColAcc1 = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int kFmt>
-constexpr uint32_t kIdescScore = idesc_f16kind(kTile, kBlk, false, kFmt);  // 128 x 64, B K-major
+constexpr uint32_t kIdescScore = idesc_f16kind(kTile, kBlk / 2, false, kFmt);  // 128 x 32 (a half block), B K-major
 template <int kFmt>
 constexpr uint32_t kIdescGrad = idesc_f16kind(kTile, kD, true, kFmt);      // 128 x 64, B MN-major
 
@@ -275,11 +275,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar_tile = bars + 0;
   uint64_t* bar_full = bars + 1;            // [kStages]
   uint64_t* bar_empty = bars + 1 + kStages;  // [kStages]
-  uint64_t* bar_s = bars + 1 + 2 * kStages;
-  uint64_t* bar_p = bar_s + 1;
-  uint64_t* bar_acc = bar_s + 2;
-  uint64_t* bar_drain = bar_s + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 4);
+  uint64_t* bar_s = bars + 1 + 2 * kStages;  // [2] scores of a half block in TMEM
+  uint64_t* bar_p = bar_s + 2;               // [2] P and dS of a half block in TMEM
+  uint64_t* bar_acc = bar_s + 4;
+  uint64_t* bar_drain = bar_s + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -289,8 +289,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(bar_full + i, 32);  // the loading warp's 32 lanes (lane 0 with the TMA bytes)
       mbar_init(bar_empty + i, 1);
     }
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s + i, 1);
+      mbar_init(bar_p + i, 128);
+    }
     mbar_init(bar_acc, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -372,46 +374,70 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t t0_lo = (smem_u32(sTile0) >> 4) | (1u << 16);
       const uint32_t t1_lo = (smem_u32(sTile1) >> 4) | (1u << 16);
       const uint32_t lbo_mn = ((uint32_t)(kBlk * 128) >> 4) << 16;
-      bool ok = wt.wait(bar_tile, 0);
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int st = j % kStages;
-        ok = wt.wait(bar_full + st, (j / kStages) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t b0_addr = smem_u32(sStage + st * kStageBytes) >> 4;
+      // Blocks go in two halves of 32 streamed rows, so the tensor cores work
+      // on one half while the compute warps work on the other:
+      //   scores(0, a) scores(0, b) | grads(j, a) scores(j+1, a) | grads(j, b) scores(j+1, b) | ...
+      // A half's scores overwrite TMEM columns whose P and dS the same half's
+      // gradient products (issued just before, executed in order) have read.
+      auto stage_addr = [&](int j) -> uint32_t { return smem_u32(sStage + (j % kStages) * kStageBytes) >> 4; };
+      auto scores = [&](int j, int hf) {
+        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * 128 >> 4);
         const uint32_t b1_addr = b0_addr + (kBlkBytes >> 4);
-        // scores: tile0 x block0^T and tile1 x block1^T (K-major operands)
+        // tile0 x block0^T and tile1 x block1^T over the half's 32 rows (K-major operands)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          mma_ss(tmem + kColS, desc_from(t0_lo + kk * 2, kDescHi), desc_from((b0_addr | (1u << 16)) + kk * 2, kDescHi),
-                 kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kColS + 32 * hf, desc_from(t0_lo + kk * 2, kDescHi),
+                 desc_from((b0_addr | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          mma_ss(tmem + kColDP, desc_from(t1_lo + kk * 2, kDescHi), desc_from((b1_addr | (1u << 16)) + kk * 2, kDescHi),
-                 kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
-        tc_commit(bar_s);
-        ok = wt.wait(bar_p, j & 1);
+          mma_ss(tmem + kColDP + 32 * hf, desc_from(t1_lo + kk * 2, kDescHi),
+                 desc_from((b1_addr | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
+        tc_commit(bar_s + hf);
+      };
+      // gradients of a half: A (P or dS, packed) from TMEM, B the half's rows read MN-major
+      auto grads = [&](int j, int hf) {
+        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * 128 >> 4);
+        const uint32_t b1_addr = b0_addr + (kBlkBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 32; ++kk) {
+          const uint32_t acc = (j > 0 || hf > 0 || kk > 0) ? 1u : 0u;
+          if (kKeys) {
+            // dV += P^T dout (block 1), dK += dS^T Q (block 0)
+            mma_ts(tmem + kColAcc0, tmem + kColS + 32 * hf + kk * 8, desc_from((b1_addr | lbo_mn) + kk * 128, kDescHi),
+                   kIdescGrad<kFmt>, acc);
+            mma_ts(tmem + kColAcc1, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
+                   kIdescGrad<kFmt>, acc);
+          } else {
+            // dQ += dS K (block 0)
+            mma_ts(tmem + kColAcc0, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
+                   kIdescGrad<kFmt>, acc);
+          }
+        }
+      };
+      bool ok = wt.wait(bar_tile, 0) && wt.wait(bar_full + 0, 0);
+      if (ok) {
+        tc_fence_after();
+        scores(0, 0);
+        scores(0, 1);
+      }
+      for (int j = 0; j < nblk && ok; ++j) {
+        const bool more = j + 1 < nblk;
+        ok = wt.wait(bar_p + 0, j & 1);
         if (!ok) break;
         tc_fence_after();
-        // gradients: A (P or dS, input format) from TMEM, B the block read MN-major
-        if (kKeys) {
-          // dV += P^T dout (block 1), dK += dS^T Q (block 0)
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tmem + kColAcc0, tmem + kColS + kk * 8, desc_from((b1_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, (j > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tmem + kColAcc1, tmem + kColDP + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, (j > 0 || kk > 0) ? 1u : 0u);
-        } else {
-          // dQ += dS K (block 0)
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk)
-            mma_ts(tmem + kColAcc0, tmem + kColDP + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, (j > 0 || kk > 0) ? 1u : 0u);
+        grads(j, 0);
+        if (more) {
+          ok = wt.wait(bar_full + (j + 1) % kStages, ((j + 1) / kStages) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          scores(j + 1, 0);
         }
-        tc_commit(bar_empty + st);
+        ok = wt.wait(bar_p + 1, j & 1);
+        if (!ok) break;
+        tc_fence_after();
+        grads(j, 1);
+        tc_commit(bar_empty + j % kStages);  // the block's shared memory is free once its products ran
+        if (more) scores(j + 1, 1);
       }
       if (ok) tc_commit(bar_acc);
       // drain: all issued MMAs complete before TMEM is released
@@ -439,17 +465,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float* sl = reinterpret_cast<const float*>(sStage + st * kStageBytes + 2 * kBlkBytes);
       const float* sd = sl + kBlk;
       if (kKeys) ok = wt.wait_warp(bar_full + st, (j / kStages) & 1);
-      if (ok) ok = wt.wait_warp(bar_s, j & 1);
       if (!ok) break;
-      tc_fence_after();
       const int b0 = s0 + j * kBlk;
       // every (row, column) pair of the block real: no masking needed
       const bool full = b0 + kBlk <= u.m && (!causal || (kKeys ? b0 >= tr : b0 + kBlk - 1 <= tr));
-      // two halves of 32 streamed rows: scores and dP in, P and dS (packed
-      // pairs) out over the first columns of the same TMEM buffers, which the
-      // first half has already read when the second half is written
+      // two halves of 32 streamed rows, each as soon as its scores are in
+      // TMEM: scores and dP in, P and dS (packed pairs) out over the first 16
+      // columns of the half's own 32
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int hf = 0; hf < 2 && ok; ++hf) {
+        ok = wt.wait_warp(bar_s + hf, j & 1);
+        if (!ok) break;
+        tc_fence_after();
         uint32_t sr[32], dr[32];
         LN_TMEM_LD32(tmem + lane_base + kColS + 32 * hf, sr);
         LN_TMEM_LD32(tmem + lane_base + kColDP + 32 * hf, dr);
@@ -460,12 +487,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           p_ds_half<kFmt, kKeys, false>(sr, dr, sl + 32 * hf, sd + 32 * hf, lse2, delta, sc2, c0, u.m, tr, causal, pk, dk);
         else
           p_ds_half<kFmt, kKeys, true>(sr, dr, sl + 32 * hf, sd + 32 * hf, lse2, delta, sc2, c0, u.m, tr, causal, pk, dk);
-        if (kKeys) LN_TMEM_ST16(tmem + lane_base + kColS + 16 * hf, pk);
-        LN_TMEM_ST16(tmem + lane_base + kColDP + 16 * hf, dk);
+        if (kKeys) LN_TMEM_ST16(tmem + lane_base + kColS + 32 * hf, pk);
+        LN_TMEM_ST16(tmem + lane_base + kColDP + 32 * hf, dk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p + hf);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p);
     }
     if (ok) ok = wt.wait_warp(bar_acc, 0);
     if (ok) {
