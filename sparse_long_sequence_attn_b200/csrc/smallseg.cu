@@ -37,6 +37,7 @@
 
 #include "device_util.cuh"
 #include "params.h"
+#include "tc_ptx.cuh"  // the tensor-map encoder lookup
 
 namespace longnet {
 namespace ss {
@@ -511,25 +512,6 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
 
 // ------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encoder() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
 // Layout of one warp pair's shared memory for these patterns; 0 if unsupported.
 int pair_bytes(const Problem& p, int* park_off, int* park_rows, int* order) {
   int n1 = 0, k = 0;
@@ -579,7 +561,7 @@ bool smallseg_supports(const Problem& p) {
 
 int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   using namespace ss;
-  EncodeTiledFn enc = get_encoder();
+  tc::EncodeTiledFn enc = tc::get_encoder();
   if (!enc) return LONGNET_ERR_CUDA;
   static Params P;
   static Maps maps;
