@@ -70,7 +70,8 @@ def _code_only(text: str) -> str:
 def kernel_source_hash(family: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_long_sequence_attn_b200", "csrc")
-    paths = [os.path.join(csrc, n) for n in (f"{family}.cu",) + _FAMILY_SOURCES]
+    src = {"patterns": "perpattern.cu"}.get(family, f"{family}.cu")
+    paths = [os.path.join(csrc, n) for n in (src,) + _FAMILY_SOURCES]
     paths.append(os.path.join(ROOT, "include", "longnet.h"))
     for path in paths:
         with open(path, encoding="utf-8") as f:
@@ -247,7 +248,7 @@ def main():
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", help="ours | reference")
     ap.add_argument("--kernel", default="auto",
-                    help="auto | simt | tcgen05 | smallseg (forward); auto | simt | tiles | tcgen05 (--pass bwd)")
+                    help="auto | simt | tcgen05 | smallseg | patterns (forward); auto | simt | tiles | tcgen05 (--pass bwd)")
     ap.add_argument("--ref-positions", type=int, default=48)
     ap.add_argument("--cpu-positions", type=int, default=0,
                     help="oracle sample size for cpu_baseline (0: calibrate to ~10 s)")
@@ -286,11 +287,12 @@ def _impl_code(name):
     from sparse_long_sequence_attn_b200 import binding as bd
 
     return {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT,
-            "tcgen05": bd.LONGNET_IMPL_TCGEN05, "smallseg": bd.LONGNET_IMPL_SMALLSEG}[name]
+            "tcgen05": bd.LONGNET_IMPL_TCGEN05, "smallseg": bd.LONGNET_IMPL_SMALLSEG,
+            "patterns": bd.LONGNET_IMPL_PATTERNS}[name]
 
 
 def _impl_name(code):
-    return {1: "simt", 2: "tcgen05", 3: "smallseg"}.get(code, str(code))
+    return {1: "simt", 2: "tcgen05", 3: "smallseg", 5: "patterns"}.get(code, str(code))
 
 
 def time_steps(fn, steps, warmup, stream, flush_buf):
@@ -450,7 +452,7 @@ def run_ours(args, wl):
         "roofline": roof,
         "e2e": {"value": weak_scaling_rate(tokens * e2e_steps, ws, e2e_total), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": (1 + len(wl.patterns) if kname == "patterns" else 1) * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
     if soak is not None:

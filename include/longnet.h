@@ -29,8 +29,8 @@
  *     When w does not divide N the last segment is the shorter rest of the
  *     sequence (no padding); w > N makes one segment of the whole sequence.
  *     Patterns may repeat and come in any order; a repeated pattern counts
- *     twice.  (The tcgen05 and small-segment kernels take N % w == 0 only;
- *     LONGNET_IMPL_AUTO falls back to the SIMT kernel otherwise.)
+ *     twice.  (The small-segment kernel takes N % w == 0 only; AUTO picks
+ *     another family otherwise.)
  *   - causal: 1 = causal inside each sparsified segment, 0 = full.
  *   - stream: a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; the call returns before it finishes.
@@ -84,9 +84,15 @@ enum longnet_impl {
   LONGNET_IMPL_SMALLSEG = 3, /* bf16 or fp16, D = 64, all patterns one segment
                                 length w <= 64 (a multiple of 8), one of them
                                 r = 1: memory-bound kernel */
-  LONGNET_IMPL_TILES = 4     /* backward only: bf16 or fp16, D = 64, any
+  LONGNET_IMPL_TILES = 4,    /* backward only: bf16 or fp16, D = 64, any
                                 patterns: 64-row tiles of the sparsified
                                 segments on mma.sync tensor cores */
+  LONGNET_IMPL_PATTERNS = 5  /* forward: bf16 or fp16, D = 64 or 128, any number
+                                of patterns, lse required with more than one:
+                                one tcgen05 launch per pattern, each merging its
+                                rows into out and lse (initialised to 0 and
+                                -inf); out is rounded to the input format
+                                between patterns */
 };
 
 /*
@@ -328,8 +334,9 @@ int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
 
 /*
  * longnet_select_impl — which family AUTO would run for these arguments
- * (a longnet_impl >= 1), or a negative longnet_status when the arguments
- * are invalid.  Host-only; touches no device.
+ * with lse requested (a longnet_impl >= 1), or a negative longnet_status
+ * when the arguments are invalid.  Host-only; touches no device.  (Without
+ * lse, a multi-pattern call the PATTERNS family would take goes to SIMT.)
  */
 int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
                         const int64_t* w, const int64_t* r, int causal,

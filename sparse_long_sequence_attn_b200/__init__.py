@@ -8,6 +8,7 @@ forward (seqpar).
 """
 from .binding import (  # noqa: F401
     LONGNET_IMPL_AUTO,
+    LONGNET_IMPL_PATTERNS,
     LONGNET_IMPL_SIMT,
     LONGNET_IMPL_SMALLSEG,
     LONGNET_IMPL_TCGEN05,

@@ -38,6 +38,7 @@ LONGNET_IMPL_SIMT = 1
 LONGNET_IMPL_TCGEN05 = 2
 LONGNET_IMPL_SMALLSEG = 3
 LONGNET_IMPL_TILES = 4
+LONGNET_IMPL_PATTERNS = 5
 
 # Every symbol include/longnet.h declares, with its ctypes signature.
 _i64 = ctypes.c_int64

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblongnet.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["api.cu", "simt.cu", "tcgen05.cu", "smallseg.cu", "backward.cu", "bwd_tcgen05.cu", "exchange.cu", "prologue.cu"]
+SOURCES = ["api.cu", "simt.cu", "tcgen05.cu", "smallseg.cu", "backward.cu", "bwd_tcgen05.cu", "exchange.cu", "prologue.cu", "perpattern.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -111,6 +111,7 @@ bool simt_supports(const Problem& p) { return p.D == 16 || p.D == 32 || p.D == 6
 int choose_impl(const Problem& p) {
   if (smallseg_supports(p)) return LONGNET_IMPL_SMALLSEG;
   if (tcgen05_supports(p)) return LONGNET_IMPL_TCGEN05;
+  if (perpattern_supports(p)) return LONGNET_IMPL_PATTERNS;
   if (simt_supports(p)) return LONGNET_IMPL_SIMT;
   return LONGNET_ERR_UNSUPPORTED;
 }
@@ -157,6 +158,9 @@ int run(Problem& pb, int impl, longnet_stream_t stream) {
     case LONGNET_IMPL_SMALLSEG:
       if (!smallseg_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
       return launch_smallseg(pb, s);
+    case LONGNET_IMPL_PATTERNS:
+      if (!perpattern_supports(pb)) return LONGNET_ERR_UNSUPPORTED;
+      return launch_perpattern(pb, s);
     default:
       return LONGNET_ERR_INVALID_ARG;
   }
@@ -174,7 +178,8 @@ int check_part(Problem& pb, int64_t q0, int64_t q1, int64_t h0, int64_t h1) {
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
             int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
             int flags, int impl, int64_t q0, int64_t q1, int64_t h0, int64_t h1, longnet_stream_t stream) {
-  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_PATTERNS || impl == LONGNET_IMPL_TILES)
+    return LONGNET_ERR_INVALID_ARG;
   if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
   int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
@@ -189,7 +194,8 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
 int forward_ws(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t N,
                int64_t H, int64_t D, int n_pat, const int64_t* w, const int64_t* r, int causal, int dtype,
                int flags, int impl, void* workspace, int64_t workspace_bytes, longnet_stream_t stream) {
-  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_SMALLSEG) return LONGNET_ERR_INVALID_ARG;
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_PATTERNS || impl == LONGNET_IMPL_TILES)
+    return LONGNET_ERR_INVALID_ARG;
   if (flags & ~(LONGNET_FLAG_QK_NORM | LONGNET_FLAG_XPOS)) return LONGNET_ERR_INVALID_ARG;
   Problem pb;
   int rc = check_args(q, k, v, out, lse, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
@@ -391,11 +397,12 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
 
 extern "C" int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
                                    const int64_t* w, const int64_t* r, int causal, int dtype) {
-  // Stand-in pointers: only their alignment is looked at here.
+  // Stand-in pointers: only their alignment (and, for lse, presence) is
+  // looked at here; the call is taken as one that asks for lse.
   static __align__(16) char dummy[16];
   Problem pb;
-  int rc = check_args(dummy, dummy, dummy, dummy, nullptr, B, N, H, D, n_pat, w, r, causal, dtype,
-                      &pb);
+  int rc = check_args(dummy, dummy, dummy, dummy, reinterpret_cast<float*>(dummy), B, N, H, D, n_pat, w, r,
+                      causal, dtype, &pb);
   if (rc) return rc;
   return choose_impl(pb);
 }

@@ -68,6 +68,8 @@ int launch_move_rows(const void* src, const int64_t* src_idx, int64_t src_rows, 
 
 // Shape checks of the specialised families (host only, no device access).
 bool tcgen05_supports(const Problem& p);
+bool perpattern_supports(const Problem& p);  // the per-pattern tcgen05 forward
+int launch_perpattern(const Problem& p, cudaStream_t stream);
 bool smallseg_supports(const Problem& p);
 bool backward_supports(const Problem& p);       // the SIMT backward
 bool tile_backward_supports(const Problem& p);  // the mma.sync tile backward

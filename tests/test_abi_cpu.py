@@ -93,8 +93,12 @@ def test_select_impl_host_logic():
     assert bd.longnet_select_impl(1, 255, 2, 16, ((64, 1),), True, f32) == bd.LONGNET_IMPL_SIMT
     # bf16 D = 64 with shorter last segments (4000 = 3 * 1024 + 928) goes to tcgen05
     assert bd.longnet_select_impl(1, 4000, 4, 64, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_TCGEN05
-    # D = 128 and fp32 inputs go to the general kernel
-    assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_SIMT
+    # D = 128 (16-bit) goes to the per-pattern tcgen05 family, fp32 to the general kernel
+    assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_PATTERNS
+    assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, f32) == bd.LONGNET_IMPL_SIMT
+    # more than 6 patterns at D = 64: per-pattern family
+    seven = tuple((256 * (i + 1), i + 1) for i in range(7))
+    assert bd.longnet_select_impl(1, 4096, 4, 64, seven, True, bf16) == bd.LONGNET_IMPL_PATTERNS
     assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 0),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
     impl = bd.longnet_select_impl(1, 32768, 12, 64, ((2048, 1), (4096, 2)), True, bf16)
     assert impl in (bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05)

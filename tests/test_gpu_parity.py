@@ -15,7 +15,7 @@ from tests import gpu_helpers as gh
 pytestmark = pytest.mark.gpu
 
 IMPLS = {"simt": bd.LONGNET_IMPL_SIMT, "tcgen05": bd.LONGNET_IMPL_TCGEN05,
-         "smallseg": bd.LONGNET_IMPL_SMALLSEG}
+         "smallseg": bd.LONGNET_IMPL_SMALLSEG, "patterns": bd.LONGNET_IMPL_PATTERNS}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -75,7 +75,7 @@ def test_small_cases_vs_oracle(case, impl_name):
 
 @pytest.mark.parametrize("case", [c for c in SMALL_CASES if c[5] in (torch.bfloat16, torch.float16) and c[4] == 64],
                          ids=[c[0] for c in SMALL_CASES if c[5] in (torch.bfloat16, torch.float16) and c[4] == 64])
-@pytest.mark.parametrize("impl_name", ["tcgen05", "smallseg"])
+@pytest.mark.parametrize("impl_name", ["tcgen05", "smallseg", "patterns"])
 def test_specialised_families_vs_oracle(case, impl_name):
     name, B, N, H, D, dtype, causal, pats = case
     q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=zlib.crc32(name.encode()) % 100000)
@@ -86,6 +86,44 @@ def test_specialised_families_vs_oracle(case, impl_name):
             pytest.skip(f"{impl_name} does not take {name}")
         raise
     gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
+
+
+# Shapes the fused tcgen05 family does not take: D = 128, more than six
+# patterns, more than eight distinct r; the per-pattern family does.
+PATTERNS_CASES = [
+    # name, B, N, H, D, dtype, causal, patterns
+    ("bf16_d128_lm_like", 2, 2048, 4, 128, torch.bfloat16, True, ((512, 1), (1024, 2), (2048, 4))),
+    ("bf16_d128_noncausal_partial", 1, 1500, 3, 128, torch.bfloat16, False, ((384, 1), (700, 3), (2000, 5))),
+    ("f16_d128_causal", 1, 1024, 2, 128, torch.float16, True, ((256, 1), (1024, 4))),
+    ("bf16_d64_seven_patterns", 1, 2048, 5, 64, torch.bfloat16, True,
+     ((128, 1), (256, 2), (384, 3), (512, 4), (768, 5), (1024, 6), (2048, 8))),
+    ("bf16_d128_one_pattern", 1, 1024, 2, 128, torch.bfloat16, True, ((256, 1),)),
+    ("bf16_d128_uncovered", 1, 960, 3, 128, torch.bfloat16, True, ((192, 3), (960, 4))),
+]
+
+
+@pytest.mark.parametrize("case", PATTERNS_CASES, ids=[c[0] for c in PATTERNS_CASES])
+@pytest.mark.parametrize("impl_name", ["auto", "patterns"])
+def test_per_pattern_family_vs_oracle(case, impl_name):
+    name, B, N, H, D, dtype, causal, pats = case
+    impl = bd.LONGNET_IMPL_AUTO if impl_name == "auto" else IMPLS[impl_name]
+    if impl_name == "auto":
+        assert bd.longnet_select_impl(B, N, H, D, pats, causal, dtype) == bd.LONGNET_IMPL_PATTERNS
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=zlib.crc32(name.encode()) % 100000)
+    o, l = gh.run_cuda(q, k, v, pats, causal, impl)
+    err = gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"{name}/{impl_name}")
+    print(f"{name}/{impl_name}: max|out - oracle| = {err:.3e}")
+
+
+def test_per_pattern_family_without_lse():
+    """One pattern needs no lse; several need it (else AUTO picks SIMT and the
+    forced family is refused)."""
+    q, k, v = wl.random_inputs(1, 1024, 2, 128, torch.bfloat16, seed=41)
+    o1, _ = gh.run_cuda(q, k, v, ((256, 1),), True, bd.LONGNET_IMPL_PATTERNS, want_lse=False)
+    gh.compare_full(o1, None, q, k, v, ((256, 1),), True, torch.bfloat16, label="one pattern, no lse")
+    with pytest.raises(bd.LongNetError) as e:
+        gh.run_cuda(q, k, v, ((256, 1), (1024, 2)), True, bd.LONGNET_IMPL_PATTERNS, want_lse=False)
+    assert e.value.code == bd.LONGNET_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("impl_name", ["auto", "tcgen05", "simt"])
