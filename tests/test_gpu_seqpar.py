@@ -19,7 +19,7 @@ from tests import gpu_helpers as gh
 pytestmark = pytest.mark.gpu
 
 IMPLS = {"auto": bd.LONGNET_IMPL_AUTO, "simt": bd.LONGNET_IMPL_SIMT, "tcgen05": bd.LONGNET_IMPL_TCGEN05,
-         "smallseg": bd.LONGNET_IMPL_SMALLSEG}
+         "smallseg": bd.LONGNET_IMPL_SMALLSEG, "patterns": bd.LONGNET_IMPL_PATTERNS}
 OUT_SENTINEL, LSE_SENTINEL = 3.0, -7.0
 POISON = 1.0e4
 
@@ -43,6 +43,7 @@ CASES = [
     ("fp32_g2", 1, 512, 2, 32, torch.float32, True, ((128, 1), (512, 2)), 2),
     ("small_segments_g2", 2, 2048, 4, 64, torch.bfloat16, True, ((64, 1), (64, 2)), 2),
     ("f16_g4", 1, 4096, 4, 64, torch.float16, True, ((1024, 1), (4096, 8)), 4),
+    ("bf16_d128_g2", 1, 4096, 2, 128, torch.bfloat16, True, ((1024, 1), (4096, 4)), 2),
 ]
 
 
@@ -89,7 +90,7 @@ def emulate_ranks(q, k, v, patterns, causal, G, impl):
 
 
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
-@pytest.mark.parametrize("impl_name", ["auto", "simt", "tcgen05"])
+@pytest.mark.parametrize("impl_name", ["auto", "simt", "tcgen05", "patterns"])
 def test_emulated_ranks_vs_oracle_and_single_device(case, impl_name):
     name, B, N, H, D, dtype, causal, pats, G = case
     impl = IMPLS[impl_name]
@@ -108,7 +109,7 @@ def test_emulated_ranks_vs_oracle_and_single_device(case, impl_name):
     assert d <= gh.TOL_OUT[dtype]
 
 
-@pytest.mark.parametrize("impl_name", ["auto", "simt", "tcgen05"])
+@pytest.mark.parametrize("impl_name", ["auto", "simt", "tcgen05", "patterns"])
 def test_head_ranges_assemble_the_full_forward(impl_name):
     """Heads split into three ranges, each computed by its own call: the
     assembled output equals the single-call forward, and nothing outside a
