@@ -772,6 +772,25 @@ def backward_line(wl, steps, warmup, dev_index=0):
            "tflops_algorithmic": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "peak_source": peak_kind}
     del q, k, v, dout, out, lse, dq, dk, dv
     torch.cuda.empty_cache()
+    # the same shape at D = 128 (half the heads, the same FLOPs)
+    H2, D2 = wl.H // 2, 2 * wl.D
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed)
+    q, k, v, dout = (torch.randn(wl.B, wl.N, H2, D2, device=dev, generator=g, dtype=torch.float32)
+                     .to(wl.torch_dtype) for _ in range(4))
+    out, lse = bd.dilated_attn(q, k, v, wl.patterns, wl.causal)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    per = time_steps(lambda: bd.longnet_dilated_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, wl.patterns,
+                                                         wl.causal, bd.LONGNET_IMPL_AUTO, stream),
+                     steps, warmup, stream, flush)
+    st = bd.longnet_last_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after the D = 128 backward: {bd.status_string(st)}")
+    t2 = sum(per) / len(per)
+    res["d128"] = {"H": H2, "D": D2, "ms": t2 * 1e3, "tflops_algorithmic": flops / t2 / 1e12,
+                   "frac_of_bf16_peak": flops / t2 / 1e12 / peaks["bf16_tflops"]}
+    del q, k, v, dout, out, lse, dq, dk, dv
+    torch.cuda.empty_cache()
     return res
 
 

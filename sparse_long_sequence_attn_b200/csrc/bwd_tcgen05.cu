@@ -64,25 +64,36 @@ namespace longnet {
 namespace tb {
 using namespace tc;
 
-constexpr int kD = 64;
 constexpr int kTile = 128;                      // rows a CTA owns (M of every MMA)
 constexpr int kBlk = 64;                        // rows of a streamed block (N of the score MMAs)
 constexpr int kMaxPat = 6;
 constexpr int kStages = 3;
 constexpr int kThreads = 192;                   // warp 0 loads, warp 1 MMAs, warps 2-5 compute
-constexpr int kTileBytes = kTile * kD * 2;      // 16 KB
-constexpr int kBlkBytes = kBlk * kD * 2;        // 8 KB
-constexpr int kStageBytes = 2 * kBlkBytes + 1024;  // two blocks, then lse and delta (key-centric)
-constexpr int kSmemBytes = 2 * kTileBytes + kStages * kStageBytes + 256 + 1024;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kTilePanel = kTile * 128;         // 16 KB: 128 rows of one 64-element swizzle panel
+constexpr int kBlkPanel = kBlk * 128;           // 8 KB
 // TMEM columns: scores (S or S^T), dP, then the accumulators.
-constexpr uint32_t kColS = 0, kColDP = 64, kColAcc0 = 128, kColAcc1 = 192;
+constexpr uint32_t kColS = 0, kColDP = 64, kColAcc0 = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Sizes for D = 64 kPanels (a row is kPanels 128-byte swizzle panels).
+template <int kPanels>
+struct BL {
+  static constexpr int kD = 64 * kPanels;
+  static constexpr int kTileBytes = kPanels * kTilePanel;
+  static constexpr int kBlkBytes = kPanels * kBlkPanel;
+  static constexpr int kStageBytes = 2 * kBlkBytes + 1024;  // two blocks, then lse and delta (key-centric)
+  static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kStageBytes + 256 + 1024;
+  static constexpr uint32_t kColAcc1 = kColAcc0 + kD;       // the key-centric kernel's second accumulator
+  // 256 columns, two CTAs per SM at D = 64; the key-centric kernel at D = 128
+  // needs 384 (512 allocated), and shared memory allows one CTA per SM there
+  template <bool kKeys>
+  __host__ __device__ static constexpr uint32_t tmem_cols() { return kColAcc0 + (kKeys ? 2 : 1) * kD <= 256 ? 256u : 512u; }
+};
 
 template <int kFmt>
 constexpr uint32_t kIdescScore = idesc_f16kind(kTile, kBlk / 2, false, kFmt);  // 128 x 32 (a half block), B K-major
-template <int kFmt>
-constexpr uint32_t kIdescGrad = idesc_f16kind(kTile, kD, true, kFmt);      // 128 x 64, B MN-major
+template <int kFmt, int kD>
+constexpr uint32_t kIdescGrad = idesc_f16kind(kTile, kD, true, kFmt);      // 128 x D, B MN-major
 
 struct PatGeo {
   int w, r;
@@ -181,12 +192,12 @@ struct Waiter {
   __device__ bool wait_warp(uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, wait(bar, parity)); }
 };
 
-// dot(a, b) of two rows of 64 16-bit elements (global memory, 16-byte aligned)
-template <int kFmt>
+// dot(a, b) of two rows of kD 16-bit elements (global memory, 16-byte aligned)
+template <int kFmt, int kD>
 __device__ __forceinline__ float row_dot(const uint16_t* a, const uint16_t* b) {
   float d = 0.f;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < kD / 8; ++c) {
     const uint4 x = reinterpret_cast<const uint4*>(a)[c];
     const uint4 y = reinterpret_cast<const uint4*>(b)[c];
     const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
@@ -251,9 +262,12 @@ __device__ __forceinline__ void p_ds_half(const uint32_t (&sr)[32], const uint32
 }
 
 // kKeys: the key-centric kernel (dk, dv); else the query-centric one (dq).
-template <int kFmt, bool kKeys>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int kFmt, bool kKeys, int kPanels>
+__global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
     bwd_tc_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
+  using L = BL<kPanels>;
+  constexpr int kD = L::kD, kTileBytes = L::kTileBytes, kBlkBytes = L::kBlkBytes, kStageBytes = L::kStageBytes;
+  constexpr uint32_t kColAcc1 = L::kColAcc1, kTmemCols = L::template tmem_cols<kKeys>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Unit u = decode_cta<kKeys>(P, blockIdx.x);
@@ -325,8 +339,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const Coord c = coord(geo, u.first + geo.r * t0, nrows);
       const CUtensorMap* mp = c.map ? mp1 : mp0;
       mbar_arrive_expect_tx(bar_tile, 2 * kTileBytes);
-      tma_load_5d(sTile0, mp + 0, bar_tile, 0, u.h, c.c, c.kk, u.b);
-      tma_load_5d(sTile1, mp + 1, bar_tile, 0, u.h, c.c, c.kk, u.b);
+#pragma unroll
+      for (int pn = 0; pn < kPanels; ++pn) {
+        tma_load_5d(sTile0 + pn * kTilePanel, mp + 0, bar_tile, 64 * pn, u.h, c.c, c.kk, u.b);
+        tma_load_5d(sTile1 + pn * kTilePanel, mp + 1, bar_tile, 64 * pn, u.h, c.c, c.kk, u.b);
+      }
     }
     for (int j = 0; j < nblk && ok; ++j) {
       const int st = j % kStages;
@@ -352,8 +369,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         const Coord c = coord(geo, u.first + geo.r * b0, need);
         const CUtensorMap* mp = c.map ? mp1 : mp0;
         mbar_arrive_expect_tx(bar_full + st, 2 * kBlkBytes);
-        tma_load_5d(stage, mp + 2, bar_full + st, 0, u.h, c.c, c.kk, u.b);
-        tma_load_5d(stage + kBlkBytes, mp + 3, bar_full + st, 0, u.h, c.c, c.kk, u.b);
+#pragma unroll
+        for (int pn = 0; pn < kPanels; ++pn) {
+          tma_load_5d(stage + pn * kBlkPanel, mp + 2, bar_full + st, 64 * pn, u.h, c.c, c.kk, u.b);
+          tma_load_5d(stage + kBlkBytes + pn * kBlkPanel, mp + 3, bar_full + st, 64 * pn, u.h, c.c, c.kk, u.b);
+        }
       } else {
         mbar_arrive(bar_full + st);
       }
@@ -383,15 +403,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       auto scores = [&](int j, int hf) {
         const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * 128 >> 4);
         const uint32_t b1_addr = b0_addr + (kBlkBytes >> 4);
-        // tile0 x block0^T and tile1 x block1^T over the half's 32 rows (K-major operands)
+        // tile0 x block0^T and tile1 x block1^T over the half's 32 rows
+        // (K-major operands, one 64-element panel of D at a time)
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          mma_ss(tmem + kColS + 32 * hf, desc_from(t0_lo + kk * 2, kDescHi),
-                 desc_from((b0_addr | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
+        for (int pn = 0; pn < kPanels; ++pn)
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          mma_ss(tmem + kColDP + 32 * hf, desc_from(t1_lo + kk * 2, kDescHi),
-                 desc_from((b1_addr | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kColS + 32 * hf, desc_from(t0_lo + pn * (kTilePanel >> 4) + kk * 2, kDescHi),
+                   desc_from(((b0_addr + pn * (kBlkPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>,
+                   (pn > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int pn = 0; pn < kPanels; ++pn)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kColDP + 32 * hf, desc_from(t1_lo + pn * (kTilePanel >> 4) + kk * 2, kDescHi),
+                   desc_from(((b1_addr + pn * (kBlkPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>,
+                   (pn > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar_s + hf);
       };
       // gradients of a half: A (P or dS, packed) from TMEM, B the half's rows read MN-major
@@ -404,13 +431,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (kKeys) {
             // dV += P^T dout (block 1), dK += dS^T Q (block 0)
             mma_ts(tmem + kColAcc0, tmem + kColS + 32 * hf + kk * 8, desc_from((b1_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, acc);
+                   kIdescGrad<kFmt, kD>, acc);
             mma_ts(tmem + kColAcc1, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, acc);
+                   kIdescGrad<kFmt, kD>, acc);
           } else {
             // dQ += dS K (block 0)
             mma_ts(tmem + kColAcc0, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
-                   kIdescGrad<kFmt>, acc);
+                   kIdescGrad<kFmt, kD>, acc);
           }
         }
       };
@@ -455,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     float lse2 = 0.f, delta = 0.f;
     if (!kKeys && row_ok) {
       lse2 = P.pb.lse[bhN + pos] * kLog2e;
-      delta = row_dot<kFmt>(static_cast<const uint16_t*>(P.g.dout) + elem,
+      delta = row_dot<kFmt, kD>(static_cast<const uint16_t*>(P.g.dout) + elem,
                             static_cast<const uint16_t*>(P.g.out) + elem);
     }
     const uint64_t sc2 = f32x2(P.scale_log2, P.scale_log2);
@@ -503,12 +530,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         float* dst = kKeys ? (a == 0 ? P.g.dv : P.g.dk) : P.g.dq;
         const float sc = (kKeys && a == 0) ? 1.f : P.scale;
 #pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
+        for (int c0 = 0; c0 < kD; c0 += 32) {
           uint32_t acc[32];
-          LN_TMEM_LD32(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + 32 * hf, acc);
+          LN_TMEM_LD32(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + c0, acc);
           tmem_wait_ld();
           if (row_ok) {
-            float4* d4 = reinterpret_cast<float4*>(dst + elem + 32 * hf);
+            float4* d4 = reinterpret_cast<float4*>(dst + elem + c0);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               atomicAdd(d4 + c, make_float4(__uint_as_float(acc[4 * c]) * sc, __uint_as_float(acc[4 * c + 1]) * sc,
@@ -528,26 +555,27 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // delta_i = <dout_i, out_i> for every row, into [B, H, N]; one thread per row.
-template <int kFmt>
+template <int kFmt, int kD>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const Problem pb, const uint16_t* out, const uint16_t* dout,
                                                         float* delta) {
   const int64_t rows = pb.B * pb.N * pb.H;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t h = i % pb.H, n = (i / pb.H) % pb.N, b = i / (pb.H * pb.N);
-    delta[(b * pb.H + h) * pb.N + n] = row_dot<kFmt>(dout + i * kD, out + i * kD);
+    delta[(b * pb.H + h) * pb.N + n] = row_dot<kFmt, kD>(dout + i * kD, out + i * kD);
   }
 }
 
-// View [B, N, H, 64] (16-bit elements, starting `shift` positions in) as
-// (d, h, c, k, b), position = r k + c, boxes of box_rows consecutive k.
+// View [B, N, H, D] (16-bit elements, starting `shift` positions in) as
+// (d, h, c, k, b), position = r k + c; boxes of one 64-element panel of D by
+// box_rows consecutive k.
 bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem& p, int64_t r, int64_t shift,
             int64_t kcount, int box_rows) {
-  const int64_t es = 2;
-  const char* ptr = static_cast<const char*>(base) + shift * p.H * kD * es;
-  cuuint64_t dims[5] = {(cuuint64_t)kD, (cuuint64_t)p.H, (cuuint64_t)r, (cuuint64_t)kcount, (cuuint64_t)p.B};
-  cuuint64_t strides[4] = {(cuuint64_t)(kD * es), (cuuint64_t)(p.H * kD * es), (cuuint64_t)(r * p.H * kD * es),
-                           (cuuint64_t)(p.N * p.H * kD * es)};
-  cuuint32_t box[5] = {(cuuint32_t)kD, 1, 1, (cuuint32_t)box_rows, 1};
+  const int64_t es = 2, D = p.D;
+  const char* ptr = static_cast<const char*>(base) + shift * p.H * D * es;
+  cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)p.H, (cuuint64_t)r, (cuuint64_t)kcount, (cuuint64_t)p.B};
+  cuuint64_t strides[4] = {(cuuint64_t)(D * es), (cuuint64_t)(p.H * D * es), (cuuint64_t)(r * p.H * D * es),
+                           (cuuint64_t)(p.N * p.H * D * es)};
+  cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapDataType ty =
       p.dtype == LONGNET_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -559,7 +587,8 @@ bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem
 // CTAs and the per-pattern geometry; false when the shape is outside this
 // family.
 bool geometry(const Problem& p, Params* P) {
-  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD || p.qk_norm) return false;
+  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || (p.D != 64 && p.D != 128) || p.qk_norm)
+    return false;
   if (p.n_pat > kMaxPat || p.N > ((int64_t)1 << 30) || p.H > 65535 || p.B > 65535) return false;
   int64_t ctas = 0;
   for (int i = 0; i < p.n_pat; ++i) {
@@ -633,17 +662,22 @@ int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t str
     return LONGNET_ERR_CUDA;
   }
   const bool f16 = p.dtype == LONGNET_DTYPE_F16;
-  auto kern_k = f16 ? bwd_tc_kernel<kFmtF16, true> : bwd_tc_kernel<kFmtBF16, true>;
-  auto kern_q = f16 ? bwd_tc_kernel<kFmtF16, false> : bwd_tc_kernel<kFmtBF16, false>;
-  auto kern_d = f16 ? bwd_delta_kernel<kFmtF16> : bwd_delta_kernel<kFmtBF16>;
-  static bool attr_set[64][2] = {};
-  if (!attr_set[dev][f16]) {
+  const int panels = (int)(p.D / 64);
+  auto kern_k = f16 ? (panels == 1 ? bwd_tc_kernel<kFmtF16, true, 1> : bwd_tc_kernel<kFmtF16, true, 2>)
+                    : (panels == 1 ? bwd_tc_kernel<kFmtBF16, true, 1> : bwd_tc_kernel<kFmtBF16, true, 2>);
+  auto kern_q = f16 ? (panels == 1 ? bwd_tc_kernel<kFmtF16, false, 1> : bwd_tc_kernel<kFmtF16, false, 2>)
+                    : (panels == 1 ? bwd_tc_kernel<kFmtBF16, false, 1> : bwd_tc_kernel<kFmtBF16, false, 2>);
+  auto kern_d = f16 ? (panels == 1 ? bwd_delta_kernel<kFmtF16, 64> : bwd_delta_kernel<kFmtF16, 128>)
+                    : (panels == 1 ? bwd_delta_kernel<kFmtBF16, 64> : bwd_delta_kernel<kFmtBF16, 128>);
+  const int kSmemBytes = panels == 1 ? BL<1>::kSmemBytes : BL<2>::kSmemBytes;
+  static bool attr_set[64][2][2] = {};
+  if (!attr_set[dev][f16][panels - 1]) {
     if (cudaFuncSetAttribute(kern_k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern_q, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
-    attr_set[dev][f16] = true;
+    attr_set[dev][f16][panels - 1] = true;
   }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);

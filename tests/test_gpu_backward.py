@@ -85,6 +85,8 @@ CASES = [
     ("bf16_d32_partial", 1, 700, 2, 32, torch.bfloat16, False, ((128, 1), (300, 2))),
     ("f16_d64_r_not_dividing", 1, 768, 5, 64, torch.float16, True, ((192, 3), (384, 4), (768, 8))),
     ("f16_d128", 1, 256, 2, 128, torch.float16, True, ((64, 1), (256, 2))),
+    ("bf16_d128_lm_like", 1, 1024, 3, 128, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
+    ("bf16_d128_noncausal_partial", 2, 700, 2, 128, torch.bfloat16, False, ((256, 1), (300, 3))),
 ]
 
 
@@ -92,6 +94,7 @@ def _impls(dtype, D):
     out = [("simt", bd.LONGNET_IMPL_SIMT)]
     if dtype != torch.float32 and D == 64:
         out.append(("tiles", bd.LONGNET_IMPL_TILES))
+    if dtype != torch.float32 and D in (64, 128):
         out.append(("tcgen05", bd.LONGNET_IMPL_TCGEN05))
     return out
 
