@@ -13,6 +13,7 @@ from .oracle import (  # noqa: F401
     num_threads,
     qk_normalize_bwd_fp64,
     qk_normalize_fp64,
+    xpos_bwd_fp64,
     xpos_fp64,
 )
 from .brute import dilated_attn_bruteforce  # noqa: F401

@@ -192,18 +192,46 @@ def qk_normalize_bwd_fp64(x, dxhat) -> np.ndarray:
     return np.where(n > 1e-12, a * proj, a * dxhat)
 
 
-def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None, qk_norm=False):
+def xpos_bwd_fp64(g, downscale=False) -> np.ndarray:
+    """Chain rule through xpos_fp64: per element pair the forward is
+    y = s R(n theta_i) x (s the pair's scale, its inverse for keys), a linear
+    map whose transpose is s R(-n theta_i).  Returns the cotangent of x given
+    g, the cotangent of y."""
+    g = _f64(g)
+    B, N, H, D = g.shape
+    n = np.arange(N, dtype=np.float64)[:, None]
+    i = np.arange(D // 2, dtype=np.float64)[None, :]
+    theta = 10000.0 ** (-2.0 * i / D)
+    zeta = (2.0 * i + 0.4 * D) / (1.4 * D)
+    s = zeta ** ((n - (N // 2)) / 512.0)
+    if downscale:
+        s = 1.0 / s
+    cos = (np.cos(n * theta) * s)[None, :, None, :]
+    sin = (np.sin(n * theta) * s)[None, :, None, :]
+    g0, g1 = g[..., 0::2], g[..., 1::2]
+    x = np.empty_like(g)
+    x[..., 0::2] = g0 * cos + g1 * sin
+    x[..., 1::2] = g1 * cos - g0 * sin
+    return x
+
+
+def dilated_attn_bwd_fp64(q, k, v, dout, patterns, causal=True, lib=None, qk_norm=False, xpos=False):
     """Full fp64 backward: the gradients of sum(dout * out) with respect to
     q, k and v, where out is the forward's output.  All tensors [B, N, H, D].
-    qk_norm: the forward normalised q and k rows first (qk_normalize_fp64);
-    the gradients then go back through that normalisation.
+    qk_norm, xpos: the forward normalised q and k rows (qk_normalize_fp64)
+    and then applied XPOS (xpos_fp64) before the scores; the gradients go
+    back through both, in the reverse order.
 
     Returns (dq, dk, dv) as float64 arrays.
     """
-    if qk_norm:
-        qh, kh = qk_normalize_fp64(q), qk_normalize_fp64(k)
+    if qk_norm or xpos:
+        qh, kh = _prologue(q, k, qk_norm, xpos)
         dqh, dkh, dv = dilated_attn_bwd_fp64(qh, kh, v, dout, patterns, causal, lib)
-        return qk_normalize_bwd_fp64(q, dqh), qk_normalize_bwd_fp64(k, dkh), dv
+        if xpos:
+            dqh, dkh = xpos_bwd_fp64(dqh), xpos_bwd_fp64(dkh, downscale=True)
+        if qk_norm:
+            dqh, dkh = qk_normalize_bwd_fp64(q, dqh), qk_normalize_bwd_fp64(k, dkh)
+        return dqh, dkh, dv
     lib = lib or load_library()
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, N, H, D = q.shape

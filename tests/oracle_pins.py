@@ -579,6 +579,44 @@ def check_bwd_qk_norm(lib):
                                            rtol=1e-12)
 
 
+def check_bwd_xpos(lib, xpos_bwd=None):
+    """The backward through XPOS (and qk_norm then XPOS): the adjoint identity
+    <xpos(x), g> = <x, xpos_bwd(g)> for queries and keys (XPOS is linear in x),
+    and central differences of the forward with the options."""
+    xpos_bwd = xpos_bwd or orc.xpos_bwd_fp64
+    B, N, H, D = 1, 40, 2, 4
+    x, g = _rand((B, N, H, D), 141), _rand((B, N, H, D), 142)
+    for down in (False, True):
+        lhs = float((orc.xpos_fp64(x, downscale=down) * g).sum())
+        rhs = float((x * xpos_bwd(g, downscale=down)).sum())
+        assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs)), (down, lhs, rhs)
+    pats = [(10, 1), (20, 2), (40, 4)]
+    q, k, v, do = (_rand((B, N, H, D), s) for s in (143, 144, 145, 146))
+    saved = orc.xpos_bwd_fp64
+    orc.xpos_bwd_fp64 = xpos_bwd
+    try:
+        for qk_norm in (False, True):
+            for causal in (True, False):
+                grads = orc.dilated_attn_bwd_fp64(q, k, v, do, pats, causal=causal, lib=lib, qk_norm=qk_norm,
+                                                  xpos=True)
+                eps = 1e-6
+                gen = np.random.default_rng(147)
+                for which in range(3):
+                    for _ in range(4):
+                        idx = (0, int(gen.integers(N)), int(gen.integers(H)), int(gen.integers(D)))
+                        vals = []
+                        for sgn in (1.0, -1.0):
+                            args = [q.copy(), k.copy(), v.copy()]
+                            args[which][idx] += sgn * eps
+                            o, _ = orc.dilated_attn_fp64(*args, pats, causal=causal, lib=lib, qk_norm=qk_norm,
+                                                         xpos=True)
+                            vals.append(float((o * do).sum()))
+                        fd = (vals[0] - vals[1]) / (2 * eps)
+                        assert abs(fd - grads[which][idx]) < 1e-6 * max(1.0, abs(fd)), (qk_norm, causal, which, idx)
+    finally:
+        orc.xpos_bwd_fp64 = saved
+
+
 ALL_CHECKS = [
     check_rows_function_direct,
     check_qk_norm,
@@ -600,4 +638,5 @@ ALL_CHECKS = [
     check_bwd_rows_function,
     check_bwd_closed_form,
     check_bwd_qk_norm,
+    check_bwd_xpos,
 ]

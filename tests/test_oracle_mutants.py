@@ -157,3 +157,36 @@ def test_xpos_pins_catch_mutant(oracle_lib, name):
 
 def test_xpos_unmutated_variant_passes(oracle_lib):
     pins.check_xpos(oracle_lib, xpos=_xpos_variant())
+
+
+def _xpos_bwd_variant(sin_sign=1.0, invert_keys=True):
+    """xpos_bwd with one planted mistake: the rotation's direction, or the key scale."""
+    import numpy as np
+
+    from oracle.oracle import _f64
+
+    def xb(g, downscale=False):
+        g = _f64(g)
+        B, N, H, D = g.shape
+        n = np.arange(N, dtype=np.float64)[:, None]
+        i = np.arange(D // 2, dtype=np.float64)[None, :]
+        theta = 10000.0 ** (-2.0 * i / D)
+        zeta = (2.0 * i + 0.4 * D) / (1.4 * D)
+        s = zeta ** ((n - N // 2) / 512.0)
+        if downscale and invert_keys:
+            s = 1.0 / s
+        cos = (np.cos(n * theta) * s)[None, :, None, :]
+        sin = (sin_sign * np.sin(n * theta) * s)[None, :, None, :]
+        g0, g1 = g[..., 0::2], g[..., 1::2]
+        x = np.empty_like(g)
+        x[..., 0::2] = g0 * cos + g1 * sin
+        x[..., 1::2] = g1 * cos - g0 * sin
+        return x
+
+    return xb
+
+
+@pytest.mark.parametrize("kw", [dict(sin_sign=-1.0), dict(invert_keys=False)], ids=["rotation_sign", "key_scale"])
+def test_xpos_backward_pins_catch_mutant(oracle_lib, kw):
+    with pytest.raises(AssertionError):
+        pins.check_bwd_xpos(oracle_lib, xpos_bwd=_xpos_bwd_variant(**kw))
