@@ -333,6 +333,31 @@ int longnet_dilated_attn_bwd(const void* q, const void* k, const void* v,
                              longnet_stream_t stream);
 
 /*
+ * longnet_dilated_attn_bwd_ws — the backward of longnet_dilated_attn_fwd_ws:
+ * the gradients of sum(dout * out) with respect to the ORIGINAL q, k, v when
+ * the forward applied the input-side options (flags: LONGNET_FLAG_QK_NORM,
+ * LONGNET_FLAG_XPOS, or both; out and lse are that forward's results).  The
+ * same prologue pass encodes q and k into the caller's workspace, the
+ * attention's backward runs on the encoded rows (any family; AUTO picks as
+ * for the plain backward, tcgen05 included), and a last pass takes dq and
+ * dk back through XPOS (per element pair the transpose s R(-n theta_i), 1/s
+ * for keys) and then the norm (a (g - xhat <xhat, g>)), in place.
+ *   workspace, workspace_bytes: as for longnet_dilated_attn_fwd_ws (the
+ *     encoded q and k are written there; contents on entry do not matter).
+ *   flags = 0: the call is longnet_dilated_attn_bwd with flags 0 (workspace
+ *     unused, may be null).  Other arguments, results and errors as
+ *     longnet_dilated_attn_bwd and longnet_dilated_attn_fwd_ws.
+ */
+int longnet_dilated_attn_bwd_ws(const void* q, const void* k, const void* v,
+                                const void* out, const float* lse, const void* dout,
+                                float* dq, float* dk, float* dv,
+                                int64_t B, int64_t N, int64_t H, int64_t D,
+                                int n_pat, const int64_t* w, const int64_t* r,
+                                int causal, int dtype, int flags, int impl,
+                                void* workspace, int64_t workspace_bytes,
+                                longnet_stream_t stream);
+
+/*
  * longnet_select_impl — which family AUTO would run for these arguments
  * with lse requested (a longnet_impl >= 1), or a negative longnet_status
  * when the arguments are invalid.  Host-only; touches no device.  (Without

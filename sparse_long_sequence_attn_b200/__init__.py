@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     dilated_attn_bwd,
     load_library,
     longnet_dilated_attn_bwd,
+    longnet_dilated_attn_bwd_ws,
     longnet_dilated_attn_fwd,
     longnet_dilated_attn_fwd_noalloc,
     longnet_dilated_attn_fwd_part,

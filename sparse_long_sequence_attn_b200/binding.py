@@ -74,6 +74,10 @@ SIGNATURES = {
                                                 _i64, _i64, _i64, _i64, ctypes.c_int, _i64p,
                                                 _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                 ctypes.c_int, _vp]),
+    "longnet_dilated_attn_bwd_ws": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                   _i64, _i64, _i64, _i64, ctypes.c_int, _i64p,
+                                                   _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, _vp, _i64, _vp]),
     "longnet_select_impl": (ctypes.c_int, [_i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
                                            ctypes.c_int, ctypes.c_int]),
     "longnet_last_device_status": (ctypes.c_int, [_vp]),
@@ -315,16 +319,15 @@ def dilated_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  impl: int = LONGNET_IMPL_AUTO, want_lse: bool = True, stream=None,
                  qk_norm: bool = False, xpos: bool = False):
     """Allocate out (and lse) with torch and run the forward.  Returns (out,
-    lse).  xpos (and qk_norm with it) goes through the prologue pass, with a
-    workspace allocated by torch; qk_norm alone is applied inside the
-    attention kernel."""
+    lse).  The options (qk_norm, xpos) go through the prologue pass, with a
+    workspace allocated by torch, so every family (tcgen05 included) runs."""
     B, N, H, D = q.shape
     out = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if want_lse else None
-    if xpos:
-        ws = torch.empty(longnet_fwd_workspace_bytes(B, N, H, D, q.dtype, qk_norm, True),
+    if qk_norm or xpos:
+        ws = torch.empty(longnet_fwd_workspace_bytes(B, N, H, D, q.dtype, qk_norm, xpos),
                          dtype=torch.uint8, device=q.device)
-        longnet_dilated_attn_fwd_ws(q, k, v, out, lse, patterns, causal, ws, impl, stream, qk_norm, True)
+        longnet_dilated_attn_fwd_ws(q, k, v, out, lse, patterns, causal, ws, impl, stream, qk_norm, xpos)
     else:
         longnet_dilated_attn_fwd(q, k, v, out, lse, patterns, causal, impl, stream, qk_norm)
     return out, lse
@@ -362,12 +365,55 @@ def longnet_dilated_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise LongNetError(rc, "longnet_dilated_attn_bwd")
 
 
+def longnet_dilated_attn_bwd_ws(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                                dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
+                                patterns: Sequence[Tuple[int, int]], causal: bool,
+                                workspace: torch.Tensor | None, impl: int = LONGNET_IMPL_AUTO, stream=None,
+                                qk_norm: bool = False, xpos: bool = False) -> None:
+    """The backward of longnet_dilated_attn_fwd_ws (out and lse from it, with
+    the same options): the prologue into `workspace`, the attention's backward
+    on the encoded rows, then dq and dk taken back through XPOS and the norm.
+    Tensors as in longnet_dilated_attn_bwd.  Raises LongNetError on a non-zero
+    status."""
+    lib = load_library()
+    B, N, H, D = q.shape
+    for t in (q, k, v, out, dout):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out, dout must be contiguous CUDA tensors of one shape and dtype")
+    for t in (dq, dk, dv):
+        if not (t.is_cuda and t.is_contiguous()) or tuple(t.shape) != (B, N, H, D) or t.dtype != torch.float32:
+            raise ValueError("dq, dk, dv must be contiguous fp32 CUDA tensors [B, N, H, D]")
+    if not (lse.is_cuda and lse.is_contiguous() and lse.dtype == torch.float32
+            and tuple(lse.shape) == (B, H, N)):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, H, N]")
+    if workspace is not None and not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_ptr = None if workspace is None else workspace.data_ptr()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_bwd_ws(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, D, n, w, r, int(bool(causal)),
+        _dtype_code(q), _flags(qk_norm, xpos), int(impl), ws_ptr, ws_bytes, _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_bwd_ws")
+
+
 def dilated_attn_bwd(q, k, v, out, lse, dout, patterns, causal: bool = True,
-                     impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False):
-    """Allocate fp32 dq, dk, dv with torch and run the backward.  Returns (dq, dk, dv)."""
+                     impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False, xpos: bool = False):
+    """Allocate fp32 dq, dk, dv (and, with options, the workspace) with torch
+    and run the backward matching dilated_attn.  Returns (dq, dk, dv)."""
     dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
-    longnet_dilated_attn_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal,
-                             impl, stream, qk_norm)
+    if qk_norm or xpos:
+        B, N, H, D = q.shape
+        ws = torch.empty(longnet_fwd_workspace_bytes(B, N, H, D, q.dtype, qk_norm, xpos), dtype=torch.uint8,
+                         device=q.device)
+        longnet_dilated_attn_bwd_ws(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal, ws,
+                                    impl, stream, qk_norm, xpos)
+    else:
+        longnet_dilated_attn_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, patterns, causal, impl,
+                                 stream)
     return dq, dk, dv
 
 
@@ -375,24 +421,24 @@ class DilatedAttnFunction(torch.autograd.Function):
     """The forward and backward entry points as one torch autograd op."""
 
     @staticmethod
-    def forward(ctx, q, k, v, patterns, causal, qk_norm=False):
-        out, lse = dilated_attn(q, k, v, patterns, causal, qk_norm=qk_norm)
+    def forward(ctx, q, k, v, patterns, causal, qk_norm=False, xpos=False):
+        out, lse = dilated_attn(q, k, v, patterns, causal, qk_norm=qk_norm, xpos=xpos)
         ctx.save_for_backward(q, k, v, out, lse)
-        ctx.patterns, ctx.causal, ctx.qk_norm = list(patterns), causal, qk_norm
+        ctx.patterns, ctx.causal, ctx.qk_norm, ctx.xpos = list(patterns), causal, qk_norm, xpos
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
         dq, dk, dv = dilated_attn_bwd(q, k, v, out, lse, dout.to(q.dtype), ctx.patterns, ctx.causal,
-                                      qk_norm=ctx.qk_norm)
+                                      qk_norm=ctx.qk_norm, xpos=ctx.xpos)
         # autograd wants each gradient in its input's dtype
-        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None, None, None
 
 
-def dilated_attention(q, k, v, patterns, causal: bool = True, qk_norm: bool = False):
+def dilated_attention(q, k, v, patterns, causal: bool = True, qk_norm: bool = False, xpos: bool = False):
     """Differentiable forward: out [B, N, H, D], gradients through the backward."""
-    return DilatedAttnFunction.apply(q, k, v, patterns, causal, qk_norm)
+    return DilatedAttnFunction.apply(q, k, v, patterns, causal, qk_norm, xpos)
 
 
 def longnet_select_impl(B: int, N: int, H: int, D: int, patterns, causal: bool, dtype) -> int:

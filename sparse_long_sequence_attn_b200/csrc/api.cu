@@ -395,6 +395,60 @@ extern "C" int longnet_dilated_attn_bwd(const void* q, const void* k, const void
   return launch_backward(pb, g, impl, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" int longnet_dilated_attn_bwd_ws(const void* q, const void* k, const void* v, const void* out,
+                                           const float* lse, const void* dout, float* dq, float* dk,
+                                           float* dv, int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
+                                           const int64_t* w, const int64_t* r, int causal, int dtype,
+                                           int flags, int impl, void* workspace, int64_t workspace_bytes,
+                                           longnet_stream_t stream) {
+  if (flags & ~(LONGNET_FLAG_QK_NORM | LONGNET_FLAG_XPOS)) return LONGNET_ERR_INVALID_ARG;
+  if (flags == 0)
+    return longnet_dilated_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, N, H, D, n_pat, w, r, causal,
+                                    dtype, 0, impl, stream);
+  if (impl != LONGNET_IMPL_AUTO && impl != LONGNET_IMPL_SIMT && impl != LONGNET_IMPL_TILES &&
+      impl != LONGNET_IMPL_TCGEN05)
+    return LONGNET_ERR_INVALID_ARG;
+  if (!out || !lse || !dout || !dq || !dk || !dv) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  int rc = check_args(q, k, v, dq, const_cast<float*>(lse), B, N, H, D, n_pat, w, r, causal, dtype, &pb);
+  if (rc) return rc;
+  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+    return LONGNET_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < prologue_workspace_bytes(B, N, H, D, dtype)) return LONGNET_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return LONGNET_ERR_MISALIGNED;
+  pb.qk_norm = (flags & LONGNET_FLAG_QK_NORM) ? 1 : 0;
+  const int xpos = (flags & LONGNET_FLAG_XPOS) ? 1 : 0;
+  if (!prologue_supports(pb, xpos)) return LONGNET_ERR_UNSUPPORTED;
+  // the attention's backward runs on the encoded rows, without options
+  Problem enc = pb;
+  char* qo = static_cast<char*>(workspace);
+  char* ko = qo + prologue_workspace_bytes(B, N, H, D, dtype) / 2;
+  enc.q = qo;
+  enc.k = ko;
+  enc.qk_norm = 0;
+  if (impl == LONGNET_IMPL_AUTO && !backward_supports(enc) && !tile_backward_supports(enc))
+    return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_SIMT && !backward_supports(enc)) return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_TILES && !tile_backward_supports(enc)) return LONGNET_ERR_UNSUPPORTED;
+  if (impl == LONGNET_IMPL_TCGEN05 && !tcgen05_backward_supports(enc)) return LONGNET_ERR_UNSUPPORTED;
+  int dev = 0;
+  rc = current_device_state(&dev, &pb.status);
+  if (rc) return rc;
+  enc.status = pb.status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  rc = launch_prologue(pb, xpos, qo, ko, s);
+  if (rc) return rc;
+  BwdArgs g;
+  g.out = out;
+  g.dout = dout;
+  g.dq = dq;
+  g.dk = dk;
+  g.dv = dv;
+  rc = launch_backward(enc, g, impl, s);
+  if (rc) return rc;
+  return launch_prologue_bwd(pb, xpos, dq, dk, s);
+}
+
 extern "C" int longnet_select_impl(int64_t B, int64_t N, int64_t H, int64_t D, int n_pat,
                                    const int64_t* w, const int64_t* r, int causal, int dtype) {
   // Stand-in pointers: only their alignment (and, for lse, presence) is

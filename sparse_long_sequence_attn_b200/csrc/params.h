@@ -58,6 +58,9 @@ int launch_backward(const Problem& p, const BwdArgs& g, int impl, cudaStream_t s
 int64_t prologue_workspace_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int dtype);
 bool prologue_supports(const Problem& p, int xpos);
 int launch_prologue(const Problem& p, int xpos, void* qo, void* ko, cudaStream_t stream);
+// Its backward: the fp32 gradients of the encoded q and k rows, in place in
+// dq and dk, become those of the original rows (p.q, p.k).
+int launch_prologue_bwd(const Problem& p, int xpos, float* dq, float* dk, cudaStream_t stream);
 
 // Row moves of the sequence-parallel exchange: dst[dst_idx[i]] = src[src_idx[i]]
 // for i < n (a null index array is the identity), rows of row_bytes (a

@@ -174,6 +174,87 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// The backward of the pass: the fp32 gradient g of the encoded rows (in
+// place, [B, N, H, D]) becomes the gradient of the original rows x: first
+// back through XPOS (per pair the transpose of s R(n theta_i): s R(-n theta_i),
+// 1/s for keys), then through the norm, a (g - xhat <xhat, g>) with
+// a = 1 / max(|x|, 1e-12) and xhat = a x (a g where |x| <= 1e-12).  One
+// thread group of TPR = D / 8 threads per row, 8 elements each.
+template <typename T, int TPR>
+__global__ void __launch_bounds__(kThreads)
+    prologue_bwd_kernel(const T* __restrict__ x, float* __restrict__ g, int64_t rows, int N, int H, int center,
+                        int qk_norm, int xpos, int is_k, const XposTable tab) {
+  constexpr int kD = TPR * 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = rows * TPR;
+  const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+  for (int64_t base = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * 32; base < total;
+       base += warps * 32) {
+    const int64_t t = base + lane;
+    const bool active = t < total;
+    const int chunk = (int)(t % TPR);
+    const int64_t row = active ? t / TPR : 0;
+    float gv[8];
+    if (active) {
+      const float4 a = reinterpret_cast<const float4*>(g + row * kD + chunk * 8)[0];
+      const float4 b2 = reinterpret_cast<const float4*>(g + row * kD + chunk * 8)[1];
+      gv[0] = a.x; gv[1] = a.y; gv[2] = a.z; gv[3] = a.w;
+      gv[4] = b2.x; gv[5] = b2.y; gv[6] = b2.z; gv[7] = b2.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gv[j] = 0.f;
+    }
+    if (xpos && active) {
+      const int n = (int)((row / H) % N);
+      const float rel = (float)(n - center) * (1.f / 512.f);
+      const double two_pi = 6.283185307179586476925286766559;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = chunk * 4 + j;
+        double a = (double)n * tab.theta[i];
+        a -= two_pi * rint(a * (1.0 / two_pi));
+        float sn, cs;
+        sincosf((float)a, &sn, &cs);
+        const float e = tab.log2zeta[i] * rel;
+        const float sc = exp2f(is_k ? -e : e);
+        const float g0 = gv[2 * j], g1 = gv[2 * j + 1];
+        gv[2 * j] = (g0 * cs + g1 * sn) * sc;
+        gv[2 * j + 1] = (g1 * cs - g0 * sn) * sc;
+      }
+    }
+    if (qk_norm) {
+      float xv[8];
+      if (active) {
+        load8(x + row * kD + chunk * 8, xv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xv[j] = 0.f;
+      }
+      float ss = 0.f, dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ss = fmaf(xv[j], xv[j], ss);
+        dot = fmaf(xv[j], gv[j], dot);
+      }
+#pragma unroll
+      for (int m = 1; m < TPR; m <<= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        dot += __shfl_xor_sync(0xffffffffu, dot, m);
+      }
+      const float nrm = sqrtf(ss);
+      const float a = 1.f / fmaxf(nrm, 1e-12f);
+      // <xhat, g> = a <x, g>; g - xhat <xhat, g> = g - x a^2 <x, g>
+      const float c = nrm > 1e-12f ? a * a * dot : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gv[j] = a * (gv[j] - xv[j] * c);
+    }
+    if (active) {
+      reinterpret_cast<float4*>(g + row * kD + chunk * 8)[0] = make_float4(gv[0], gv[1], gv[2], gv[3]);
+      reinterpret_cast<float4*>(g + row * kD + chunk * 8)[1] = make_float4(gv[4], gv[5], gv[6], gv[7]);
+    }
+  }
+}
+
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 int64_t elem_bytes(int dtype) { return dtype == LONGNET_DTYPE_F32 ? 4 : 2; }
@@ -208,7 +289,61 @@ int launch_typed(const Problem& p, void* qo, void* ko, const XposTable& tab, int
   return cudaGetLastError() == cudaSuccess ? LONGNET_OK : LONGNET_ERR_CUDA;
 }
 
+template <typename T>
+int launch_bwd_typed(const Problem& p, int xpos, float* dq, float* dk, const XposTable& tab, cudaStream_t s) {
+  const int64_t rows = p.B * p.N * p.H;
+  const int tpr = (int)(p.D / 8);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  int64_t blocks = (rows * tpr + kThreads - 1) / kThreads;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  const int center = (int)(p.N / 2);
+  for (int which = 0; which < 2; ++which) {
+    const T* x = static_cast<const T*>(which ? p.k : p.q);
+    float* g = which ? dk : dq;
+#define LN_PROLOGUE_BWD(TPRV)                                                                               \
+  prologue_bwd_kernel<T, TPRV><<<(unsigned)blocks, kThreads, 0, s>>>(x, g, rows, (int)p.N, (int)p.H, center, \
+                                                                   p.qk_norm, xpos, which, tab)
+    switch (tpr) {
+      case 2: LN_PROLOGUE_BWD(2); break;
+      case 4: LN_PROLOGUE_BWD(4); break;
+      case 8: LN_PROLOGUE_BWD(8); break;
+      case 16: LN_PROLOGUE_BWD(16); break;
+      default: return LONGNET_ERR_UNSUPPORTED;
+    }
+#undef LN_PROLOGUE_BWD
+    if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
+  }
+  return LONGNET_OK;
+}
+
+XposTable make_table(int64_t D) {
+  XposTable tab;
+  const int n_pairs = (int)(D / 2);
+  for (int i = 0; i < kMaxPairs; ++i) {
+    if (i < n_pairs) {
+      tab.theta[i] = pow(10000.0, -2.0 * i / (double)D);
+      tab.log2zeta[i] = (float)log2((2.0 * i + 0.4 * (double)D) / (1.4 * (double)D));
+    } else {
+      tab.theta[i] = 0.0;
+      tab.log2zeta[i] = 0.f;
+    }
+  }
+  return tab;
+}
+
 }  // namespace
+
+int launch_prologue_bwd(const Problem& p, int xpos, float* dq, float* dk, cudaStream_t s) {
+  const XposTable tab = make_table(p.D);
+  switch (p.dtype) {
+    case LONGNET_DTYPE_F32: return launch_bwd_typed<float>(p, xpos, dq, dk, tab, s);
+    case LONGNET_DTYPE_BF16: return launch_bwd_typed<__nv_bfloat16>(p, xpos, dq, dk, tab, s);
+    case LONGNET_DTYPE_F16: return launch_bwd_typed<__half>(p, xpos, dq, dk, tab, s);
+    default: return LONGNET_ERR_INVALID_ARG;
+  }
+}
 
 int64_t prologue_workspace_bytes(int64_t B, int64_t N, int64_t H, int64_t D, int dtype) {
   return 2 * round_up(B * N * H * D * elem_bytes(dtype), 256);
@@ -234,17 +369,7 @@ bool prologue_supports(const Problem& p, int xpos) {
 }
 
 int launch_prologue(const Problem& p, int xpos, void* qo, void* ko, cudaStream_t s) {
-  XposTable tab;
-  const int n_pairs = (int)(p.D / 2);
-  for (int i = 0; i < kMaxPairs; ++i) {
-    if (i < n_pairs) {
-      tab.theta[i] = pow(10000.0, -2.0 * i / (double)p.D);
-      tab.log2zeta[i] = (float)log2((2.0 * i + 0.4 * (double)p.D) / (1.4 * (double)p.D));
-    } else {
-      tab.theta[i] = 0.0;
-      tab.log2zeta[i] = 0.f;
-    }
-  }
+  const XposTable tab = make_table(p.D);
   switch (p.dtype) {
     case LONGNET_DTYPE_F32: return launch_typed<float>(p, qo, ko, tab, xpos, s);
     case LONGNET_DTYPE_BF16: return launch_typed<__nv_bfloat16>(p, qo, ko, tab, xpos, s);

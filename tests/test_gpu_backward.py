@@ -256,3 +256,66 @@ def test_backward_qk_norm(case, impl_name, impl):
     check(got, ref, dtype, f"{name} ({impl_name})")
     bound = 10 * TOL_GRAD[dtype] * max(1.0, float(np.abs(zero[1]).max()))
     assert np.abs(zero[0] - zero[1]).max() <= bound, "zero key row (1/eps branch)"
+
+
+# The backward of the workspace forward (longnet_dilated_attn_fwd_ws): the
+# options qk_norm and XPOS on the encoded rows, gradients taken back through
+# them, against the oracle's backward with the same options.
+WS_CASES = [
+    ("ws_bf16_d64_lm_like", 1, 1024, 3, 64, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
+    ("ws_f16_d64_noncausal", 2, 512, 2, 64, torch.float16, False, ((128, 1), (512, 4))),
+    ("ws_bf16_d128", 1, 1024, 2, 128, torch.bfloat16, True, ((256, 1), (1024, 2))),
+    ("ws_fp32_d32_partial", 1, 300, 2, 32, torch.float32, True, ((64, 1), (128, 3))),
+]
+WS_OPTIONS = {"qk_norm": (True, False), "xpos": (False, True), "both": (True, True)}
+
+
+@pytest.mark.parametrize("case", WS_CASES, ids=[c[0] for c in WS_CASES])
+@pytest.mark.parametrize("opt", sorted(WS_OPTIONS))
+@pytest.mark.parametrize("impl_name", ["auto", "tcgen05", "tiles", "simt"])
+def test_backward_through_the_prologue(case, opt, impl_name):
+    name, B, N, H, D, dtype, causal, pats = case
+    qk_norm, xpos = WS_OPTIONS[opt]
+    impl = {"auto": bd.LONGNET_IMPL_AUTO, "tcgen05": bd.LONGNET_IMPL_TCGEN05, "tiles": bd.LONGNET_IMPL_TILES,
+            "simt": bd.LONGNET_IMPL_SIMT}[impl_name]
+    seed = zlib.crc32((name + opt).encode()) % 100000
+    q, k, v = wl.random_inputs(B, N, H, D, dtype, seed=seed, scale=3.0 if qk_norm else 1.0)
+    dout = wl.random_cotangent(B, N, H, D, dtype, seed=seed)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (x.to(dev).contiguous() for x in (q, k, v, dout))
+    out, lse = bd.dilated_attn(qd, kd, vd, pats, causal, qk_norm=qk_norm, xpos=xpos)
+    n = q.numel()
+    G = gh.GUARD
+    bufs = [torch.full((n + 2 * G,), float("nan"), dtype=torch.float32, device=dev) for _ in range(3)]
+    views = [b[G:G + n].view(q.shape) for b in bufs]
+    ws = torch.empty(bd.longnet_fwd_workspace_bytes(B, N, H, D, dtype, qk_norm, xpos), dtype=torch.uint8,
+                     device=dev)
+    try:
+        bd.longnet_dilated_attn_bwd_ws(qd, kd, vd, out, lse, dod, *views, pats, causal, ws, impl,
+                                       qk_norm=qk_norm, xpos=xpos)
+    except bd.LongNetError as e:
+        if e.code == bd.LONGNET_ERR_UNSUPPORTED:
+            pytest.skip("the family does not take this case")
+        raise
+    assert bd.longnet_last_device_status() == 0
+    for b in bufs:
+        assert torch.isnan(b[:G]).all() and torch.isnan(b[-G:]).all(), "write outside a gradient"
+    got = [x.double().cpu().numpy() for x in views]
+    ref = oracle.dilated_attn_bwd_fp64(q, k, v, dout, pats, causal, qk_norm=qk_norm, xpos=xpos)
+    check(got, ref, dtype, f"{name}/{opt} ({impl_name})")
+
+
+def test_autograd_with_xpos_matches_direct_calls():
+    B, N, H, D = 1, 1024, 2, 64
+    pats = ((256, 1), (1024, 4))
+    q, k, v = (x.cuda().requires_grad_(True) for x in wl.random_inputs(B, N, H, D, torch.bfloat16, seed=23))
+    dout = wl.random_cotangent(B, N, H, D, torch.bfloat16, seed=23).cuda()
+    out = bd.dilated_attention(q, k, v, pats, True, qk_norm=True, xpos=True)
+    (out.float() * dout.float()).sum().backward()
+    with torch.no_grad():
+        o2, l2 = bd.dilated_attn(q.detach(), k.detach(), v.detach(), pats, True, qk_norm=True, xpos=True)
+        dq, dk, dv = bd.dilated_attn_bwd(q.detach(), k.detach(), v.detach(), o2, l2, dout, pats, True,
+                                         qk_norm=True, xpos=True)
+    assert torch.equal(out.detach(), o2)
+    for a, b in ((q.grad, dq), (k.grad, dk), (v.grad, dv)):
+        assert (a.float() - b.to(torch.bfloat16).float()).abs().max() <= 1e-2 * max(1.0, b.abs().max().item())
