@@ -30,6 +30,10 @@
 //    format, and at the end the merge into out and lse.
 //  * TMEM: two 64-column score buffers and a D-column O: 256 columns, two
 //    CTAs per SM.
+//  * The pattern launches overlap: each is a programmatic dependent launch,
+//    whose CTAs compute their attention while the previous launch finishes
+//    and wait for it (griddepcontrol.wait) only before the merge, so a
+//    launch's last, longest CTAs do not leave the GPU idle.
 //  * Every wait is bounded; on a timeout the kernel records the status word,
 //    stops issuing, drains what it issued and returns.
 #include <cuda.h>
@@ -133,6 +137,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the next pattern's launch may start as soon as every CTA of this one has:
+  // its attention reads only q, k and v, and its merge waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // CTA -> (batch, head of the part, segment, tile): tiles fastest, longest first
   int64_t rem = blockIdx.x;
   const int tile = P.tiles - 1 - (int)(rem % P.tiles);
@@ -368,6 +375,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(bar_p + (j & 1));
     }
     if (ok) ok = wt.wait_warp(bar_of, 0);
+    // out and lse as the previous launch (the init pass or the previous
+    // pattern) left them: that grid has completed and its writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (ok) {
       tc_fence_after();
       const int64_t pos = (int64_t)first + (int64_t)P.r * (tr < m ? tr : t0);
@@ -421,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // out = 0, lse = -inf over the computed part (rows no pattern keeps keep them).
 template <int kD>
 __global__ void __launch_bounds__(256) pp_init_kernel(const Problem pb) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t Nr = pb.q1 - pb.q0, Hr = pb.h1 - pb.h0;
   const int64_t rows = pb.B * Nr * Hr;
   constexpr int kChunks = kD * 2 / 16;  // 16-byte chunks per row
@@ -505,8 +516,23 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
         if (!encode(enc, &maps.m[sh][t], bases[t], pb, P.r, sh ? P.tail : 0, P.kfull, t == 0 ? kTile : kBlk))
           return LONGNET_ERR_CUDA;
     const int64_t ctas = pb.B * (pb.h1 - pb.h0) * (int64_t)P.n_seg * P.tiles;
-    pp_fwd_kernel<kFmt, kPanels><<<(unsigned)ctas, kThreads, L::kSmem, stream>>>(P, maps);
-    if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
+    // programmatic dependent launch: the kernel's CTAs may start while the
+    // previous launch on the stream is finishing; each waits for it
+    // (griddepcontrol.wait) before it reads or writes out and lse
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, pp_fwd_kernel<kFmt, kPanels>, P, maps) != cudaSuccess) {
+      cudaGetLastError();
+      return LONGNET_ERR_CUDA;
+    }
   }
   return LONGNET_OK;
 }
