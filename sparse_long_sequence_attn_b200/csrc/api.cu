@@ -110,6 +110,9 @@ bool simt_supports(const Problem& p) { return p.D == 16 || p.D == 32 || p.D == 6
 
 int choose_impl(const Problem& p) {
   if (smallseg_supports(p)) return LONGNET_IMPL_SMALLSEG;
+  // The fused family first: the per-pattern one is as fast at 32K and faster
+  // on longer sequences, but rounds out to the input format after every
+  // pattern's merge, which on six patterns exceeds the bf16 error bound.
   if (tcgen05_supports(p)) return LONGNET_IMPL_TCGEN05;
   if (perpattern_supports(p)) return LONGNET_IMPL_PATTERNS;
   if (simt_supports(p)) return LONGNET_IMPL_SIMT;

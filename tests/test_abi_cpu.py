@@ -100,8 +100,9 @@ def test_select_impl_host_logic():
     seven = tuple((256 * (i + 1), i + 1) for i in range(7))
     assert bd.longnet_select_impl(1, 4096, 4, 64, seven, True, bf16) == bd.LONGNET_IMPL_PATTERNS
     assert bd.longnet_select_impl(1, 256, 2, 16, ((64, 0),), True, f32) == bd.LONGNET_ERR_INVALID_ARG
+    # the fused family takes 16-bit D = 64 shapes with up to six patterns
     impl = bd.longnet_select_impl(1, 32768, 12, 64, ((2048, 1), (4096, 2)), True, bf16)
-    assert impl in (bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_TCGEN05)
+    assert impl == bd.LONGNET_IMPL_TCGEN05
 
 
 def _call_bwd(lib, B=1, N=64, H=2, D=16, pats=((16, 1),), causal=1, dtype=0, flags=0,

@@ -201,16 +201,19 @@ def test_named_tiny_workload_fp32():
     assert err <= 1e-4
 
 
-@pytest.mark.parametrize("name", ["lm", "long32k", "smallseg"])
-def test_named_workloads_every_element(name):
+@pytest.mark.parametrize("name,impl_name", [("lm", "auto"), ("long32k", "auto"), ("smallseg", "auto"),
+                                             ("lm", "patterns"), ("long32k", "patterns")])
+def test_named_workloads_every_element(name, impl_name):
     """Full-size workloads in the launch configuration the benchmark times
-    (AUTO), every element of out and lse against the full fp64 oracle."""
+    (AUTO), and on the per-pattern family, every element of out and lse
+    against the full fp64 oracle."""
     w = wl.WORKLOADS[name]
     q, k, v = wl.make_inputs(w)
-    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, bd.LONGNET_IMPL_AUTO)
+    impl = bd.LONGNET_IMPL_AUTO if impl_name == "auto" else IMPLS[impl_name]
+    o, l = gh.run_cuda(q, k, v, w.patterns, w.causal, impl)
     assert gh.lse_is_finite_everywhere(l)  # every row is kept by an r = 1 pattern
-    err = gh.compare_full(o, l, q, k, v, w.patterns, w.causal, torch.bfloat16, label=name)
-    print(f"{name}: max|out - oracle| = {err:.3e} over {o.size} elements")
+    err = gh.compare_full(o, l, q, k, v, w.patterns, w.causal, torch.bfloat16, label=f"{name}/{impl_name}")
+    print(f"{name}/{impl_name}: max|out - oracle| = {err:.3e} over {o.size} elements")
 
 
 @pytest.mark.parametrize("N", wl.SWEEP_NS)
@@ -229,8 +232,9 @@ def test_sweep_sampled_rows(N):
     print(f"sweep{N}: max|out - oracle| = {err:.3e} over {len(rows)} rows")
 
 
+@pytest.mark.parametrize("impl_name", ["auto", "patterns"])
 @pytest.mark.parametrize("causal", [True, False])
-def test_partial_last_segments_full_size(causal):
+def test_partial_last_segments_full_size(causal, impl_name):
     """The 32K-token shape 64 positions short, so every pattern's last segment
     is cut by the sequence's end (and the longest segment exceeds it), in the
     benchmark's launch configuration (AUTO): sampled rows, including every
@@ -238,15 +242,14 @@ def test_partial_last_segments_full_size(causal):
     positions, against the oracle."""
     w = wl.WORKLOADS["long32k"]
     N = w.N - 64
-    assert bd.longnet_select_impl(w.B, N, w.H, w.D, w.patterns, causal, torch.bfloat16) == \
-        bd.LONGNET_IMPL_TCGEN05
     q, k, v = wl.make_inputs(w, N=N)
-    o, l = gh.run_cuda(q, k, v, w.patterns, causal, bd.LONGNET_IMPL_AUTO)
+    impl = bd.LONGNET_IMPL_AUTO if impl_name == "auto" else IMPLS[impl_name]
+    o, l = gh.run_cuda(q, k, v, w.patterns, causal, impl)
     rows = gh.sample_rows(w.B, N, w.H, w.patterns, n_random=1000, seed=17, boundary=4096)
     tail = np.array([(0, x, h) for x in range(N - 2048, N) for h in range(w.H)], dtype=np.int64)
     rows = np.unique(np.concatenate([rows, tail]), axis=0)
     err = gh.compare_rows(o, l, q, k, v, w.patterns, causal, torch.bfloat16, rows, label=f"long32k-64/{causal}")
-    print(f"long32k-64 causal={causal}: max|out - oracle| = {err:.3e} over {len(rows)} rows")
+    print(f"long32k-64 causal={causal} {impl_name}: max|out - oracle| = {err:.3e} over {len(rows)} rows")
 
 
 def test_lse_optional_and_deterministic():
