@@ -26,7 +26,11 @@ def test_committed_counters_reported_only_for_current_sources():
     assert entries
     for key, ent in entries.items():
         family, workload = key.split(":", 1)
-        assert ent["dram_bytes_per_launch"] == ent["dram_read_bytes"] + ent["dram_write_bytes"]
+        if ent["dram_bytes_per_launch"] is None:
+            # a capture that does not cover a whole call records no total
+            assert ent.get("note"), key
+        else:
+            assert ent["dram_bytes_per_launch"] == ent["dram_read_bytes"] + ent["dram_write_bytes"]
         assert os.path.exists(os.path.join(ROOT, ent["capture"])), ent["capture"]
         current = ent["source_hash"] == bench.kernel_source_hash(family)
         expected = ent["dram_bytes_per_launch"] if current else None
