@@ -82,8 +82,10 @@ enum longnet_impl {
                                 tcgen05/TMEM flash kernel, patterns fused in
                                 shared memory */
   LONGNET_IMPL_SMALLSEG = 3, /* bf16 or fp16, D = 64, all patterns one segment
-                                length w <= 64 (a multiple of 8), one of them
-                                r = 1: memory-bound kernel */
+                                length w <= 64 (a multiple of 8), up to 8
+                                patterns when every r divides 8, else up to
+                                4; q, k, v, out 16-byte aligned: memory-bound
+                                kernel, one weighted softmax per segment */
   LONGNET_IMPL_TILES = 4,    /* backward only: bf16 or fp16, D = 64, any
                                 patterns: 64-row tiles of the sparsified
                                 segments on mma.sync tensor cores */

@@ -4,27 +4,37 @@
 // (the DilatedAttention usage example of the "LongNet" docs page: segment 64,
 // dilation 2), so this kernel is built for HBM bandwidth, not tensor peak.
 //
+// One softmax per segment.  With a common segment length, every pattern's
+// sparsified segment of head h is a subset of the same W positions: pattern
+// p keeps the positions i = o_p (mod r_p), o_p = h mod r_p.  Combining the
+// patterns' outputs with weights equal to their softmax denominators
+// ("LONGNET: Scaling Transformer to 1 billion tokens", section "Token
+// expansion reaches 1 billion+", read as the denominator-weighted
+// combination) gives, for a row i,
+//     out_i = sum_j c_ij e^{s_ij} v_j / sum_j c_ij e^{s_ij},
+//     c_ij  = #{p : i and j both kept by p}   (and j <= i when causal),
+// and the combined lse is log sum_j c_ij e^{s_ij}: the patterns' numerators
+// and denominators simply add.  So one Q K^T over the segment, one softmax
+// whose exponent carries log2 c_ij, and one P V replace the per-pattern
+// passes and their merge; no partial result is rounded or parked.
+//
 // Each pair of warps owns one (batch, segment, head) item at a time, in a
-// persistent grid (one CTA per SM, several pairs); the two warps split every
-// pattern's 16-row chunks:
+// persistent grid (one CTA per SM, several pairs); the two warps split the
+// segment's 16-row chunks:
 //   * three TMA tile loads (Q, K, V: W rows x 128 B, 128-byte swizzle) bring
 //     the segment's rows of that head into the pair's shared memory;
-//   * every pattern's sparsified segment (head offset o = h mod r, rows
-//     o + r*k < W) is read straight from shared memory by ldmatrix (the
-//     dilated gather is just a choice of row addresses) and attended with
-//     mma.sync m16n8k16 (bf16 or fp16 in, fp32 accumulate) and an fp32 softmax;
-//   * patterns other than the r = 1 one park their normalised rows (16-byte
-//     chunks rotated by row, like the TMA swizzle, so a fragment's 8 rows hit
-//     distinct banks) and lse in the pair's shared memory;
-//   * the r = 1 pattern, processed last, merges them row by row with weights
-//     e^{lse_p} ("LONGNET: Scaling Transformer to 1 billion tokens", section
-//     "Token expansion reaches 1 billion+", read as the softmax-denominator-
-//     weighted combination) and the rows go out as coalesced 128-byte stores.
+//   * S = Q K^T and O = P V by mma.sync m16n8k16 (bf16 or fp16 in, fp32
+//     accumulate) on ldmatrix fragments, fp32 softmax with exp2;
+//   * the weights: in the accumulator layout a lane holds rows g, g + 8 and
+//     columns 8 nt + 2 t4 + {0, 1}; when every r divides 8 these are the same
+//     residues mod r for every chunk and every nt, so log2 c is one packed
+//     pair per lane, read from a table indexed by h mod 8 and the lane (the
+//     exponent costs nothing extra).  Other dilations take a general variant
+//     that counts c per element from per-pattern bit masks;
+//   * the normalised rows are staged over the rows' own Q rows (same swizzled
+//     layout) and leave by one TMA tile store per item.
 // Pairs of an SM sit at different points of their load/compute/store cycle,
-// which keeps bytes in flight while others compute.  The work per item is
-// issue-bound (index arithmetic, softmax, mma.sync), so the per-item set-up
-// is hoisted and the unmasked case (non-causal, m a multiple of 16) has its
-// own instantiation; six pairs leave 168 registers per thread.
+// which keeps bytes in flight while others compute.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -44,27 +54,33 @@ namespace ss {
 
 constexpr int kD = 64;
 constexpr int kMaxW = 64;
-constexpr int kMaxPat = 4;
-constexpr int kMaxPairs = 6;  // 12 warps, 3 per SM sub-partition: up to 168 registers each
+constexpr int kMaxPat = 8;         // patterns when every r divides 8
+constexpr int kMaxPatGeneral = 4;  // patterns otherwise (per-pattern masks per lane)
+constexpr int kMaxPairs = 6;       // 12 warps, 3 per SM sub-partition: up to 168 registers each
 constexpr int kTile = kMaxW * kD * 2;  // 8 KB
 constexpr int kSmemLimit = 232448;
+constexpr int kTableBytes = 8 * 32 * 8;  // [h mod 8][lane] packed log2 c pair
+
+// Softmax variants.
+//   kModeFull:    every r divides 8, some r = 1, not causal, W a multiple of 16:
+//                 every key of every row has weight >= 1, no column is masked;
+//   kModeMasked:  every r divides 8, otherwise (causal, W not a multiple of
+//                 16, or keys of weight 0);
+//   kModeGeneral: some r does not divide 8: weights counted per element.
+constexpr int kModeFull = 0, kModeMasked = 1, kModeGeneral = 2;
 
 struct Params {
   Problem pb;
-  int W;                    // common segment length
-  int order[kMaxPat];       // patterns in processing order (the r = 1 one last)
-  int park_off[kMaxPat];    // byte offset of each parked pattern's rows in a pair's region
-  int park_rows[kMaxPat];   // rows reserved for it (ceil(W / r))
-  int r32[kMaxPat];         // dilations (the host checks they fit)
-  uint32_t rcp16[kMaxPat];  // ceil(2^16 / r): (x * rcp16) >> 16 = x / r for 0 <= x < 64
-  int pair_bytes;           // shared memory per warp pair (1024-aligned)
+  int W;                  // common segment length
+  int r32[kMaxPat];       // dilations (the host checks they fit)
+  int pair_bytes;         // shared memory per warp pair (1024-aligned)
   int n_pairs;
-  int64_t n_items;          // B * (segments of the part) * (heads of the part)
+  int64_t n_items;        // B * (segments of the part) * (heads of the part)
   uint64_t wait_limit_ns;
 };
 
 struct __align__(64) Maps {
-  CUtensorMap m[3];  // q, k, v: (d, h, n, b), box (64, 1, W, 1)
+  CUtensorMap m[4];  // q, k, v, out: (d, h, n, b), box (64, 1, W, 1)
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -162,19 +178,36 @@ __device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int ch) {
   return base + (uint32_t)row * 128u + ((uint32_t)(ch ^ (row & 7)) << 4);
 }
 
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The issuing thread's bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The issuing thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------ kernel
 
-// One 16-row chunk (rows [16 rc, 16 rc + 16) of a sparsified segment with m
-// kept rows at o, o + r, ...): S = Q K^T over its m keys, softmax, O = P V,
-// normalised.  In the mma fragment layout this lane holds rows g and g + 8 of
-// the chunk; their O goes to ov and their lse (log2 domain) to lse0, lse1.
-// kMasked: some of the n_kt * 16 key columns are not keys of every row
-// (causal, or m not a multiple of 16).
-template <int kFmt, bool kMasked>
-__device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, uint32_t v_base, int o,
-                                             int r, int m, int n_kt, int rc, bool causal,
-                                             float scale_log2, int lane, float (&ov)[8][4],
-                                             float& lse0, float& lse1) {
+// One 16-row chunk (segment rows [16 rc, 16 rc + 16)) against the segment's W
+// keys: S = Q K^T, the weighted softmax, O = P V, normalised.  In the mma
+// fragment layout this lane holds rows g and g + 8 of the chunk and key
+// columns 8 nt + 2 t4 + {0, 1}; their O goes to ov and their lse (log2
+// domain, -inf for a row no pattern keeps) to lse0, lse1.
+//   kModeFull / kModeMasked: lb = (log2 c, log2 c) of this lane's two key
+//     parities (-inf for weight 0), the same for both rows;
+//   kModeGeneral: cw0, cw1 = the weights of the lane's 16 key columns for
+//     rows g and g + 8, one nibble per column (nibble 2 nt + e).
+template <int kFmt, int kMode>
+__device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, uint32_t v_base, int W, int n_kt,
+                                             int rc, bool causal, float scale_log2, int lane, float2 lb,
+                                             uint64_t cw0, uint64_t cw1, float (&ov)[8][4], float& lse0,
+                                             float& lse1) {
   const int g = lane >> 2, t4 = lane & 3;
   float acc[8][4];
 #pragma unroll
@@ -183,22 +216,20 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   {
     // A fragments address row 16 rc + (lane & 15); B fragments key
-    // 16 np + (lane & 7) + 8 (lane >> 4); rows past m are clamped (their
-    // results are never used, their keys are masked or absent)
+    // 16 np + (lane & 7) + 8 (lane >> 4); rows and keys past W are clamped
+    // (their results are never used, their keys are masked or absent)
     int qi = rc * 16 + (lane & 15);
-    if (qi >= m) qi = m - 1;
-    const int qrow = o + r * qi;
-    const uint32_t qa = q_base + (uint32_t)qrow * 128u;
-    const int qsw = qrow & 7;
+    if (qi >= W) qi = W - 1;
+    const uint32_t qa = q_base + (uint32_t)qi * 128u;
+    const int qsw = qi & 7;
     uint32_t ka[4];
     int ksw[4];
 #pragma unroll
     for (int np = 0; np < 4; ++np) {
       int kj = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-      if (kj >= m) kj = m - 1;
-      const int krow = o + r * kj;
-      ka[np] = k_base + (uint32_t)krow * 128u;
-      ksw[np] = krow & 7;
+      if (kj >= W) kj = W - 1;
+      ka[np] = k_base + (uint32_t)kj * 128u;
+      ksw[np] = kj & 7;
     }
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
@@ -215,44 +246,101 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
       }
     }
   }
-  // ---- softmax over the keys (rows g and g + 8 of this chunk)
+  // ---- weighted softmax over the keys (rows g and g + 8 of this chunk)
   const int row0 = rc * 16 + g, row1 = row0 + 8;
-  float mx0 = -INFINITY, mx1 = -INFINITY;
+  float l0 = 0.f, l1 = 0.f;
+  float m0, m1;  // the exponents' stabilisers (log2 domain)
+  uint32_t pa[4][4];  // P as A fragments, one per 16-key step
+  if constexpr (kMode == kModeFull) {
+    // every weight >= 1: the largest raw score of the row stabilises
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    if (nt < 2 * n_kt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        if (kMasked) {
-          const int c = nt * 8 + 2 * t4 + e;
-          const bool k_ok = c < m;
-          if (!(k_ok && (!causal || c <= row0))) acc[nt][e] = -INFINITY;
-          if (!(k_ok && (!causal || c <= row1))) acc[nt][2 + e] = -INFINITY;
-        }
-        mx0 = fmaxf(mx0, acc[nt][e]);
-        mx1 = fmaxf(mx1, acc[nt][2 + e]);
+    for (int nt = 0; nt < 8; ++nt) {
+      if (nt < 2 * n_kt) {
+        mx0 = fmaxf(mx0, fmaxf(acc[nt][0], acc[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(acc[nt][2], acc[nt][3]));
       }
     }
-  }
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-  const float ms0 = mx0 * scale_log2, ms1 = mx1 * scale_log2;  // every row has a key: finite
-  float l0 = 0.f, l1 = 0.f;
-  uint32_t pa[4][4];  // P as A fragments, one per 16-key step
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    m0 = mx0 * scale_log2;
+    m1 = mx1 * scale_log2;
+    // p = 2^(s * scale + log2 c - m) = c 2^(s * scale - m) <= c
+    const uint64_t sc2 = f32x2(scale_log2, scale_log2);
+    const uint64_t a0 = f32x2(lb.x - m0, lb.y - m0), a1 = f32x2(lb.x - m1, lb.y - m1);
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    if (nt < 2 * n_kt) {
-      float x0, x1, x2, x3;
-      f32x2_split(fma_f32x2(f32x2(acc[nt][0], acc[nt][1]), f32x2(scale_log2, scale_log2), f32x2(-ms0, -ms0)), x0, x1);
-      f32x2_split(fma_f32x2(f32x2(acc[nt][2], acc[nt][3]), f32x2(scale_log2, scale_log2), f32x2(-ms1, -ms1)), x2, x3);
-      const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-      l0 += p0 + p1;
-      l1 += p2 + p3;
-      const int kk = nt >> 1, hi = nt & 1;
-      pa[kk][hi * 2 + 0] = pack2<kFmt>(p0, p1);
-      pa[kk][hi * 2 + 1] = pack2<kFmt>(p2, p3);
+    for (int nt = 0; nt < 8; ++nt) {
+      if (nt < 2 * n_kt) {
+        float x0, x1, x2, x3;
+        f32x2_split(fma_f32x2(f32x2(acc[nt][0], acc[nt][1]), sc2, a0), x0, x1);
+        f32x2_split(fma_f32x2(f32x2(acc[nt][2], acc[nt][3]), sc2, a1), x2, x3);
+        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+        l0 += p0 + p1;
+        l1 += p2 + p3;
+        const int kk = nt >> 1, hi = nt & 1;
+        pa[kk][hi * 2 + 0] = pack2<kFmt>(p0, p1);
+        pa[kk][hi * 2 + 1] = pack2<kFmt>(p2, p3);
+      }
+    }
+  } else {
+    // x = s * scale + log2 c, -inf where the key is past W, after the row
+    // (causal) or of weight 0; the row's largest x stabilises
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      if (nt < 2 * n_kt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = nt * 8 + 2 * t4 + e;
+          const bool ok0 = c < W && (!causal || c <= row0);
+          const bool ok1 = c < W && (!causal || c <= row1);
+          if constexpr (kMode == kModeMasked) {
+            const float b = e ? lb.y : lb.x;
+            acc[nt][e] = ok0 ? fmaf(acc[nt][e], scale_log2, b) : -INFINITY;
+            acc[nt][2 + e] = ok1 ? fmaf(acc[nt][2 + e], scale_log2, b) : -INFINITY;
+          } else {
+            const int sh = 4 * (2 * nt + e);
+            const bool w0 = ((cw0 >> sh) & 15u) != 0, w1 = ((cw1 >> sh) & 15u) != 0;
+            acc[nt][e] = ok0 && w0 ? acc[nt][e] * scale_log2 : -INFINITY;
+            acc[nt][2 + e] = ok1 && w1 ? acc[nt][2 + e] * scale_log2 : -INFINITY;
+          }
+          mx0 = fmaxf(mx0, acc[nt][e]);
+          mx1 = fmaxf(mx1, acc[nt][2 + e]);
+        }
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    // a row with no key of positive weight (no pattern keeps it) has mx =
+    // -inf: any finite stabiliser gives p = 0 and l = 0
+    m0 = mx0 == -INFINITY ? 0.f : mx0;
+    m1 = mx1 == -INFINITY ? 0.f : mx1;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      if (nt < 2 * n_kt) {
+        float p0 = ex2(acc[nt][0] - m0), p1 = ex2(acc[nt][1] - m0);
+        float p2 = ex2(acc[nt][2] - m1), p3 = ex2(acc[nt][3] - m1);
+        if constexpr (kMode == kModeGeneral) {
+          // times the weight (a nibble, as float through the 2^23 magic number)
+          const int sh = 4 * (2 * nt);
+          auto wf = [](uint64_t w, int s) {
+            return __uint_as_float(0x4B000000u | (uint32_t)((w >> s) & 15u)) - 8388608.f;
+          };
+          p0 *= wf(cw0, sh);
+          p1 *= wf(cw0, sh + 4);
+          p2 *= wf(cw1, sh);
+          p3 *= wf(cw1, sh + 4);
+        }
+        l0 += p0 + p1;
+        l1 += p2 + p3;
+        const int kk = nt >> 1, hi = nt & 1;
+        pa[kk][hi * 2 + 0] = pack2<kFmt>(p0, p1);
+        pa[kk][hi * 2 + 1] = pack2<kFmt>(p2, p3);
+      }
     }
   }
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -268,10 +356,9 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
   for (int kk = 0; kk < 4; ++kk) {
     if (kk < n_kt) {
       int vj = kk * 16 + (lane & 15);
-      if (vj >= m) vj = m - 1;  // keys past m have P = 0
-      const int vrow = o + r * vj;
-      const uint32_t va = v_base + (uint32_t)vrow * 128u;
-      const int vsw = vrow & 7;
+      if (vj >= W) vj = W - 1;  // keys past W have P = 0
+      const uint32_t va = v_base + (uint32_t)vj * 128u;
+      const int vsw = vj & 7;
 #pragma unroll
       for (int dp = 0; dp < 4; ++dp) {  // pairs of 8-dim tiles
         uint32_t b0, b1, b2, b3;
@@ -281,17 +368,55 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
       }
     }
   }
-  const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+  if constexpr (kMode == kModeFull) {
+    // l >= 1: the row's largest score has weight >= 1 and exponent >= 0
+    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    f32x2_split(mul_f32x2(f32x2(ov[nt][0], ov[nt][1]), f32x2(inv0, inv0)), ov[nt][0], ov[nt][1]);
-    f32x2_split(mul_f32x2(f32x2(ov[nt][2], ov[nt][3]), f32x2(inv1, inv1)), ov[nt][2], ov[nt][3]);
+    for (int nt = 0; nt < 8; ++nt) {
+      f32x2_split(mul_f32x2(f32x2(ov[nt][0], ov[nt][1]), f32x2(inv0, inv0)), ov[nt][0], ov[nt][1]);
+      f32x2_split(mul_f32x2(f32x2(ov[nt][2], ov[nt][3]), f32x2(inv1, inv1)), ov[nt][2], ov[nt][3]);
+    }
+    lse0 = m0 + __log2f(l0);
+    lse1 = m1 + __log2f(l1);
+  } else {
+    // a row no pattern keeps: out = 0, lse = -inf
+    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      f32x2_split(mul_f32x2(f32x2(ov[nt][0], ov[nt][1]), f32x2(inv0, inv0)), ov[nt][0], ov[nt][1]);
+      f32x2_split(mul_f32x2(f32x2(ov[nt][2], ov[nt][3]), f32x2(inv1, inv1)), ov[nt][2], ov[nt][3]);
+    }
+    lse0 = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
+    lse1 = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
   }
-  lse0 = ms0 + __log2f(l0);
-  lse1 = ms1 + __log2f(l1);
 }
 
-template <int kFmt>
+// Weight nibbles of this lane's 16 key columns (nibble 2 nt + e for column
+// 8 nt + 2 t4 + e) under the patterns keeping `row`: c = the number of
+// patterns p with row = o_p and column = o_p (mod r_p).
+__device__ __forceinline__ uint64_t weight_nibbles(int row, int t4, int n_pat, const int* rp, const int* op) {
+  uint64_t w = 0;
+#pragma unroll
+  for (int p = 0; p < kMaxPatGeneral; ++p) {
+    if (p >= n_pat) break;
+    const int r = rp[p], o = op[p];
+    if (row % r != o) continue;
+    const int step = 8 % r;
+    int m0 = (2 * t4) % r, m1 = (2 * t4 + 1) % r;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      w += (uint64_t)(m0 == o) << (4 * (2 * nt));
+      w += (uint64_t)(m1 == o) << (4 * (2 * nt + 1));
+      m0 += step;
+      m0 -= m0 >= r ? r : 0;
+      m1 += step;
+      m1 -= m1 >= r ? r : 0;
+    }
+  }
+  return w;
+}
+
+template <int kFmt, int kMode>
 __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     smallseg_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   extern __shared__ uint8_t smem_raw[];
@@ -302,14 +427,32 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
   uint8_t* sQ = region;
   uint8_t* sK = region + kTile;
   uint8_t* sV = region + 2 * kTile;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(region + P.pair_bytes - 32);  // TMA landed
-  uint64_t* pbar = bar + 1;                                                 // the pair's hand-off
+  uint64_t* bar = reinterpret_cast<uint64_t*>(region + 3 * kTile);  // TMA landed
+  uint64_t* pbar = bar + 1;                                         // the pair's hand-off
+  float2* wtab = reinterpret_cast<float2*>(smem + (size_t)P.n_pairs * P.pair_bytes);  // [h mod 8][lane]
+  const int n_pat = P.pb.n_pat;
   if (wsub == 0 && lane == 0) {
     mbar_init(bar, 1);
     mbar_init(pbar, 64);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int t = 0; t < 3; ++t)
+    for (int t = 0; t < 4; ++t)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[t])) : "memory");
+  }
+  if constexpr (kMode != kModeGeneral) {
+    // log2 of the weights of a lane's two key parities, for each h mod 8:
+    // rows g (and g + 8, 16 rc + g) and columns 2 t4 + e (+ 8 nt) have the
+    // same residues mod every r dividing 8
+    for (int i = threadIdx.x; i < 8 * 32; i += blockDim.x) {
+      const int hc = i >> 5, g = (i & 31) >> 2, t4 = i & 3;
+      int c[2] = {0, 0};
+      for (int p = 0; p < n_pat; ++p) {
+        const int r = P.r32[p], o = hc % r;
+        if (g % r != o) continue;
+        c[0] += (2 * t4) % r == o;
+        c[1] += (2 * t4 + 1) % r == o;
+      }
+      wtab[i] = make_float2(c[0] ? log2f((float)c[0]) : -INFINITY, c[1] ? log2f((float)c[1]) : -INFINITY);
+    }
   }
   __syncthreads();
   uint32_t pphase = 0;
@@ -321,14 +464,16 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     if (!ok) record_status(P.pb.status, kStatusTimeout);
     return ok;
   };
+  const bool issuer = wsub == 0 && lane == 0;  // TMA loads and the bulk store of the pair
 
-  const int W = P.W, n_pat = P.pb.n_pat;
+  const int W = P.W;
   const int H = (int)P.pb.H;
   const int64_t N = P.pb.N;
   const int seg0 = (int)(P.pb.q0 / W), n_seg = (int)((P.pb.q1 - P.pb.q0) / W);
   const int h0 = (int)P.pb.h0, Hr = (int)(P.pb.h1 - P.pb.h0);
   const bool causal = P.pb.causal != 0;
   const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
+  const int n_kt = (W + 15) >> 4;          // 16-key steps and 16-row chunks
   const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
   const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
   uint32_t phase = 0;
@@ -340,10 +485,12 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     const int seg = seg0 + (int)(bs % n_seg);
     const int b = (int)(bs / n_seg);
     // ---- load the segment's rows of this head (both warps are done with the
-    // previous item: the pair synchronised at its end)
+    // previous item: the pair synchronised before its store)
     __syncwarp();
-    if (wsub == 0 && lane == 0) {
-      // the previous item's rows were staged here with ordinary stores
+    if (issuer) {
+      // the previous item's store has read the staged rows out of sQ, and
+      // rows written with ordinary stores are ordered before the async proxy
+      bulk_wait_read();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                    "r"((uint32_t)(3 * W * 128))
@@ -352,16 +499,20 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
       tma_load_4d(sK, &maps.m[1], bar, 0, h, seg * W, b);
       tma_load_4d(sV, &maps.m[2], bar, 0, h, seg * W, b);
     }
-    // per-item pattern table: head offset of every pattern, computed once
-    int oq[kMaxPat];
+    float2 lb = make_float2(0.f, 0.f);
+    int op[kMaxPatGeneral];
+    if constexpr (kMode != kModeGeneral) {
+      lb = wtab[(h & 7) * 32 + lane];
+    } else {
 #pragma unroll
-    for (int pi = 0; pi < kMaxPat; ++pi) oq[pi] = pi < n_pat ? h % P.r32[P.order[pi]] : 0;
-    const int64_t row0_pos = (int64_t)b * N + (int64_t)seg * W;  // position of the segment's row 0
+      for (int p = 0; p < kMaxPatGeneral; ++p) op[p] = p < n_pat ? h % P.r32[p] : 0;
+    }
     if (!mbar_wait(bar, phase, P.wait_limit_ns)) {
       record_status(P.pb.status, kStatusTimeout);
       // the segment's loads may still be in flight into this pair's shared
       // memory: wait for them once more (bounded) before the warps leave
       mbar_wait(bar, phase, P.wait_limit_ns);
+      if (issuer) bulk_wait_all();
       return;
     }
     if (P.pb.qk_norm) {
@@ -396,148 +547,59 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
           *reinterpret_cast<uint4*>(tile + sw_addr(0, row, ch)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
       }
-      if (!pair_sync()) return;  // every row is normalised before any is read
+      if (!pair_sync()) {  // every row is normalised before any is read
+        if (issuer) bulk_wait_all();
+        return;
+      }
     }
 
-    bool ok = true;
-    for (int pi = 0; pi < n_pat; ++pi) {
-      const int p = P.order[pi];
-      const bool last = pi == n_pat - 1;
-      // the other warp's parked rows are complete before the merging pattern
-      if (last && pi > 0 && !(ok = pair_sync())) break;
-      const int r = P.r32[p];
-      int o = 0;
+    const int64_t seg_pos = (int64_t)seg * W;  // position of the segment's row 0
+    for (int rc = wsub; rc < n_kt; rc += 2) {
+      uint64_t cw0 = 0, cw1 = 0;
+      if constexpr (kMode == kModeGeneral) {
+        cw0 = weight_nibbles(rc * 16 + g, t4, n_pat, P.r32, op);
+        cw1 = weight_nibbles(rc * 16 + g + 8, t4, n_pat, P.r32, op);
+      }
+      float ov[8][4];
+      float lse0, lse1;
+      attend_chunk<kFmt, kMode>(q_base, k_base, v_base, W, n_kt, rc, causal, scale_log2, lane, lb, cw0, cw1, ov,
+                                lse0, lse1);
+      // ---- stage the rows over their own Q rows (no longer read: later
+      // chunks read other rows) in the same swizzled layout
 #pragma unroll
-      for (int q = 0; q < kMaxPat; ++q)
-        if (q == pi) o = oq[q];
-      const int m = o >= W ? 0 : (W - o + r - 1) / r;  // kept rows of this head
-      if (m == 0) continue;
-      const int n_kt = (m + 15) >> 4;  // 16-key steps
-      const bool masked = causal || (m & 15) != 0;
-      uint8_t* park = region + P.park_off[p];
-      float* park_l = reinterpret_cast<float*>(park + P.park_rows[p] * 128);
-      for (int rc = wsub; rc < n_kt; rc += 2) {
-        float ov[8][4];
-        float lse0, lse1;
-        if (masked)
-          attend_chunk<kFmt, true>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
-        else
-          attend_chunk<kFmt, false>(q_base, k_base, v_base, o, r, m, n_kt, rc, causal, scale_log2, lane, ov, lse0, lse1);
-        const int row0 = rc * 16 + g, row1 = row0 + 8;
-        if (!last) {
-          // ---- park the normalised rows (16-byte chunks rotated by row)
+      for (int half = 0; half < 2; ++half) {
+        const int row = rc * 16 + g + 8 * half;
+        if (row < W) {
+          uint8_t* sr = sQ + row * 128 + 4 * t4;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int row = half ? row1 : row0;
-            if (row < m) {
-              uint8_t* pr = park + row * 128 + 4 * t4;
-#pragma unroll
-              for (int nt = 0; nt < 8; ++nt)
-                *reinterpret_cast<uint32_t*>(pr + ((nt ^ (row & 7)) << 4)) =
-                    pack2<kFmt>(ov[nt][2 * half], ov[nt][2 * half + 1]);
-              if (t4 == 0) park_l[row] = half ? lse1 : lse0;
-            }
-          }
-        } else {
-          // ---- merge with the parked patterns, stage over the row's own Q row
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int row = half ? row1 : row0;  // sparse index = position in segment (r = 1)
-            float lse = half ? lse1 : lse0;
-            if (row < m) {
-#pragma unroll
-              for (int qi = 0; qi < kMaxPat - 1; ++qi) {
-                if (qi >= pi) break;
-                const int q = P.order[qi];
-                const int rq = P.r32[q];
-                const int rel = row - oq[qi];
-                const int kq = (int)(((uint32_t)rel * P.rcp16[q]) >> 16);  // rel / rq, exact for rel < 64
-                if (rel < 0 || kq * rq != rel) continue;
-                const uint8_t* pk = region + P.park_off[q];
-                const float lq = reinterpret_cast<const float*>(pk + P.park_rows[q] * 128)[kq];
-                const float mxl = fmaxf(lse, lq);
-                const float wa = ex2(lse - mxl), wb = ex2(lq - mxl);
-                const float iw = 1.f / (wa + wb);
-                const float ca = wa * iw, cb = wb * iw;
-                const uint8_t* pq = pk + kq * 128 + 4 * t4;
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                  float plo, phi;
-                  unpack2<kFmt>(*reinterpret_cast<const uint32_t*>(pq + ((nt ^ (kq & 7)) << 4)), plo, phi);
-                  ov[nt][2 * half] = fmaf(plo, cb, ov[nt][2 * half] * ca);
-                  ov[nt][2 * half + 1] = fmaf(phi, cb, ov[nt][2 * half + 1] * ca);
-                }
-                lse = mxl + __log2f(wa + wb);
-              }
-              // stage the row over its own Q row (no longer read: later chunks
-              // read other rows) in the same swizzled layout
-              uint8_t* sr = sQ + row * 128 + 4 * t4;
-#pragma unroll
-              for (int nt = 0; nt < 8; ++nt)
-                *reinterpret_cast<uint32_t*>(sr + ((nt ^ (row & 7)) << 4)) =
-                    pack2<kFmt>(ov[nt][2 * half], ov[nt][2 * half + 1]);
-              if (t4 == 0 && P.pb.lse)
-                P.pb.lse[((int64_t)b * H + h) * N + (int64_t)seg * W + row] = lse * 0.69314718055994531f;
-            }
-          }
+          for (int nt = 0; nt < 8; ++nt)
+            *reinterpret_cast<uint32_t*>(sr + ((nt ^ (row & 7)) << 4)) =
+                pack2<kFmt>(ov[nt][2 * half], ov[nt][2 * half + 1]);
+          if (t4 == 0 && P.pb.lse)
+            P.pb.lse[((int64_t)b * H + h) * N + seg_pos + row] = (half ? lse1 : lse0) * 0.69314718055994531f;
         }
-        __syncwarp();
       }
     }
-    if (!ok) return;
-    // rows this thread wrote with ordinary stores (normalised q and k, staged
-    // output) may next be overwritten by the async proxy (the next item's TMA)
+    // staged rows (and normalised q and k) are ordered before the async
+    // proxy's store and the next item's loads
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    // ---- coalesced store of the rows this warp staged (its 16-row chunks):
-    // 16-byte chunks, 8 per row
-    __syncwarp();
-    {
-      uint16_t* out_seg = static_cast<uint16_t*>(P.pb.out) + (row0_pos * H + h) * kD;  // 16-bit elements
-      const int64_t row_stride = (int64_t)H * kD;
-      for (int rc = wsub; rc * 16 < W; rc += 2) {
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int idx = it * 32 + lane;
-          const int row = rc * 16 + (idx >> 3), ch = idx & 7;
-          if (row < W) {
-            const uint4 u = *reinterpret_cast<const uint4*>(sQ + sw_addr(0, row, ch));
-            *reinterpret_cast<uint4*>(out_seg + row * row_stride + ch * 8) = u;
-          }
-        }
-      }
+    if (!pair_sync()) {
+      if (issuer) bulk_wait_all();
+      return;
     }
-    if (!pair_sync()) return;
+    if (issuer) tma_store_4d(&maps.m[3], sQ, 0, h, seg * W, b);
   }
+  if (issuer) bulk_wait_all();
 }
 
 // ------------------------------------------------------------ host side
 
-// Layout of one warp pair's shared memory for these patterns; 0 if unsupported.
-int pair_bytes(const Problem& p, int* park_off, int* park_rows, int* order) {
-  int n1 = 0, k = 0;
-  for (int i = 0; i < p.n_pat; ++i) {
-    if (p.r[i] == 1) ++n1;
-  }
-  if (n1 != 1) return 0;
-  int off = 3 * kTile;
-  for (int i = 0; i < p.n_pat; ++i) {
-    if (p.r[i] != 1) {
-      order[k++] = i;
-      park_off[i] = off;
-      park_rows[i] = (int)((p.w[0] + p.r[i] - 1) / p.r[i]);
-      off += park_rows[i] * 128 + park_rows[i] * 4;
-    }
-  }
-  for (int i = 0; i < p.n_pat; ++i) {
-    if (p.r[i] == 1) {
-      order[k++] = i;
-      park_off[i] = 0;
-      park_rows[i] = 0;
-    }
-  }
-  off += 32;                                 // mbarriers
-  return (off + 1023) & ~1023;
-}
+namespace {
+bool divides8(int64_t r) { return r == 1 || r == 2 || r == 4 || r == 8; }
+}  // namespace
+
+// Shared memory of one warp pair: Q, K, V tiles and two mbarriers.
+constexpr int kPairBytes = (3 * kTile + 16 + 1023) & ~1023;
 
 }  // namespace ss
 
@@ -545,6 +607,9 @@ bool smallseg_supports(const Problem& p) {
   using namespace ss;
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
   if (p.n_pat < 1 || p.n_pat > kMaxPat) return false;
+  bool general = false;
+  for (int i = 0; i < p.n_pat; ++i) general |= !divides8(p.r[i]);
+  if (general && p.n_pat > kMaxPatGeneral) return false;
   const int64_t W = p.w[0];
   if (W < 1 || W > kMaxW || W % 8 != 0) return false;
   for (int i = 0; i < p.n_pat; ++i)
@@ -554,9 +619,11 @@ bool smallseg_supports(const Problem& p) {
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.r[i] < 1 || p.r[i] > (int64_t)INT32_MAX) return false;
-  int off[kMaxPat], rows[kMaxPat], order[kMaxPat];
-  const int pb = pair_bytes(p, off, rows, order);
-  return pb > 0 && pb + 1024 <= kSmemLimit;
+  // the tensor maps' base addresses (the strides are multiples of 128 B)
+  const void* ptrs[4] = {p.q, p.k, p.v, p.out};
+  for (const void* ptr : ptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return false;
+  return true;
 }
 
 int launch_smallseg(const Problem& pb, cudaStream_t stream) {
@@ -571,15 +638,15 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   P.pb = pb;
   P.W = (int)pb.w[0];
   P.wait_limit_ns = kWaitLimitNs;
-  P.pair_bytes = pair_bytes(pb, P.park_off, P.park_rows, P.order);
+  P.pair_bytes = kPairBytes;
+  bool general = false, has_r1 = false;
   for (int i = 0; i < pb.n_pat; ++i) {
     P.r32[i] = (int)pb.r[i];
-    P.rcp16[i] = (uint32_t)((65536 + pb.r[i] - 1) / pb.r[i]);
+    general |= !divides8(pb.r[i]);
+    has_r1 |= pb.r[i] == 1;
   }
-  if (P.pair_bytes <= 0) return LONGNET_ERR_UNSUPPORTED;
-  P.n_pairs = (kSmemLimit - 1024) / P.pair_bytes;
+  P.n_pairs = (kSmemLimit - 1024 - kTableBytes) / P.pair_bytes;
   if (P.n_pairs > kMaxPairs) P.n_pairs = kMaxPairs;
-  if (P.n_pairs < 1) return LONGNET_ERR_UNSUPPORTED;
   // items of the computed part: (b, segment, head) with segments in
   // [q0 / W, q1 / W) and heads in [h0, h1)
   P.n_items = pb.B * ((pb.q1 - pb.q0) / P.W) * (pb.h1 - pb.h0);
@@ -593,17 +660,18 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
     const void* q;
     const void* k;
     const void* v;
+    const void* out;
     int64_t B, N, H, W, dtype;
   };
   static MapKey last[64] = {};
   static Maps last_maps[64];
-  const MapKey key{pb.q, pb.k, pb.v, pb.B, pb.N, pb.H, P.W, pb.dtype};
+  const MapKey key{pb.q, pb.k, pb.v, pb.out, pb.B, pb.N, pb.H, P.W, pb.dtype};
   if (memcmp(&last[dev], &key, sizeof(key)) == 0) {
     maps = last_maps[dev];
   } else {
     last[dev] = MapKey{};
-    const void* bases[3] = {pb.q, pb.k, pb.v};
-    for (int t = 0; t < 3; ++t) {
+    const void* bases[4] = {pb.q, pb.k, pb.v, pb.out};
+    for (int t = 0; t < 4; ++t) {
       cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)pb.H, (cuuint64_t)pb.N, (cuuint64_t)pb.B};
       cuuint64_t strides[3] = {(cuuint64_t)(kD * 2), (cuuint64_t)(pb.H * kD * 2),
                                (cuuint64_t)(pb.N * pb.H * kD * 2)};
@@ -618,14 +686,23 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
     last[dev] = key;
   }
   const bool f16 = pb.dtype == LONGNET_DTYPE_F16;
-  auto kernel = f16 ? smallseg_kernel<kFmtF16> : smallseg_kernel<kFmtBF16>;
-  static bool attr_set[64][2] = {};
-  if (!attr_set[dev][f16]) {
+  const int mode = general ? kModeGeneral
+                   : (has_r1 && !pb.causal && P.W % 16 == 0) ? kModeFull
+                                                               : kModeMasked;
+  using KernelFn = void (*)(Params, Maps);
+  static const KernelFn kernels[2][3] = {
+      {smallseg_kernel<kFmtF16, kModeFull>, smallseg_kernel<kFmtF16, kModeMasked>,
+       smallseg_kernel<kFmtF16, kModeGeneral>},
+      {smallseg_kernel<kFmtBF16, kModeFull>, smallseg_kernel<kFmtBF16, kModeMasked>,
+       smallseg_kernel<kFmtBF16, kModeGeneral>}};
+  const KernelFn kernel = kernels[f16 ? 0 : 1][mode];
+  static bool attr_set[64][2][3] = {};
+  if (!attr_set[dev][f16][mode]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
-    attr_set[dev][f16] = true;
+    attr_set[dev][f16][mode] = true;
   }
-  const int smem = P.n_pairs * P.pair_bytes + 1024;
+  const int smem = P.n_pairs * P.pair_bytes + kTableBytes + 1024;
   int64_t grid = (P.n_items + P.n_pairs - 1) / P.n_pairs;
   if (grid > n_sm) grid = n_sm;
   kernel<<<(unsigned)grid, P.n_pairs * 64, smem, stream>>>(P, maps);
