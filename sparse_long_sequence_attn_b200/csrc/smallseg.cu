@@ -34,7 +34,9 @@
 //   * the normalised rows are staged over the rows' own Q rows (same swizzled
 //     layout) and leave by one TMA tile store per item.
 // Pairs of an SM sit at different points of their load/compute/store cycle,
-// which keeps bytes in flight while others compute.
+// which keeps bytes in flight while others compute; each pair also has its
+// next item's tiles brought into L2 (TMA prefetch) when it loads the current
+// one, so the next loads wait for L2, not HBM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -191,6 +193,13 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // The issuing thread's bulk stores are complete.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Brings a tile into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
 
 // ------------------------------------------------------------ kernel
 
@@ -391,28 +400,32 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
   }
 }
 
-// Weight nibbles of this lane's 16 key columns (nibble 2 nt + e for column
-// 8 nt + 2 t4 + e) under the patterns keeping `row`: c = the number of
-// patterns p with row = o_p and column = o_p (mod r_p).
-__device__ __forceinline__ uint64_t weight_nibbles(int row, int t4, int n_pat, const int* rp, const int* op) {
+// Pattern (r, o)'s mask of this lane's 16 key columns: nibble 2 nt + e is 1
+// when column 8 nt + 2 t4 + e = o (mod r).
+__device__ __forceinline__ uint64_t column_nibbles(int r, int o, int t4) {
+  uint64_t w = 0;
+  const int step = 8 % r;
+  int m0 = (2 * t4) % r, m1 = (2 * t4 + 1) % r;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    w |= (uint64_t)(m0 == o) << (4 * (2 * nt));
+    w |= (uint64_t)(m1 == o) << (4 * (2 * nt + 1));
+    m0 += step;
+    m0 -= m0 >= r ? r : 0;
+    m1 += step;
+    m1 -= m1 >= r ? r : 0;
+  }
+  return w;
+}
+// Weight nibbles of this lane's key columns for `row`: the sum of the column
+// masks of the patterns keeping the row (c = #{p : row = o_p and
+// column = o_p (mod r_p)}).
+__device__ __forceinline__ uint64_t weight_nibbles(int row, int n_pat, const int* rp, const int* op,
+                                                   const uint64_t* cols) {
   uint64_t w = 0;
 #pragma unroll
-  for (int p = 0; p < kMaxPatGeneral; ++p) {
-    if (p >= n_pat) break;
-    const int r = rp[p], o = op[p];
-    if (row % r != o) continue;
-    const int step = 8 % r;
-    int m0 = (2 * t4) % r, m1 = (2 * t4 + 1) % r;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      w += (uint64_t)(m0 == o) << (4 * (2 * nt));
-      w += (uint64_t)(m1 == o) << (4 * (2 * nt + 1));
-      m0 += step;
-      m0 -= m0 >= r ? r : 0;
-      m1 += step;
-      m1 -= m1 >= r ? r : 0;
-    }
-  }
+  for (int p = 0; p < kMaxPatGeneral; ++p)
+    if (p < n_pat && row % rp[p] == op[p]) w += cols[p];
   return w;
 }
 
@@ -498,14 +511,26 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
       tma_load_4d(sQ, &maps.m[0], bar, 0, h, seg * W, b);
       tma_load_4d(sK, &maps.m[1], bar, 0, h, seg * W, b);
       tma_load_4d(sV, &maps.m[2], bar, 0, h, seg * W, b);
+      // this pair's next item into L2, so that its loads find it there
+      const int64_t nx = item + (int64_t)gridDim.x * P.n_pairs;
+      if (nx < P.n_items) {
+        const int hn = h0 + (int)(nx % Hr);
+        const int64_t bsn = nx / Hr;
+        const int segn = seg0 + (int)(bsn % n_seg), bn = (int)(bsn / n_seg);
+        for (int t = 0; t < 3; ++t) tma_prefetch_4d(&maps.m[t], 0, hn, segn * W, bn);
+      }
     }
     float2 lb = make_float2(0.f, 0.f);
     int op[kMaxPatGeneral];
+    uint64_t cols[kMaxPatGeneral];
     if constexpr (kMode != kModeGeneral) {
       lb = wtab[(h & 7) * 32 + lane];
     } else {
 #pragma unroll
-      for (int p = 0; p < kMaxPatGeneral; ++p) op[p] = p < n_pat ? h % P.r32[p] : 0;
+      for (int p = 0; p < kMaxPatGeneral; ++p) {
+        op[p] = p < n_pat ? h % P.r32[p] : 0;
+        cols[p] = p < n_pat ? column_nibbles(P.r32[p], op[p], t4) : 0;
+      }
     }
     if (!mbar_wait(bar, phase, P.wait_limit_ns)) {
       record_status(P.pb.status, kStatusTimeout);
@@ -557,8 +582,8 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     for (int rc = wsub; rc < n_kt; rc += 2) {
       uint64_t cw0 = 0, cw1 = 0;
       if constexpr (kMode == kModeGeneral) {
-        cw0 = weight_nibbles(rc * 16 + g, t4, n_pat, P.r32, op);
-        cw1 = weight_nibbles(rc * 16 + g + 8, t4, n_pat, P.r32, op);
+        cw0 = weight_nibbles(rc * 16 + g, n_pat, P.r32, op, cols);
+        cw1 = weight_nibbles(rc * 16 + g + 8, n_pat, P.r32, op, cols);
       }
       float ov[8][4];
       float lse0, lse1;
