@@ -51,6 +51,12 @@ SMALL_CASES = [
     ("bf16_d64_seg40_4pat", 1, 800, 5, 64, torch.bfloat16, True, ((40, 1), (40, 3), (40, 7), (40, 48))),
     ("bf16_d64_seg8_noncausal", 2, 256, 3, 64, torch.bfloat16, False, ((8, 1), (8, 2))),
     ("bf16_d64_seg56_r5", 1, 560, 6, 64, torch.bfloat16, False, ((56, 5), (56, 1), (56, 2))),
+    # one segment length: eight patterns (repeats count twice), no r = 1 (rows
+    # no pattern keeps), W not a multiple of 16 with every r dividing 8
+    ("bf16_d64_seg64_eight_patterns", 2, 1024, 8, 64, torch.bfloat16, False,
+     ((64, 1), (64, 2), (64, 4), (64, 8), (64, 2), (64, 4), (64, 8), (64, 1))),
+    ("bf16_d64_seg32_no_r1_causal", 1, 512, 8, 64, torch.bfloat16, True, ((32, 2), (32, 4), (32, 8))),
+    ("f16_d64_seg48_r8_causal", 2, 480, 9, 64, torch.float16, True, ((48, 1), (48, 8), (48, 4))),
     # fp16 inputs (every family)
     ("f16_d64_lm_like", 2, 2048, 4, 64, torch.float16, True, ((512, 1), (1024, 2), (2048, 4))),
     ("f16_d64_r_not_dividing", 1, 1536, 5, 64, torch.float16, True, ((384, 3), (768, 4), (1536, 8))),
