@@ -237,6 +237,56 @@ int longnet_dilated_attn_fwd_noalloc(const void* q, const void* k, const void* v
                                      longnet_stream_t stream);
 
 /*
+ * longnet_dilated_attn_fwd_host — the forward on inputs and outputs in HOST
+ * memory, with the host<->device copies overlapped with the attention.  The
+ * pages have no counterpart (they say nothing about where a model's tensors
+ * live); it is the call of a host program whose q, k, v come from, and whose
+ * out goes back to, host memory.  The work is cut into pieces that are
+ * pipelined: the copy in of piece c + 1 runs while piece c is attended and
+ * piece c - 1 is copied out.  The cut follows the method's independences:
+ *   B >= 2: ranges of batches (each batch attends on its own);
+ *   B = 1 and H >= 4, or not causal: ranges of heads (each head attends with
+ *     its own rows), copied as strided 2-D blocks;
+ *   B = 1, H < 4, causal: ranges of positions, in order (a row attends to
+ *     keys at or before it, which arrived with its piece or an earlier one),
+ *     each attended as a part (longnet_dilated_attn_fwd_part).
+ *   q_host, k_host, v_host: [B, N, H, D] inputs in host memory; out_host
+ *     [B, N, H, D] and lse_host [B, H, N] (may be NULL) outputs in host
+ *     memory.  Page-locked (pinned) memory lets the copies run asynchronously;
+ *     pageable memory works but each copy then waits on the host.
+ *   q_dev, k_dev, v_dev, out_dev: device buffers of the same shape, and
+ *     lse_dev [B, H, N] (required when lse_host is given), owned by the
+ *     caller and used as the copies' staging; the call allocates nothing.
+ *     Their alignment rules are those of longnet_dilated_attn_fwd.
+ *   pieces: how many pieces (0 = 8 ranges of batches or positions, 6 of
+ *     heads); never more than the batches, positions (in blocks of 256) or
+ *     heads there are, nor more than 64.
+ *   flags: 0 or LONGNET_FLAG_QK_NORM (applied inside the kernels that take
+ *     it, as in longnet_dilated_attn_fwd_ex); impl: as there.
+ *   stream: the call enqueues on `stream` and on two copy streams of its own;
+ *     the copies start after the work already on `stream`, and `stream`
+ *     waits for the last copies before anything enqueued on it later, so
+ *     synchronising `stream` means out_host and lse_host hold the results.
+ *     The call returns once everything is enqueued.
+ *   First call on a device: it creates the two copy streams and their events
+ *     (kept for later calls); make that first call before any stream capture
+ *     begins.  Calls are enqueued one at a time (a lock), so several host
+ *     threads may call; their copies and kernels are then ordered only by
+ *     their streams.
+ * Returns LONGNET_ERR_INVALID_ARG for a NULL host pointer, lse_host without
+ * lse_dev, pieces < 0 or any argument the plain forward rejects (checked
+ * before anything is enqueued); LONGNET_ERR_CUDA when a copy cannot be
+ * enqueued; otherwise the status of the first piece's forward that failed.
+ */
+int longnet_dilated_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                                  void* out_host, float* lse_host,
+                                  void* q_dev, void* k_dev, void* v_dev, void* out_dev, float* lse_dev,
+                                  int64_t B, int64_t N, int64_t H, int64_t D,
+                                  int n_pat, const int64_t* w, const int64_t* r,
+                                  int causal, int dtype, int flags, int impl,
+                                  int64_t pieces, longnet_stream_t stream);
+
+/*
  * longnet_dilated_attn_fwd_part — the forward with options and a family (as
  * longnet_dilated_attn_fwd_ex), computing only part of the output: positions
  * [q_begin, q_end) and heads [h_begin, h_end) of out and lse; every other

@@ -23,6 +23,7 @@ from .binding import (  # noqa: F401
     longnet_dilated_attn_bwd_ws,
     longnet_dilated_attn_fwd,
     longnet_dilated_attn_fwd_noalloc,
+    longnet_dilated_attn_fwd_host,
     longnet_dilated_attn_fwd_part,
     longnet_dilated_attn_fwd_ws,
     longnet_fwd_workspace_bytes,

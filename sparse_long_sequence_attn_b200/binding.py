@@ -60,6 +60,10 @@ SIGNATURES = {
                                                      _i64, ctypes.c_int, _i64p, _i64p,
                                                      ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                      ctypes.c_int, _i64, _i64, _i64, _i64, _vp]),
+    "longnet_dilated_attn_fwd_host": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                     _i64, _i64, _i64, _i64, ctypes.c_int, _i64p, _i64p,
+                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     _i64, _vp]),
     "longnet_fwd_workspace_bytes": (ctypes.c_int64, [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int]),
     "longnet_dilated_attn_fwd_ws": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                                    ctypes.c_int, _i64p, _i64p, ctypes.c_int,
@@ -274,6 +278,44 @@ def longnet_dilated_attn_fwd_part(q: torch.Tensor, k: torch.Tensor, v: torch.Ten
         int(q_range[1]), int(h0), int(h1), _stream_handle(stream))
     if rc != LONGNET_OK:
         raise LongNetError(rc, "longnet_dilated_attn_fwd_part")
+
+
+def longnet_dilated_attn_fwd_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+                                  out_host: torch.Tensor, lse_host: torch.Tensor | None,
+                                  q_dev: torch.Tensor, k_dev: torch.Tensor, v_dev: torch.Tensor,
+                                  out_dev: torch.Tensor, lse_dev: torch.Tensor | None,
+                                  patterns: Sequence[Tuple[int, int]], causal: bool = True,
+                                  impl: int = LONGNET_IMPL_AUTO, stream=None, qk_norm: bool = False,
+                                  pieces: int = 0) -> None:
+    """Enqueue the forward on host tensors (pinned for asynchronous copies):
+    the work is cut into `pieces` ranges (0: the library's choice) of batches
+    (B >= 2), heads (B = 1 with H >= 4, or full attention) or positions
+    (B = 1, H < 4, causal), and each piece's copy in, attention and copy out
+    overlap with its neighbours'.
+    The *_dev tensors are the caller's device staging of the same shapes.
+    Synchronise `stream` before reading out_host / lse_host.  Raises
+    LongNetError on a non-zero status."""
+    lib = load_library()
+    B, N, H, D = q_host.shape
+    for t in (q_host, k_host, v_host, out_host):
+        if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, N, H, D) or t.dtype != q_host.dtype:
+            raise ValueError("q_host, k_host, v_host, out_host: contiguous host tensors [B, N, H, D] of one dtype")
+    for t in (q_dev, k_dev, v_dev, out_dev):
+        if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, N, H, D) or t.dtype != q_host.dtype:
+            raise ValueError("q_dev, k_dev, v_dev, out_dev: contiguous CUDA tensors of the host tensors' shape")
+    for t, want_cuda in ((lse_host, False), (lse_dev, True)):
+        if t is not None and (t.is_cuda != want_cuda or t.dtype != torch.float32 or not t.is_contiguous()
+                              or tuple(t.shape) != (B, H, N)):
+            raise ValueError("lse_host / lse_dev: contiguous fp32 [B, H, N] (host / CUDA)")
+    n, w, r = _patterns(patterns)
+    rc = lib.longnet_dilated_attn_fwd_host(
+        q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), out_host.data_ptr(),
+        None if lse_host is None else lse_host.data_ptr(), q_dev.data_ptr(), k_dev.data_ptr(), v_dev.data_ptr(),
+        out_dev.data_ptr(), None if lse_dev is None else lse_dev.data_ptr(), B, N, H, D, n, w, r,
+        int(bool(causal)), _dtype_code(q_host), LONGNET_FLAG_QK_NORM if qk_norm else 0, int(impl),
+        int(pieces), _stream_handle(stream))
+    if rc != LONGNET_OK:
+        raise LongNetError(rc, "longnet_dilated_attn_fwd_host")
 
 
 def _rows_view(t: torch.Tensor, row_elems: int):

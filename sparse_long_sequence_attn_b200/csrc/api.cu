@@ -301,6 +301,164 @@ extern "C" int longnet_dilated_attn_fwd_noalloc(const void* q, const void* k, co
                     LONGNET_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+namespace longnet {
+namespace {
+// Copy streams and events of the host-buffer forward, per device, created on
+// its first call on that device.  The events are reused from call to call:
+// calls are enqueued one at a time (g_pipe_mutex), and a wait takes the
+// state of an event's latest record at the time the wait is enqueued.
+constexpr int kMaxChunks = 64;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, out_done = nullptr;
+  cudaEvent_t in_done[kMaxChunks] = {};
+  cudaEvent_t comp_done[kMaxChunks] = {};
+};
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.out_done, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; ok && c < kMaxChunks; ++c)
+      ok = cudaEventCreateWithFlags(&hp.in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp_done[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return LONGNET_ERR_CUDA;  // what was created stays for the next attempt to replace
+    }
+    hp.ready = true;
+  }
+  *out = &hp;
+  return LONGNET_OK;
+}
+
+int elem_bytes(int dtype) { return dtype == LONGNET_DTYPE_F32 ? 4 : 2; }
+}  // namespace
+}  // namespace longnet
+
+extern "C" int longnet_dilated_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                                             void* out_host, float* lse_host, void* q_dev, void* k_dev,
+                                             void* v_dev, void* out_dev, float* lse_dev, int64_t B,
+                                             int64_t N, int64_t H, int64_t D, int n_pat, const int64_t* w,
+                                             const int64_t* r, int causal, int dtype, int flags, int impl,
+                                             int64_t pieces, longnet_stream_t stream) {
+  using namespace longnet;
+  // every argument first, on the host: nothing is enqueued for a bad call
+  if (!q_host || !k_host || !v_host || !out_host || (lse_host && !lse_dev)) return LONGNET_ERR_INVALID_ARG;
+  if (pieces < 0) return LONGNET_ERR_INVALID_ARG;
+  if (impl < LONGNET_IMPL_AUTO || impl > LONGNET_IMPL_PATTERNS || impl == LONGNET_IMPL_TILES)
+    return LONGNET_ERR_INVALID_ARG;
+  if (flags & ~LONGNET_FLAG_QK_NORM) return LONGNET_ERR_INVALID_ARG;
+  Problem pb;
+  int rc = check_args(q_dev, k_dev, v_dev, out_dev, lse_dev, B, N, H, D, n_pat, w, r, causal, dtype, &pb);
+  if (rc) return rc;
+  // How the work is cut (each piece: copy in, attend, copy out):
+  //  * B >= 2: ranges of batches (independent, contiguous in memory);
+  //  * B = 1, H >= 4 or not causal: ranges of heads (each head attends with
+  //    its own rows), copied as strided 2-D blocks; every piece has the same
+  //    work, so the last one, whose attention and copy out are not hidden,
+  //    is short;
+  //  * B = 1, H < 4, causal: ranges of positions, in order (a row's keys are
+  //    at or before it, so they arrived with its piece or an earlier one),
+  //    each attended as a part of the forward.
+  int mode;  // 0 batches, 1 positions, 2 heads
+  int64_t per, n_pieces;
+  if (B >= 2) {
+    mode = 0;
+    n_pieces = pieces > 0 ? pieces : 8;
+    if (n_pieces > B) n_pieces = B;
+    per = (B + n_pieces - 1) / n_pieces;
+  } else if (H < 4 && causal) {
+    mode = 1;
+    n_pieces = pieces > 0 ? pieces : 8;
+    per = (N + n_pieces - 1) / n_pieces;
+    per = (per + 255) / 256 * 256;  // whole 256-position blocks
+  } else {
+    mode = 2;
+    n_pieces = pieces > 0 ? pieces : 6;
+    if (n_pieces > H) n_pieces = H;
+    per = (H + n_pieces - 1) / n_pieces;
+  }
+  const int64_t extent = mode == 0 ? B : mode == 1 ? N : H;
+  if (per > extent) per = extent;
+  if ((extent + per - 1) / per > kMaxChunks) per = (extent + kMaxChunks - 1) / kMaxChunks;
+  n_pieces = (extent + per - 1) / per;
+  int dev = 0;
+  int* status = nullptr;
+  rc = current_device_state(&dev, &status);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe* hp = nullptr;
+  rc = host_pipe(dev, &hp);
+  if (rc) return rc;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t eb = (size_t)elem_bytes(dtype);
+  const size_t row = (size_t)H * (size_t)D * eb;  // one position of all heads
+  auto cu = [](cudaError_t e) { return e == cudaSuccess; };
+  auto at = [](const void* base, size_t off) { return static_cast<const char*>(base) + off; };
+  auto atw = [](void* base, size_t off) { return static_cast<char*>(base) + off; };
+  // the copies start after the work already on the caller's stream (an
+  // earlier call may still read these device buffers)
+  bool ok = cu(cudaEventRecord(hp->start, cs)) && cu(cudaStreamWaitEvent(hp->in, hp->start, 0)) &&
+            cu(cudaStreamWaitEvent(hp->out, hp->start, 0));
+  int frc = LONGNET_OK;
+  const void* hin[3] = {q_host, k_host, v_host};
+  void* din[3] = {q_dev, k_dev, v_dev};
+  for (int64_t c = 0; ok && frc == LONGNET_OK && c < n_pieces; ++c) {
+    const int64_t a0 = c * per, a1 = a0 + per < extent ? a0 + per : extent;
+    // the piece as a box: batches [b0, b1), positions [n0, n1), heads [h0, h1)
+    const int64_t b0 = mode == 0 ? a0 : 0, b1 = mode == 0 ? a1 : B;
+    const int64_t n0 = mode == 1 ? a0 : 0, n1 = mode == 1 ? a1 : N;
+    const int64_t h0 = mode == 2 ? a0 : 0, h1 = mode == 2 ? a1 : H;
+    // in memory: `rows` rows of `width` bytes, `pitch` apart, from byte `off`
+    const size_t off = ((size_t)b0 * (size_t)N + (size_t)n0) * row + (size_t)h0 * (size_t)D * eb;
+    const size_t width = (size_t)(h1 - h0) * (size_t)D * eb;
+    const size_t rows = (size_t)(b1 - b0) * (size_t)(n1 - n0);
+    for (int t = 0; ok && t < 3; ++t)
+      ok = mode == 2 ? cu(cudaMemcpy2DAsync(atw(din[t], off), row, at(hin[t], off), row, width, rows,
+                                            cudaMemcpyHostToDevice, hp->in))
+                     : cu(cudaMemcpyAsync(atw(din[t], off), at(hin[t], off), rows * row, cudaMemcpyHostToDevice,
+                                          hp->in));
+    ok = ok && cu(cudaEventRecord(hp->in_done[c], hp->in)) && cu(cudaStreamWaitEvent(cs, hp->in_done[c], 0));
+    if (!ok) break;
+    // the batches of the piece as a problem of their own (B' = b1 - b0)
+    const size_t boff = (size_t)b0 * (size_t)N * row;
+    frc = forward(at(q_dev, boff), at(k_dev, boff), at(v_dev, boff), atw(out_dev, boff),
+                  lse_dev ? lse_dev + b0 * H * N : nullptr, b1 - b0, N, H, D, n_pat, w, r, causal, dtype, flags,
+                  impl, n0, n1, h0, h1, stream);
+    if (frc != LONGNET_OK) break;
+    ok = cu(cudaEventRecord(hp->comp_done[c], cs)) && cu(cudaStreamWaitEvent(hp->out, hp->comp_done[c], 0));
+    ok = ok && (mode == 2 ? cu(cudaMemcpy2DAsync(atw(out_host, off), row, at(out_dev, off), row, width, rows,
+                                                 cudaMemcpyDeviceToHost, hp->out))
+                          : cu(cudaMemcpyAsync(atw(out_host, off), at(out_dev, off), rows * row,
+                                               cudaMemcpyDeviceToHost, hp->out)));
+    if (ok && lse_host) {
+      // lse [B, H, N]: (b1 - b0) * (h1 - h0) runs of (n1 - n0) values; one
+      // 2-D copy per batch
+      for (int64_t b = b0; ok && b < b1; ++b) {
+        const size_t lo = ((size_t)b * (size_t)H + (size_t)h0) * (size_t)N + (size_t)n0;
+        ok = cu(cudaMemcpy2DAsync(lse_host + lo, (size_t)N * 4, lse_dev + lo, (size_t)N * 4,
+                                  (size_t)(n1 - n0) * 4, (size_t)(h1 - h0), cudaMemcpyDeviceToHost, hp->out));
+      }
+    }
+  }
+  // the caller's stream waits for the last copies, whatever happened above,
+  // so the copy streams never run ahead of it into a later call
+  const bool joined = cu(cudaEventRecord(hp->out_done, hp->out)) && cu(cudaStreamWaitEvent(cs, hp->out_done, 0)) &&
+                      cu(cudaEventRecord(hp->out_done, hp->in)) && cu(cudaStreamWaitEvent(cs, hp->out_done, 0));
+  if (!ok || !joined) {
+    cudaGetLastError();
+    return LONGNET_ERR_CUDA;
+  }
+  return frc;
+}
+
 extern "C" int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,
                                              void* out, float* lse, int64_t B, int64_t N,
                                              int64_t H, int64_t D, int n_pat, const int64_t* w,

@@ -275,3 +275,27 @@ def test_noalloc_entry_checked_on_host():
     if not torch.cuda.is_available():
         assert call(1024, 2, 1) == bd.LONGNET_ERR_NO_DEVICE
         assert call(32768, 8, 0) == bd.LONGNET_ERR_NO_DEVICE  # no options: no scratch needed
+
+
+def test_host_buffer_entry_checked_on_host():
+    """longnet_dilated_attn_fwd_host rejects bad arguments before touching a
+    device, and a valid call without a device reports no device."""
+    lib = bd.load_library()
+    buf = ctypes.c_void_p(0x1000)  # never dereferenced on the host
+    w = (ctypes.c_int64 * 1)(16)
+    r = (ctypes.c_int64 * 1)(1)
+
+    def call(q_host=buf, lse_host=None, lse_dev=None, flags=0, impl=0, pieces=0, D=64, dev=buf):
+        return lib.longnet_dilated_attn_fwd_host(q_host, buf, buf, buf, lse_host, dev, buf, buf, buf, lse_dev,
+                                                 1, 256, 4, D, 1, w, r, 1, 1, flags, impl, pieces, None)
+
+    assert call(q_host=None) == bd.LONGNET_ERR_INVALID_ARG
+    assert call(lse_host=buf) == bd.LONGNET_ERR_INVALID_ARG  # lse_host without lse_dev
+    assert call(pieces=-1) == bd.LONGNET_ERR_INVALID_ARG
+    assert call(flags=bd.LONGNET_FLAG_XPOS) == bd.LONGNET_ERR_INVALID_ARG  # XPOS needs a workspace
+    assert call(impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_INVALID_ARG  # backward-only family
+    assert call(D=0) == bd.LONGNET_ERR_INVALID_ARG
+    assert call(dev=ctypes.c_void_p(0x1004)) == bd.LONGNET_ERR_MISALIGNED
+    if not torch.cuda.is_available():
+        assert call() == bd.LONGNET_ERR_NO_DEVICE
+        assert call(lse_host=buf, lse_dev=buf, pieces=3) == bd.LONGNET_ERR_NO_DEVICE
