@@ -980,7 +980,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
         {
           uint32_t pk[32];
-#pragma unroll
           const uint64_t sc2 = f32x2(scale_log2, scale_log2), nm2 = f32x2(-m_use, -m_use);
           uint64_t ls[4] = {0, 0, 0, 0};  // row sum of P in packed pairs
 #pragma unroll
