@@ -849,8 +849,8 @@ def variant_lines(steps, warmup, dev_index=0):
         if st != 0:
             raise RuntimeError(f"device status after variant {name}: {bd.status_string(st)}")
         fam = _impl_name(bd.longnet_select_impl(base.B, N, H, D, base.patterns, base.causal, torch.bfloat16))
-        if mode == "ex_norm":
-            fam = "simt or smallseg (the families that apply qk_norm in the kernel)"
+        if mode == "ex_norm" and fam == "patterns":
+            fam = "simt"  # the per-pattern family does not apply qk_norm in the kernel
         t = sum(per) / len(per)
         res.append({"variant": name, "N": N, "H": H, "D": D, "family": fam, "steps": n,
                     "ms": t * 1e3, "tokens_per_s": base.B * N / t})

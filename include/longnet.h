@@ -124,12 +124,14 @@ enum longnet_flags {
   /* Scale every q row and every k row (over D) to unit L2 norm before the
    * scores: x / max(|x|, 1e-12), computed in fp32.  The reading adopted for
    * the qk_norm option of the DilatedAttention module ("LongNet" docs page,
-   * usage example).  Through longnet_dilated_attn_fwd_ex the SIMT and
-   * small-segment kernels apply it inside the attention (the small-segment
-   * kernel then rounds the rows back to the input format, the SIMT kernel
-   * keeps them in fp32) and the tcgen05 kernel declines it (AUTO falls
-   * back); through longnet_dilated_attn_fwd_ws a prologue pass applies it
-   * and every family takes the result. */
+   * usage example).  Through longnet_dilated_attn_fwd_ex the SIMT,
+   * small-segment and tcgen05 kernels apply it inside the attention (the
+   * small-segment kernel rounds the normalised rows back to the input
+   * format, the SIMT kernel keeps them in fp32, the tcgen05 kernel scales
+   * the scores of the rows as given by both inverse norms in fp32); the
+   * per-pattern family declines it (AUTO falls back); through
+   * longnet_dilated_attn_fwd_ws a prologue pass applies it and every family
+   * takes the result. */
   LONGNET_FLAG_QK_NORM = 1,
   /* XPOS on q and k, the rotary position encoding with exponential scaling
    * that the use_xpos option names ("LongNet论文精读", section "Dilated

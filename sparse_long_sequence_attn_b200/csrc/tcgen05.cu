@@ -120,6 +120,7 @@ struct SmemLayout {
   int slot_o;  // n_pat x 128 parked rows (input format)
   int slot_l;  // n_pat x 128 parked lse (fp32, log2 domain)
   int stats;   // [stream][O buffer][use parity][row] (m, l)
+  int ikn;     // qk_norm: [stream][block parity][64] inverse key norms
   int meta;    // tile queues, stage descriptors, pattern table, counters
   int walker;  // the TMA thread's block-sequence state (kept out of local memory)
   int bars;
@@ -133,7 +134,8 @@ struct SmemLayout {
     slot_o = kv + stages * 2 * kKVBytes;
     slot_l = slot_o + n_pat * kTileBytes;
     stats = slot_l + n_pat * kBM * 4;
-    meta = stats + 2 * 2 * 2 * kBM * 8;
+    ikn = stats + 2 * 2 * 2 * kBM * 8;
+    meta = ikn + 2 * 2 * kBN * 4;
     walker = meta + kMetaBytes;
     bars = walker + 2 * kWalkerBytes;
     misc = bars + 48 * 8;
@@ -570,7 +572,12 @@ enum : uint32_t {
 // ---------------------------------------------------------------- kernel
 
 
-template <int kFmt>
+// kNorm: LONGNET_FLAG_QK_NORM, q and k rows taken at unit L2 norm.  The
+// scores are computed from the rows as given and scaled afterwards, row i by
+// 1 / max(|q_i|, 1e-12) and column j by 1 / max(|k_j|, 1e-12) (fp32), which is
+// the dot product of the normalised rows; the norms come from the Q tile and
+// the K blocks in shared memory.
+template <int kFmt, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1)
     dilated_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ TmaMaps maps) {
   extern __shared__ uint8_t smem_raw[];
@@ -602,6 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_drain = bars + 23;        // [2]
   uint64_t* bar_kv_full = bars + 26;      // [2][kMaxStages]
   uint64_t* bar_kv_empty = bars + 26 + 2 * kMaxStages;  // [2][kMaxStages]
+  uint64_t* bar_ikn = bars + 26 + 4 * kMaxStages;       // qk_norm: [2][2] stream, block parity
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 8);
 
@@ -623,7 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar_q_full + g, 1);
-      mbar_init(bar_q_empty + g, 1);
+      // with qk_norm the softmax warps read their Q rows too before the
+      // buffer may be refilled
+      mbar_init(bar_q_empty + g, kNorm ? 1 + 128 : 1);
+      for (int b2 = 0; b2 < 2; ++b2) mbar_init(bar_ikn + 2 * g + b2, 128);
       for (int sb = 0; sb < 2; ++sb) {
         mbar_init(bar_s_full + 2 * g + sb, 1);
         mbar_init(bar_p_full + 2 * g + sb, 128);
@@ -916,9 +927,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
+    float row_scale = scale_log2;  // with qk_norm times this row's inverse q norm
     uint32_t s_cnt = 0, od_cnt = 0;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
+    const int NSg = ring_stages(P.stages, g);
+    const uint8_t* ring_g = sKV + (g ? ring_stages(P.stages, 0) : 0) * 2 * kKVBytes;
+    float* ikn = reinterpret_cast<float*>(smem + L.ikn) + g * 2 * kBN;
     for (int i = 0; ok; ++i) {  // this stream's tiles
       ok = wait_count(cnt_elem + g, i);
       ok = __all_sync(0xffffffffu, ok);
@@ -942,14 +957,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sb = s_cnt & 1;
         ok = sy.wait_warp(bar_s_full + 2 * g + sb, (s_cnt >> 1) & 1);
         if (!ok) break;
-        ++s_cnt;
+        const uint32_t blk = s_cnt++;  // this stream's block count
         tc_fence_after();
         const uint32_t s_col = tmem + lane_base + col_s(g, sb);
         const int lim = causal ? em.lim0 + row - j * kBN : em.lim0 - j * kBN;
+        if constexpr (kNorm) {
+          // This block's keys: rows of the K block of ring stage blk mod NS,
+          // which stays until this block's P V has run.  Thread t sums half
+          // of key row t / 2; the 64 inverse norms go to shared memory.
+          const uint8_t* kb = ring_g + (int)(blk % (uint32_t)NSg) * 2 * kKVBytes;
+          const int kr = row >> 1, half = row & 1;
+          float ss = 0.f;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int ch = half * 4 + c4;
+            const uint4 u = *reinterpret_cast<const uint4*>(kb + kr * 128 + ((ch ^ (kr & 7)) << 4));
+            const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float lo, hi;
+              unpack2<kFmt>(wv[e], lo, hi);
+              ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+            }
+          }
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          float* ikb = ikn + (blk & 1) * kBN;
+          if (half == 0) ikb[kr] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+          if (j == 0) {
+            // the row's inverse q norm, from the tile's Q buffer (which is
+            // refilled only after these reads: the q-empty barrier counts them)
+            const uint8_t* qt = sQ + g * kTileBytes + row * 128;
+            float qs = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint4 u = *reinterpret_cast<const uint4*>(qt + ((ch ^ (row & 7)) << 4));
+              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float lo, hi;
+                unpack2<kFmt>(wv[e], lo, hi);
+                qs = fmaf(lo, lo, fmaf(hi, hi, qs));
+              }
+            }
+            row_scale = scale_log2 / fmaxf(sqrtf(qs), 1e-12f);
+            mbar_arrive(bar_q_empty + g);
+          }
+          // every thread's inverse norm is written before any is read; the
+          // other parity's array is rewritten only after all 128 threads
+          // arrived for the block in between
+          mbar_arrive(bar_ikn + 2 * g + (blk & 1));
+          ok = sy.wait_warp(bar_ikn + 2 * g + (blk & 1), (blk >> 1) & 1);
+          if (!ok) break;
+        }
         uint32_t sr[kBN];
         LN_TMEM_LD32(s_col + 0, (sr + 0));
         LN_TMEM_LD32(s_col + 32, (sr + 32));
         tmem_wait_ld();
+        if constexpr (kNorm) {
+          const float4* ik4 = reinterpret_cast<const float4*>(ikn + (blk & 1) * kBN);
+#pragma unroll
+          for (int c4 = 0; c4 < kBN / 4; ++c4) {
+            const float4 f = ik4[c4];
+            sr[4 * c4 + 0] = __float_as_uint(__uint_as_float(sr[4 * c4 + 0]) * f.x);
+            sr[4 * c4 + 1] = __float_as_uint(__uint_as_float(sr[4 * c4 + 1]) * f.y);
+            sr[4 * c4 + 2] = __float_as_uint(__uint_as_float(sr[4 * c4 + 2]) * f.z);
+            sr[4 * c4 + 3] = __float_as_uint(__uint_as_float(sr[4 * c4 + 3]) * f.w);
+          }
+        }
         if (lim < kBN - 1) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
@@ -962,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
         const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        const float m_blk = mx * scale_log2;
+        const float m_blk = mx * row_scale;
         float corr = 1.f;
         bool rescale = false;
         if (m_blk > m_use + 8.f || m_use == -INFINITY) {
@@ -980,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
         {
           uint32_t pk[32];
-          const uint64_t sc2 = f32x2(scale_log2, scale_log2), nm2 = f32x2(-m_use, -m_use);
+          const uint64_t sc2 = f32x2(row_scale, row_scale), nm2 = f32x2(-m_use, -m_use);
           uint64_t ls[4] = {0, 0, 0, 0};  // row sum of P in packed pairs
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -1247,7 +1321,6 @@ int64_t range_cost(const Problem& pb, int64_t A, int64_t Bnd) {
 bool tcgen05_supports(const Problem& p) {
   using namespace tc;
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || p.D != kD) return false;
-  if (p.qk_norm) return false;  // no normalisation pass on this path
   static_assert(sizeof(BlockSeq) <= kWalkerBytes, "block-sequence state must fit its shared-memory slot");
   if (p.n_pat > kMaxPat || pick_stages(p.n_pat) < 4) return false;
   if (p.H > 65535 || p.B > 65535) return false;
@@ -1478,13 +1551,14 @@ int launch_tcgen05(const Problem& pb, cudaStream_t stream) {
     c.v = pb.v;
   }
   const int smem_bytes = P.smem_bytes;
-  const bool f16 = pb.dtype == LONGNET_DTYPE_F16;
-  auto kernel = f16 ? dilated_fwd_kernel<kFmtF16> : dilated_fwd_kernel<kFmtBF16>;
-  static bool attr_set[64][2] = {};
-  if (!attr_set[dev][f16]) {
+  const bool f16 = pb.dtype == LONGNET_DTYPE_F16, norm = pb.qk_norm != 0;
+  auto kernel = f16 ? (norm ? dilated_fwd_kernel<kFmtF16, true> : dilated_fwd_kernel<kFmtF16, false>)
+                    : (norm ? dilated_fwd_kernel<kFmtBF16, true> : dilated_fwd_kernel<kFmtBF16, false>);
+  static bool attr_set[64][2][2] = {};
+  if (!attr_set[dev][f16][norm]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
       return LONGNET_ERR_CUDA;
-    attr_set[dev][f16] = true;
+    attr_set[dev][f16][norm] = true;
   }
   const int64_t grid = (int64_t)P.n_units * pb.B * (pb.h1 - pb.h0);
   kernel<<<(unsigned)grid, kThreads, smem_bytes, stream>>>(P, c.maps);
