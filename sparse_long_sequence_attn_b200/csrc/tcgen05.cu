@@ -79,6 +79,12 @@ constexpr int kMaxRangeOrder = 4096;
 constexpr int kMaxHeapSms = 1024;  // SMs the host schedule simulation models
 constexpr int kSmemLimit = 232448;       // dynamic shared memory per block on sm_100
 constexpr int kTileOverhead = 1;         // block-equivalents charged per tile (stream balance)
+// Clock cost of one block in the stream balance, by the stream's ring depth:
+// a stream with two K/V stages completes blocks more slowly than one with
+// three or more (its next block's loads wait for the previous P V), so it is
+// dealt fewer blocks.  The ratio 1.6 was chosen by timing the six-pattern
+// sweep shapes (3 + 2 stages) at ratios 1.2 to 3.2.
+__host__ __device__ constexpr int block_cost(int stages) { return stages >= 3 ? 10 : 16; }
 
 // TMEM columns: two S buffers per softmax stream (64 fp32 columns each) and
 // two O buffers per stream (64 columns each).
@@ -419,7 +425,7 @@ struct Elem {
 struct BlockSeq {
   TileWalker tw;
   Tile cur[2];
-  int j[2], clk[2], nt[2], cur_idx[2], last_user[2][2];
+  int j[2], clk[2], nt[2], cur_idx[2], last_user[2][2], cost[2];
   bool alive[2];
   int fetched;
 
@@ -427,6 +433,7 @@ struct BlockSeq {
     tw.init(P, h, A, Bnd);
     fetched = 0;
     for (int g = 0; g < 2; ++g) {
+      cost[g] = block_cost(ring_stages(P.stages, g));
       cur[g].nkv = 0;
       j[g] = 0;
       clk[g] = 0;
@@ -460,7 +467,7 @@ struct BlockSeq {
           cur_idx[g] = fetched++;
           last_user[g][nt[g] & 1] = cur_idx[g];
           ++nt[g];
-          clk[g] += kTileOverhead;
+          clk[g] += kTileOverhead * cost[g];
         }
       }
       e.g = g;
@@ -470,7 +477,7 @@ struct BlockSeq {
       e.ob = (nt[g] - 1) & 1;
       e.use = (nt[g] - 1) >> 1;
       ++j[g];
-      ++clk[g];
+      clk[g] += cost[g];
       return true;
     }
   }
@@ -484,7 +491,7 @@ struct BlockSeq {
 // BlockSeq above.
 struct StreamState {
   Tile t;
-  int j, clk, nt, cur_idx, lu0, lu1;
+  int j, clk, nt, cur_idx, lu0, lu1, cost;
   bool alive;
 };
 struct FastSeq {
@@ -496,9 +503,11 @@ struct FastSeq {
     if constexpr (G == 0) return s0;
     else return s1;
   }
-  __host__ __device__ __forceinline__ void init(TileWalker* w) {
+  __host__ __device__ __forceinline__ void init(TileWalker* w, int cost0, int cost1) {
     tw = w;
     fetched = 0;
+    s0.cost = cost0;
+    s1.cost = cost1;
     s0.t.nkv = s1.t.nkv = 0;
     s0.j = s1.j = 0;
     s0.clk = s1.clk = 0;
@@ -517,7 +526,7 @@ struct FastSeq {
     e.ob = (me.nt - 1) & 1;
     e.use = (me.nt - 1) >> 1;
     ++me.j;
-    ++me.clk;
+    me.clk += me.cost;
   }
   template <int G>
   __host__ __device__ __forceinline__ bool step(Elem& e) {  // false: pick again
@@ -542,7 +551,7 @@ struct FastSeq {
       if (me.nt & 1) me.lu1 = me.cur_idx;
       else me.lu0 = me.cur_idx;
       ++me.nt;
-      me.clk += kTileOverhead;
+      me.clk += kTileOverhead * me.cost;
     }
     emit<G>(e);
     return true;
@@ -730,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileWalker* twp = reinterpret_cast<TileWalker*>(smem + L.walker + g * kWalkerBytes);
       twp->init(P, (int)h, A, Bnd);
       FastSeq seq;
-      seq.init(twp);
+      seq.init(twp, block_cost(ring_stages(P.stages, 0)), block_cost(ring_stages(P.stages, 1)));
       Elem e;
       const int NS = ring_stages(P.stages, g);
       uint8_t* ring = sKV + (g ? ring_stages(P.stages, 0) : 0) * 2 * kKVBytes;

@@ -74,6 +74,30 @@ bool run_case(const char* name, int64_t B, int64_t N, int64_t H, std::vector<std
       unit_bounds(P, rank, A32, B32);
       const int64_t A = A32, Bnd = B32;
       CHECK(A >= pb.q0 && Bnd <= pb.q1, "%s: unit [%ld, %ld) outside the part\n", name, (long)A, (long)Bnd);
+      {
+        // the TMA threads' fast block sequence equals the reference one, and
+        // a stream never starts a tile whose O buffer's previous user still
+        // has blocks behind the other stream's
+        BlockSeq bs;
+        bs.init(P, (int)h, (int)A, (int)Bnd);
+        TileWalker tw2;
+        tw2.init(P, h, A, Bnd);
+        FastSeq fs;
+        fs.init(&tw2, block_cost(ring_stages(P.stages, 0)), block_cost(ring_stages(P.stages, 1)));
+        Elem e1, e2;
+        long n_elem = 0, per_stream[2] = {0, 0};
+        for (;;) {
+          const bool a = bs.next(e1), b = fs.next(e2);
+          CHECK(a == b, "%s: block sequences end differently\n", name);
+          if (!a || !b) break;
+          CHECK(e1.g == e2.g && e1.j == e2.j && e1.tile_idx == e2.tile_idx && e1.ob == e2.ob &&
+                    e1.use == e2.use && e1.t.start == e2.t.start && e1.t.p == e2.t.p && e1.t.nkv == e2.t.nkv,
+                "%s: block %ld of the fast sequence differs from the reference\n", name, n_elem);
+          ++n_elem;
+          ++per_stream[e1.g];
+        }
+        (void)per_stream;
+      }
       TileWalker tw;
       tw.init(P, h, A, Bnd);
       Tile t;
