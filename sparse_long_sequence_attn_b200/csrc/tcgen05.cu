@@ -1482,8 +1482,11 @@ void fill_params(const Problem& pb, tc::Params& P, int n_sm) {
     int best_k = 0;
     const bool can_split = R % 2 == 0 && R / 2 >= kBM && (int64_t)P.n_ranges * BH <= 262144;
     if (can_split) {
+      // up to 64 ranges split (the unit array holds kMaxRangeOrder + 8), the
+      // search stopping once 8 more splits in a row have not helped
       int64_t best = makespan(units_for(0));
-      for (int k = 1; k <= std::min(8, P.n_ranges); ++k) {
+      const int k_max = std::min(std::min(64, P.n_ranges), kMaxRangeOrder + 8 - P.n_ranges);
+      for (int k = 1; k <= k_max && k - best_k <= 8; ++k) {
         const int n = units_for(k);
         if (n > kMaxRangeOrder) break;
         const int64_t m = makespan(n);
