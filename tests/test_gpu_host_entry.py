@@ -101,3 +101,24 @@ def test_two_calls_in_a_row_reuse_the_staging_buffers():
         o2, l2 = gh.run_cuda(q, k, v, pats, True, bd.LONGNET_IMPL_AUTO)
         assert float(np.abs(oh.float().numpy() - o2).max()) <= gh.TOL_OUT[dtype]
         assert float(np.abs(lh.numpy() - l2).max()) <= gh.TOL_LSE
+
+
+def test_host_entry_with_qk_norm():
+    """The flag passes through to the pieces' forwards (the fused kernel's
+    qk_norm variant here)."""
+    dev = torch.device("cuda:0")
+    B, N, H, D, dtype, pats = 2, 2048, 4, 64, torch.bfloat16, ((256, 1), (512, 2), (2048, 4))
+    q, k, _ = wl.random_inputs(B, N, H, D, dtype, seed=41, scale=3.0)
+    _, _, v = wl.random_inputs(B, N, H, D, dtype, seed=42)
+    qh, kh, vh = (_host(x, True) for x in (q, k, v))
+    out_h = torch.full((B, N, H, D), float("nan"), dtype=dtype, pin_memory=True)
+    lse_h = torch.full((B, H, N), float("nan"), dtype=torch.float32, pin_memory=True)
+    qd, kd, vd, od = (torch.empty(B, N, H, D, dtype=dtype, device=dev) for _ in range(4))
+    ld = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    bd.longnet_dilated_attn_fwd_host(qh, kh, vh, out_h, lse_h, qd, kd, vd, od, ld, pats, True, stream=stream,
+                                     qk_norm=True)
+    stream.synchronize()
+    assert bd.longnet_last_device_status(stream) == 0
+    gh.compare_full(out_h.float().numpy(), lse_h.numpy(), q, k, v, pats, True, dtype, label="host entry qk_norm",
+                    qk_norm=True)

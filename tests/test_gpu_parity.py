@@ -180,6 +180,9 @@ QK_NORM_CASES = [
     ("lm_like_bf16", 1, 1024, 3, 64, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
     ("paper_like_f16_partial", 1, 3000, 4, 64, torch.float16, True, ((256, 1), (512, 2), (1024, 4), (3000, 6))),
     ("long_noncausal_bf16", 2, 2048, 2, 64, torch.bfloat16, False, ((512, 1), (2048, 4))),
+    # six patterns: the fused kernel's streams get 3 + 2 ring stages
+    ("six_patterns_bf16", 1, 3072, 2, 64, torch.bfloat16, True,
+     ((256, 1), (512, 2), (768, 3), (1024, 4), (1536, 6), (3072, 12))),
     ("fp32_d32", 1, 384, 2, 32, torch.float32, True, ((96, 1), (192, 5), (384, 7))),
 ]
 
