@@ -799,8 +799,8 @@ def variant_lines(steps, warmup, dev_index=0):
     flush between steps): the input options through the prologue pass
     (longnet_dilated_attn_fwd_ws: qk_norm, XPOS), qk_norm inside the kernel
     (longnet_dilated_attn_fwd_ex, which AUTO sends to the family that takes
-    it), a sequence 64 tokens short (a partial last segment) and D = 128
-    (H 6).  Reports the family AUTO picked for each.  Inputs drawn on the
+    it), a sequence 64 tokens short (a partial last segment), D = 128
+    (H 6) and D = 32 (H 24).  Reports the family AUTO picked for each.  Inputs drawn on the
     device; parity of each variant is tested separately."""
     import torch
 
@@ -816,7 +816,7 @@ def variant_lines(steps, warmup, dev_index=0):
              ("xpos_prologue", base.N, base.H, base.D, "ws_xpos"),
              ("qk_norm_in_kernel", base.N, base.H, base.D, "ex_norm"),
              ("partial_last_segment", base.N - 64, base.H, base.D, "plain"),
-             ("d128", base.N, base.H // 2, 128, "plain")]
+             ("d128", base.N, base.H // 2, 128, "plain"), ("d32", base.N, base.H * 2, 32, "plain")]
     for name, N, H, D, mode in cases:
         g = torch.Generator(device=dev)
         g.manual_seed(base.seed)

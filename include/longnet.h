@@ -89,7 +89,7 @@ enum longnet_impl {
   LONGNET_IMPL_TILES = 4,    /* backward only: bf16 or fp16, D = 64, any
                                 patterns: 64-row tiles of the sparsified
                                 segments on mma.sync tensor cores */
-  LONGNET_IMPL_PATTERNS = 5  /* forward: bf16 or fp16, D = 64 or 128, any number
+  LONGNET_IMPL_PATTERNS = 5  /* forward: bf16 or fp16, D = 16, 32, 64 or 128, any number
                                 of patterns, lse required with more than one:
                                 one tcgen05 launch per pattern, each merging its
                                 rows into out and lse (initialised to 0 and

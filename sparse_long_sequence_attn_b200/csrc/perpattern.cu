@@ -1,6 +1,6 @@
 // Kernel family PATTERNS: the multi-pattern dilated-attention forward one
 // pattern at a time, on the 5th-generation tensor cores, for bf16 or fp16 at
-// D = 64 or 128 and any number of patterns.
+// D = 16, 32, 64 or 128 and any number of patterns.
 //
 // What it computes is the forward of the fused tcgen05 family ("LONGNET:
 // Scaling Transformer to 1 billion tokens", section "LongNet's attention
@@ -57,18 +57,27 @@ using namespace tc;
 constexpr int kTile = 128;   // rows per CTA (M of the MMAs)
 constexpr int kBlk = 64;     // keys per block (N of S = Q K^T)
 constexpr int kThreads = 192;
-constexpr int kPanelRowBytes = 128;              // one 64-element swizzle panel row
-constexpr int kQPanel = kTile * kPanelRowBytes;  // 16 KB
-constexpr int kKVPanel = kBlk * kPanelRowBytes;  // 8 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;  // scores at 0 and 64
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994531f;
 
-// kPanels = D / 64; ring stages: 3 at D = 64, 2 at D = 128 (two CTAs per SM)
-template <int kPanels>
+// Rows of D elements as swizzle panels: D = 64 or 128 is one or two panels of
+// 64 elements (128-byte rows, 128-byte swizzle); D = 32 or 16 is one panel of
+// D elements (64- or 32-byte rows, 64- or 32-byte swizzle).  Ring stages: 3 up
+// to D = 64, 2 at D = 128 (two CTAs per SM).
+template <int kD>
 struct Layout {
-  static constexpr int kStages = kPanels == 1 ? 3 : 2;
+  static constexpr int kPanels = kD >= 64 ? kD / 64 : 1;
+  static constexpr int kPanelElems = kD >= 64 ? 64 : kD;
+  static constexpr int kRowBytes = kPanelElems * 2;  // one panel row
+  static constexpr int kQPanel = kTile * kRowBytes;
+  static constexpr int kKVPanel = kBlk * kRowBytes;
+  // descriptor high word: stride between 8-row groups, sm_100 version, layout
+  // type (128-byte swizzle 2, 64-byte 4, 32-byte 6)
+  static constexpr uint32_t kDescHi = (uint32_t)(8 * kRowBytes >> 4) | (1u << 14) |
+                                      ((kRowBytes == 128 ? 2u : kRowBytes == 64 ? 4u : 6u) << 29);
+  static constexpr int kStages = kD <= 64 ? 3 : 2;
   static constexpr int kQBytes = kPanels * kQPanel;
   static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
   static constexpr int kBars = kQBytes + kStages * kStageBytes;
@@ -129,11 +138,30 @@ struct Waiter {
   __device__ bool wait_warp(uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, wait(bar, parity)); }
 };
 
-template <int kFmt, int kPanels>
+template <int kFmt, int kD>
 __global__ void __launch_bounds__(kThreads, 2)
     pp_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
-  using L = Layout<kPanels>;
-  constexpr int kD = 64 * kPanels;
+  using L = Layout<kD>;
+  constexpr int kPanels = L::kPanels;
+  constexpr int kQPanel = L::kQPanel, kKVPanel = L::kKVPanel;
+  constexpr uint32_t kDescHi = L::kDescHi;
+  // O moves between TMEM and registers kOChunk columns at a time (16 at D = 16)
+  constexpr int kOChunk = kD < 32 ? kD : 32;
+  auto o_load = [](uint32_t taddr, uint32_t(&r)[kOChunk]) {
+    if constexpr (kOChunk == 32) {
+      LN_TMEM_LD32(taddr, r);
+    } else {
+      LN_TMEM_LD16(taddr, r);
+    }
+    tmem_wait_ld();
+  };
+  auto o_store = [](uint32_t taddr, uint32_t(&r)[kOChunk]) {
+    if constexpr (kOChunk == 32) {
+      LN_TMEM_ST32(taddr, r);
+    } else {
+      LN_TMEM_ST16(taddr, r);
+    }
+  };
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -222,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive_expect_tx(bar_q, L::kQBytes);
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn)
-          tma_load_5d(sQ + pn * kQPanel, &maps.m[c.map][0], bar_q, 64 * pn, h, c.c, c.kk, b);
+          tma_load_5d(sQ + pn * kQPanel, &maps.m[c.map][0], bar_q, L::kPanelElems * pn, h, c.c, c.kk, b);
       }
       int issued = 0;
       for (int j = 0; j < nblk && ok; ++j) {
@@ -236,8 +264,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive_expect_tx(bar_full + st, L::kStageBytes);
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn) {
-          tma_load_5d(stage + pn * kKVPanel, &maps.m[c.map][1], bar_full + st, 64 * pn, h, c.c, c.kk, b);
-          tma_load_5d(stage + (kPanels + pn) * kKVPanel, &maps.m[c.map][2], bar_full + st, 64 * pn, h, c.c, c.kk, b);
+          tma_load_5d(stage + pn * kKVPanel, &maps.m[c.map][1], bar_full + st, L::kPanelElems * pn, h, c.c, c.kk,
+                      b);
+          tma_load_5d(stage + (kPanels + pn) * kKVPanel, &maps.m[c.map][2], bar_full + st, L::kPanelElems * pn, h,
+                      c.c, c.kk, b);
         }
         issued = j + 1;
       }
@@ -262,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t v_lo = (smem_u32(sStage + (jj % S) * L::kStageBytes) >> 4) + (uint32_t)(kPanels * kKVPanel >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          mma_ts(tmem + kColO, tmem + 64 * (jj & 1) + kk * 8, desc_from((v_lo | lbo_mn) + kk * 128, kDescHi), kIdO,
+          mma_ts(tmem + kColO, tmem + 64 * (jj & 1) + kk * 8,
+                 desc_from((v_lo | lbo_mn) + kk * (16 * L::kRowBytes >> 4), kDescHi), kIdO,
                  (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar_empty + jj % S);
         tc_commit(bar_od);
@@ -279,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < L::kPanelElems / 16; ++kk)
             mma_ss(tmem + 64 * (j & 1), desc_from(((q_lo + pn * (kQPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi),
                    desc_from(((k_lo + pn * (kKVPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi), kIdS,
                    (pn > 0 || kk > 0) ? 1u : 0u);
@@ -361,13 +392,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-          uint32_t rr[32];
-          LN_TMEM_LD32(tmem + lane_base + kColO + c0, rr);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < kD; c0 += kOChunk) {
+          uint32_t rr[kOChunk];
+          o_load(tmem + lane_base + kColO + c0, rr);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
-          LN_TMEM_ST32(tmem + lane_base + kColO + c0, rr);
+          for (int c = 0; c < kOChunk; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * corr);
+          o_store(tmem + lane_base + kColO + c0, rr);
         }
         tmem_wait_st();
       }
@@ -394,13 +424,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float ca = wa * inv, cb = wb * inv / l_run;
       uint16_t* orow = static_cast<uint16_t*>(P.pb.out) + elem;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
-        uint32_t rr[32];
-        LN_TMEM_LD32(tmem + lane_base + kColO + c0, rr);
-        tmem_wait_ld();
+      for (int c0 = 0; c0 < kD; c0 += kOChunk) {
+        uint32_t rr[kOChunk];
+        o_load(tmem + lane_base + kColO + c0, rr);
         if (write) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {  // 8 elements (16 bytes) at a time
+          for (int q = 0; q < kOChunk / 8; ++q) {  // 8 elements (16 bytes) at a time
             uint4 old = make_uint4(0, 0, 0, 0);
             if (!P.first_call) old = reinterpret_cast<const uint4*>(orow + c0)[q];
             const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
@@ -447,7 +476,8 @@ __global__ void __launch_bounds__(256) pp_init_kernel(const Problem pb) {
 }
 
 // View [B, N, H, D] (16-bit elements, starting `shift` positions in) as
-// (d, h, c, k, b), position = r k + c; boxes of 64 elements x box_rows k.
+// (d, h, c, k, b), position = r k + c; boxes of one panel row (64 elements,
+// or D below 64) x box_rows k.
 bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem& p, int64_t r, int64_t shift,
             int64_t kcount, int box_rows) {
   const int64_t es = 2, D = p.D;
@@ -455,18 +485,20 @@ bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem
   cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)p.H, (cuuint64_t)r, (cuuint64_t)kcount, (cuuint64_t)p.B};
   cuuint64_t strides[4] = {(cuuint64_t)(D * es), (cuuint64_t)(p.H * D * es), (cuuint64_t)(r * p.H * D * es),
                            (cuuint64_t)(p.N * p.H * D * es)};
-  cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
+  const int64_t pe = D >= 64 ? 64 : D;  // elements of a panel row
+  cuuint32_t box[5] = {(cuuint32_t)pe, 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapDataType ty =
       p.dtype == LONGNET_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return enc(map, ty, 5, const_cast<char*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             pe == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : pe == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kFmt, int kPanels>
+template <int kFmt, int kD>
 int launch_typed(const Problem& pb, cudaStream_t stream) {
-  using L = Layout<kPanels>;
+  using L = Layout<kD>;
   EncodeTiledFn enc = get_encoder();
   if (!enc) return LONGNET_ERR_CUDA;
   int dev = 0;
@@ -478,7 +510,7 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(pp_fwd_kernel<kFmt, kPanels>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
+    if (cudaFuncSetAttribute(pp_fwd_kernel<kFmt, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
         cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
@@ -491,7 +523,7 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
     const int64_t work = pb.B * (pb.q1 - pb.q0) * (pb.h1 - pb.h0) * (pb.D / 8);
     int64_t blocks = (work + 255) / 256;
     if (blocks > (int64_t)n_sm * 16) blocks = (int64_t)n_sm * 16;
-    pp_init_kernel<64 * kPanels><<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, stream>>>(pb);
+    pp_init_kernel<kD><<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, stream>>>(pb);
     if (cudaGetLastError() != cudaSuccess) return LONGNET_ERR_CUDA;
   }
   for (int i = 0; i < pb.n_pat; ++i) {
@@ -529,7 +561,7 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, pp_fwd_kernel<kFmt, kPanels>, P, maps) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, pp_fwd_kernel<kFmt, kD>, P, maps) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
@@ -540,7 +572,9 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
 }  // namespace pp
 
 bool perpattern_supports(const Problem& p) {
-  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || (p.D != 64 && p.D != 128)) return false;
+  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) ||
+      (p.D != 16 && p.D != 32 && p.D != 64 && p.D != 128))
+    return false;
   if (p.qk_norm) return false;           // the prologue entry takes qk_norm
   if (p.n_pat > 1 && !p.lse) return false;  // the merge runs through lse
   if (p.N > ((int64_t)1 << 30) || p.H > 65535 || p.B > 65535) return false;
@@ -559,8 +593,16 @@ bool perpattern_supports(const Problem& p) {
 
 int launch_perpattern(const Problem& p, cudaStream_t stream) {
   const bool f16 = p.dtype == LONGNET_DTYPE_F16;
-  if (p.D == 64) return f16 ? pp::launch_typed<tc::kFmtF16, 1>(p, stream) : pp::launch_typed<tc::kFmtBF16, 1>(p, stream);
-  return f16 ? pp::launch_typed<tc::kFmtF16, 2>(p, stream) : pp::launch_typed<tc::kFmtBF16, 2>(p, stream);
+  switch (p.D) {
+    case 16:
+      return f16 ? pp::launch_typed<tc::kFmtF16, 16>(p, stream) : pp::launch_typed<tc::kFmtBF16, 16>(p, stream);
+    case 32:
+      return f16 ? pp::launch_typed<tc::kFmtF16, 32>(p, stream) : pp::launch_typed<tc::kFmtBF16, 32>(p, stream);
+    case 64:
+      return f16 ? pp::launch_typed<tc::kFmtF16, 64>(p, stream) : pp::launch_typed<tc::kFmtBF16, 64>(p, stream);
+    default:
+      return f16 ? pp::launch_typed<tc::kFmtF16, 128>(p, stream) : pp::launch_typed<tc::kFmtBF16, 128>(p, stream);
+  }
 }
 
 }  // namespace longnet

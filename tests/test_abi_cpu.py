@@ -96,6 +96,9 @@ def test_select_impl_host_logic():
     # D = 128 (16-bit) goes to the per-pattern tcgen05 family, fp32 to the general kernel
     assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_PATTERNS
     assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, f32) == bd.LONGNET_IMPL_SIMT
+    # so do D = 32 and 16 (16-bit)
+    for D in (16, 32):
+        assert bd.longnet_select_impl(1, 4096, 4, D, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_PATTERNS
     # more than 6 patterns at D = 64: per-pattern family
     seven = tuple((256 * (i + 1), i + 1) for i in range(7))
     assert bd.longnet_select_impl(1, 4096, 4, 64, seven, True, bf16) == bd.LONGNET_IMPL_PATTERNS

@@ -105,6 +105,11 @@ PATTERNS_CASES = [
      ((128, 1), (256, 2), (384, 3), (512, 4), (768, 5), (1024, 6), (2048, 8))),
     ("bf16_d128_one_pattern", 1, 1024, 2, 128, torch.bfloat16, True, ((256, 1),)),
     ("bf16_d128_uncovered", 1, 960, 3, 128, torch.bfloat16, True, ((192, 3), (960, 4))),
+    # narrow heads: one 64- or 32-byte swizzle panel per row
+    ("bf16_d32_lm_like", 2, 2048, 4, 32, torch.bfloat16, True, ((512, 1), (1024, 2), (2048, 4))),
+    ("f16_d32_noncausal_partial", 1, 1500, 3, 32, torch.float16, False, ((384, 1), (700, 3), (2000, 5))),
+    ("bf16_d16_causal", 1, 2048, 4, 16, torch.bfloat16, True, ((256, 1), (1024, 4))),
+    ("f16_d16_noncausal", 2, 1024, 2, 16, torch.float16, False, ((128, 1), (512, 2), (1024, 8))),
 ]
 
 
