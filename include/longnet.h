@@ -366,9 +366,9 @@ int longnet_scatter_rows(const void* src, int64_t n, const int64_t* idx, void* d
  *     a = 1 / max(|x|, 1e-12); a g for a row with |x| <= 1e-12).  Other bits:
  *     LONGNET_ERR_INVALID_ARG.
  *   - impl: LONGNET_IMPL_AUTO (tcgen05 where it applies, else the tile
- *     kernels, else SIMT), LONGNET_IMPL_TCGEN05 (bf16/fp16, D = 64, no
- *     qk_norm, up to 6 patterns: TMA-fed tcgen05 tensor cores with TMEM
- *     accumulators), LONGNET_IMPL_TILES (bf16/fp16, D = 64: mma.sync tensor
+ *     kernels, else SIMT), LONGNET_IMPL_TCGEN05 (bf16/fp16, D = 16, 32, 64
+ *     or 128, no qk_norm, up to 6 patterns: TMA-fed tcgen05 tensor cores with
+ *     TMEM accumulators), LONGNET_IMPL_TILES (bf16/fp16, D = 64: mma.sync tensor
  *     cores) or LONGNET_IMPL_SIMT (fp32 FMA, D in {16, 32, 64, 128}, every
  *     dtype).  A family that does not cover the call: LONGNET_ERR_UNSUPPORTED.
  *   - Enqueued on stream; allocates nothing.  The tcgen05 and tile kernels

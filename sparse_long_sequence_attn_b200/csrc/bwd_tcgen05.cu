@@ -69,16 +69,25 @@ constexpr int kBlk = 64;                        // rows of a streamed block (N o
 constexpr int kMaxPat = 6;
 constexpr int kStages = 3;
 constexpr int kThreads = 192;                   // warp 0 loads, warp 1 MMAs, warps 2-5 compute
-constexpr int kTilePanel = kTile * 128;         // 16 KB: 128 rows of one 64-element swizzle panel
-constexpr int kBlkPanel = kBlk * 128;           // 8 KB
 // TMEM columns: scores (S or S^T), dP, then the accumulators.
 constexpr uint32_t kColS = 0, kColDP = 64, kColAcc0 = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Sizes for D = 64 kPanels (a row is kPanels 128-byte swizzle panels).
-template <int kPanels>
+// Sizes for a row of D elements: one or two 64-element panels (128-byte rows,
+// 128-byte swizzle) at D = 64 or 128, one panel of D elements (64- or 32-byte
+// rows and swizzle) at D = 32 or 16.
+template <int kDim>
 struct BL {
-  static constexpr int kD = 64 * kPanels;
+  static constexpr int kD = kDim;
+  static constexpr int kPanels = kD >= 64 ? kD / 64 : 1;
+  static constexpr int kPanelElems = kD >= 64 ? 64 : kD;
+  static constexpr int kRowBytes = kPanelElems * 2;
+  static constexpr int kTilePanel = kTile * kRowBytes;  // 128 rows of one panel
+  static constexpr int kBlkPanel = kBlk * kRowBytes;
+  // descriptor high word: stride between 8-row groups, sm_100 version, layout
+  // type (128-byte swizzle 2, 64-byte 4, 32-byte 6)
+  static constexpr uint32_t kDescHi = (uint32_t)(8 * kRowBytes >> 4) | (1u << 14) |
+                                      ((kRowBytes == 128 ? 2u : kRowBytes == 64 ? 4u : 6u) << 29);
   static constexpr int kTileBytes = kPanels * kTilePanel;
   static constexpr int kBlkBytes = kPanels * kBlkPanel;
   static constexpr int kStageBytes = 2 * kBlkBytes + 1024;  // two blocks, then lse and delta (key-centric)
@@ -262,10 +271,13 @@ __device__ __forceinline__ void p_ds_half(const uint32_t (&sr)[32], const uint32
 }
 
 // kKeys: the key-centric kernel (dk, dv); else the query-centric one (dq).
-template <int kFmt, bool kKeys, int kPanels>
-__global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
+template <int kFmt, bool kKeys, int kDim>
+__global__ void __launch_bounds__(kThreads, kDim <= 64 ? 2 : 1)
     bwd_tc_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
-  using L = BL<kPanels>;
+  using L = BL<kDim>;
+  constexpr int kPanels = L::kPanels;
+  constexpr int kTilePanel = L::kTilePanel, kBlkPanel = L::kBlkPanel;
+  constexpr uint32_t kDescHi = L::kDescHi;
   constexpr int kD = L::kD, kTileBytes = L::kTileBytes, kBlkBytes = L::kBlkBytes, kStageBytes = L::kStageBytes;
   constexpr uint32_t kColAcc1 = L::kColAcc1, kTmemCols = L::template tmem_cols<kKeys>();
   extern __shared__ uint8_t smem_raw[];
@@ -341,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
       mbar_arrive_expect_tx(bar_tile, 2 * kTileBytes);
 #pragma unroll
       for (int pn = 0; pn < kPanels; ++pn) {
-        tma_load_5d(sTile0 + pn * kTilePanel, mp + 0, bar_tile, 64 * pn, u.h, c.c, c.kk, u.b);
-        tma_load_5d(sTile1 + pn * kTilePanel, mp + 1, bar_tile, 64 * pn, u.h, c.c, c.kk, u.b);
+        tma_load_5d(sTile0 + pn * kTilePanel, mp + 0, bar_tile, L::kPanelElems * pn, u.h, c.c, c.kk, u.b);
+        tma_load_5d(sTile1 + pn * kTilePanel, mp + 1, bar_tile, L::kPanelElems * pn, u.h, c.c, c.kk, u.b);
       }
     }
     for (int j = 0; j < nblk && ok; ++j) {
@@ -371,8 +383,9 @@ __global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
         mbar_arrive_expect_tx(bar_full + st, 2 * kBlkBytes);
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn) {
-          tma_load_5d(stage + pn * kBlkPanel, mp + 2, bar_full + st, 64 * pn, u.h, c.c, c.kk, u.b);
-          tma_load_5d(stage + kBlkBytes + pn * kBlkPanel, mp + 3, bar_full + st, 64 * pn, u.h, c.c, c.kk, u.b);
+          tma_load_5d(stage + pn * kBlkPanel, mp + 2, bar_full + st, L::kPanelElems * pn, u.h, c.c, c.kk, u.b);
+          tma_load_5d(stage + kBlkBytes + pn * kBlkPanel, mp + 3, bar_full + st, L::kPanelElems * pn, u.h, c.c,
+                      c.kk, u.b);
         }
       } else {
         mbar_arrive(bar_full + st);
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
     if (lane == 0) {
       const uint32_t t0_lo = (smem_u32(sTile0) >> 4) | (1u << 16);
       const uint32_t t1_lo = (smem_u32(sTile1) >> 4) | (1u << 16);
-      const uint32_t lbo_mn = ((uint32_t)(kBlk * 128) >> 4) << 16;
+      const uint32_t lbo_mn = ((uint32_t)kBlkPanel >> 4) << 16;  // the panel stride along D
       // Blocks go in two halves of 32 streamed rows, so the tensor cores work
       // on one half while the compute warps work on the other:
       //   scores(0, a) scores(0, b) | grads(j, a) scores(j+1, a) | grads(j, b) scores(j+1, b) | ...
@@ -401,42 +414,43 @@ __global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
       // gradient products (issued just before, executed in order) have read.
       auto stage_addr = [&](int j) -> uint32_t { return smem_u32(sStage + (j % kStages) * kStageBytes) >> 4; };
       auto scores = [&](int j, int hf) {
-        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * 128 >> 4);
+        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * L::kRowBytes >> 4);
         const uint32_t b1_addr = b0_addr + (kBlkBytes >> 4);
         // tile0 x block0^T and tile1 x block1^T over the half's 32 rows
         // (K-major operands, one 64-element panel of D at a time)
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < L::kPanelElems / 16; ++kk)
             mma_ss(tmem + kColS + 32 * hf, desc_from(t0_lo + pn * (kTilePanel >> 4) + kk * 2, kDescHi),
                    desc_from(((b0_addr + pn * (kBlkPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>,
                    (pn > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int pn = 0; pn < kPanels; ++pn)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < L::kPanelElems / 16; ++kk)
             mma_ss(tmem + kColDP + 32 * hf, desc_from(t1_lo + pn * (kTilePanel >> 4) + kk * 2, kDescHi),
                    desc_from(((b1_addr + pn * (kBlkPanel >> 4)) | (1u << 16)) + kk * 2, kDescHi), kIdescScore<kFmt>,
                    (pn > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar_s + hf);
       };
       // gradients of a half: A (P or dS, packed) from TMEM, B the half's rows read MN-major
+      constexpr uint32_t kStep16 = 16 * L::kRowBytes >> 4;  // 16 rows of an MN-major operand
       auto grads = [&](int j, int hf) {
-        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * 128 >> 4);
+        const uint32_t b0_addr = stage_addr(j) + (uint32_t)(hf * 32 * L::kRowBytes >> 4);
         const uint32_t b1_addr = b0_addr + (kBlkBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 32; ++kk) {
           const uint32_t acc = (j > 0 || hf > 0 || kk > 0) ? 1u : 0u;
           if (kKeys) {
             // dV += P^T dout (block 1), dK += dS^T Q (block 0)
-            mma_ts(tmem + kColAcc0, tmem + kColS + 32 * hf + kk * 8, desc_from((b1_addr | lbo_mn) + kk * 128, kDescHi),
+            mma_ts(tmem + kColAcc0, tmem + kColS + 32 * hf + kk * 8, desc_from((b1_addr | lbo_mn) + kk * kStep16, kDescHi),
                    kIdescGrad<kFmt, kD>, acc);
-            mma_ts(tmem + kColAcc1, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
+            mma_ts(tmem + kColAcc1, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * kStep16, kDescHi),
                    kIdescGrad<kFmt, kD>, acc);
           } else {
             // dQ += dS K (block 0)
-            mma_ts(tmem + kColAcc0, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * 128, kDescHi),
+            mma_ts(tmem + kColAcc0, tmem + kColDP + 32 * hf + kk * 8, desc_from((b0_addr | lbo_mn) + kk * kStep16, kDescHi),
                    kIdescGrad<kFmt, kD>, acc);
           }
         }
@@ -529,15 +543,20 @@ __global__ void __launch_bounds__(kThreads, kPanels == 1 ? 2 : 1)
       for (int a = 0; a < (kKeys ? 2 : 1); ++a) {
         float* dst = kKeys ? (a == 0 ? P.g.dv : P.g.dk) : P.g.dq;
         const float sc = (kKeys && a == 0) ? 1.f : P.scale;
+        constexpr int kChunk = kD < 32 ? kD : 32;  // accumulator columns per TMEM load
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-          uint32_t acc[32];
-          LN_TMEM_LD32(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + c0, acc);
+        for (int c0 = 0; c0 < kD; c0 += kChunk) {
+          uint32_t acc[kChunk];
+          if constexpr (kChunk == 32) {
+            LN_TMEM_LD32(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + c0, acc);
+          } else {
+            LN_TMEM_LD16(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + c0, acc);
+          }
           tmem_wait_ld();
           if (row_ok) {
             float4* d4 = reinterpret_cast<float4*>(dst + elem + c0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
+            for (int c = 0; c < kChunk / 4; ++c)
               atomicAdd(d4 + c, make_float4(__uint_as_float(acc[4 * c]) * sc, __uint_as_float(acc[4 * c + 1]) * sc,
                                             __uint_as_float(acc[4 * c + 2]) * sc,
                                             __uint_as_float(acc[4 * c + 3]) * sc));
@@ -575,19 +594,22 @@ bool encode(EncodeTiledFn enc, CUtensorMap* map, const void* base, const Problem
   cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)p.H, (cuuint64_t)r, (cuuint64_t)kcount, (cuuint64_t)p.B};
   cuuint64_t strides[4] = {(cuuint64_t)(D * es), (cuuint64_t)(p.H * D * es), (cuuint64_t)(r * p.H * D * es),
                            (cuuint64_t)(p.N * p.H * D * es)};
-  cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
+  const int64_t pe = D >= 64 ? 64 : D;  // elements of a panel row
+  cuuint32_t box[5] = {(cuuint32_t)pe, 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapDataType ty =
       p.dtype == LONGNET_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return enc(map, ty, 5, const_cast<char*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             pe == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : pe == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // CTAs and the per-pattern geometry; false when the shape is outside this
 // family.
 bool geometry(const Problem& p, Params* P) {
-  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) || (p.D != 64 && p.D != 128) || p.qk_norm)
+  if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) ||
+      (p.D != 16 && p.D != 32 && p.D != 64 && p.D != 128) || p.qk_norm)
     return false;
   if (p.n_pat > kMaxPat || p.N > ((int64_t)1 << 30) || p.H > 65535 || p.B > 65535) return false;
   int64_t ctas = 0;
@@ -662,22 +684,36 @@ int launch_tcgen05_backward(const Problem& p, const BwdArgs& g, cudaStream_t str
     return LONGNET_ERR_CUDA;
   }
   const bool f16 = p.dtype == LONGNET_DTYPE_F16;
-  const int panels = (int)(p.D / 64);
-  auto kern_k = f16 ? (panels == 1 ? bwd_tc_kernel<kFmtF16, true, 1> : bwd_tc_kernel<kFmtF16, true, 2>)
-                    : (panels == 1 ? bwd_tc_kernel<kFmtBF16, true, 1> : bwd_tc_kernel<kFmtBF16, true, 2>);
-  auto kern_q = f16 ? (panels == 1 ? bwd_tc_kernel<kFmtF16, false, 1> : bwd_tc_kernel<kFmtF16, false, 2>)
-                    : (panels == 1 ? bwd_tc_kernel<kFmtBF16, false, 1> : bwd_tc_kernel<kFmtBF16, false, 2>);
-  auto kern_d = f16 ? (panels == 1 ? bwd_delta_kernel<kFmtF16, 64> : bwd_delta_kernel<kFmtF16, 128>)
-                    : (panels == 1 ? bwd_delta_kernel<kFmtBF16, 64> : bwd_delta_kernel<kFmtBF16, 128>);
-  const int kSmemBytes = panels == 1 ? BL<1>::kSmemBytes : BL<2>::kSmemBytes;
-  static bool attr_set[64][2][2] = {};
-  if (!attr_set[dev][f16][panels - 1]) {
+  using KFn = void (*)(Params, Maps);
+  using DFn = void (*)(const Problem, const uint16_t*, const uint16_t*, float*);
+  const int di = p.D == 16 ? 0 : p.D == 32 ? 1 : p.D == 64 ? 2 : 3;
+  static const KFn kk_tab[2][4] = {
+      {bwd_tc_kernel<kFmtBF16, true, 16>, bwd_tc_kernel<kFmtBF16, true, 32>, bwd_tc_kernel<kFmtBF16, true, 64>,
+       bwd_tc_kernel<kFmtBF16, true, 128>},
+      {bwd_tc_kernel<kFmtF16, true, 16>, bwd_tc_kernel<kFmtF16, true, 32>, bwd_tc_kernel<kFmtF16, true, 64>,
+       bwd_tc_kernel<kFmtF16, true, 128>}};
+  static const KFn kq_tab[2][4] = {
+      {bwd_tc_kernel<kFmtBF16, false, 16>, bwd_tc_kernel<kFmtBF16, false, 32>, bwd_tc_kernel<kFmtBF16, false, 64>,
+       bwd_tc_kernel<kFmtBF16, false, 128>},
+      {bwd_tc_kernel<kFmtF16, false, 16>, bwd_tc_kernel<kFmtF16, false, 32>, bwd_tc_kernel<kFmtF16, false, 64>,
+       bwd_tc_kernel<kFmtF16, false, 128>}};
+  static const DFn kd_tab[2][4] = {
+      {bwd_delta_kernel<kFmtBF16, 16>, bwd_delta_kernel<kFmtBF16, 32>, bwd_delta_kernel<kFmtBF16, 64>,
+       bwd_delta_kernel<kFmtBF16, 128>},
+      {bwd_delta_kernel<kFmtF16, 16>, bwd_delta_kernel<kFmtF16, 32>, bwd_delta_kernel<kFmtF16, 64>,
+       bwd_delta_kernel<kFmtF16, 128>}};
+  static const int smem_tab[4] = {BL<16>::kSmemBytes, BL<32>::kSmemBytes, BL<64>::kSmemBytes, BL<128>::kSmemBytes};
+  const KFn kern_k = kk_tab[f16][di], kern_q = kq_tab[f16][di];
+  const DFn kern_d = kd_tab[f16][di];
+  const int kSmemBytes = smem_tab[di];
+  static bool attr_set[64][2][4] = {};
+  if (!attr_set[dev][f16][di]) {
     if (cudaFuncSetAttribute(kern_k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern_q, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
-    attr_set[dev][f16][panels - 1] = true;
+    attr_set[dev][f16][di] = true;
   }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);

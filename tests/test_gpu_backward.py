@@ -87,6 +87,10 @@ CASES = [
     ("f16_d128", 1, 256, 2, 128, torch.float16, True, ((64, 1), (256, 2))),
     ("bf16_d128_lm_like", 1, 1024, 3, 128, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
     ("bf16_d128_noncausal_partial", 2, 700, 2, 128, torch.bfloat16, False, ((256, 1), (300, 3))),
+    # narrow heads on the tensor cores: one 64- or 32-byte swizzle panel per row
+    ("bf16_d32_lm_like", 1, 1024, 3, 32, torch.bfloat16, True, ((256, 1), (512, 2), (1024, 4))),
+    ("f16_d32_noncausal", 2, 512, 2, 32, torch.float16, False, ((128, 1), (512, 4))),
+    ("bf16_d16_causal", 1, 1024, 4, 16, torch.bfloat16, True, ((256, 1), (1024, 4))),
 ]
 
 
@@ -94,7 +98,7 @@ def _impls(dtype, D):
     out = [("simt", bd.LONGNET_IMPL_SIMT)]
     if dtype != torch.float32 and D == 64:
         out.append(("tiles", bd.LONGNET_IMPL_TILES))
-    if dtype != torch.float32 and D in (64, 128):
+    if dtype != torch.float32 and D in (16, 32, 64, 128):
         out.append(("tcgen05", bd.LONGNET_IMPL_TCGEN05))
     return out
 
