@@ -135,11 +135,13 @@ def test_backward_argument_checks_on_host():
     assert _call_bwd(lib, causal=3) == bd.LONGNET_ERR_INVALID_ARG
     for impl in (3, 5, -1):
         assert _call_bwd(lib, impl=impl) == bd.LONGNET_ERR_INVALID_ARG, impl
-    # the tensor-core families: bf16/fp16 and D = 64 only; tcgen05 also
-    # without qk_norm and with at most 6 patterns
+    # the tensor-core families: bf16/fp16 only; the tile family at D = 64, the
+    # tcgen05 one at D = 16, 32, 64 or 128, without qk_norm, with at most 6
+    # patterns
     for impl in (bd.LONGNET_IMPL_TILES, bd.LONGNET_IMPL_TCGEN05):
         assert _call_bwd(lib, impl=impl) == bd.LONGNET_ERR_UNSUPPORTED
-        assert _call_bwd(lib, impl=impl, dtype=1, D=32) == bd.LONGNET_ERR_UNSUPPORTED
+        assert _call_bwd(lib, impl=impl, dtype=1, D=48) == bd.LONGNET_ERR_UNSUPPORTED
+    assert _call_bwd(lib, impl=bd.LONGNET_IMPL_TILES, dtype=1, D=32) == bd.LONGNET_ERR_UNSUPPORTED
     assert _call_bwd(lib, impl=bd.LONGNET_IMPL_TCGEN05, dtype=1, D=64,
                      flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_UNSUPPORTED
     assert _call_bwd(lib, impl=bd.LONGNET_IMPL_TCGEN05, dtype=1, D=64,
@@ -159,6 +161,7 @@ def test_backward_valid_call_without_device_reports_no_device():
         assert _call_bwd(lib, dtype=dtype, pats=((24, 1), (64, 4))) == bd.LONGNET_ERR_NO_DEVICE
     assert _call_bwd(lib, dtype=1, D=64, impl=bd.LONGNET_IMPL_TILES) == bd.LONGNET_ERR_NO_DEVICE
     assert _call_bwd(lib, dtype=1, D=64, impl=bd.LONGNET_IMPL_TCGEN05) == bd.LONGNET_ERR_NO_DEVICE
+    assert _call_bwd(lib, dtype=1, D=32, impl=bd.LONGNET_IMPL_TCGEN05) == bd.LONGNET_ERR_NO_DEVICE
     # qk_norm is taken by both families
     assert _call_bwd(lib, flags=bd.LONGNET_FLAG_QK_NORM) == bd.LONGNET_ERR_NO_DEVICE
     assert _call_bwd(lib, dtype=2, D=64, flags=bd.LONGNET_FLAG_QK_NORM,
