@@ -270,6 +270,7 @@ WS_CASES = [
     ("ws_f16_d64_noncausal", 2, 512, 2, 64, torch.float16, False, ((128, 1), (512, 4))),
     ("ws_bf16_d128", 1, 1024, 2, 128, torch.bfloat16, True, ((256, 1), (1024, 2))),
     ("ws_fp32_d32_partial", 1, 300, 2, 32, torch.float32, True, ((64, 1), (128, 3))),
+    ("ws_bf16_d32", 1, 1024, 2, 32, torch.bfloat16, True, ((256, 1), (1024, 4))),
 ]
 WS_OPTIONS = {"qk_norm": (True, False), "xpos": (False, True), "both": (True, True)}
 
