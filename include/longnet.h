@@ -29,8 +29,7 @@
  *     When w does not divide N the last segment is the shorter rest of the
  *     sequence (no padding); w > N makes one segment of the whole sequence.
  *     Patterns may repeat and come in any order; a repeated pattern counts
- *     twice.  (The small-segment kernel takes N % w == 0 only; AUTO picks
- *     another family otherwise.)
+ *     twice.
  *   - causal: 1 = causal inside each sparsified segment, 0 = full.
  *   - stream: a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued asynchronously; the call returns before it finishes.
@@ -82,7 +81,8 @@ enum longnet_impl {
                                 tcgen05/TMEM flash kernel, patterns fused in
                                 shared memory */
   LONGNET_IMPL_SMALLSEG = 3, /* bf16 or fp16, D = 64, all patterns one segment
-                                length w <= 64 (a multiple of 8), up to 8
+                                length w <= 64 (a multiple of 8; the last
+                                segment may be shorter), up to 8
                                 patterns when every r divides 8, else up to
                                 4; q, k, v, out 16-byte aligned: memory-bound
                                 kernel, one weighted softmax per segment */
@@ -305,8 +305,8 @@ int longnet_dilated_attn_fwd_host(const void* q_host, const void* k_host, const 
  * the keys and values of longer segments coming from the other devices), and
  * the step of a split by heads.  0 <= q_begin < q_end <= N and
  * 0 <= h_begin < h_end <= H, else LONGNET_ERR_INVALID_ARG.  The small-segment
- * kernel takes parts made of whole segments only (AUTO then picks another
- * family).  The other conventions are those of the full forward.
+ * kernel takes parts made of whole segments only (the sequence's shorter last
+ * one included; AUTO otherwise picks another family).  The other conventions are those of the full forward.
  */
 int longnet_dilated_attn_fwd_part(const void* q, const void* k, const void* v,
                                   void* out, float* lse,

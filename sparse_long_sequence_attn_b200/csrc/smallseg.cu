@@ -1,6 +1,7 @@
 // Kernel family SMALLSEG: the multi-pattern dilated-attention forward when
 // every pattern's segments are short (all patterns share one segment length
-// W <= 64, bf16 or fp16, D = 64).  Such shapes move far more bytes than they compute
+// W <= 64, bf16 or fp16, D = 64; the last segment may be the shorter rest of
+// the sequence).  Such shapes move far more bytes than they compute
 // (the DilatedAttention usage example of the "LongNet" docs page: segment 64,
 // dilation 2), so this kernel is built for HBM bandwidth, not tensor peak.
 //
@@ -65,7 +66,8 @@ constexpr int kTableBytes = 8 * 32 * 8;  // [h mod 8][lane] packed log2 c pair
 
 // Softmax variants.
 //   kModeFull:    every r divides 8, some r = 1, not causal, W a multiple of 16:
-//                 every key of every row has weight >= 1, no column is masked;
+//                 every key of every row has weight >= 1, no column is masked
+//                 (but the keys past the end of a short last segment);
 //   kModeMasked:  every r divides 8, otherwise (causal, W not a multiple of
 //                 16, or keys of weight 0);
 //   kModeGeneral: some r does not divide 8: weights counted per element.
@@ -261,6 +263,15 @@ __device__ __forceinline__ void attend_chunk(uint32_t q_base, uint32_t k_base, u
   float m0, m1;  // the exponents' stabilisers (log2 domain)
   uint32_t pa[4][4];  // P as A fragments, one per 16-key step
   if constexpr (kMode == kModeFull) {
+    if (W & 15) {
+      // a short last segment: the keys past its end (zeros from the load)
+      // inside the last 16-key step get no weight
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (nt * 8 + 2 * t4 + e >= W) acc[nt][e] = acc[nt][2 + e] = -INFINITY;
+    }
     // every weight >= 1: the largest raw score of the row stabilises
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -482,11 +493,11 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
   const int W = P.W;
   const int H = (int)P.pb.H;
   const int64_t N = P.pb.N;
-  const int seg0 = (int)(P.pb.q0 / W), n_seg = (int)((P.pb.q1 - P.pb.q0) / W);
+  // segments of the part; the last one may be the shorter rest of the sequence
+  const int seg0 = (int)(P.pb.q0 / W), n_seg = (int)((P.pb.q1 - P.pb.q0 + W - 1) / W);
   const int h0 = (int)P.pb.h0, Hr = (int)(P.pb.h1 - P.pb.h0);
   const bool causal = P.pb.causal != 0;
   const int g = lane >> 2, t4 = lane & 3;  // mma fragment coordinates
-  const int n_kt = (W + 15) >> 4;          // 16-key steps and 16-row chunks
   const float scale_log2 = 1.4426950408889634f * rsqrtf((float)kD);
   const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
   uint32_t phase = 0;
@@ -497,6 +508,10 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
     const int64_t bs = item / Hr;
     const int seg = seg0 + (int)(bs % n_seg);
     const int b = (int)(bs / n_seg);
+    // rows (and keys) of this segment: W, or the rest of the sequence; the
+    // tiles' rows past N load as zeros and are not stored
+    const int Wr = N - (int64_t)seg * W < W ? (int)(N - (int64_t)seg * W) : W;
+    const int n_kt = (Wr + 15) >> 4;  // 16-key steps and 16-row chunks
     // ---- load the segment's rows of this head (both warps are done with the
     // previous item: the pair synchronised before its store)
     __syncwarp();
@@ -587,14 +602,14 @@ __global__ void __launch_bounds__(kMaxPairs * 64, 1)
       }
       float ov[8][4];
       float lse0, lse1;
-      attend_chunk<kFmt, kMode>(q_base, k_base, v_base, W, n_kt, rc, causal, scale_log2, lane, lb, cw0, cw1, ov,
+      attend_chunk<kFmt, kMode>(q_base, k_base, v_base, Wr, n_kt, rc, causal, scale_log2, lane, lb, cw0, cw1, ov,
                                 lse0, lse1);
       // ---- stage the rows over their own Q rows (no longer read: later
       // chunks read other rows) in the same swizzled layout
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int row = rc * 16 + g + 8 * half;
-        if (row < W) {
+        if (row < Wr) {
           uint8_t* sr = sQ + row * 128 + 4 * t4;
 #pragma unroll
           for (int nt = 0; nt < 8; ++nt)
@@ -639,8 +654,8 @@ bool smallseg_supports(const Problem& p) {
   if (W < 1 || W > kMaxW || W % 8 != 0) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.w[i] != W) return false;
-  if (W > p.N || p.N % W != 0) return false;  // whole segments only
-  if (p.q0 % W != 0 || p.q1 % W != 0) return false;  // a part of whole segments
+  // a part of whole segments (the sequence's last one may be shorter)
+  if (p.q0 % W != 0 || (p.q1 % W != 0 && p.q1 != p.N)) return false;
   if (p.H > 65535 || p.B > 65535 || p.N > (int64_t)INT32_MAX) return false;
   for (int i = 0; i < p.n_pat; ++i)
     if (p.r[i] < 1 || p.r[i] > (int64_t)INT32_MAX) return false;
@@ -674,7 +689,7 @@ int launch_smallseg(const Problem& pb, cudaStream_t stream) {
   if (P.n_pairs > kMaxPairs) P.n_pairs = kMaxPairs;
   // items of the computed part: (b, segment, head) with segments in
   // [q0 / W, q1 / W) and heads in [h0, h1)
-  P.n_items = pb.B * ((pb.q1 - pb.q0) / P.W) * (pb.h1 - pb.h0);
+  P.n_items = pb.B * ((pb.q1 - pb.q0 + P.W - 1) / P.W) * (pb.h1 - pb.h0);
   int dev = 0, n_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
       cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

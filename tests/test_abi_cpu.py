@@ -96,6 +96,8 @@ def test_select_impl_host_logic():
     # D = 128 (16-bit) goes to the per-pattern tcgen05 family, fp32 to the general kernel
     assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_PATTERNS
     assert bd.longnet_select_impl(1, 4096, 4, 128, ((1024, 1), (2048, 2)), True, f32) == bd.LONGNET_IMPL_SIMT
+    # one short segment length with a shorter last segment: the small-segment family
+    assert bd.longnet_select_impl(2, 1000, 4, 64, ((64, 1), (64, 2)), False, bf16) == bd.LONGNET_IMPL_SMALLSEG
     # so do D = 32 and 16 (16-bit)
     for D in (16, 32):
         assert bd.longnet_select_impl(1, 4096, 4, D, ((1024, 1), (2048, 2)), True, bf16) == bd.LONGNET_IMPL_PATTERNS

@@ -57,6 +57,11 @@ SMALL_CASES = [
      ((64, 1), (64, 2), (64, 4), (64, 8), (64, 2), (64, 4), (64, 8), (64, 1))),
     ("bf16_d64_seg32_no_r1_causal", 1, 512, 8, 64, torch.bfloat16, True, ((32, 2), (32, 4), (32, 8))),
     ("f16_d64_seg48_r8_causal", 2, 480, 9, 64, torch.float16, True, ((48, 1), (48, 8), (48, 4))),
+    # one segment length, the last segment the shorter rest (or w > N)
+    ("bf16_d64_seg64_partial_noncausal", 2, 1000, 4, 64, torch.bfloat16, False, ((64, 1), (64, 2))),
+    ("f16_d64_seg32_partial_causal", 1, 500, 3, 64, torch.float16, True, ((32, 1), (32, 4))),
+    ("bf16_d64_seg48_w_gt_n", 2, 40, 2, 64, torch.bfloat16, False, ((48, 1), (48, 2), (48, 3))),
+    ("f16_d64_seg32_odd_n", 1, 1001, 2, 64, torch.float16, False, ((32, 1), (32, 2), (32, 4))),
     # fp16 inputs (every family)
     ("f16_d64_lm_like", 2, 2048, 4, 64, torch.float16, True, ((512, 1), (1024, 2), (2048, 4))),
     ("f16_d64_r_not_dividing", 1, 1536, 5, 64, torch.float16, True, ((384, 3), (768, 4), (1536, 8))),
