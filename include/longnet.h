@@ -251,7 +251,9 @@ int longnet_dilated_attn_fwd_noalloc(const void* q, const void* k, const void* v
  *     its own rows), copied as strided 2-D blocks;
  *   B = 1, H < 4, causal: ranges of positions, in order (a row attends to
  *     keys at or before it, which arrived with its piece or an earlier one),
- *     each attended as a part (longnet_dilated_attn_fwd_part).
+ *     each attended as a part (longnet_dilated_attn_fwd_part); the rows of
+ *     k_dev and v_dev past the first piece are zeroed before any copy, since
+ *     a part may read later key rows (masked) that must be finite.
  *   q_host, k_host, v_host: [B, N, H, D] inputs in host memory; out_host
  *     [B, N, H, D] and lse_host [B, H, N] (may be NULL) outputs in host
  *     memory.  Page-locked (pinned) memory lets the copies run asynchronously;

@@ -407,6 +407,14 @@ extern "C" int longnet_dilated_attn_fwd_host(const void* q_host, const void* k_h
   // earlier call may still read these device buffers)
   bool ok = cu(cudaEventRecord(hp->start, cs)) && cu(cudaStreamWaitEvent(hp->in, hp->start, 0)) &&
             cu(cudaStreamWaitEvent(hp->out, hp->start, 0));
+  if (ok && mode == 1 && per < N) {
+    // A piece's attention may read key and value rows past its end (a tile's
+    // K/V block reaches further and masks them), which later pieces bring
+    // in: until then they must be finite, so they start as zeros (B = 1).
+    const size_t tail = (size_t)(N - per) * row;
+    ok = cu(cudaMemsetAsync(atw(k_dev, (size_t)per * row), 0, tail, hp->in)) &&
+         cu(cudaMemsetAsync(atw(v_dev, (size_t)per * row), 0, tail, hp->in));
+  }
   int frc = LONGNET_OK;
   const void* hin[3] = {q_host, k_host, v_host};
   void* din[3] = {q_dev, k_dev, v_dev};

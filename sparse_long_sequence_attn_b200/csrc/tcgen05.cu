@@ -1022,39 +1022,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         LN_TMEM_LD32(s_col + 0, (sr + 0));
         LN_TMEM_LD32(s_col + 32, (sr + 32));
         tmem_wait_ld();
-        if constexpr (kNorm) {
-          const float4* ik4 = reinterpret_cast<const float4*>(ikn + (blk & 1) * kBN);
-#pragma unroll
-          for (int c4 = 0; c4 < kBN / 4; ++c4) {
-            const float4 f = ik4[c4];
-            sr[4 * c4 + 0] = __float_as_uint(__uint_as_float(sr[4 * c4 + 0]) * f.x);
-            sr[4 * c4 + 1] = __float_as_uint(__uint_as_float(sr[4 * c4 + 1]) * f.y);
-            sr[4 * c4 + 2] = __float_as_uint(__uint_as_float(sr[4 * c4 + 2]) * f.z);
-            sr[4 * c4 + 3] = __float_as_uint(__uint_as_float(sr[4 * c4 + 3]) * f.w);
-          }
-        }
         if (lim < kBN - 1) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (c > lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        float pm[8];
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
-#pragma unroll
-        for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        const float m_blk = mx * row_scale;
         float corr = 1.f;
         bool rescale = false;
-        if (m_blk > m_use + 8.f || m_use == -INFINITY) {
-          if (m_blk != -INFINITY) {
-            if (m_use != -INFINITY) {
-              corr = ex2(m_use - m_blk);
-              rescale = true;
+        if constexpr (kNorm) {
+          // unit rows: a logit s |q|^-1 |k|^-1 scale_log2 is a cosine times
+          // scale_log2, so scale_log2 bounds it (up to rounding) and serves as
+          // the stabiliser of every block: no row maximum, no rescaling
+          m_use = scale_log2;
+        } else {
+          float pm[8];
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
+#pragma unroll
+          for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
+          const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          const float m_blk = mx * row_scale;
+          if (m_blk > m_use + 8.f || m_use == -INFINITY) {
+            if (m_blk != -INFINITY) {
+              if (m_use != -INFINITY) {
+                corr = ex2(m_use - m_blk);
+                rescale = true;
+              }
+              m_use = m_blk;
             }
-            m_use = m_blk;
           }
         }
         // P = 2^(s*scale - m) in the input format over the first 32 columns of this S buffer
@@ -1065,10 +1061,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[32];
           const uint64_t sc2 = f32x2(row_scale, row_scale), nm2 = f32x2(-m_use, -m_use);
           uint64_t ls[4] = {0, 0, 0, 0};  // row sum of P in packed pairs
+          // qk_norm: the block's inverse key norms as packed pairs
+          const ulonglong2* ik2 = reinterpret_cast<const ulonglong2*>(ikn + (blk & 1) * kBN);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
+            uint64_t coef = sc2;  // the scale of keys 2c and 2c + 1
+            if constexpr (kNorm) {
+              const ulonglong2 pr = ik2[c >> 1];
+              coef = mul_f32x2((c & 1) ? pr.y : pr.x, sc2);
+            }
             float xa, xb;
-            f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sc2, nm2), xa, xb);
+            f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), coef, nm2), xa, xb);
             const float a = ex2(xa), bq = ex2(xb);
             ls[c & 3] = add_f32x2(ls[c & 3], f32x2(a, bq));
             pk[c] = pack2<kFmt>(a, bq);

@@ -57,9 +57,11 @@ def test_host_entry_matches_oracle_and_device_entry(case):
     qh, kh, vh = (_host(x, pinned) for x in (q, k, v))
     out_h = torch.full((B, N, H, D), float("nan"), dtype=dtype, pin_memory=pinned)
     lse_h = torch.full((B, H, N), float("nan"), dtype=torch.float32, pin_memory=pinned) if with_lse else None
-    qd, kd, vd = (torch.empty(B, N, H, D, dtype=dtype, device=dev) for _ in range(3))
-    out_d = torch.empty(B, N, H, D, dtype=dtype, device=dev)
-    lse_d = torch.empty(B, H, N, dtype=torch.float32, device=dev) if with_lse else None
+    # device staging full of NaN: a row read before its copy arrived, or an
+    # output row never written, shows
+    qd, kd, vd = (torch.full((B, N, H, D), float("nan"), dtype=dtype, device=dev) for _ in range(3))
+    out_d = torch.full((B, N, H, D), float("nan"), dtype=dtype, device=dev)
+    lse_d = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev) if with_lse else None
     stream = torch.cuda.Stream(device=dev)
     bd.longnet_dilated_attn_fwd_host(qh, kh, vh, out_h, lse_h, qd, kd, vd, out_d, lse_d, pats, causal,
                                      stream=stream, pieces=chunk)
@@ -80,17 +82,19 @@ def test_host_entry_matches_oracle_and_device_entry(case):
     print(f"{name}: max|out - oracle| = {err:.3e}, max|out - device entry| = {d:.3e}")
 
 
-def test_two_calls_in_a_row_reuse_the_staging_buffers():
-    """The second call's copies in wait for the first call's attention (the
-    staging buffers are shared), and each call's results are its own."""
+@pytest.mark.parametrize("H", [8, 2], ids=["heads", "positions"])
+def test_two_calls_in_a_row_reuse_the_staging_buffers(H):
+    """The second call's copies in (and, by positions, the zeroing of the
+    key and value rows still to come) wait for the first call's attention
+    (the staging buffers are shared), and each call's results are its own."""
     dev = torch.device("cuda:0")
-    B, N, H, D, dtype, pats = 1, 4096, 8, 64, torch.bfloat16, ((512, 1), (2048, 4))
+    B, N, D, dtype, pats = 1, 4096, 64, torch.bfloat16, ((512, 1), (2048, 4))
     sets = [wl.random_inputs(B, N, H, D, dtype, seed=s) for s in (31, 32)]
     hosts = [tuple(_host(x, True) for x in s) for s in sets]
     outs = [torch.empty(B, N, H, D, dtype=dtype, pin_memory=True) for _ in range(2)]
     lses = [torch.empty(B, H, N, dtype=torch.float32, pin_memory=True) for _ in range(2)]
-    qd, kd, vd, od = (torch.empty(B, N, H, D, dtype=dtype, device=dev) for _ in range(4))
-    ld = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    qd, kd, vd, od = (torch.full((B, N, H, D), float("nan"), dtype=dtype, device=dev) for _ in range(4))
+    ld = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     for (qh, kh, vh), oh, lh in zip(hosts, outs, lses):
         bd.longnet_dilated_attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, pats, True, stream=stream,
@@ -113,8 +117,8 @@ def test_host_entry_with_qk_norm():
     qh, kh, vh = (_host(x, True) for x in (q, k, v))
     out_h = torch.full((B, N, H, D), float("nan"), dtype=dtype, pin_memory=True)
     lse_h = torch.full((B, H, N), float("nan"), dtype=torch.float32, pin_memory=True)
-    qd, kd, vd, od = (torch.empty(B, N, H, D, dtype=dtype, device=dev) for _ in range(4))
-    ld = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    qd, kd, vd, od = (torch.full((B, N, H, D), float("nan"), dtype=dtype, device=dev) for _ in range(4))
+    ld = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     bd.longnet_dilated_attn_fwd_host(qh, kh, vh, out_h, lse_h, qd, kd, vd, od, ld, pats, True, stream=stream,
                                      qk_norm=True)
