@@ -90,7 +90,8 @@ enum longnet_impl {
                                 patterns: 64-row tiles of the sparsified
                                 segments on mma.sync tensor cores */
   LONGNET_IMPL_PATTERNS = 5  /* forward: bf16 or fp16, D = 16, 32, 64 or 128, any number
-                                of patterns, lse required with more than one:
+                                of patterns, qk_norm or not, lse required with
+                                more than one:
                                 one tcgen05 launch per pattern, each merging its
                                 rows into out and lse (initialised to 0 and
                                 -inf); out is rounded to the input format
@@ -124,12 +125,11 @@ enum longnet_flags {
   /* Scale every q row and every k row (over D) to unit L2 norm before the
    * scores: x / max(|x|, 1e-12), computed in fp32.  The reading adopted for
    * the qk_norm option of the DilatedAttention module ("LongNet" docs page,
-   * usage example).  Through longnet_dilated_attn_fwd_ex the SIMT,
-   * small-segment and tcgen05 kernels apply it inside the attention (the
-   * small-segment kernel rounds the normalised rows back to the input
-   * format, the SIMT kernel keeps them in fp32, the tcgen05 kernel scales
-   * the scores of the rows as given by both inverse norms in fp32); the
-   * per-pattern family declines it (AUTO falls back); through
+   * usage example).  Through longnet_dilated_attn_fwd_ex every forward
+   * family applies it inside the attention (the small-segment kernel rounds
+   * the normalised rows back to the input format, the SIMT kernel keeps them
+   * in fp32, the tcgen05 and per-pattern kernels scale the scores of the rows
+   * as given by both inverse norms in fp32); through
    * longnet_dilated_attn_fwd_ws a prologue pass applies it and every family
    * takes the result. */
   LONGNET_FLAG_QK_NORM = 1,

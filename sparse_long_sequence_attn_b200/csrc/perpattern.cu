@@ -83,7 +83,8 @@ struct Layout {
   static constexpr int kBars = kQBytes + kStages * kStageBytes;
   // at least 80 KB, so no third CTA (whose 256 TMEM columns would not fit)
   // shares an SM
-  static constexpr int kSmem = kBars + 256 + 1024 > 80 * 1024 ? kBars + 256 + 1024 : 80 * 1024;
+  // barriers (256 B), then qk_norm's inverse key norms [2][kBlk] (512 B)
+  static constexpr int kSmem = kBars + 768 + 1024 > 80 * 1024 ? kBars + 768 + 1024 : 80 * 1024;
 };
 
 struct Params {
@@ -138,7 +139,11 @@ struct Waiter {
   __device__ bool wait_warp(uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, wait(bar, parity)); }
 };
 
-template <int kFmt, int kD>
+// kNorm: LONGNET_FLAG_QK_NORM, q and k rows taken at unit L2 norm: the
+// scores are scaled in fp32 by the row's and the key's inverse norms, which
+// bounds a scaled logit by the softmax scale (a cosine times it), the fixed
+// stabiliser of every block.
+template <int kFmt, int kD, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 2)
     pp_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   using L = Layout<kD>;
@@ -207,6 +212,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar_drain = bar_s + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* bar_ikn = bar_s + 8;  // qk_norm: [2] block parity, one arrival per softmax thread
+  float* ikn = reinterpret_cast<float*>(smem + L::kBars + 256);  // qk_norm: [2][kBlk]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -222,6 +229,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bar_od, 1);
     mbar_init(bar_of, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_ikn + 0, 128);
+    mbar_init(bar_ikn + 1, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -329,8 +338,49 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int tr = t0 + row;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    const uint64_t sc2 = f32x2(P.scale_log2, P.scale_log2);
+    // Sum of squares of a row of 16-bit elements in a swizzled tile: the
+    // swizzle only permutes the 16-byte chunks inside each row's bytes, so
+    // chunks [c0, c1) of the row (panel after panel) are summed in place.
+    auto row_sumsq = [](const uint8_t* tile, int panel_bytes, int r, int c0, int c1) -> float {
+      constexpr int kCpr = L::kRowBytes / 16;  // chunks per panel row
+      float acc = 0.f;
+#pragma unroll
+      for (int i = c0; i < c1; ++i) {
+        const uint4 u = *reinterpret_cast<const uint4*>(tile + (i / kCpr) * panel_bytes + r * L::kRowBytes +
+                                                         (i % kCpr) * 16);
+        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float lo, hi;
+          unpack2<kFmt>(wv[e], lo, hi);
+          acc = fmaf(lo, lo, fmaf(hi, hi, acc));
+        }
+      }
+      return acc;
+    };
+    float row_scale = P.scale_log2;  // with qk_norm times the row's inverse q norm
+    if constexpr (kNorm) {
+      ok = wt.wait_warp(bar_q, 0);
+      if (ok) row_scale = P.scale_log2 / fmaxf(sqrtf(row_sumsq(sQ, kQPanel, row, 0, kD / 8)), 1e-12f);
+    }
+    const uint64_t sc2 = f32x2(row_scale, row_scale);
     for (int j = 0; j < nblk && ok; ++j) {
+      if constexpr (kNorm) {
+        // this block's inverse key norms (its K block stays in its stage until
+        // its P V has run): thread t sums half of key row t / 2
+        ok = wt.wait_warp(bar_full + j % S, (j / S) & 1);
+        if (!ok) break;
+        const int kr = row >> 1, half = row & 1;
+        float ss = row_sumsq(sStage + (j % S) * L::kStageBytes, kKVPanel, kr, half * (kD / 16),
+                             (half + 1) * (kD / 16));
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        // block j - 2's array (this parity) is read by everyone before any
+        // thread arrives for block j - 1, so it may be rewritten now
+        if (half == 0) ikn[(j & 1) * kBlk + kr] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+        mbar_arrive(bar_ikn + (j & 1));
+        ok = wt.wait_warp(bar_ikn + (j & 1), (j >> 1) & 1);
+        if (!ok) break;
+      }
       ok = wt.wait_warp(bar_s + (j & 1), (j >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
@@ -347,22 +397,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int c = 0; c < kBlk; ++c)
           if (c > lim) sr[c] = __float_as_uint(-INFINITY);
       }
-      float pm[8];
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
-#pragma unroll
-      for (int c = 8; c < kBlk; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      const float m_blk = mx * P.scale_log2;
       float corr = 1.f;
       bool rescale = false;
-      if (m_blk > m_use + 8.f || m_use == -INFINITY) {
-        if (m_blk != -INFINITY) {
-          if (m_use != -INFINITY) {
-            corr = ex2(m_use - m_blk);
-            rescale = true;
+      if constexpr (kNorm) {
+        m_use = P.scale_log2;  // the bound of every scaled logit
+      } else {
+        float pm[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(sr[q8]);
+#pragma unroll
+        for (int c = 8; c < kBlk; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float m_blk = mx * P.scale_log2;
+        if (m_blk > m_use + 8.f || m_use == -INFINITY) {
+          if (m_blk != -INFINITY) {
+            if (m_use != -INFINITY) {
+              corr = ex2(m_use - m_blk);
+              rescale = true;
+            }
+            m_use = m_blk;
           }
-          m_use = m_blk;
         }
       }
       // P = 2^(s scale - m) in the input format over the first 32 columns
@@ -371,10 +425,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint32_t pk[32];
         const uint64_t nm2 = f32x2(-m_use, -m_use);
         uint64_t ls[4] = {0, 0, 0, 0};
+        const ulonglong2* ik2 = reinterpret_cast<const ulonglong2*>(ikn + (j & 1) * kBlk);  // qk_norm
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
+          uint64_t coef = sc2;  // the scale of keys 2c and 2c + 1
+          if constexpr (kNorm) {
+            const ulonglong2 pr = ik2[c >> 1];
+            coef = mul_f32x2((c & 1) ? pr.y : pr.x, sc2);
+          }
           float xa, xb;
-          f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sc2, nm2), xa, xb);
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), coef, nm2), xa, xb);
           const float a = ex2(xa), bq = ex2(xb);
           ls[c & 3] = add_f32x2(ls[c & 3], f32x2(a, bq));
           pk[c] = pack2<kFmt>(a, bq);
@@ -506,16 +566,17 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
     cudaGetLastError();
     return LONGNET_ERR_CUDA;
   }
-  static bool attr_set[64] = {};
+  const bool norm = pb.qk_norm != 0;
+  auto kernel = norm ? pp_fwd_kernel<kFmt, kD, true> : pp_fwd_kernel<kFmt, kD, false>;
+  static bool attr_set[64][2] = {};
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(pp_fwd_kernel<kFmt, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
-        cudaSuccess) {
+  if (!attr_set[dev][norm]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
-    attr_set[dev] = true;
+    attr_set[dev][norm] = true;
   }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
@@ -561,7 +622,7 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, pp_fwd_kernel<kFmt, kD>, P, maps) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kernel, P, maps) != cudaSuccess) {
       cudaGetLastError();
       return LONGNET_ERR_CUDA;
     }
@@ -575,7 +636,6 @@ bool perpattern_supports(const Problem& p) {
   if ((p.dtype != LONGNET_DTYPE_BF16 && p.dtype != LONGNET_DTYPE_F16) ||
       (p.D != 16 && p.D != 32 && p.D != 64 && p.D != 128))
     return false;
-  if (p.qk_norm) return false;           // the prologue entry takes qk_norm
   if (p.n_pat > 1 && !p.lse) return false;  // the merge runs through lse
   if (p.N > ((int64_t)1 << 30) || p.H > 65535 || p.B > 65535) return false;
   int64_t ctas = 0;

@@ -194,6 +194,10 @@ QK_NORM_CASES = [
     ("six_patterns_bf16", 1, 3072, 2, 64, torch.bfloat16, True,
      ((256, 1), (512, 2), (768, 3), (1024, 4), (1536, 6), (3072, 12))),
     ("fp32_d32", 1, 384, 2, 32, torch.float32, True, ((96, 1), (192, 5), (384, 7))),
+    # head sizes other than 64: the per-pattern family (several tiles, a partial one)
+    ("d128_bf16", 1, 1280, 2, 128, torch.bfloat16, True, ((256, 1), (1280, 4))),
+    ("d32_f16_noncausal", 2, 640, 3, 32, torch.float16, False, ((128, 1), (640, 2))),
+    ("d16_bf16", 1, 896, 2, 16, torch.bfloat16, True, ((256, 1), (896, 3))),
 ]
 
 
@@ -202,17 +206,19 @@ def test_qk_norm_option(case):
     """LONGNET_FLAG_QK_NORM on raw q and k (rows of norm about 3*sqrt(D); v
     of unit scale, so the 16-bit bounds keep their meaning), against the
     oracle with its q, k rows normalised in fp64; AUTO, SIMT, the small-
-    segment kernel and the tcgen05 kernel (which scales the scores by the
-    rows' inverse norms) take it where they take the shape."""
+    segment kernel, the tcgen05 and the per-pattern kernels (which scale the
+    scores by the rows' inverse norms) take it where they take the shape."""
     name, B, N, H, D, dtype, causal, pats = case
     seed = zlib.crc32(name.encode()) % 100000
     q, k, _ = wl.random_inputs(B, N, H, D, dtype, seed=seed, scale=3.0)
     _, _, v = wl.random_inputs(B, N, H, D, dtype, seed=seed + 1)
-    for impl in (bd.LONGNET_IMPL_AUTO, bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_SMALLSEG, bd.LONGNET_IMPL_TCGEN05):
+    for impl in (bd.LONGNET_IMPL_AUTO, bd.LONGNET_IMPL_SIMT, bd.LONGNET_IMPL_SMALLSEG, bd.LONGNET_IMPL_TCGEN05,
+                 bd.LONGNET_IMPL_PATTERNS):
         try:
             o, l = gh.run_cuda(q, k, v, pats, causal, impl, qk_norm=True)
         except bd.LongNetError as e:
-            assert impl in (bd.LONGNET_IMPL_SMALLSEG, bd.LONGNET_IMPL_TCGEN05) and e.code == bd.LONGNET_ERR_UNSUPPORTED
+            assert impl in (bd.LONGNET_IMPL_SMALLSEG, bd.LONGNET_IMPL_TCGEN05, bd.LONGNET_IMPL_PATTERNS)
+            assert e.code == bd.LONGNET_ERR_UNSUPPORTED
             continue
         gh.compare_full(o, l, q, k, v, pats, causal, dtype, label=f"qk_norm {name}/{impl}", qk_norm=True)
 
