@@ -815,6 +815,7 @@ def variant_lines(steps, warmup, dev_index=0):
     cases = [("plain", base.N, base.H, base.D, "plain"), ("qk_norm_prologue", base.N, base.H, base.D, "ws_norm"),
              ("xpos_prologue", base.N, base.H, base.D, "ws_xpos"),
              ("qk_norm_in_kernel", base.N, base.H, base.D, "ex_norm"),
+             ("qk_norm_in_kernel_d128", base.N, base.H // 2, 128, "ex_norm"),
              ("partial_last_segment", base.N - 64, base.H, base.D, "plain"),
              ("d128", base.N, base.H // 2, 128, "plain"), ("d32", base.N, base.H * 2, 32, "plain")]
     for name, N, H, D, mode in cases:
@@ -849,8 +850,6 @@ def variant_lines(steps, warmup, dev_index=0):
         if st != 0:
             raise RuntimeError(f"device status after variant {name}: {bd.status_string(st)}")
         fam = _impl_name(bd.longnet_select_impl(base.B, N, H, D, base.patterns, base.causal, torch.bfloat16))
-        if mode == "ex_norm" and fam == "patterns":
-            fam = "simt"  # the per-pattern family does not apply qk_norm in the kernel
         t = sum(per) / len(per)
         res.append({"variant": name, "N": N, "H": H, "D": D, "family": fam, "steps": n,
                     "ms": t * 1e3, "tokens_per_s": base.B * N / t})
