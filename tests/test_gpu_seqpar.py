@@ -208,3 +208,41 @@ def test_sequence_parallel_forward_single_rank_group():
         assert np.array_equal(o.float().cpu().numpy(), o1) and np.array_equal(l.cpu().numpy(), l1)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("impl_name,D", [("auto", 128), ("patterns", 64), ("tcgen05", 64), ("auto", 32)])
+def test_qk_norm_parts_assemble_the_full_forward(impl_name, D):
+    """qk_norm through the part entry: ranges of positions, then ranges of
+    heads, each computed by its own call (as the sequence-parallel and head
+    splits make them).  Each assembled output equals the single call and the
+    oracle on normalised rows; nothing outside a call's part is written."""
+    B, N, H = 1, 3000, max(1, 256 // D)
+    pats = ((512, 1), (1024, 2), (3000, 4))
+    q, k, _ = wl.random_inputs(B, N, H, D, torch.bfloat16, seed=91 + D, scale=3.0)
+    _, _, v = wl.random_inputs(B, N, H, D, torch.bfloat16, seed=92 + D)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    impl = IMPLS[impl_name]
+    o1, l1 = gh.run_cuda(q, k, v, pats, True, impl, qk_norm=True)
+    splits = {"positions": [((a, e), None) for a, e in ((0, 1000), (1000, 2200), (2200, N))],
+              "heads": [((0, N), (h0, h1)) for h0, h1 in ((0, 1), (1, H))] if H > 1 else [((0, N), (0, 1))]}
+    for kind, parts in splits.items():
+        out = np.full_like(o1, np.nan)
+        lse = np.full_like(l1, np.nan)
+        for (a, e), hr in parts:
+            h0, h1 = hr if hr is not None else (0, H)
+            o = torch.full((B, N, H, D), OUT_SENTINEL, dtype=q.dtype, device=dev)
+            l = torch.full((B, H, N), LSE_SENTINEL, dtype=torch.float32, device=dev)
+            bd.longnet_dilated_attn_fwd_part(qd, kd, vd, o, l, pats, True, (a, e), hr, impl, qk_norm=True)
+            assert bd.longnet_last_device_status() == 0
+            oc, lc = o.float().cpu().numpy(), l.cpu().numpy()
+            inside = np.zeros((N, H), dtype=bool)
+            inside[a:e, h0:h1] = True
+            assert (oc[:, ~inside] == OUT_SENTINEL).all(), f"{kind}: a write outside the part"
+            assert (lc.transpose(0, 2, 1)[:, ~inside] == LSE_SENTINEL).all(), f"{kind}: an lse write outside"
+            out[:, a:e, h0:h1] = oc[:, a:e, h0:h1]
+            lse[:, h0:h1, a:e] = lc[:, h0:h1, a:e]
+        assert not np.isnan(out).any() and not np.isnan(lse).any()
+        assert float(np.abs(out - o1).max()) <= gh.TOL_OUT[torch.bfloat16], kind
+        gh.compare_full(out, lse, q, k, v, pats, True, torch.bfloat16, label=f"qk_norm {kind}/{impl_name}/D{D}",
+                        qk_norm=True)
