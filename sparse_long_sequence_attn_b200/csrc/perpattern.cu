@@ -56,7 +56,8 @@ using namespace tc;
 
 constexpr int kTile = 128;   // rows per CTA (M of the MMAs)
 constexpr int kBlk = 64;     // keys per block (N of S = Q K^T)
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;      // loads, MMA issue, four softmax warps
+constexpr int kThreadsNorm = 256;  // with qk_norm, and two warps for the key norms
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;  // scores at 0 and 64
 constexpr float kLog2e = 1.4426950408889634f;
@@ -144,7 +145,7 @@ struct Waiter {
 // bounds a scaled logit by the softmax scale (a cosine times it), the fixed
 // stabiliser of every block.
 template <int kFmt, int kD, bool kNorm>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kNorm ? kThreadsNorm : kThreads, 2)
     pp_fwd_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps maps) {
   using L = Layout<kD>;
   constexpr int kPanels = L::kPanels;
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar_drain = bar_s + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* bar_ikn = bar_s + 8;  // qk_norm: [2] block parity, one arrival per softmax thread
+  uint64_t* bar_ikn = bar_s + 8;  // qk_norm: [2] block parity, one arrival per lane of the norm warps
   float* ikn = reinterpret_cast<float*>(smem + L::kBars + 256);  // qk_norm: [2][kBlk]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -229,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bar_od, 1);
     mbar_init(bar_of, 1);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_ikn + 0, 128);
-    mbar_init(bar_ikn + 1, 128);
+    mbar_init(bar_ikn + 0, 64);
+    mbar_init(bar_ikn + 1, 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -249,6 +250,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Waiter wt{abort_flag, P.pb.status, P.wait_limit_ns};
+  // qk_norm: sum of squares of a row of 16-bit elements in a swizzled tile;
+  // the swizzle only permutes the 16-byte chunks inside each row's bytes, so
+  // the row's chunks (panel after panel) are summed in place
+  auto row_sumsq = [](const uint8_t* tile, int panel_bytes, int r) -> float {
+    constexpr int kCpr = L::kRowBytes / 16;  // chunks per panel row
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) {
+      const uint4 u =
+          *reinterpret_cast<const uint4*>(tile + (i / kCpr) * panel_bytes + r * L::kRowBytes + (i % kCpr) * 16);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        unpack2<kFmt>(wv[e], lo, hi);
+        acc = fmaf(lo, lo, fmaf(hi, hi, acc));
+      }
+    }
+    return acc;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
@@ -331,6 +352,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_commit(bar_drain);
       if (!mbar_wait(bar_drain, 0, P.wait_limit_ns)) record_status(P.pb.status, kStatusTimeout);
     }
+  } else if (kNorm && warp >= 6) {
+    // ------------------------------------------------------------ key norms (qk_norm)
+    // Per block: the inverse norms of its 64 K rows (the K block stays in its
+    // stage until its P V has run) into the array of the block's parity, once
+    // the block has landed and, from block 2 on, every softmax thread has
+    // written block j - 2's P, which it does after its last read of that
+    // block's array (the same parity).  Warps 6 and 7, one key per lane.
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      ok = wt.wait_warp(bar_full + j % S, (j / S) & 1);
+      if (ok && j >= 2) ok = wt.wait_warp(bar_p + (j & 1), ((j - 2) >> 1) & 1);
+      if (!ok) break;
+      const uint8_t* kb = sStage + (j % S) * L::kStageBytes;
+      const int kr = 32 * (warp - 6) + lane;
+      ikn[(j & 1) * kBlk + kr] = 1.f / fmaxf(sqrtf(row_sumsq(kb, kKVPanel, kr)), 1e-12f);
+      mbar_arrive(bar_ikn + (j & 1));
+    }
   } else {
     // ------------------------------------------------------------ softmax and the merge
     const int row = 32 * (warp & 3) + lane;  // TMEM lane = tile row
@@ -338,46 +376,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int tr = t0 + row;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // Sum of squares of a row of 16-bit elements in a swizzled tile: the
-    // swizzle only permutes the 16-byte chunks inside each row's bytes, so
-    // chunks [c0, c1) of the row (panel after panel) are summed in place.
-    auto row_sumsq = [](const uint8_t* tile, int panel_bytes, int r, int c0, int c1) -> float {
-      constexpr int kCpr = L::kRowBytes / 16;  // chunks per panel row
-      float acc = 0.f;
-#pragma unroll
-      for (int i = c0; i < c1; ++i) {
-        const uint4 u = *reinterpret_cast<const uint4*>(tile + (i / kCpr) * panel_bytes + r * L::kRowBytes +
-                                                         (i % kCpr) * 16);
-        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float lo, hi;
-          unpack2<kFmt>(wv[e], lo, hi);
-          acc = fmaf(lo, lo, fmaf(hi, hi, acc));
-        }
-      }
-      return acc;
-    };
     float row_scale = P.scale_log2;  // with qk_norm times the row's inverse q norm
     if constexpr (kNorm) {
       ok = wt.wait_warp(bar_q, 0);
-      if (ok) row_scale = P.scale_log2 / fmaxf(sqrtf(row_sumsq(sQ, kQPanel, row, 0, kD / 8)), 1e-12f);
+      if (ok) row_scale = P.scale_log2 / fmaxf(sqrtf(row_sumsq(sQ, kQPanel, row)), 1e-12f);
     }
     const uint64_t sc2 = f32x2(row_scale, row_scale);
     for (int j = 0; j < nblk && ok; ++j) {
       if constexpr (kNorm) {
-        // this block's inverse key norms (its K block stays in its stage until
-        // its P V has run): thread t sums half of key row t / 2
-        ok = wt.wait_warp(bar_full + j % S, (j / S) & 1);
-        if (!ok) break;
-        const int kr = row >> 1, half = row & 1;
-        float ss = row_sumsq(sStage + (j % S) * L::kStageBytes, kKVPanel, kr, half * (kD / 16),
-                             (half + 1) * (kD / 16));
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        // block j - 2's array (this parity) is read by everyone before any
-        // thread arrives for block j - 1, so it may be rewritten now
-        if (half == 0) ikn[(j & 1) * kBlk + kr] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
-        mbar_arrive(bar_ikn + (j & 1));
+        // this block's inverse key norms, from the norm warp
         ok = wt.wait_warp(bar_ikn + (j & 1), (j >> 1) & 1);
         if (!ok) break;
       }
@@ -614,7 +621,7 @@ int launch_typed(const Problem& pb, cudaStream_t stream) {
     // (griddepcontrol.wait) before it reads or writes out and lse
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(norm ? kThreadsNorm : kThreads);
     cfg.dynamicSmemBytes = L::kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
